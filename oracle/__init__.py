@@ -1,0 +1,230 @@
+"""Plain CPU oracle for the MoE expert-epilogue ops (numpy front end).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import this package.  The
+product path (``moe_expert_epilogue_b200``) never imports it, and the two share
+no code: the arithmetic lives in ``moe_oracle.c`` (plain C, fp32 evaluation of
+each documented formula, one rounding to the storage dtype), built here into
+``libmoe_oracle.so`` with gcc and called through ctypes.
+
+Array conventions: bf16 and fp16 tensors are passed as ``numpy.uint16`` arrays
+holding the raw bits; fp32 as ``numpy.float32``; index maps as ``numpy.int32``.
+Every function allocates and returns its outputs.
+
+Pins: see ``tests/test_oracle_pins.py``.  Every op has at least one pin that is
+independent of this code (library routines, closed forms, float64 finite
+differences, brute force on tiny inputs); no function is left unpinned.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libmoe_oracle.so")
+_LOCK = threading.Lock()
+_LIB = None
+
+BF16, F16, F32 = 0, 1, 2
+SQRELU, SQRELU_CLAMP, SWIGLU = 0, 1, 2
+ERR_COUNT, ERR_MAP, ERR_INVERSE = 1, 2, 4
+
+_CFLAGS = ["-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no FMA contraction, no fast math)."""
+    stale = (not os.path.exists(_LIB_PATH)
+             or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *_CFLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _lib():
+    global _LIB
+    with _LOCK:
+        if _LIB is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            P, I64, I32, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
+            sig = {
+                "orc_bf16_from_f32": (ctypes.c_uint16, [F]),
+                "orc_f32_from_bf16": (F, [ctypes.c_uint16]),
+                "orc_f16_from_f32": (ctypes.c_uint16, [F]),
+                "orc_f32_from_f16": (F, [ctypes.c_uint16]),
+                "orc_swiglu_clamped_fwd": (None, [P, P, P, I64, I64, I64, I64, F]),
+                "orc_swiglu_clamped_bwd": (None, [P, P, P, P, P, P, I64, I64, I64, I64, I64, F]),
+                "orc_swiglu_clamped_fwd_f64": (None, [P, P, P, P, I64, ctypes.c_double]),
+                "orc_router_weight_fwd": (None, [P, ctypes.c_int, P, P, ctypes.c_int, I64, I64]),
+                "orc_router_weight_bwd": (None, [P, ctypes.c_int, P, ctypes.c_int, P, P, P, P,
+                                                 I64, I64]),
+                "orc_act_with_probs_permuted": (ctypes.c_int, [ctypes.c_int, P, P, P, I32, P, I64,
+                                                               I64, I64, F, ctypes.c_int]),
+                "orc_unpermute_ordered": (ctypes.c_int, [P, ctypes.c_int, I64, P, I32, P,
+                                                         ctypes.c_int, I64, I64, I32]),
+                "orc_residual_add": (None, [P, P, P, P, I64, ctypes.c_int]),
+            }
+            for name, (res, args) in sig.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _LIB = lib
+    return _LIB
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    if a is None:
+        return None
+    a = np.ascontiguousarray(a)
+    if a.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {a.dtype}")
+    return a
+
+
+def _storage_np(dt):
+    return np.float32 if dt == F32 else np.uint16
+
+
+# ------------------------------------------------------------ scalar dtypes
+
+def bf16_from_f32(values) -> np.ndarray:
+    """Round fp32 values to bf16 bits (RNE), elementwise."""
+    lib = _lib()
+    v = np.asarray(values, dtype=np.float32).ravel()
+    return np.array([lib.orc_bf16_from_f32(float(x)) for x in v], dtype=np.uint16)
+
+
+def f32_from_bf16(bits) -> np.ndarray:
+    lib = _lib()
+    b = np.asarray(bits, dtype=np.uint16).ravel()
+    return np.array([lib.orc_f32_from_bf16(int(x)) for x in b], dtype=np.float32)
+
+
+def f16_from_f32(values) -> np.ndarray:
+    lib = _lib()
+    v = np.asarray(values, dtype=np.float32).ravel()
+    return np.array([lib.orc_f16_from_f32(float(x)) for x in v], dtype=np.uint16)
+
+
+def f32_from_f16(bits) -> np.ndarray:
+    lib = _lib()
+    b = np.asarray(bits, dtype=np.uint16).ravel()
+    return np.array([lib.orc_f32_from_f16(int(x)) for x in b], dtype=np.float32)
+
+
+# -------------------------------------------------------------- the ops
+
+def swiglu_clamped_fwd(x: np.ndarray, probs: np.ndarray, limit: float) -> np.ndarray:
+    """x: uint16 bf16 bits [rows, 2*inter]; probs: float32 [rows] or [rows, 1].
+    Returns y: uint16 bf16 bits [rows, inter]."""
+    x = _c(x, np.uint16)
+    rows, two_i = x.shape
+    inter = two_i // 2
+    probs = _c(np.asarray(probs, np.float32).reshape(rows), np.float32)
+    y = np.empty((rows, inter), np.uint16)
+    _lib().orc_swiglu_clamped_fwd(_p(x), _p(probs), _p(y), rows, inter, two_i, inter,
+                                  float(limit))
+    return y
+
+
+def swiglu_clamped_bwd(x, probs, grad_y, limit):
+    """Returns (grad_x uint16 [rows, 2*inter], grad_probs float64 [rows],
+    grad_probs_abs float64 [rows])."""
+    x = _c(x, np.uint16)
+    rows, two_i = x.shape
+    inter = two_i // 2
+    probs = _c(np.asarray(probs, np.float32).reshape(rows), np.float32)
+    grad_y = _c(grad_y, np.uint16)
+    assert grad_y.shape == (rows, inter)
+    gx = np.empty((rows, two_i), np.uint16)
+    gp = np.empty(rows, np.float64)
+    ga = np.empty(rows, np.float64)
+    _lib().orc_swiglu_clamped_bwd(_p(x), _p(probs), _p(grad_y), _p(gx), _p(gp), _p(ga),
+                                  rows, inter, two_i, inter, two_i, float(limit))
+    return gx, gp, ga
+
+
+def swiglu_clamped_fwd_f64(g, u, p, limit) -> np.ndarray:
+    g = _c(np.asarray(g, np.float64).ravel(), np.float64)
+    u = _c(np.asarray(u, np.float64).ravel(), np.float64)
+    p = _c(np.asarray(p, np.float64).ravel(), np.float64)
+    y = np.empty_like(g)
+    _lib().orc_swiglu_clamped_fwd_f64(_p(g), _p(u), _p(p), _p(y), g.size, float(limit))
+    return y
+
+
+def router_weight_fwd(x, x_dt, probs, out_dt):
+    x = _c(x, _storage_np(x_dt))
+    rows, hidden = x.shape
+    probs = _c(np.asarray(probs, np.float32).reshape(rows), np.float32)
+    out = np.empty((rows, hidden), _storage_np(out_dt))
+    _lib().orc_router_weight_fwd(_p(x), x_dt, _p(probs), _p(out), out_dt, rows, hidden)
+    return out
+
+
+def router_weight_bwd(grad_out, g_dt, x, x_dt, probs):
+    """x may be None (forward did not save x).  Returns (grad_x, grad_probs f64
+    or None, grad_probs_abs f64 or None)."""
+    grad_out = _c(grad_out, _storage_np(g_dt))
+    rows, hidden = grad_out.shape
+    x = _c(x, _storage_np(x_dt))
+    probs = _c(np.asarray(probs, np.float32).reshape(rows), np.float32)
+    gx = np.empty((rows, hidden), _storage_np(x_dt))
+    gp = np.empty(rows, np.float64) if x is not None else None
+    ga = np.empty(rows, np.float64) if x is not None else None
+    _lib().orc_router_weight_bwd(_p(grad_out), g_dt, _p(x), x_dt, _p(probs), _p(gx),
+                                 _p(gp), _p(ga), rows, hidden)
+    return gx, gp, ga
+
+
+def act_with_probs_permuted(act, x, out_init, permutation_map, n_used, probs, width,
+                            clamp_scale=1.0, zero_padding=False):
+    """x: uint16 [max_rows, width or 2*width]; out_init: uint16 [max_rows, width]
+    (its contents stand for whatever the output buffer held before the call).
+    Returns (out, error_bits)."""
+    x = _c(x, np.uint16)
+    out = np.array(out_init, dtype=np.uint16, copy=True)
+    max_rows = out.shape[0]
+    pm = _c(permutation_map, np.int32)
+    probs = _c(np.asarray(probs, np.float32).ravel(), np.float32)
+    err = _lib().orc_act_with_probs_permuted(act, _p(x), _p(out), _p(pm), int(n_used),
+                                             _p(probs), probs.size, max_rows, width,
+                                             float(clamp_scale), int(bool(zero_padding)))
+    return out, err
+
+
+def unpermute_ordered(expert_output, in_dt, inverse_map, valid_tokens, out_init, out_dt):
+    """expert_output [max_rows, hidden]; inverse_map int32 [tokens, E];
+    out_init [tokens, hidden] (prior contents).  Returns (out, error_bits)."""
+    eo = _c(expert_output, _storage_np(in_dt))
+    max_rows, hidden = eo.shape
+    inv = _c(inverse_map, np.int32)
+    tokens, n_exp = inv.shape
+    out = np.array(out_init, dtype=_storage_np(out_dt), copy=True)
+    assert out.shape == (tokens, hidden)
+    err = _lib().orc_unpermute_ordered(_p(eo), in_dt, max_rows, _p(inv), int(valid_tokens),
+                                       _p(out), out_dt, tokens, hidden, n_exp)
+    return out, err
+
+
+def residual_add(expert_output, shared_expert_output, residual, dt):
+    st = _storage_np(dt)
+    e = _c(expert_output, st)
+    s = _c(shared_expert_output, st)
+    r = _c(residual, st)
+    assert e.shape == s.shape == r.shape
+    out = np.empty_like(r)
+    _lib().orc_residual_add(_p(e), _p(s), _p(r), _p(out), e.size, dt)
+    return out
