@@ -1,0 +1,596 @@
+#!/usr/bin/env python
+"""Throughput of the MoE expert-epilogue pass on B200: achieved HBM GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole epilogue over one batch of seeded synthetic
+inputs that are resident in HBM before timing starts:
+
+    clamped SwiGLU fwd and bwd      rows 65536 (8192 tokens x top-8), inter 2048, L 10
+    router-weight multiply fwd/bwd  [16384, 7168] bf16, fp32 probs, save_x on
+    permuted activation x3          8192 tokens, top-8 of 64 experts, 128-row alignment,
+                                    width 1536: SQRELU, SQRELU_CLAMP (scale 7), SWIGLU,
+                                    zero padding on
+    fixed-order unpermute           -> [8192, 4096] bf16
+    residual add                    [32768, 7168] bf16; its expert_output's first
+                                    16384 rows are the router-weight forward's output
+
+value = algorithmic bytes of all steps on all ranks / max-over-ranks device
+time (CUDA events on the launching stream, barrier + synchronize on both
+sides).  Every kernel's working set exceeds the 126 MB L2, so no flush is
+needed between steps.  Multi-GPU runs (torchrun) are weak scaling: each rank
+runs the full step on its own inputs; the only collectives are the barrier and
+the max of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import contextlib
+import datetime
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "clamped-SwiGLU fwd+bwd achieved HBM GB/s and % of B200 peak; rows/s"
+FALLBACK_HBM_GBS = 6650.0
+
+# ---------------------------------------------------------------- workload
+
+SWIGLU = dict(rows=65536, inter=2048, limit=10.0, sigma=3.0)
+ROUTER = dict(rows=16384, hidden=7168)
+PERMUTED = dict(tokens=8192, top_k=8, experts=64, align=128, width=1536, hidden=4096, scale=7.0)
+RESIDUAL = dict(rows=32768, hidden=7168)
+
+WORKLOAD_NAME = ("moe_expert_epilogue_pass: clamped SwiGLU fwd+bwd rows=65536 inter=2048 L=10; "
+                 "router-weight fwd+bwd [16384,7168]; permuted SQRELU/SQRELU_CLAMP/SWIGLU + "
+                 "ordered unpermute (8192 tok, top-8 of 64, align 128, width 1536, hidden 4096); "
+                 "residual add [32768,7168]; all bf16 with fp32 probs")
+
+
+def algorithmic_bytes(n_used: int) -> dict:
+    """Minimal bytes per launch: each input byte read once, each output byte
+    written once; padding rows count as written (zero padding), never as read."""
+    R, I = SWIGLU["rows"], SWIGLU["inter"]
+    Rr, H = ROUTER["rows"], ROUTER["hidden"]
+    live = PERMUTED["tokens"] * PERMUTED["top_k"]
+    W = PERMUTED["width"]
+    T, E, Hu = PERMUTED["tokens"], PERMUTED["experts"], PERMUTED["hidden"]
+    meta = 4 * n_used + 4 * live          # permutation map rows + gathered probs
+    return {
+        "swiglu_fwd": R * (2 * I * 2 + 4 + I * 2),
+        "swiglu_bwd": R * (2 * I * 2 + I * 2 + 4 + 2 * I * 2 + 4),
+        "router_weight_fwd": Rr * H * 2 * 2 + Rr * 4,
+        "router_weight_bwd": Rr * H * 2 * 3 + Rr * 8,
+        "act_sqrelu": live * W * 2 + n_used * W * 2 + meta,
+        "act_sqrelu_clamp": live * W * 2 + n_used * W * 2 + meta,
+        "act_swiglu": live * 2 * W * 2 + n_used * W * 2 + meta,
+        "unpermute": live * Hu * 2 + T * E * 4 + T * Hu * 2,
+        "residual_add": 4 * RESIDUAL["rows"] * RESIDUAL["hidden"] * 2,
+    }
+
+
+ROWS = {  # rows (or tokens) one launch processes, for rows/s
+    "swiglu_fwd": SWIGLU["rows"], "swiglu_bwd": SWIGLU["rows"],
+    "router_weight_fwd": ROUTER["rows"], "router_weight_bwd": ROUTER["rows"],
+    "act_sqrelu": None, "act_sqrelu_clamp": None, "act_swiglu": None,
+    "unpermute": PERMUTED["tokens"], "residual_add": RESIDUAL["rows"],
+}
+
+KERNEL_SOURCES = {
+    "swiglu_fwd": "swiglu_clamped.cu", "swiglu_bwd": "swiglu_clamped.cu",
+    "router_weight_fwd": "router_weight.cu", "router_weight_bwd": "router_weight.cu",
+    "act_sqrelu": "act_permuted.cu", "act_sqrelu_clamp": "act_permuted.cu",
+    "act_swiglu": "act_permuted.cu", "unpermute": "unpermute_ordered.cu",
+    "residual_add": "residual_add.cu",
+}
+
+
+class Batch:
+    """All inputs and outputs of one step, on one device."""
+
+    def __init__(self, device, seed):
+        from moe_expert_epilogue_b200 import inputs
+        gen_dev = device if device.type == "cuda" else "cpu"
+        sw = inputs.swiglu_inputs(SWIGLU["rows"], SWIGLU["inter"], sigma=SWIGLU["sigma"],
+                                  probs="topk_softmax", seed=seed, device=gen_dev)
+        self.sw_x, self.sw_p, self.sw_gy = sw["x"], sw["probs"], sw["grad_y"]
+        rw = inputs.router_weight_inputs(ROUTER["rows"], ROUTER["hidden"], seed=seed + 1,
+                                         device=gen_dev)
+        self.rw_x, self.rw_p, self.rw_g = rw["x"], rw["probs"], rw["grad_out"]
+        rt = inputs.routing(PERMUTED["tokens"], PERMUTED["top_k"], PERMUTED["experts"],
+                            PERMUTED["align"], seed=seed + 2, device=gen_dev)
+        self.rt = rt
+        W = PERMUTED["width"]
+        self.act_x = inputs.permuted_activation_input(rt, W, swiglu=False, seed=seed + 3,
+                                                      device=gen_dev)
+        self.act_x2 = inputs.permuted_activation_input(rt, W, swiglu=True, seed=seed + 4,
+                                                       device=gen_dev)
+        self.pmap, self.probs = rt.permutation_map, rt.probs
+        self.n_used = torch.tensor([rt.n_used], dtype=torch.int32, device=gen_dev)
+        self.eo = inputs.expert_output_input(rt, PERMUTED["hidden"], seed=seed + 5, device=gen_dev)
+        self.inv = rt.inverse_map
+        self.valid = torch.tensor([rt.tokens], dtype=torch.int32, device=gen_dev)
+        res = inputs.residual_inputs((RESIDUAL["rows"], RESIDUAL["hidden"]), torch.bfloat16,
+                                     seed=seed + 6, device=gen_dev)
+        self.res_e, self.res_s, self.res_r = (res["expert_output"], res["shared_expert_output"],
+                                              res["residual"])
+        self.to(device)
+        # outputs
+        z = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device=device)  # noqa: E731
+        R, I = SWIGLU["rows"], SWIGLU["inter"]
+        self.sw_y, self.sw_gx, self.sw_gp = z(R, I), z(R, 2 * I), z(R, 1, dt=torch.float32)
+        self.rw_gx, self.rw_gp = z(ROUTER["rows"], ROUTER["hidden"]), z(ROUTER["rows"], 1,
+                                                                        dt=torch.float32)
+        self.act_o1, self.act_o2, self.act_o3 = (z(rt.max_rows, W) for _ in range(3))
+        self.unp_out = z(PERMUTED["tokens"], PERMUTED["hidden"])
+        self.res_out = z(RESIDUAL["rows"], RESIDUAL["hidden"])
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
+
+    INPUT_NAMES = ("sw_x", "sw_p", "sw_gy", "rw_x", "rw_p", "rw_g", "act_x", "act_x2", "pmap",
+                   "probs", "n_used", "eo", "inv", "valid", "res_e", "res_s", "res_r")
+    OUTPUT_NAMES = ("sw_y", "sw_gx", "sw_gp", "rw_gx", "rw_gp", "act_o1", "act_o2", "act_o3",
+                    "unp_out", "res_out")
+
+    def to(self, device):
+        for k in self.INPUT_NAMES:
+            setattr(self, k, getattr(self, k).to(device))
+
+    def kernels(self):
+        """(name, launch) pairs of one step, in MoE-layer order."""
+        from moe_expert_epilogue_b200 import ops
+        L = SWIGLU["limit"]
+        P = PERMUTED
+        half = ROUTER["rows"]
+        # the router-weight forward writes the first half of the residual's expert output
+        rw_out = self.res_e[:half]
+        return [
+            ("swiglu_fwd", lambda: ops.swiglu_clamped_fwd(self.sw_x, self.sw_p, L, out=self.sw_y)),
+            ("router_weight_fwd", lambda: ops.router_weight_mul_fwd(
+                self.rw_x, self.rw_p, torch.bfloat16, out=rw_out)),
+            ("act_sqrelu", lambda: ops.act_with_probs_permuted(
+                ops.MOE_ACT_SQRELU, self.act_x, self.pmap, self.n_used, self.probs, 1.0, True,
+                out=self.act_o1, dev_err=self.dev_err)),
+            ("act_sqrelu_clamp", lambda: ops.act_with_probs_permuted(
+                ops.MOE_ACT_SQRELU_CLAMP, self.act_x, self.pmap, self.n_used, self.probs,
+                P["scale"], True, out=self.act_o2, dev_err=self.dev_err)),
+            ("act_swiglu", lambda: ops.act_with_probs_permuted(
+                ops.MOE_ACT_SWIGLU, self.act_x2, self.pmap, self.n_used, self.probs, 1.0, True,
+                out=self.act_o3, dev_err=self.dev_err)),
+            ("unpermute", lambda: ops.unpermute_ordered(self.eo, self.inv, self.valid,
+                                                        self.unp_out, dev_err=self.dev_err)),
+            ("residual_add", lambda: ops.residual_add(self.res_e, self.res_s, self.res_r,
+                                                      out=self.res_out)),
+            ("router_weight_bwd", lambda: ops.router_weight_mul_bwd(
+                self.rw_g, self.rw_x, self.rw_p, grad_x=self.rw_gx, grad_probs=self.rw_gp)),
+            ("swiglu_bwd", lambda: ops.swiglu_clamped_bwd(self.sw_x, self.sw_p, self.sw_gy, L,
+                                                          grad_x=self.sw_gx,
+                                                          grad_probs=self.sw_gp)),
+        ]
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Max of a scalar over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate_value(bytes_per_step: int, steps: int, world: int, max_seconds: float) -> float:
+    """Whole-job GB/s: every rank's bytes over the slowest rank's time."""
+    return bytes_per_step * steps * world / max_seconds / 1e9
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        self.path = tempfile.mktemp(suffix=".csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            t0 = time.time()
+            while time.time() - t0 < 5 and os.path.getsize(self.path) == 0:
+                time.sleep(0.02)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            self.proc.wait(timeout=5)
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), max=float(parts[2]),
+                                 power=float(parts[3]) if parts[3] not in ("[N/A]", "") else 0.0,
+                                 active=parts[4], hw=parts[5], hwt=parts[6], swt=parts[7],
+                                 pcap=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] > 250.0] or rows
+        sms = sorted(r["sm"] for r in loaded)
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": sms[len(sms) // 2], "sm_max_mhz": loaded[0]["max"],
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# ---------------------------------------------------------------- peaks, traffic
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest(fn: str) -> str:
+    csrc = os.path.join(ROOT, "moe_expert_epilogue_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted([fn, "common.cuh"]):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel's source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            entry = json.load(f)[kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    if entry.get("source_digest") != source_digest(KERNEL_SOURCES[kernel]):
+        return None
+    return entry.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args):
+    from moe_expert_epilogue_b200 import build as mbuild
+    rank, local_rank, world = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=device,
+                                timeout=datetime.timedelta(seconds=120))
+    if not mbuild.up_to_date():
+        if rank == 0:
+            mbuild.build()
+        barrier(device)
+
+    batch = Batch(device, seed=1000 * rank)
+    kernels = batch.kernels()
+    nbytes = algorithmic_bytes(batch.rt.n_used)
+    bytes_per_step = sum(nbytes.values())
+    stream = torch.cuda.current_stream(device)
+
+    for _ in range(args.warmup):
+        for _, fn in kernels:
+            fn()
+    torch.cuda.synchronize(device)
+
+    K = args.steps
+    ev = {name: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(K)] for name, _ in kernels}
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(device.index) if not args.no_clocks else contextlib.nullcontext()
+    with sampler:
+        barrier(device)
+        torch.cuda.synchronize(device)
+        t_start.record(stream)
+        for k in range(K):
+            for name, fn in kernels:
+                ev[name][k][0].record(stream)
+                fn()
+                ev[name][k][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+    elapsed_ms = t_start.elapsed_time(t_end)
+    max_ms = max_over_ranks(elapsed_ms, device)
+    clocks = sampler.summary() if not args.no_clocks else None
+
+    per_kernel = {}
+    peak, peak_kind = hbm_peak()
+    for name, _ in kernels:
+        times = sorted(a.elapsed_time(b) for a, b in ev[name])
+        avg_ms = sum(times) / len(times)
+        gbs = nbytes[name] / (avg_ms * 1e-3) / 1e9
+        per_kernel[name] = {"us": round(avg_ms * 1e3, 2), "median_us": round(times[len(times) // 2] * 1e3, 2),
+                            "bytes": nbytes[name], "gbs": round(gbs, 1),
+                            "frac": round(gbs / peak, 4),
+                            "share": None}
+        if ROWS[name]:
+            per_kernel[name]["rows_per_s"] = ROWS[name] / (avg_ms * 1e-3)
+    total_kernel_ms = sum(v["us"] for v in per_kernel.values())
+    for v in per_kernel.values():
+        v["share"] = round(v["us"] / total_kernel_ms, 4)
+    dominant = max(per_kernel, key=lambda n: per_kernel[n]["us"])
+    d = per_kernel[dominant]
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(batch, kernels, nbytes, args, device)
+
+    sw_bytes = nbytes["swiglu_fwd"] + nbytes["swiglu_bwd"]
+    sw_us = per_kernel["swiglu_fwd"]["us"] + per_kernel["swiglu_bwd"]["us"]
+    line = {
+        "metric": METRIC,
+        "value": round(aggregate_value(bytes_per_step, K, world, max_ms * 1e-3), 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(max_ms / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAME, "bytes_per_step": bytes_per_step,
+                   "l2": "no flush: every kernel streams > 126 MB (inputs larger than L2)",
+                   "parallelism": f"weak: {world} independent replica(s), one per GPU",
+                   "n_used": batch.rt.n_used},
+        "swiglu_fwd_bwd": {"gbs": round(sw_bytes / (sw_us * 1e-6) / 1e9, 1),
+                           "frac": round(sw_bytes / (sw_us * 1e-6) / 1e9 / peak, 4),
+                           "rows_per_s": SWIGLU["rows"] / (sw_us * 1e-6),
+                           "fwd_frac": per_kernel["swiglu_fwd"]["frac"],
+                           "bwd_frac": per_kernel["swiglu_bwd"]["frac"]},
+        "roofline": {"kernel": dominant, "bound": "hbm", "achieved": d["gbs"], "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": d["frac"],
+                     "algorithmic_bytes": d["bytes"], "traffic": ncu_traffic(dominant)},
+        "kernels": per_kernel,
+        "gpu_launches": K * len(kernels),
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_sample, steps=1)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(batch, kernels, nbytes, args, device):
+    """The same step through the public API with inputs in pinned host memory:
+    host->device copies of every input, the kernels, and device->host copies
+    of every output, all inside the timed region."""
+    host_in = {k: torch.empty_like(getattr(batch, k), device="cpu").pin_memory()
+               for k in batch.INPUT_NAMES}
+    for k, h in host_in.items():
+        h.copy_(getattr(batch, k))
+    host_out = {k: torch.empty_like(getattr(batch, k), device="cpu").pin_memory()
+                for k in batch.OUTPUT_NAMES}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        for k, h in host_in.items():
+            getattr(batch, k).copy_(h, non_blocking=True)
+        for _, fn in kernels:
+            fn()
+        for k, h in host_out.items():
+            h.copy_(getattr(batch, k), non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        step()
+    torch.cuda.synchronize(device)
+    n = args.e2e_steps
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    ms = max_over_ranks(a.elapsed_time(b), device)
+    _, _, world = dist_env()
+    return {"value": round(aggregate_value(sum(nbytes.values()), n, world, ms * 1e-3), 2),
+            "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": n, "ms_per_step": round(ms / n, 3)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def cpu_sample_workload(frac: float, seed: int = 0):
+    """A bounded sample of the same workload on the host: the first `frac` of
+    the rows (tokens) of every op, same distributions."""
+    import numpy as np  # noqa: F401
+    from moe_expert_epilogue_b200 import inputs
+    R = max(8, int(SWIGLU["rows"] * frac) // 8 * 8)
+    Rr = max(1, int(ROUTER["rows"] * frac))
+    T = max(8, int(PERMUTED["tokens"] * frac))
+    Rs = max(1, int(RESIDUAL["rows"] * frac))
+    sw = inputs.swiglu_inputs(R, SWIGLU["inter"], sigma=SWIGLU["sigma"], probs="topk_softmax",
+                              seed=seed)
+    rw = inputs.router_weight_inputs(Rr, ROUTER["hidden"], seed=seed + 1)
+    rt = inputs.routing(T, PERMUTED["top_k"], PERMUTED["experts"], PERMUTED["align"], seed=seed + 2)
+    ax = inputs.permuted_activation_input(rt, PERMUTED["width"], swiglu=False, seed=seed + 3)
+    ax2 = inputs.permuted_activation_input(rt, PERMUTED["width"], swiglu=True, seed=seed + 4)
+    eo = inputs.expert_output_input(rt, PERMUTED["hidden"], seed=seed + 5)
+    res = inputs.residual_inputs((Rs, RESIDUAL["hidden"]), torch.bfloat16, seed=seed + 6)
+    return dict(R=R, Rr=Rr, T=T, Rs=Rs, sw=sw, rw=rw, rt=rt, ax=ax, ax2=ax2, eo=eo, res=res)
+
+
+def oracle_step(w):
+    """One pass of the oracle over the sampled workload; returns its algorithmic bytes."""
+    import numpy as np
+    import oracle
+    from moe_expert_epilogue_b200.inputs import bits
+    L, I, W, Hu = SWIGLU["limit"], SWIGLU["inter"], PERMUTED["width"], PERMUTED["hidden"]
+    sw, rw, rt, res = w["sw"], w["rw"], w["rt"], w["res"]
+    xb, pb, gb = bits(sw["x"]), bits(sw["probs"]), bits(sw["grad_y"])
+    oracle.swiglu_clamped_fwd(xb, pb, L)
+    rxb, rpb, rgb = bits(rw["x"]), bits(rw["probs"]), bits(rw["grad_out"])
+    e = oracle.router_weight_fwd(rxb, oracle.BF16, rpb, oracle.BF16)
+    pm, pr = bits(rt.permutation_map), bits(rt.probs)
+    init = np.zeros((rt.max_rows, W), np.uint16)
+    for act, x in ((oracle.SQRELU, w["ax"]), (oracle.SQRELU_CLAMP, w["ax"]), (oracle.SWIGLU, w["ax2"])):
+        oracle.act_with_probs_permuted(act, bits(x), init, pm, rt.n_used, pr, W, PERMUTED["scale"],
+                                       True)
+    oracle.unpermute_ordered(bits(w["eo"]), oracle.BF16, bits(rt.inverse_map), rt.tokens,
+                             np.zeros((rt.tokens, Hu), np.uint16), oracle.BF16)
+    ee = bits(res["expert_output"]).copy()
+    ee[: min(ee.shape[0], e.shape[0])] = e[: ee.shape[0]]
+    oracle.residual_add(ee, bits(res["shared_expert_output"]), bits(res["residual"]), oracle.BF16)
+    oracle.router_weight_bwd(rgb, oracle.BF16, rxb, oracle.BF16, rpb)
+    oracle.swiglu_clamped_bwd(xb, pb, gb, L)
+    live = rt.tokens * rt.top_k
+    R, Rr, Rs, T = w["R"], w["Rr"], w["Rs"], w["T"]
+    meta = 4 * rt.n_used + 4 * live
+    return (R * (2 * I * 2 + 4 + I * 2) + R * (2 * I * 2 + I * 2 + 4 + 2 * I * 2 + 4)
+            + Rr * ROUTER["hidden"] * 4 + Rr * 4 + Rr * ROUTER["hidden"] * 6 + Rr * 8
+            + 2 * (live * W * 2 + rt.n_used * W * 2 + meta)
+            + (live * 2 * W * 2 + rt.n_used * W * 2 + meta)
+            + live * Hu * 2 + T * rt.experts * 4 + T * Hu * 2
+            + 4 * Rs * RESIDUAL["hidden"] * 2)
+
+
+def cpu_baseline(frac, steps=1):
+    w = cpu_sample_workload(frac)
+    t0 = time.perf_counter()
+    b = 0
+    for _ in range(steps):
+        b += oracle_step(w)
+    dt = time.perf_counter() - t0
+    return {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "seconds": round(dt, 2), "host_cpu": _cpu_model(), "host_nproc": os.cpu_count(),
+            "sample": f"first {frac:g} of the rows/tokens of every op of the step "
+                      f"(swiglu rows {w['R']}, router rows {w['Rr']}, tokens {w['T']}, "
+                      f"residual rows {w['Rs']}); single-threaded C oracle, -O2"}
+
+
+def _cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    w = cpu_sample_workload(args.cpu_sample)
+    for _ in range(args.warmup):
+        oracle_step(w)
+    t0 = time.perf_counter()
+    b = 0
+    for _ in range(args.steps):
+        b += oracle_step(w)
+    dt = time.perf_counter() - t0
+    value = round(b / dt / 1e9, 4)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAME, "sample_fraction": args.cpu_sample},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"first {args.cpu_sample:g} of the rows/tokens of every op per "
+                                   "step; single-threaded C oracle"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-sample", type=float, default=0.25,
+                    help="fraction of the rows of every op the CPU oracle runs")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        raise SystemExit("--warmup must be >= 3")
+    _, _, world = dist_env()
+    if world != args.gpus and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,238 @@
+/*
+ * moe_epilogue.h -- C ABI of the B200 (sm_100a) MoE expert-epilogue library.
+ *
+ * Seven memory-bound ops that sit between the grouped GEMMs of a
+ * Mixture-of-Experts layer and the residual stream.  Each entry point takes
+ * caller-owned DEVICE pointers, sizes and a CUDA stream, validates its
+ * arguments on the host, enqueues exactly one kernel on `stream` and returns.
+ *
+ * Common contract
+ *   - Ownership: every pointer is owned by the caller and must stay valid
+ *     until the enqueued kernel has finished.  The library allocates nothing,
+ *     keeps no per-call state and never synchronises, so calls may be captured
+ *     in a CUDA graph.
+ *   - Layout: 2-D tensors are row-major.  `ld_*` arguments are leading
+ *     dimensions in ELEMENTS (the distance between the starts of two rows);
+ *     where no leading dimension is taken, rows are contiguous.
+ *   - Counts that change at run time (n_used, valid_tokens) are int32 values
+ *     in DEVICE memory, read by the kernel, so a captured graph stays valid as
+ *     they change.  The matching maximum sizes are host arguments.
+ *   - Alignment: every pointer must be aligned to its element size
+ *     (MOE_ERR_ALIGN otherwise).  16-byte aligned pointers and leading
+ *     dimensions / widths that are multiples of 8 elements take the
+ *     vectorised path; anything else takes an element-wise path inside the
+ *     same kernel family with identical results.
+ *   - Aliasing: outputs must not overlap inputs, except that
+ *     moe_residual_add may run in place (out == residual).
+ *   - Errors: the return value is MOE_OK or one of the MOE_ERR_* codes below.
+ *     Argument errors are detected before anything is enqueued.  MOE_ERR_CUDA
+ *     means a CUDA runtime call failed (moe_last_cuda_error() gives the
+ *     cudaError_t); note that an asynchronous error left pending by earlier
+ *     work on the device can surface here too.  Sizes of zero are valid no-ops.
+ *   - Device error word: the two ops that read routing metadata from device
+ *     memory take an optional `int32_t* dev_err` (device memory, may be
+ *     NULL).  Out-of-range metadata never causes an out-of-bounds access:
+ *     the kernel clamps or skips and ORs MOE_DEVERR_* bits into *dev_err.
+ *   - Numerics: inputs are widened to fp32, the documented formula is
+ *     evaluated in fp32 and each output is rounded once to its dtype with
+ *     round-to-nearest-even.  Every result is independent of the grid size,
+ *     of the other rows / tokens in the batch and of the run (no atomics in
+ *     any reduction).
+ *
+ * Sources (API reference pages, cited by page title and documented symbol):
+ *   [OPT] nemo_automodel.components.moe.optimized_ops
+ *   [SWI] nemo_automodel.components.moe.swiglu_triton
+ *   [BI]  core.inference.moe.batch_invariant
+ *   [RES] core.fusions.fused_moe_residual_add
+ */
+#ifndef MOE_EPILOGUE_H
+#define MOE_EPILOGUE_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { MOE_BF16 = 0, MOE_FP16 = 1, MOE_FP32 = 2 } moe_dtype;
+
+typedef enum {
+  MOE_ACT_SQRELU = 0,       /* squared ReLU, square rounded to bf16 first        */
+  MOE_ACT_SQRELU_CLAMP = 1, /* tanh soft clamp, then squared ReLU, all in fp32   */
+  MOE_ACT_SWIGLU = 2        /* silu(gate) * up, gate = first half of the row     */
+} moe_act;
+
+enum {
+  MOE_OK = 0,
+  MOE_ERR_NULL = 1,  /* a required pointer is NULL                              */
+  MOE_ERR_SHAPE = 2, /* negative size, leading dim below the row width, or a
+                        size beyond the documented maximum                     */
+  MOE_ERR_DTYPE = 3, /* dtype (or activation) not supported for that argument   */
+  MOE_ERR_ALIGN = 4, /* a pointer not aligned to its element size               */
+  MOE_ERR_LIMIT = 5, /* limit or clamp_scale not a positive number              */
+  MOE_ERR_CUDA = 6   /* a CUDA runtime call or the launch failed                */
+};
+
+/* Bits ORed into the optional device error word. */
+enum {
+  MOE_DEVERR_COUNT = 1,  /* *n_used / *valid_tokens outside [0, max]: clamped    */
+  MOE_DEVERR_MAP = 2,    /* permutation_map entry >= num_probs: row skipped       */
+  MOE_DEVERR_INVERSE = 4 /* inverse_map entry >= max_rows: contribution skipped   */
+};
+
+/* Human-readable name of a status code (static storage). */
+MOE_API const char* moe_status_string(int status);
+
+/* cudaError_t of the most recent MOE_ERR_CUDA on the calling thread (0 if none). */
+MOE_API int moe_last_cuda_error(void);
+
+/* Library ABI version, currently 1. */
+MOE_API int moe_abi_version(void);
+
+/* ------------------------------------------------------------------------
+ * Clamped, probability-weighted SwiGLU, forward.
+ * [SWI] module docstring and the forward kernel (_swiglu_clamped_fwd_kernel):
+ *   y[r, j] = silu(clamp(g, max=L)) * clamp(u, -L, L) * probs[r]
+ *   with g = x[r, j], u = x[r, inter + j], silu(z) = z * sigmoid(z);
+ *   fp32 math, one rounding to bf16.  clamp is torch.clamp (NaN propagates).
+ * x      bf16 [rows, ld_x], columns [0, inter) gate, [inter, 2*inter) up; ld_x >= 2*inter
+ * probs  fp32 [rows] (one routing probability per row, i.e. [rows, 1])
+ * y      bf16 [rows, ld_y], ld_y >= inter; columns >= inter are not written
+ * limit  L > 0, may be +inf (no clamping); NaN or <= 0 -> MOE_ERR_LIMIT
+ * dt     MOE_BF16 (others -> MOE_ERR_DTYPE)
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_swiglu_clamped_fwd(const void* x, const float* probs, void* y, int64_t rows,
+                           int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
+                           moe_dtype dt, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Clamped SwiGLU, one-pass backward.
+ * [SWI] module docstring and the backward kernel (_swiglu_clamped_bwd_kernel):
+ *   a = dy * p,   s = silu(gc),   gc = clamp(g, max=L),  uc = clamp(u, -L, L)
+ *   grad_x[r, j]         = a * uc * silu'(gc)  where g <= L,        else 0
+ *   grad_x[r, inter + j] = a * s               where -L <= u <= L,  else 0
+ *   grad_probs[r]        = sum_j dy * s * uc   (fp32, reduced per row)
+ *   silu'(z) = sigmoid(z) * (1 + z * (1 - sigmoid(z))); the masks are
+ *   torch.clamp's inclusive ranges on the input values; grad_x is rounded
+ *   once to bf16.  grad_probs is reduced in a fixed order (per-thread
+ *   partials over a fixed column assignment, a fixed warp butterfly, warps
+ *   in index order), independent of the grid and of the batch.
+ * x           bf16 [rows, ld_x]   (the forward's input, recomputed from)
+ * probs       fp32 [rows]
+ * grad_y      bf16 [rows, ld_gy], ld_gy >= inter
+ * grad_x      bf16 [rows, ld_gx], ld_gx >= 2*inter  (output)
+ * grad_probs  fp32 [rows]                           (output)
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_swiglu_clamped_bwd(const void* x, const float* probs, const void* grad_y,
+                           void* grad_x, float* grad_probs, int64_t rows, int64_t inter,
+                           int64_t ld_x, int64_t ld_gy, int64_t ld_gx, float limit,
+                           moe_dtype dt, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Router-weight multiply in fp32, forward.
+ * [OPT] _rw_fwd_core and _RouterWeightMulFunction.forward:
+ *   out[r, h] = (x[r, h].float() * probs[r]).to(out_dtype)
+ *   one fp32 multiply and one rounding: bitwise identical to the eager op.
+ * x      x_dt [rows, hidden] contiguous;  x_dt in {BF16, FP16, FP32}
+ * probs  fp32 [rows]
+ * out    out_dt [rows, hidden] contiguous; out_dt in {BF16, FP16, FP32}
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_router_weight_mul_fwd(const void* x, moe_dtype x_dt, const float* probs, void* out,
+                              moe_dtype out_dt, int64_t rows, int64_t hidden,
+                              cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Router-weight multiply, backward (both gradients in one pass).
+ * [OPT] _rw_bwd_x_core, _rw_bwd_probs_core, _RouterWeightMulFunction.backward:
+ *   grad_x[r, h]  = (g[r, h].float() * probs[r]).to(x_dt)         (bitwise)
+ *   grad_probs[r] = sum_h g[r, h].float() * x[r, h].float()       (fp32)
+ * grad_out    g_dt [rows, hidden] contiguous (the forward output's dtype)
+ * x           x_dt [rows, hidden] contiguous, or NULL when the forward did
+ *             not save x (save_x false): then grad_probs must be NULL too and
+ *             only grad_x is computed (x is never read).
+ * probs       fp32 [rows]
+ * grad_x      x_dt [rows, hidden]  (output)
+ * grad_probs  fp32 [rows] or NULL  (output; fixed-order row reduction)
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_router_weight_mul_bwd(const void* grad_out, moe_dtype g_dt, const void* x,
+                              moe_dtype x_dt, const float* probs, void* grad_x,
+                              float* grad_probs, int64_t rows, int64_t hidden,
+                              cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Batch-invariant activation with router probabilities over a padded,
+ * expert-grouped row layout.
+ * [BI] _squared_relu_with_probs_kernel, squared_relu_with_probs,
+ *      _swiglu_with_probs_kernel, swiglu_with_probs:
+ *   for each row r < *n_used: m = permutation_map[r];
+ *     m >= 0: out[r, :] = act(x[r, :]) * probs[m]       (one bf16 rounding,
+ *             except SQRELU, whose square is rounded to bf16 first)
+ *     m <  0: alignment padding row -- zero-filled if zero_padding, else
+ *             left untouched
+ *   rows r >= *n_used are neither read nor written.
+ *   SQRELU:       out = bf16(bf16(relu(x)^2) * p)
+ *   SQRELU_CLAMP: z = clamp_scale * tanh(x / clamp_scale); out = bf16(relu(z)^2 * p)
+ *   SWIGLU:       out = bf16(silu(gate) * up * p), gate = x[r, 0:width],
+ *                 up = x[r, width:2*width]
+ * x                bf16 [max_rows, width] (SWIGLU: [max_rows, 2*width]) contiguous
+ * out              bf16 [max_rows, width] contiguous
+ * permutation_map  int32 [max_rows] (device): flat index into probs, or < 0
+ * n_used           int32 (device): rows in the live, padded prefix
+ * probs            fp32 [num_probs] (device), indexed by permutation_map
+ * clamp_scale      SQRELU_CLAMP only: finite and > 0 (MOE_ERR_LIMIT otherwise);
+ *                  ignored for the other activations
+ * dev_err          optional int32 (device): MOE_DEVERR_COUNT, MOE_DEVERR_MAP
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_act_with_probs_permuted(moe_act act, const void* x, void* out,
+                                const int32_t* permutation_map, const int32_t* n_used,
+                                const float* probs, int64_t num_probs, int64_t max_rows,
+                                int64_t width, float clamp_scale, int zero_padding,
+                                int32_t* dev_err, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Token-local unpermute that sums expert contributions in a fixed order.
+ * [BI] _unpermute_tokens_in_expert_order_kernel, unpermute_tokens_in_expert_order:
+ *   for each token t < *valid_tokens:
+ *     acc = +0.0f;  for e = 0, 1, ..., E-1 (increasing local expert id):
+ *       if inverse_map[t, e] >= 0: acc += expert_output[inverse_map[t, e], :]
+ *     out[t, :] = acc rounded once to out_dt
+ *   fp32 sequential adds, no atomics; tokens t >= *valid_tokens untouched.
+ * expert_output  in_dt [max_rows, hidden] contiguous
+ * inverse_map    int32 [tokens, num_local_experts] (device): row or < 0
+ * valid_tokens   int32 (device)
+ * out            out_dt [tokens, hidden] contiguous
+ * num_local_experts  1 .. 4096
+ * dev_err        optional int32 (device): MOE_DEVERR_COUNT, MOE_DEVERR_INVERSE
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_unpermute_ordered(const void* expert_output, moe_dtype in_dt, int64_t max_rows,
+                          const int32_t* inverse_map, const int32_t* valid_tokens, void* out,
+                          moe_dtype out_dt, int64_t tokens, int64_t hidden,
+                          int32_t num_local_experts, int32_t* dev_err, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Fused MoE residual add.
+ * [RES] module docstring, _moe_residual_add_kernel, fused_moe_residual_add:
+ *   out = residual + round_dt(expert_output + shared_expert_output)
+ *   each add in fp32, each result rounded to dt: bit-identical to the two
+ *   unfused adds.  Reads the three inputs once and writes out once.  The
+ *   backward passes grad_out unchanged to all three inputs, so it has no
+ *   kernel.
+ * all four tensors dt [numel] contiguous, dt in {BF16, FP16, FP32};
+ * out may equal residual (in place).
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_residual_add(const void* expert_output, const void* shared_expert_output,
+                     const void* residual, void* out, int64_t numel, moe_dtype dt,
+                     cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_EPILOGUE_H */

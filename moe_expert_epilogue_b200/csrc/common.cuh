@@ -1,0 +1,239 @@
+// common.cuh -- device helpers shared by the epilogue kernels (sm_100a).
+//
+// Everything on this path is a memory-bound stream: 16-byte vector loads and
+// stores that bypass L1 allocation, fp32 arithmetic in registers, and one
+// rounding to the storage dtype per output element.  Nothing here is a dense
+// contraction, so no tensor-core path exists.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kThreads = 256;  // threads per CTA for every kernel in the library
+constexpr int kVec = 8;        // elements per vector unit ("chunk")
+
+// Storage-type tags.  Each knows how to widen 8 consecutive elements to fp32
+// and how to round 8 fp32 values (RNE) back.
+struct BF16 { using T = uint16_t; static constexpr int kBytes = 2; };
+struct F16  { using T = uint16_t; static constexpr int kBytes = 2; };
+struct F32  { using T = float;    static constexpr int kBytes = 4; };
+
+// ------------------------------------------------------------ raw access
+
+// 16-byte streaming load through the non-coherent path, no L1 allocation
+// (no element is reused), with a 256-byte L2 prefetch hint (a warp reads
+// 512 contiguous bytes per load instruction).
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
+// 16-byte coherent load, no L1 allocation: for data that the same kernel
+// also writes (the in-place residual add).
+__device__ __forceinline__ uint4 ld_coherent(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
+// 16-byte store, no L1 allocation.
+__device__ __forceinline__ void st_stream(void* p, uint4 v) {
+  asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// ------------------------------------------------------------ conversions
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Two fp32 -> packed bf16x2 with round-to-nearest-even; `lo` lands at the lower address.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float f16_to_f32(uint16_t h) {
+  float f;
+  asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"(h));
+  return f;
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16(float f) {
+  uint16_t r;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(f));
+  return r;
+}
+
+__device__ __forceinline__ uint16_t f32_to_f16(float f) {
+  uint16_t r;
+  asm("cvt.rn.f16.f32 %0, %1;" : "=h"(r) : "f"(f));
+  return r;
+}
+
+// Scalar widen / round for the unaligned (element-granular) paths.
+template <class D> __device__ __forceinline__ float load1(const typename D::T* p);
+template <> __device__ __forceinline__ float load1<BF16>(const uint16_t* p) {
+  return __uint_as_float((uint32_t)__ldg(p) << 16);
+}
+template <> __device__ __forceinline__ float load1<F16>(const uint16_t* p) {
+  return f16_to_f32(__ldg(p));
+}
+template <> __device__ __forceinline__ float load1<F32>(const float* p) { return __ldg(p); }
+
+// Coherent scalar widen (plain load, for data the kernel may also write).
+template <class D> __device__ __forceinline__ float load1c(const typename D::T* p);
+template <> __device__ __forceinline__ float load1c<BF16>(const uint16_t* p) {
+  return __uint_as_float((uint32_t)*p << 16);
+}
+template <> __device__ __forceinline__ float load1c<F16>(const uint16_t* p) { return f16_to_f32(*p); }
+template <> __device__ __forceinline__ float load1c<F32>(const float* p) { return *p; }
+
+template <class D> __device__ __forceinline__ void store1(typename D::T* p, float v);
+template <> __device__ __forceinline__ void store1<BF16>(uint16_t* p, float v) { *p = f32_to_bf16(v); }
+template <> __device__ __forceinline__ void store1<F16>(uint16_t* p, float v) { *p = f32_to_f16(v); }
+template <> __device__ __forceinline__ void store1<F32>(float* p, float v) { *p = v; }
+
+// Round-trip through the storage dtype (what materialising a tensor does).
+template <class D> __device__ __forceinline__ float round_to(float v);
+template <> __device__ __forceinline__ float round_to<BF16>(float v) {
+  return __uint_as_float((uint32_t)f32_to_bf16(v) << 16);
+}
+template <> __device__ __forceinline__ float round_to<F16>(float v) {
+  return f16_to_f32(f32_to_f16(v));
+}
+template <> __device__ __forceinline__ float round_to<F32>(float v) { return v; }
+
+// ------------------------------------------------- 8-element vector units
+
+// A chunk of 8 elements in registers as raw bits: one 16-byte word for the
+// 16-bit types, two for fp32.
+template <class D> struct Raw8 { uint4 w[D::kBytes / 2]; };
+
+// NC = true: read-only streaming path; false: coherent path (data the
+// kernel may also write).
+template <class D, bool NC = true>
+__device__ __forceinline__ Raw8<D> load8(const typename D::T* p) {
+  Raw8<D> r;
+#pragma unroll
+  for (int i = 0; i < D::kBytes / 2; ++i) {
+    const uint4* w = reinterpret_cast<const uint4*>(p) + i;
+    r.w[i] = NC ? ld_stream(w) : ld_coherent(w);
+  }
+  return r;
+}
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& w, float (&v)[8]) {
+  v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+  v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+}
+
+template <class D> __device__ __forceinline__ void widen8(const Raw8<D>& r, float (&v)[8]);
+template <> __device__ __forceinline__ void widen8<BF16>(const Raw8<BF16>& r, float (&v)[8]) {
+  unpack_bf16x8(r.w[0], v);
+}
+template <> __device__ __forceinline__ void widen8<F16>(const Raw8<F16>& r, float (&v)[8]) {
+  const uint32_t* u = reinterpret_cast<const uint32_t*>(&r.w[0]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = f16_to_f32((uint16_t)(u[i] & 0xffffu));
+    v[2 * i + 1] = f16_to_f32((uint16_t)(u[i] >> 16));
+  }
+}
+template <> __device__ __forceinline__ void widen8<F32>(const Raw8<F32>& r, float (&v)[8]) {
+  v[0] = __uint_as_float(r.w[0].x); v[1] = __uint_as_float(r.w[0].y);
+  v[2] = __uint_as_float(r.w[0].z); v[3] = __uint_as_float(r.w[0].w);
+  v[4] = __uint_as_float(r.w[1].x); v[5] = __uint_as_float(r.w[1].y);
+  v[6] = __uint_as_float(r.w[1].z); v[7] = __uint_as_float(r.w[1].w);
+}
+
+// Round 8 fp32 values to the storage dtype (RNE) and store them.
+template <class D> __device__ __forceinline__ void store8(typename D::T* p, const float (&v)[8]);
+template <> __device__ __forceinline__ void store8<BF16>(uint16_t* p, const float (&v)[8]) {
+  st_stream(p, make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                          pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7])));
+}
+template <> __device__ __forceinline__ void store8<F16>(uint16_t* p, const float (&v)[8]) {
+  st_stream(p, make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]),
+                          pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7])));
+}
+template <> __device__ __forceinline__ void store8<F32>(float* p, const float (&v)[8]) {
+  st_stream(p, make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
+                          __float_as_uint(v[3])));
+  st_stream(p + 4, make_uint4(__float_as_uint(v[4]), __float_as_uint(v[5]),
+                              __float_as_uint(v[6]), __float_as_uint(v[7])));
+}
+
+// ------------------------------------------------------------ math
+
+// e^x = 2^(x * log2 e), with the hardware base-2 exponential (PTX
+// ex2.approx.f32; subnormal results are kept) -- then the logistic function
+// 1 / (1 + e^-z) with the hardware reciprocal (PTX rcp.approx.f32).  Both
+// approximations are within a few fp32 ulp, far below half a bf16 ulp.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float sigmoid(float z) {
+  return rcp_approx(1.0f + ex2_approx(z * -kLog2e));
+}
+
+// torch.clamp semantics: a NaN input stays NaN (every comparison is false).
+__device__ __forceinline__ float clamp_max(float v, float hi) { return v > hi ? hi : v; }
+__device__ __forceinline__ float clamp_sym(float v, float lim) {
+  return v < -lim ? -lim : (v > lim ? lim : v);
+}
+
+// Fixed xor-butterfly sum over the 32 lanes of a warp: the same tree every
+// call, so the bits do not depend on the grid.
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Walks a flat chunk index q over a [rows, cpr] grid in strides of S without
+// a division per step: (r, c) = divmod(q, cpr), (dr, dc) = divmod(S, cpr).
+struct RowCursor {
+  int64_t r, c, dr, dc, cpr;
+  __device__ __forceinline__ RowCursor(int64_t q, int64_t stride, int64_t cpr_)
+      : r(q / cpr_), c(q % cpr_), dr(stride / cpr_), dc(stride % cpr_), cpr(cpr_) {}
+  __device__ __forceinline__ void advance() {
+    c += dc;
+    r += dr;
+    if (c >= cpr) { c -= cpr; r += 1; }
+  }
+};
+
+// Device-side error word: set bits, never trap.
+__device__ __forceinline__ void flag_error(int32_t* err, int32_t bits) {
+  if (err) atomicOr(err, bits);
+}
+
+}  // namespace moe

@@ -1,0 +1,53 @@
+// launch.cuh -- host-side launch helpers shared by the op launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe_epilogue.h"
+
+namespace moe {
+
+// Records a failing CUDA call for moe_last_cuda_error() and returns MOE_ERR_CUDA.
+int cuda_fail(cudaError_t e);
+
+// Persistent grid for `kernel` launched with kThreads threads and `smem`
+// bytes of dynamic shared memory: resident CTAs per SM (occupancy, cached per
+// kernel) times the SM count of the current device (cached per device), but
+// no more than `useful_blocks`, and at least 1.
+int persistent_grid(const void* kernel, size_t smem, int64_t useful_blocks, int* grid);
+
+// MOE_ERR_CUDA if the launch just issued failed.
+int check_launch();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Launchers (one per op family); arguments already validated.
+int launch_swiglu_clamped_fwd(const uint16_t* x, const float* probs, uint16_t* y, int64_t rows,
+                              int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
+                              cudaStream_t stream);
+int launch_swiglu_clamped_bwd(const uint16_t* x, const float* probs, const uint16_t* grad_y,
+                              uint16_t* grad_x, float* grad_probs, int64_t rows, int64_t inter,
+                              int64_t ld_x, int64_t ld_gy, int64_t ld_gx, float limit,
+                              cudaStream_t stream);
+int launch_router_weight_fwd(const void* x, moe_dtype x_dt, const float* probs, void* out,
+                             moe_dtype out_dt, int64_t rows, int64_t hidden,
+                             cudaStream_t stream);
+int launch_router_weight_bwd(const void* grad_out, moe_dtype g_dt, const void* x,
+                             moe_dtype x_dt, const float* probs, void* grad_x,
+                             float* grad_probs, int64_t rows, int64_t hidden,
+                             cudaStream_t stream);
+int launch_act_with_probs_permuted(moe_act act, const uint16_t* x, uint16_t* out,
+                                   const int32_t* permutation_map, const int32_t* n_used,
+                                   const float* probs, int64_t num_probs, int64_t max_rows,
+                                   int64_t width, float clamp_scale, int zero_padding,
+                                   int32_t* dev_err, cudaStream_t stream);
+int launch_unpermute_ordered(const void* expert_output, moe_dtype in_dt, int64_t max_rows,
+                             const int32_t* inverse_map, const int32_t* valid_tokens,
+                             void* out, moe_dtype out_dt, int64_t tokens, int64_t hidden,
+                             int32_t num_local_experts, int32_t* dev_err,
+                             cudaStream_t stream);
+int launch_residual_add(const void* e, const void* s, const void* r, void* out, int64_t numel,
+                        moe_dtype dt, cudaStream_t stream);
+
+}  // namespace moe

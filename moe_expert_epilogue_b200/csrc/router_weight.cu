@@ -1,0 +1,261 @@
+// router_weight.cu -- router-weight multiply in fp32, forward and backward
+// (nemo_automodel.components.moe.optimized_ops: _rw_fwd_core, _rw_bwd_x_core,
+// _rw_bwd_probs_core, _RouterWeightMulFunction).
+//
+//   fwd:  out    = (x.float() * p).to(out_dtype)             one multiply, one rounding
+//   bwd:  grad_x = (g.float() * p).to(x_dtype)               one multiply, one rounding
+//         grad_p = sum_h g.float() * x.float()               fp32 row reduction
+//
+// The forward and the x-only backward are flat grid-stride streams over
+// 8-element chunks.  The backward with the probability gradient walks rows
+// like the SwiGLU backward: W threads per row, fixed column assignment, fixed
+// reduction tree, no fp32 intermediate ever leaves the registers.
+#include "common.cuh"
+#include "launch.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kUnroll = 2;
+
+// out[r, :] = cast(in[r, :] * p[r]) over a [rows, cpr] chunk grid.
+template <class DI, class DO>
+__global__ void __launch_bounds__(kThreads)
+scale_rows_vec(const typename DI::T* __restrict__ in, const float* __restrict__ probs,
+               typename DO::T* __restrict__ out, int64_t rows, int64_t hidden) {
+  const int64_t cpr = hidden / kVec;
+  const int64_t total = rows * cpr;
+  const int64_t S = (int64_t)gridDim.x * kThreads;
+  int64_t q = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (q >= total) return;
+  RowCursor cur(q, S, cpr);
+  for (; q < total; q += kUnroll * S) {
+    Raw8<DI> raw[kUnroll];
+    float p[kUnroll];
+    int64_t off[kUnroll];
+#pragma unroll
+    for (int k = 0; k < kUnroll; ++k) {
+      if (q + k * S < total) {
+        off[k] = cur.r * hidden + cur.c * kVec;
+        raw[k] = load8<DI>(in + off[k]);
+        p[k] = __ldg(probs + cur.r);
+      }
+      cur.advance();
+    }
+#pragma unroll
+    for (int k = 0; k < kUnroll; ++k) {
+      if (q + k * S < total) {
+        float v[8];
+        widen8<DI>(raw[k], v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = v[i] * p[k];
+        store8<DO>(out + off[k], v);
+      }
+    }
+  }
+}
+
+template <class DI, class DO>
+__global__ void __launch_bounds__(kThreads)
+scale_rows_scalar(const typename DI::T* __restrict__ in, const float* __restrict__ probs,
+                  typename DO::T* __restrict__ out, int64_t rows, int64_t hidden) {
+  const int64_t total = rows * hidden;
+  const int64_t S = (int64_t)gridDim.x * kThreads;
+  int64_t q = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (q >= total) return;
+  RowCursor cur(q, S, hidden);
+  for (; q < total; q += S, cur.advance())
+    store1<DO>(out + q, load1<DI>(in + q) * __ldg(probs + cur.r));
+}
+
+template <int W>
+__device__ __forceinline__ float row_reduce(float acc, float (*red)[kThreads / 32], int parity) {
+  acc = warp_sum(acc);
+  if constexpr (W == 32) {
+    return acc;
+  } else {
+    if ((threadIdx.x & 31) == 0) red[parity][threadIdx.x >> 5] = acc;
+    __syncthreads();
+    const int first = (threadIdx.x / W) * (W / 32);
+    float s = 0.0f;
+#pragma unroll
+    for (int w = 0; w < W / 32; ++w) s += red[parity][first + w];
+    return s;
+  }
+}
+
+// Backward with the probability gradient.  VEC selects 8-element chunks
+// (hidden % 8 == 0, 16-byte aligned) or single elements.
+template <class DG, class DX, int W, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+rw_bwd_rows(const typename DG::T* __restrict__ g, const typename DX::T* __restrict__ x,
+            const float* __restrict__ probs, typename DX::T* __restrict__ gx,
+            float* __restrict__ gp, int64_t rows, int64_t hidden) {
+  constexpr int G = kThreads / W;
+  __shared__ float red[2][kThreads / 32];
+  const int sub = threadIdx.x / W, lane = threadIdx.x % W;
+  int parity = 0;
+  for (int64_t r0 = (int64_t)blockIdx.x * G; r0 < rows; r0 += (int64_t)gridDim.x * G) {
+    const int64_t r = r0 + sub;
+    float acc = 0.0f;
+    if (r < rows) {
+      const float p = __ldg(probs + r);
+      const int64_t base = r * hidden;
+      if constexpr (VEC) {
+        const int64_t cpr = hidden / kVec;
+        for (int64_t c0 = lane; c0 < cpr; c0 += (int64_t)kUnroll * W) {
+          Raw8<DG> rg[kUnroll];
+          Raw8<DX> rx[kUnroll];
+#pragma unroll
+          for (int k = 0; k < kUnroll; ++k) {
+            const int64_t c = c0 + (int64_t)k * W;
+            if (c < cpr) {
+              rg[k] = load8<DG>(g + base + c * kVec);
+              rx[k] = load8<DX>(x + base + c * kVec);
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < kUnroll; ++k) {
+            const int64_t c = c0 + (int64_t)k * W;
+            if (c < cpr) {
+              float gv[8], xv[8], o[8];
+              widen8<DG>(rg[k], gv);
+              widen8<DX>(rx[k], xv);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                o[i] = gv[i] * p;
+                acc += gv[i] * xv[i];
+              }
+              store8<DX>(gx + base + c * kVec, o);
+            }
+          }
+        }
+      } else {
+        for (int64_t j = lane; j < hidden; j += W) {
+          const float gv = load1<DG>(g + base + j);
+          store1<DX>(gx + base + j, gv * p);
+          acc += gv * load1<DX>(x + base + j);
+        }
+      }
+    }
+    const float s = row_reduce<W>(acc, red, parity);
+    if (r < rows && lane == 0) gp[r] = s;
+    parity ^= 1;
+  }
+}
+
+inline int threads_per_row(int64_t units) {
+  if (units <= 32) return 32;
+  if (units <= 64) return 64;
+  if (units <= 128) return 128;
+  return 256;
+}
+
+template <class DI, class DO>
+int launch_scale(const void* in, const float* probs, void* out, int64_t rows, int64_t hidden,
+                 cudaStream_t stream) {
+  const auto* i = static_cast<const typename DI::T*>(in);
+  auto* o = static_cast<typename DO::T*>(out);
+  int grid;
+  if (hidden % kVec == 0 && aligned16(in) && aligned16(out)) {
+    auto k = scale_rows_vec<DI, DO>;
+    const int64_t units = rows * (hidden / kVec);
+    if (int rc = persistent_grid((const void*)k, 0,
+                                 (units + kThreads * kUnroll - 1) / (kThreads * kUnroll), &grid))
+      return rc;
+    k<<<grid, kThreads, 0, stream>>>(i, probs, o, rows, hidden);
+  } else {
+    auto k = scale_rows_scalar<DI, DO>;
+    if (int rc = persistent_grid((const void*)k, 0, (rows * hidden + kThreads - 1) / kThreads,
+                                 &grid))
+      return rc;
+    k<<<grid, kThreads, 0, stream>>>(i, probs, o, rows, hidden);
+  }
+  return check_launch();
+}
+
+template <class DG, class DX, int W, bool VEC>
+int launch_rows(const void* g, const void* x, const float* probs, void* gx, float* gp,
+                int64_t rows, int64_t hidden, cudaStream_t stream) {
+  auto k = rw_bwd_rows<DG, DX, W, VEC>;
+  int grid;
+  const int64_t blocks = (rows + kThreads / W - 1) / (kThreads / W);
+  if (int rc = persistent_grid((const void*)k, 0, blocks, &grid)) return rc;
+  k<<<grid, kThreads, 0, stream>>>(static_cast<const typename DG::T*>(g),
+                                   static_cast<const typename DX::T*>(x), probs,
+                                   static_cast<typename DX::T*>(gx), gp, rows, hidden);
+  return check_launch();
+}
+
+template <class DG, class DX>
+int launch_bwd_with_probs(const void* g, const void* x, const float* probs, void* gx, float* gp,
+                          int64_t rows, int64_t hidden, cudaStream_t stream) {
+  const bool vec = hidden % kVec == 0 && aligned16(g) && aligned16(x) && aligned16(gx);
+  const int W = threads_per_row(vec ? hidden / kVec : hidden);
+#define MOE_RW_ARGS g, x, probs, gx, gp, rows, hidden, stream
+  if (vec) {
+    switch (W) {
+      case 32: return launch_rows<DG, DX, 32, true>(MOE_RW_ARGS);
+      case 64: return launch_rows<DG, DX, 64, true>(MOE_RW_ARGS);
+      case 128: return launch_rows<DG, DX, 128, true>(MOE_RW_ARGS);
+      default: return launch_rows<DG, DX, 256, true>(MOE_RW_ARGS);
+    }
+  }
+  switch (W) {
+    case 32: return launch_rows<DG, DX, 32, false>(MOE_RW_ARGS);
+    case 64: return launch_rows<DG, DX, 64, false>(MOE_RW_ARGS);
+    case 128: return launch_rows<DG, DX, 128, false>(MOE_RW_ARGS);
+    default: return launch_rows<DG, DX, 256, false>(MOE_RW_ARGS);
+  }
+#undef MOE_RW_ARGS
+}
+
+// Dispatch a (dtype, dtype) pair to a template taking two storage tags.
+template <template <class, class> class F, class... A>
+int dispatch2(moe_dtype a, moe_dtype b, A... args) {
+#define MOE_CASE_B(TA)                                                   \
+  switch (b) {                                                           \
+    case MOE_BF16: return F<TA, BF16>::run(args...);                     \
+    case MOE_FP16: return F<TA, F16>::run(args...);                      \
+    default: return F<TA, F32>::run(args...);                            \
+  }
+  switch (a) {
+    case MOE_BF16: MOE_CASE_B(BF16)
+    case MOE_FP16: MOE_CASE_B(F16)
+    default: MOE_CASE_B(F32)
+  }
+#undef MOE_CASE_B
+}
+
+template <class DI, class DO> struct Fwd {
+  static int run(const void* x, const float* p, void* out, int64_t rows, int64_t hidden,
+                 cudaStream_t s) {
+    return launch_scale<DI, DO>(x, p, out, rows, hidden, s);
+  }
+};
+
+template <class DG, class DX> struct Bwd {
+  static int run(const void* g, const void* x, const float* p, void* gx, float* gp, int64_t rows,
+                 int64_t hidden, cudaStream_t s) {
+    if (x == nullptr) return launch_scale<DG, DX>(g, p, gx, rows, hidden, s);
+    return launch_bwd_with_probs<DG, DX>(g, x, p, gx, gp, rows, hidden, s);
+  }
+};
+
+}  // namespace
+
+int launch_router_weight_fwd(const void* x, moe_dtype x_dt, const float* probs, void* out,
+                             moe_dtype out_dt, int64_t rows, int64_t hidden,
+                             cudaStream_t stream) {
+  return dispatch2<Fwd>(x_dt, out_dt, x, probs, out, rows, hidden, stream);
+}
+
+int launch_router_weight_bwd(const void* grad_out, moe_dtype g_dt, const void* x,
+                             moe_dtype x_dt, const float* probs, void* grad_x,
+                             float* grad_probs, int64_t rows, int64_t hidden,
+                             cudaStream_t stream) {
+  return dispatch2<Bwd>(g_dt, x_dt, grad_out, x, probs, grad_x, grad_probs, rows, hidden,
+                        stream);
+}
+
+}  // namespace moe

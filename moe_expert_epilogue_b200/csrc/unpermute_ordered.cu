@@ -1,0 +1,143 @@
+// unpermute_ordered.cu -- token-local, batch-invariant unpermute
+// (core.inference.moe.batch_invariant: _unpermute_tokens_in_expert_order_kernel,
+// unpermute_tokens_in_expert_order).
+//
+//   out[t, :] = cast( ((+0 + eo[row_0, :]) + eo[row_1, :]) + ... )
+//
+// where row_0, row_1, ... are the inverse-map entries of token t in
+// increasing local expert id.  fp32 sequential adds, no atomics: the bits of
+// a token depend only on that token's rows, never on the grid or the batch.
+//
+// One CTA owns one token at a time (persistent loop up to the
+// device-resident valid_tokens).  Warp 0 compacts the token's inverse-map row
+// into an ordered list of live rows in shared memory (ballot + popc keeps
+// the increasing-expert order); then every thread takes 8-column chunks of
+// the hidden dimension and issues the loads of up to 8 contributing rows
+// before it adds them in list order.
+#include "common.cuh"
+#include "launch.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kBatch = 8;  // contributing rows loaded before they are summed
+
+template <class DI, class DO, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+unpermute_kernel(const typename DI::T* __restrict__ eo, int64_t max_rows,
+                 const int32_t* __restrict__ inv, const int32_t* __restrict__ valid_tokens,
+                 typename DO::T* __restrict__ out, int64_t tokens, int64_t hidden, int E,
+                 int32_t* err) {
+  extern __shared__ int32_t s_list[];  // [2][E]: double-buffered row lists
+  __shared__ int s_count[2];
+  int64_t n = __ldg(valid_tokens);
+  if (n < 0 || n > tokens) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(err, MOE_DEVERR_COUNT);
+    n = n < 0 ? 0 : tokens;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int parity = 0;
+  for (int64_t t = blockIdx.x; t < n; t += gridDim.x, parity ^= 1) {
+    int32_t* list = s_list + parity * E;
+    if (warp == 0) {
+      int count = 0;
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        int32_t row = e < E ? __ldg(inv + t * E + e) : -1;
+        if (row >= max_rows) {
+          flag_error(err, MOE_DEVERR_INVERSE);
+          row = -1;
+        }
+        const unsigned live = __ballot_sync(0xffffffffu, row >= 0);
+        if (row >= 0) list[count + __popc(live & ((1u << lane) - 1u))] = row;
+        count += __popc(live);
+      }
+      if (lane == 0) s_count[parity] = count;
+    }
+    __syncthreads();
+    const int count = s_count[parity];
+    if constexpr (VEC) {
+      const int64_t cpr = hidden / kVec;
+      for (int64_t c = threadIdx.x; c < cpr; c += kThreads) {
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        for (int j0 = 0; j0 < count; j0 += kBatch) {
+          Raw8<DI> raw[kBatch];
+#pragma unroll
+          for (int j = 0; j < kBatch; ++j)
+            if (j0 + j < count) raw[j] = load8<DI>(eo + (int64_t)list[j0 + j] * hidden + c * kVec);
+#pragma unroll
+          for (int j = 0; j < kBatch; ++j) {
+            if (j0 + j < count) {
+              float v[8];
+              widen8<DI>(raw[j], v);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc[i] = acc[i] + v[i];
+            }
+          }
+        }
+        store8<DO>(out + t * hidden + c * kVec, acc);
+      }
+    } else {
+      for (int64_t h = threadIdx.x; h < hidden; h += kThreads) {
+        float acc = 0.0f;
+        for (int j = 0; j < count; ++j) acc = acc + load1<DI>(eo + (int64_t)list[j] * hidden + h);
+        store1<DO>(out + t * hidden + h, acc);
+      }
+    }
+  }
+}
+
+template <class DI, class DO>
+int launch_unpermute(const void* eo, int64_t max_rows, const int32_t* inv,
+                     const int32_t* valid_tokens, void* out, int64_t tokens, int64_t hidden,
+                     int E, int32_t* err, cudaStream_t stream) {
+  const bool vec = hidden % kVec == 0 && aligned16(eo) && aligned16(out);
+  const size_t smem = 2 * (size_t)E * sizeof(int32_t);
+  auto k = vec ? unpermute_kernel<DI, DO, true> : unpermute_kernel<DI, DO, false>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute((const void*)k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  int grid;
+  if (int rc = persistent_grid((const void*)k, smem, tokens > 0 ? tokens : 1, &grid)) return rc;
+  k<<<grid, kThreads, smem, stream>>>(static_cast<const typename DI::T*>(eo), max_rows, inv,
+                                      valid_tokens, static_cast<typename DO::T*>(out), tokens,
+                                      hidden, E, err);
+  return check_launch();
+}
+
+template <class DI>
+int dispatch_out(moe_dtype out_dt, const void* eo, int64_t max_rows, const int32_t* inv,
+                 const int32_t* vt, void* out, int64_t tokens, int64_t hidden, int E,
+                 int32_t* err, cudaStream_t s) {
+  switch (out_dt) {
+    case MOE_BF16: return launch_unpermute<DI, BF16>(eo, max_rows, inv, vt, out, tokens, hidden, E, err, s);
+    case MOE_FP16: return launch_unpermute<DI, F16>(eo, max_rows, inv, vt, out, tokens, hidden, E, err, s);
+    default: return launch_unpermute<DI, F32>(eo, max_rows, inv, vt, out, tokens, hidden, E, err, s);
+  }
+}
+
+}  // namespace
+
+int launch_unpermute_ordered(const void* expert_output, moe_dtype in_dt, int64_t max_rows,
+                             const int32_t* inverse_map, const int32_t* valid_tokens,
+                             void* out, moe_dtype out_dt, int64_t tokens, int64_t hidden,
+                             int32_t num_local_experts, int32_t* dev_err,
+                             cudaStream_t stream) {
+  switch (in_dt) {
+    case MOE_BF16:
+      return dispatch_out<BF16>(out_dt, expert_output, max_rows, inverse_map, valid_tokens, out,
+                                tokens, hidden, num_local_experts, dev_err, stream);
+    case MOE_FP16:
+      return dispatch_out<F16>(out_dt, expert_output, max_rows, inverse_map, valid_tokens, out,
+                               tokens, hidden, num_local_experts, dev_err, stream);
+    default:
+      return dispatch_out<F32>(out_dt, expert_output, max_rows, inverse_map, valid_tokens, out,
+                               tokens, hidden, num_local_experts, dev_err, stream);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,106 @@
+"""The C-ABI library builds, loads and exports every declared symbol; host-side
+argument validation rejects bad calls before anything touches a device (not gpu)."""
+import os
+import re
+
+import pytest
+
+from moe_expert_epilogue_b200 import _abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _abi.lib()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(_abi.SIGNATURES) <= set(names)
+
+
+def test_status_strings_and_version(lib):
+    assert lib.moe_abi_version() == 1
+    for s in range(7):
+        assert lib.moe_status_string(s).decode().startswith("MOE_")
+    assert lib.moe_last_cuda_error() == 0
+
+
+FAKE = 0x10000  # never dereferenced: every case below fails validation first
+
+
+def _status(fn, *args):
+    with pytest.raises(_abi.MoeError) as e:
+        fn(*args)
+    return e.value.status
+
+
+def test_swiglu_validation(lib):
+    f = _abi.moe_swiglu_clamped_fwd
+    assert _status(f, FAKE, FAKE, FAKE, 4, 8, 16, 8, 7.0, _abi.MOE_FP16, 0) == _abi.MOE_ERR_DTYPE
+    assert _status(f, FAKE, FAKE, FAKE, 4, 8, 15, 8, 7.0, _abi.MOE_BF16, 0) == _abi.MOE_ERR_SHAPE
+    assert _status(f, FAKE, FAKE, FAKE, -1, 8, 16, 8, 7.0, _abi.MOE_BF16, 0) == _abi.MOE_ERR_SHAPE
+    for bad in (0.0, -1.0, float("nan")):
+        assert _status(f, FAKE, FAKE, FAKE, 4, 8, 16, 8, bad, _abi.MOE_BF16, 0) == _abi.MOE_ERR_LIMIT
+    assert _status(f, None, FAKE, FAKE, 4, 8, 16, 8, 7.0, _abi.MOE_BF16, 0) == _abi.MOE_ERR_NULL
+    assert _status(f, FAKE + 1, FAKE, FAKE, 4, 8, 16, 8, 7.0, _abi.MOE_BF16, 0) == _abi.MOE_ERR_ALIGN
+    f(None, None, None, 0, 8, 16, 8, 7.0, _abi.MOE_BF16, 0)      # empty: a no-op
+    b = _abi.moe_swiglu_clamped_bwd
+    assert _status(b, FAKE, FAKE, FAKE, FAKE, None, 4, 8, 16, 8, 16, 7.0, 0, 0) == _abi.MOE_ERR_NULL
+    assert _status(b, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 16, 8, 15, 7.0, 0, 0) == _abi.MOE_ERR_SHAPE
+
+
+def test_router_weight_validation(lib):
+    f = _abi.moe_router_weight_mul_fwd
+    assert _status(f, FAKE, 7, FAKE, FAKE, 0, 4, 8, 0) == _abi.MOE_ERR_DTYPE
+    assert _status(f, FAKE + 2, _abi.MOE_FP32, FAKE, FAKE, 0, 4, 8, 0) == _abi.MOE_ERR_ALIGN
+    b = _abi.moe_router_weight_mul_bwd
+    # x and grad_probs must be given together
+    assert _status(b, FAKE, 0, FAKE, 0, FAKE, FAKE, None, 4, 8, 0) == _abi.MOE_ERR_NULL
+    assert _status(b, FAKE, 0, None, 0, FAKE, FAKE, FAKE, 4, 8, 0) == _abi.MOE_ERR_NULL
+
+
+def test_permuted_and_unpermute_validation(lib):
+    a = _abi.moe_act_with_probs_permuted
+    assert _status(a, 9, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 4, 8, 1.0, 0, None, 0) == _abi.MOE_ERR_DTYPE
+    for bad in (0.0, float("inf"), float("nan")):
+        assert _status(a, _abi.MOE_ACT_SQRELU_CLAMP, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 4, 8, bad, 0,
+                       None, 0) == _abi.MOE_ERR_LIMIT
+    assert _status(a, 0, FAKE, FAKE, None, FAKE, FAKE, 4, 4, 8, 1.0, 0, None, 0) == _abi.MOE_ERR_NULL
+    u = _abi.moe_unpermute_ordered
+    assert _status(u, FAKE, 0, 4, FAKE, FAKE, FAKE, 0, 4, 8, 0, None, 0) == _abi.MOE_ERR_SHAPE
+    assert _status(u, FAKE, 0, 4, FAKE, FAKE, FAKE, 0, 4, 8, 5000, None, 0) == _abi.MOE_ERR_SHAPE
+    assert _status(u, FAKE, 0, 4, FAKE, FAKE + 2, FAKE, 0, 4, 8, 4, None, 0) == _abi.MOE_ERR_ALIGN
+
+
+def test_residual_validation(lib):
+    r = _abi.moe_residual_add
+    assert _status(r, FAKE, FAKE, FAKE, FAKE, 16, 3, 0) == _abi.MOE_ERR_DTYPE
+    assert _status(r, FAKE, FAKE, None, FAKE, 16, 0, 0) == _abi.MOE_ERR_NULL
+    assert _status(r, FAKE, FAKE, FAKE, FAKE + 2, 16, _abi.MOE_FP32, 0) == _abi.MOE_ERR_ALIGN
+    assert _status(r, FAKE, FAKE, FAKE, FAKE, -3, 0, 0) == _abi.MOE_ERR_SHAPE
+    r(None, None, None, None, 0, 0, 0)                             # empty: a no-op
+
+
+def test_product_path_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "moe_expert_epilogue_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert "import oracle" not in text and "from oracle" not in text, fn
+                assert "moe_oracle" not in text, fn

@@ -1,0 +1,176 @@
+"""Parity of the batch-invariant permuted activation and of the fixed-order
+unpermute with the CPU oracle (gpu).
+
+SQRELU, padding, untouched rows and the unpermute are bit-exact; SQRELU_CLAMP
+and SWIGLU are within 1 bf16 ulp (tanh / exp implementations differ).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_expert_epilogue_b200 import _abi, inputs, ops
+from tests._util import assert_bits_equal, assert_within_ulp16, bits
+
+pytestmark = pytest.mark.gpu
+
+ACTS = [(_abi.MOE_ACT_SQRELU, oracle.SQRELU, 0), (_abi.MOE_ACT_SQRELU_CLAMP, oracle.SQRELU_CLAMP, 1),
+        (_abi.MOE_ACT_SWIGLU, oracle.SWIGLU, 1)]
+CANARY = 0x1234
+
+
+def _run_act(dev, act, rt, x, width, scale, zero_padding, n_used=None, pmap=None, err=None):
+    out = torch.full((rt.max_rows, width), 0, dtype=torch.int16, device=dev).fill_(CANARY) \
+        .view(torch.bfloat16)
+    nu = torch.tensor([rt.n_used if n_used is None else n_used], dtype=torch.int32, device=dev)
+    pm = (rt.permutation_map if pmap is None else pmap).to(dev)
+    ops.act_with_probs_permuted(act, x.to(dev), pm, nu, rt.probs.to(dev), scale, zero_padding,
+                                out=out, dev_err=err)
+    torch.cuda.synchronize()
+    return bits(out)
+
+
+@pytest.mark.parametrize("act,oact,tol", ACTS)
+@pytest.mark.parametrize("zero_padding", [False, True])
+@pytest.mark.parametrize("tokens,top_k,experts,align,width", [
+    (12, 2, 4, 4, 24), (100, 4, 8, 16, 1001), (257, 8, 16, 128, 1536)])
+def test_act_permuted_parity(cuda_device, act, oact, tol, zero_padding, tokens, top_k, experts,
+                             align, width):
+    rt = inputs.routing(tokens, top_k, experts, align, seed=tokens)
+    x = inputs.permuted_activation_input(rt, width, swiglu=(oact == oracle.SWIGLU), seed=tokens + 1)
+    got = _run_act(cuda_device, act, rt, x, width, 7.0, zero_padding)
+    ref, err = oracle.act_with_probs_permuted(oact, bits(x), np.full((rt.max_rows, width), CANARY,
+                                                                     np.uint16),
+                                              bits(rt.permutation_map), rt.n_used, bits(rt.probs),
+                                              width, 7.0, zero_padding)
+    assert err == 0
+    if tol == 0:
+        assert_bits_equal(got, ref, "act")
+    else:
+        assert_within_ulp16(got, ref, tol, what="act")
+        # padding / untouched rows are exact whatever the activation
+        dead = bits(rt.permutation_map) < 0
+        assert_bits_equal(got[dead], ref[dead], "padding rows")
+
+
+@pytest.mark.parametrize("act,oact,tol", ACTS)
+def test_act_permuted_full_workload_sampled(cuda_device, act, oact, tol):
+    """8192 tokens, top-8 of 64 experts, rows padded to 128 per expert
+    (max_rows 73728), hidden 1536 / ffn 1536, zero padding on."""
+    rt = inputs.routing(8192, 8, 64, 128, seed=0)
+    width = 1536
+    x = inputs.permuted_activation_input(rt, width, swiglu=(oact == oracle.SWIGLU), seed=1)
+    got = _run_act(cuda_device, act, rt, x, width, 7.0, True)
+    pm = bits(rt.permutation_map)
+    rng = np.random.default_rng(2)
+    idx = np.unique(np.concatenate([[0, rt.n_used - 1, rt.n_used, rt.max_rows - 1],
+                                    rng.integers(0, rt.max_rows, 400),
+                                    np.flatnonzero(pm < 0)[:50]]))
+    sub_map = pm[idx]
+    # the oracle on the sampled rows: a compacted problem with the same map entries
+    ref, err = oracle.act_with_probs_permuted(
+        oact, bits(x)[idx], np.full((idx.size, width), CANARY, np.uint16),
+        np.where(idx < rt.n_used, sub_map, -1).astype(np.int32), idx.size, bits(rt.probs), width,
+        7.0, True)
+    live_or_pad = idx < rt.n_used
+    ref[~live_or_pad] = CANARY                      # rows past n_used are not touched
+    if tol == 0:
+        assert_bits_equal(got[idx], ref, "act")
+    else:
+        assert_within_ulp16(got[idx], ref, tol, what="act")
+    assert (got[rt.n_used:] == CANARY).all()
+    assert (got[:rt.n_used][pm[:rt.n_used] < 0] == 0).all()
+
+
+def test_act_permuted_bad_metadata_sets_error_bits(cuda_device):
+    rt = inputs.routing(40, 2, 4, 8, seed=3)
+    width = 16
+    x = inputs.permuted_activation_input(rt, width, swiglu=False, seed=4)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    got = _run_act(cuda_device, _abi.MOE_ACT_SQRELU, rt, x, width, 1.0, True,
+                   n_used=rt.max_rows + 100, err=err)
+    assert int(err) & _abi.MOE_DEVERR_COUNT
+    # clamped to max_rows: rows past the old n_used are padding (map < 0) -> zero-filled
+    assert (got[rt.n_used:] == 0).all()
+    pm = rt.permutation_map.clone()
+    live = torch.nonzero(pm >= 0).flatten()
+    pm[live[0]] = 1 << 30
+    err.zero_()
+    got = _run_act(cuda_device, _abi.MOE_ACT_SQRELU, rt, x, width, 1.0, True, pmap=pm, err=err)
+    assert int(err) == _abi.MOE_DEVERR_MAP
+    assert (got[int(live[0])] == CANARY).all()
+    err.zero_()
+    _run_act(cuda_device, _abi.MOE_ACT_SQRELU, rt, x, width, 1.0, True, n_used=-5, err=err)
+    assert int(err) == _abi.MOE_DEVERR_COUNT
+
+
+# ------------------------------------------------------------------ unpermute
+
+ODT = {torch.bfloat16: oracle.BF16, torch.float16: oracle.F16, torch.float32: oracle.F32}
+
+
+def _run_unpermute(dev, rt, eo, out_dtype, valid, inv=None, err=None):
+    out = torch.full((rt.tokens, eo.shape[1]), 3.0, dtype=out_dtype, device=dev)
+    vt = torch.tensor([valid], dtype=torch.int32, device=dev)
+    ops.unpermute_ordered(eo.to(dev), (rt.inverse_map if inv is None else inv).to(dev), vt, out,
+                          dev_err=err)
+    torch.cuda.synchronize()
+    return bits(out)
+
+
+@pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32, torch.float16])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32, torch.float16])
+@pytest.mark.parametrize("tokens,top_k,experts,align,hidden,valid", [
+    (50, 2, 4, 4, 72, 50), (300, 8, 64, 16, 1001, 290), (129, 6, 10, 128, 4096, 100)])
+def test_unpermute_bitwise(cuda_device, in_dtype, out_dtype, tokens, top_k, experts, align, hidden,
+                           valid):
+    rt = inputs.routing(tokens, top_k, experts, align, seed=hidden)
+    eo = inputs.expert_output_input(rt, hidden, dtype=in_dtype, seed=hidden + 1)
+    got = _run_unpermute(cuda_device, rt, eo, out_dtype, valid)
+    init = bits(torch.full((tokens, hidden), 3.0, dtype=out_dtype))
+    ref, err = oracle.unpermute_ordered(bits(eo), ODT[in_dtype], bits(rt.inverse_map), valid, init,
+                                        ODT[out_dtype])
+    assert err == 0
+    assert_bits_equal(got, ref, "unpermute", kind="f16" if out_dtype == torch.float16 else "bf16")
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_unpermute_full_workload_bitwise(cuda_device, out_dtype):
+    """8192 tokens x top-8 of 64 experts, hidden 4096: the whole output."""
+    rt = inputs.routing(8192, 8, 64, 128, seed=0)
+    eo = inputs.expert_output_input(rt, 4096, seed=2)
+    got = _run_unpermute(cuda_device, rt, eo, out_dtype, rt.tokens)
+    init = bits(torch.full((rt.tokens, 4096), 3.0, dtype=out_dtype))
+    ref, _ = oracle.unpermute_ordered(bits(eo), oracle.BF16, bits(rt.inverse_map), rt.tokens, init,
+                                      ODT[out_dtype])
+    assert_bits_equal(got, ref, "unpermute")
+
+
+def test_unpermute_order_witness_and_bad_entries(cuda_device):
+    # contributions 1, 2^24, -2^24 in expert order 0, 1, 2: fp32 gives 0, not 1
+    rt = inputs.Routing(2, 3, 3, 1, 3, 3, torch.tensor([0, 1, 2], dtype=torch.int32),
+                        torch.tensor([[0, 1, 2], [2, 1, 0]], dtype=torch.int32),
+                        torch.ones(6), torch.tensor([2, 2, 2]))
+    eo = torch.tensor([[1.0] * 8, [2.0 ** 24] * 8, [-(2.0 ** 24)] * 8], dtype=torch.bfloat16)
+    got = _run_unpermute(cuda_device, rt, eo, torch.float32, 2)
+    assert (got[0] == 0.0).all() and (got[1] == 1.0).all()
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    inv = rt.inverse_map.clone()
+    inv[0, 1] = 99
+    got = _run_unpermute(cuda_device, rt, eo, torch.float32, 5, inv=inv, err=err)
+    assert int(err) == _abi.MOE_DEVERR_COUNT | _abi.MOE_DEVERR_INVERSE
+    assert (got[0] == 1.0 - 2.0 ** 24).all()
+
+
+def test_unpermute_batch_invariant(cuda_device):
+    """A token's bits do not depend on the other tokens: shuffling the rest of
+    the batch (and its size) leaves them unchanged."""
+    rt = inputs.routing(512, 8, 64, 16, seed=5)
+    eo = inputs.expert_output_input(rt, 2048, seed=6)
+    full = _run_unpermute(cuda_device, rt, eo, torch.bfloat16, rt.tokens)
+    perm = torch.randperm(rt.tokens, generator=torch.Generator().manual_seed(7))
+    sub = perm[:37]
+    rt2 = inputs.Routing(37, 8, 64, 16, rt.max_rows, rt.n_used, rt.permutation_map,
+                         rt.inverse_map[sub].contiguous(), rt.probs, rt.counts)
+    part = _run_unpermute(cuda_device, rt2, eo, torch.bfloat16, 37)
+    assert_bits_equal(part, full[sub.numpy()], "batch invariance")

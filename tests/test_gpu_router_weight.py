@@ -1,0 +1,95 @@
+"""Parity of the router-weight multiply kernels with the CPU oracle (gpu).
+
+Forward and grad_x are single fp32 multiplies with one rounding: bit-exact.
+grad_probs is a row reduction: within 1e-5 * max(|ref|, sum_h |t_h|).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_expert_epilogue_b200 import inputs, ops
+from tests._util import assert_bits_equal, assert_sum_close, bits
+
+pytestmark = pytest.mark.gpu
+
+ODT = {torch.bfloat16: oracle.BF16, torch.float16: oracle.F16, torch.float32: oracle.F32}
+DTYPES = [torch.bfloat16, torch.float16, torch.float32]
+
+
+@pytest.mark.parametrize("rows,hidden", [(129, 7176), (300, 1001), (1, 8), (7, 3), (2048, 256)])
+@pytest.mark.parametrize("x_dtype", DTYPES)
+@pytest.mark.parametrize("out_dtype", DTYPES)
+def test_router_weight_fwd_bitwise(cuda_device, rows, hidden, x_dtype, out_dtype):
+    d = inputs.router_weight_inputs(rows, hidden, seed=rows + hidden)
+    x = d["x"].to(x_dtype)
+    out = ops.router_weight_mul_fwd(x.to(cuda_device), d["probs"].to(cuda_device), out_dtype)
+    torch.cuda.synchronize()
+    ref = oracle.router_weight_fwd(bits(x), ODT[x_dtype], bits(d["probs"]), ODT[out_dtype])
+    assert_bits_equal(bits(out), ref, "fwd", kind="f16" if out_dtype == torch.float16 else "bf16")
+
+
+@pytest.mark.parametrize("rows,hidden", [(129, 7176), (300, 1001), (1, 8), (3000, 40)])
+@pytest.mark.parametrize("g_dtype", [torch.bfloat16, torch.float32, torch.float16])
+@pytest.mark.parametrize("x_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("save_x", [True, False])
+def test_router_weight_bwd(cuda_device, rows, hidden, g_dtype, x_dtype, save_x):
+    d = inputs.router_weight_inputs(rows, hidden, out_dtype=g_dtype, seed=rows * 3 + hidden)
+    x = d["x"].to(x_dtype)
+    gx, gp = ops.router_weight_mul_bwd(d["grad_out"].to(cuda_device),
+                                       x.to(cuda_device) if save_x else None,
+                                       d["probs"].to(cuda_device), x_dtype=x_dtype)
+    torch.cuda.synchronize()
+    gx_ref, gp_ref, gabs = oracle.router_weight_bwd(bits(d["grad_out"]), ODT[g_dtype],
+                                                    bits(x) if save_x else None, ODT[x_dtype],
+                                                    bits(d["probs"]))
+    assert_bits_equal(bits(gx), gx_ref, "grad_x")
+    if save_x:
+        assert_sum_close(bits(gp).ravel(), gp_ref, gabs, 1e-5, "grad_probs")
+    else:
+        assert gp is None
+
+
+def test_router_weight_unaligned(cuda_device):
+    rows, hidden = 33, 64
+    d = inputs.router_weight_inputs(rows, hidden, seed=5)
+    buf = torch.empty(rows * hidden + 1, dtype=torch.bfloat16, device=cuda_device)
+    x = buf[1:].view(rows, hidden)
+    x.copy_(d["x"].to(cuda_device))
+    p = d["probs"].to(cuda_device)
+    out = ops.router_weight_mul_fwd(x, p, torch.float32)
+    gx, gp = ops.router_weight_mul_bwd(d["grad_out"].to(cuda_device), x, p)
+    torch.cuda.synchronize()
+    assert_bits_equal(bits(out), oracle.router_weight_fwd(bits(d["x"]), oracle.BF16,
+                                                          bits(d["probs"]), oracle.F32), "fwd")
+    gx_ref, gp_ref, gabs = oracle.router_weight_bwd(bits(d["grad_out"]), oracle.BF16,
+                                                    bits(d["x"]), oracle.BF16, bits(d["probs"]))
+    assert_bits_equal(bits(gx), gx_ref, "grad_x")
+    assert_sum_close(bits(gp).ravel(), gp_ref, gabs, 1e-5, "grad_probs")
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_router_weight_full_workload_sampled_rows(cuda_device, out_dtype):
+    """[16384, 7168] expert outputs, U(0.01, 1) probs: the full launches,
+    checked on sampled rows (fwd and both grads, save_x on and off)."""
+    rows, hidden = 16384, 7168
+    d = inputs.router_weight_inputs(rows, hidden, out_dtype=out_dtype, seed=0)
+    x, p, g = (d[k].to(cuda_device) for k in ("x", "probs", "grad_out"))
+    out = ops.router_weight_mul_fwd(x, p, out_dtype)
+    gx, gp = ops.router_weight_mul_bwd(g, x, p)
+    gx2, _ = ops.router_weight_mul_bwd(g, None, p, x_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(1)
+    idx = np.unique(np.concatenate([[0, rows - 1], rng.integers(0, rows, 254)]))
+    ti = torch.from_numpy(idx)
+    xb, pb, gb = bits(d["x"])[idx], bits(d["probs"])[idx], bits(d["grad_out"])[idx]
+    assert_bits_equal(bits(out.cpu()[ti]),
+                      oracle.router_weight_fwd(xb, oracle.BF16, pb, ODT[out_dtype]), "fwd")
+    gx_ref, gp_ref, gabs = oracle.router_weight_bwd(gb, ODT[out_dtype], xb, oracle.BF16, pb)
+    assert_bits_equal(bits(gx.cpu()[ti]), gx_ref, "grad_x")
+    assert_bits_equal(bits(gx2.cpu()[ti]), gx_ref, "grad_x (x not saved)")
+    assert_sum_close(bits(gp.cpu()[ti]).ravel(), gp_ref, gabs, 1e-5, "grad_probs")
+    # eager torch on the device computes the same forward bits (the page's definition)
+    assert torch.equal((x.float() * p).to(out_dtype).view(torch.int8 if out_dtype != torch.float32
+                                                          else torch.int32).cpu()[ti],
+                       out.view(torch.int8 if out_dtype != torch.float32 else torch.int32).cpu()[ti])

@@ -1,0 +1,173 @@
+"""Parity of the clamped-SwiGLU kernels with the CPU oracle (gpu).
+
+Tolerances (pass criteria of the op): y and grad_x within 1 bf16 ulp (the two
+sides use different exp / reciprocal implementations), grad_probs within
+1e-5 * max(|ref|, sum_j |t_j|) of the float64 sum of the fp32 terms.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_expert_epilogue_b200 import inputs, ops
+from tests._util import assert_bits_equal, assert_sum_close, assert_within_ulp16, bits
+
+pytestmark = pytest.mark.gpu
+INF = float("inf")
+
+
+def _check(d, limit, y, gx, gp, rows_idx=None):
+    xb, pb, gyb = bits(d["x"]), bits(d["probs"]), bits(d["grad_y"])
+    if rows_idx is not None:
+        xb, pb, gyb = xb[rows_idx], pb[rows_idx], gyb[rows_idx]
+    y_ref = oracle.swiglu_clamped_fwd(xb, pb, limit)
+    assert_within_ulp16(y, y_ref, 1, what="y")
+    gx_ref, gp_ref, gabs = oracle.swiglu_clamped_bwd(xb, pb, gyb, limit)
+    assert_within_ulp16(gx, gx_ref, 1, what="grad_x")
+    assert_sum_close(np.asarray(gp).ravel(), gp_ref, gabs, 1e-5, "grad_probs")
+
+
+def _ties_ok(limit):
+    return limit != INF and float(torch.tensor(limit, dtype=torch.bfloat16)) == limit
+
+
+@pytest.mark.parametrize("rows,inter,limit,sigma", [
+    (256, 512, 7.0, 2.0),      # the small workload, L = 7
+    (256, 512, INF, 2.0),      # the small workload, unclamped
+    (777, 1032, 7.0, 3.0),     # ragged rows, inter % 256 != 0
+    (300, 2048, 10.0, 5.1),    # the large workload's row shape
+    (64, 7168, 7.3, 4.0),      # long rows, limit not representable in bf16
+    (333, 1001, 10.0, 3.0),    # odd inter: element-wise path
+    (5, 8, 7.0, 8.0),
+    (1, 1, 7.0, 8.0),
+    (1000, 40, 7.0, 8.0),      # short rows: one warp per row
+])
+def test_swiglu_fwd_bwd_parity(cuda_device, rows, inter, limit, sigma):
+    d = inputs.swiglu_inputs(rows, inter, sigma=sigma, limit=limit, plant_ties=_ties_ok(limit),
+                             seed=rows + inter)
+    x, p, gy = (d[k].to(cuda_device) for k in ("x", "probs", "grad_y"))
+    y = ops.swiglu_clamped_fwd(x, p, limit)
+    gx, gp = ops.swiglu_clamped_bwd(x, p, gy, limit)
+    torch.cuda.synchronize()
+    _check(d, limit, bits(y), bits(gx), bits(gp))
+
+
+def test_swiglu_strided_rows_and_untouched_padding(cuda_device):
+    rows, inter, L = 130, 264, 7.0
+    d = inputs.swiglu_inputs(rows, inter, sigma=3.0, limit=L, plant_ties=True, seed=11)
+    xw = torch.full((rows, 2 * inter + 24), float("nan"), dtype=torch.bfloat16)
+    xw[:, :2 * inter] = d["x"]
+    gyw = torch.full((rows, inter + 16), float("nan"), dtype=torch.bfloat16)
+    gyw[:, :inter] = d["grad_y"]
+    xw, gyw = xw.to(cuda_device), gyw.to(cuda_device)
+    p = d["probs"].to(cuda_device)
+    yw = torch.full((rows, inter + 8), 3.0, dtype=torch.bfloat16, device=cuda_device)
+    gxw = torch.full((rows, 2 * inter + 8), 5.0, dtype=torch.bfloat16, device=cuda_device)
+    ops.swiglu_clamped_fwd(xw[:, :2 * inter], p, L, out=yw[:, :inter])
+    ops.swiglu_clamped_bwd(xw[:, :2 * inter], p, gyw[:, :inter], L, grad_x=gxw[:, :2 * inter])
+    gp = torch.empty(rows, 1, device=cuda_device)
+    ops.swiglu_clamped_bwd(xw[:, :2 * inter], p, gyw[:, :inter], L, grad_x=gxw[:, :2 * inter],
+                           grad_probs=gp)
+    torch.cuda.synchronize()
+    _check(d, L, bits(yw[:, :inter]), bits(gxw[:, :2 * inter]), bits(gp))
+    assert (yw[:, inter:] == 3.0).all() and (gxw[:, 2 * inter:] == 5.0).all()
+
+
+def test_swiglu_unaligned_pointers_take_the_elementwise_path(cuda_device):
+    rows, inter, L = 97, 256, 7.0
+    d = inputs.swiglu_inputs(rows, inter, sigma=3.0, limit=L, plant_ties=True, seed=12)
+    buf = torch.empty(rows * 2 * inter + 1, dtype=torch.bfloat16, device=cuda_device)
+    x = buf[1:].view(rows, 2 * inter)
+    x.copy_(d["x"].to(cuda_device))
+    assert x.data_ptr() % 16 != 0
+    p, gy = d["probs"].to(cuda_device), d["grad_y"].to(cuda_device)
+    y = ops.swiglu_clamped_fwd(x, p, L)
+    gx, gp = ops.swiglu_clamped_bwd(x, p, gy, L)
+    torch.cuda.synchronize()
+    _check(d, L, bits(y), bits(gx), bits(gp))
+
+
+def test_swiglu_nan_and_extreme_inputs(cuda_device):
+    vals = [float("nan"), -100.0, -88.5, -87.0, -20.0, -1.2734375, -1.28125, 0.0, -0.0, 7.0,
+            7.03125, 100.0, 3e38, -3e38, 1e-38, -1e-40]
+    g = torch.tensor(vals, dtype=torch.bfloat16)
+    u = torch.tensor(vals[::-1], dtype=torch.bfloat16)
+    rows = len(vals)
+    x = torch.zeros(rows, 16, dtype=torch.bfloat16)
+    x[:, :8] = g[:, None]
+    x[:, 8:] = u[:, None]
+    d = {"x": x, "probs": torch.linspace(0.1, 1.0, rows).reshape(rows, 1),
+         "grad_y": torch.ones(rows, 8, dtype=torch.bfloat16)}
+    for L in (7.0, INF):
+        xd, p, gy = (d[k].to(cuda_device) for k in ("x", "probs", "grad_y"))
+        y = ops.swiglu_clamped_fwd(xd, p, L)
+        gx, gp = ops.swiglu_clamped_bwd(xd, p, gy, L)
+        torch.cuda.synchronize()
+        xb, pb = bits(d["x"]), bits(d["probs"])
+        assert_within_ulp16(bits(y), oracle.swiglu_clamped_fwd(xb, pb, L), 1, what="y")
+        gx_ref, gp_ref, _ = oracle.swiglu_clamped_bwd(xb, pb, bits(d["grad_y"]), L)
+        assert_within_ulp16(bits(gx), gx_ref, 1, what="grad_x")
+        got = bits(gp).ravel()
+        fin = np.isfinite(gp_ref) & (np.abs(gp_ref) < 1e37)   # no fp32 overflow in the sum
+        assert np.array_equal(np.isnan(got), np.isnan(gp_ref))
+        np.testing.assert_allclose(got[fin], gp_ref[fin], rtol=1e-5, atol=1e-30)
+
+
+def test_swiglu_deterministic_and_batch_invariant(cuda_device):
+    rows, inter, L = 1500, 2048, 10.0
+    d = inputs.swiglu_inputs(rows, inter, sigma=3.0, seed=13)
+    x, p, gy = (d[k].to(cuda_device) for k in ("x", "probs", "grad_y"))
+    y1 = ops.swiglu_clamped_fwd(x, p, L)
+    g1, q1 = ops.swiglu_clamped_bwd(x, p, gy, L)
+    y2 = ops.swiglu_clamped_fwd(x, p, L)
+    g2, q2 = ops.swiglu_clamped_bwd(x, p, gy, L)
+    # a sub-batch (different grid, different neighbours) gives the same bits
+    sl = slice(700, 703)
+    y3 = ops.swiglu_clamped_fwd(x[sl].contiguous(), p[sl].contiguous(), L)
+    g3, q3 = ops.swiglu_clamped_bwd(x[sl].contiguous(), p[sl].contiguous(), gy[sl].contiguous(), L)
+    torch.cuda.synchronize()
+    for a, b in ((y1, y2), (g1, g2), (q1, q2), (y1[sl], y3), (g1[sl], g3), (q1[sl], q3)):
+        assert_bits_equal(bits(a), bits(b), "determinism / batch invariance")
+
+
+def test_swiglu_cuda_graph_replay(cuda_device):
+    rows, inter, L = 512, 2048, 10.0
+    d = inputs.swiglu_inputs(rows, inter, sigma=3.0, seed=14)
+    x, p, gy = (d[k].to(cuda_device) for k in ("x", "probs", "grad_y"))
+    y = torch.empty(rows, inter, dtype=torch.bfloat16, device=cuda_device)
+    gx = torch.empty_like(x)
+    gp = torch.empty(rows, 1, device=cuda_device)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):                       # warm-up outside capture
+        ops.swiglu_clamped_fwd(x, p, L, out=y)
+        ops.swiglu_clamped_bwd(x, p, gy, L, grad_x=gx, grad_probs=gp)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ops.swiglu_clamped_fwd(x, p, L, out=y)
+        ops.swiglu_clamped_bwd(x, p, gy, L, grad_x=gx, grad_probs=gp)
+    y.zero_(); gx.zero_(); gp.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    _check(d, L, bits(y), bits(gx), bits(gp))
+
+
+@pytest.mark.parametrize("sigma", [3.0, 5.1])
+def test_swiglu_large_workload_sampled_rows(cuda_device, sigma):
+    """rows = 65536 (8192 tokens x top-8), inter = 2048, L = 10, top-8 softmax
+    probs: the full launch the benchmark times, checked on sampled rows."""
+    rows, inter, L = 65536, 2048, 10.0
+    d = inputs.swiglu_inputs(rows, inter, sigma=sigma, probs="topk_softmax", seed=0)
+    x, p, gy = (d[k].to(cuda_device) for k in ("x", "probs", "grad_y"))
+    y = ops.swiglu_clamped_fwd(x, p, L)
+    gx, gp = ops.swiglu_clamped_bwd(x, p, gy, L)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(int(sigma * 10))
+    idx = np.unique(np.concatenate([[0, 1, rows - 1], rng.integers(0, rows, 509)]))
+    ti = torch.from_numpy(idx)
+    _check(d, L, bits(y.cpu()[ti]), bits(gx.cpu()[ti]), bits(gp.cpu()[ti]), rows_idx=idx)
+    # whole-tensor properties: masks exactly where the inputs leave the range
+    gate, up = x[:, :inter], x[:, inter:]
+    assert bool((gx[:, :inter][gate > L] == 0).all())
+    assert bool((gx[:, inter:][(up > L) | (up < -L)] == 0).all())
+    assert bool(torch.isfinite(y.float()).all()) and bool(torch.isfinite(gp).all())
