@@ -49,20 +49,32 @@ ROUTER = dict(rows=16384, hidden=7168)
 PERMUTED = dict(tokens=8192, top_k=8, experts=64, align=128, width=1536, hidden=4096, scale=7.0)
 RESIDUAL = dict(rows=32768, hidden=7168)
 
+
+def scaled(scale: float) -> dict:
+    """The workload with every op's row (token) count multiplied by `scale`
+    (1.0 = the benchmark; smaller scales serve short profiler captures)."""
+    f = lambda n, m=8: max(m, int(n * scale) // m * m)  # noqa: E731
+    return {"swiglu": dict(SWIGLU, rows=f(SWIGLU["rows"])),
+            "router": dict(ROUTER, rows=f(ROUTER["rows"])),
+            "permuted": dict(PERMUTED, tokens=f(PERMUTED["tokens"])),
+            "residual": dict(RESIDUAL, rows=f(RESIDUAL["rows"]))}
+
+
 WORKLOAD_NAME = ("moe_expert_epilogue_pass: clamped SwiGLU fwd+bwd rows=65536 inter=2048 L=10; "
                  "router-weight fwd+bwd [16384,7168]; permuted SQRELU/SQRELU_CLAMP/SWIGLU + "
                  "ordered unpermute (8192 tok, top-8 of 64, align 128, width 1536, hidden 4096); "
                  "residual add [32768,7168]; all bf16 with fp32 probs")
 
 
-def algorithmic_bytes(n_used: int) -> dict:
+def algorithmic_bytes(n_used: int, scale: float = 1.0) -> dict:
     """Minimal bytes per launch: each input byte read once, each output byte
     written once; padding rows count as written (zero padding), never as read."""
-    R, I = SWIGLU["rows"], SWIGLU["inter"]
-    Rr, H = ROUTER["rows"], ROUTER["hidden"]
-    live = PERMUTED["tokens"] * PERMUTED["top_k"]
+    w = scaled(scale)
+    R, I = w["swiglu"]["rows"], SWIGLU["inter"]
+    Rr, H = w["router"]["rows"], ROUTER["hidden"]
+    live = w["permuted"]["tokens"] * PERMUTED["top_k"]
     W = PERMUTED["width"]
-    T, E, Hu = PERMUTED["tokens"], PERMUTED["experts"], PERMUTED["hidden"]
+    T, E, Hu = w["permuted"]["tokens"], PERMUTED["experts"], PERMUTED["hidden"]
     meta = 4 * n_used + 4 * live          # permutation map rows + gathered probs
     return {
         "swiglu_fwd": R * (2 * I * 2 + 4 + I * 2),
@@ -73,16 +85,17 @@ def algorithmic_bytes(n_used: int) -> dict:
         "act_sqrelu_clamp": live * W * 2 + n_used * W * 2 + meta,
         "act_swiglu": live * 2 * W * 2 + n_used * W * 2 + meta,
         "unpermute": live * Hu * 2 + T * E * 4 + T * Hu * 2,
-        "residual_add": 4 * RESIDUAL["rows"] * RESIDUAL["hidden"] * 2,
+        "residual_add": 4 * w["residual"]["rows"] * RESIDUAL["hidden"] * 2,
     }
 
 
-ROWS = {  # rows (or tokens) one launch processes, for rows/s
-    "swiglu_fwd": SWIGLU["rows"], "swiglu_bwd": SWIGLU["rows"],
-    "router_weight_fwd": ROUTER["rows"], "router_weight_bwd": ROUTER["rows"],
-    "act_sqrelu": None, "act_sqrelu_clamp": None, "act_swiglu": None,
-    "unpermute": PERMUTED["tokens"], "residual_add": RESIDUAL["rows"],
-}
+def rows_per_launch(scale: float = 1.0) -> dict:
+    """Rows (tokens) one launch processes, for rows/s."""
+    w = scaled(scale)
+    return {"swiglu_fwd": w["swiglu"]["rows"], "swiglu_bwd": w["swiglu"]["rows"],
+            "router_weight_fwd": w["router"]["rows"], "router_weight_bwd": w["router"]["rows"],
+            "act_sqrelu": None, "act_sqrelu_clamp": None, "act_swiglu": None,
+            "unpermute": w["permuted"]["tokens"], "residual_add": w["residual"]["rows"]}
 
 KERNEL_SOURCES = {
     "swiglu_fwd": "swiglu_clamped.cu", "swiglu_bwd": "swiglu_clamped.cu",
@@ -96,16 +109,18 @@ KERNEL_SOURCES = {
 class Batch:
     """All inputs and outputs of one step, on one device."""
 
-    def __init__(self, device, seed):
+    def __init__(self, device, seed, scale=1.0):
         from moe_expert_epilogue_b200 import inputs
+        self.scale = scale
+        w = scaled(scale)
         gen_dev = device if device.type == "cuda" else "cpu"
-        sw = inputs.swiglu_inputs(SWIGLU["rows"], SWIGLU["inter"], sigma=SWIGLU["sigma"],
+        sw = inputs.swiglu_inputs(w["swiglu"]["rows"], SWIGLU["inter"], sigma=SWIGLU["sigma"],
                                   probs="topk_softmax", seed=seed, device=gen_dev)
         self.sw_x, self.sw_p, self.sw_gy = sw["x"], sw["probs"], sw["grad_y"]
-        rw = inputs.router_weight_inputs(ROUTER["rows"], ROUTER["hidden"], seed=seed + 1,
+        rw = inputs.router_weight_inputs(w["router"]["rows"], ROUTER["hidden"], seed=seed + 1,
                                          device=gen_dev)
         self.rw_x, self.rw_p, self.rw_g = rw["x"], rw["probs"], rw["grad_out"]
-        rt = inputs.routing(PERMUTED["tokens"], PERMUTED["top_k"], PERMUTED["experts"],
+        rt = inputs.routing(w["permuted"]["tokens"], PERMUTED["top_k"], PERMUTED["experts"],
                             PERMUTED["align"], seed=seed + 2, device=gen_dev)
         self.rt = rt
         W = PERMUTED["width"]
@@ -118,20 +133,20 @@ class Batch:
         self.eo = inputs.expert_output_input(rt, PERMUTED["hidden"], seed=seed + 5, device=gen_dev)
         self.inv = rt.inverse_map
         self.valid = torch.tensor([rt.tokens], dtype=torch.int32, device=gen_dev)
-        res = inputs.residual_inputs((RESIDUAL["rows"], RESIDUAL["hidden"]), torch.bfloat16,
+        res = inputs.residual_inputs((w["residual"]["rows"], RESIDUAL["hidden"]), torch.bfloat16,
                                      seed=seed + 6, device=gen_dev)
         self.res_e, self.res_s, self.res_r = (res["expert_output"], res["shared_expert_output"],
                                               res["residual"])
         self.to(device)
         # outputs
         z = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device=device)  # noqa: E731
-        R, I = SWIGLU["rows"], SWIGLU["inter"]
+        R, I = w["swiglu"]["rows"], SWIGLU["inter"]
+        Rr = w["router"]["rows"]
         self.sw_y, self.sw_gx, self.sw_gp = z(R, I), z(R, 2 * I), z(R, 1, dt=torch.float32)
-        self.rw_gx, self.rw_gp = z(ROUTER["rows"], ROUTER["hidden"]), z(ROUTER["rows"], 1,
-                                                                        dt=torch.float32)
+        self.rw_gx, self.rw_gp = z(Rr, ROUTER["hidden"]), z(Rr, 1, dt=torch.float32)
         self.act_o1, self.act_o2, self.act_o3 = (z(rt.max_rows, W) for _ in range(3))
-        self.unp_out = z(PERMUTED["tokens"], PERMUTED["hidden"])
-        self.res_out = z(RESIDUAL["rows"], RESIDUAL["hidden"])
+        self.unp_out = z(w["permuted"]["tokens"], PERMUTED["hidden"])
+        self.res_out = z(w["residual"]["rows"], RESIDUAL["hidden"])
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
 
     INPUT_NAMES = ("sw_x", "sw_p", "sw_gy", "rw_x", "rw_p", "rw_g", "act_x", "act_x2", "pmap",
@@ -148,9 +163,8 @@ class Batch:
         from moe_expert_epilogue_b200 import ops
         L = SWIGLU["limit"]
         P = PERMUTED
-        half = ROUTER["rows"]
-        # the router-weight forward writes the first half of the residual's expert output
-        rw_out = self.res_e[:half]
+        # the router-weight forward writes the first rows of the residual's expert output
+        rw_out = self.res_e[:self.rw_x.shape[0]]
         return [
             ("swiglu_fwd", lambda: ops.swiglu_clamped_fwd(self.sw_x, self.sw_p, L, out=self.sw_y)),
             ("router_weight_fwd", lambda: ops.router_weight_mul_fwd(
@@ -324,9 +338,15 @@ def run_ours(args):
             mbuild.build()
         barrier(device)
 
-    batch = Batch(device, seed=1000 * rank)
+    batch = Batch(device, seed=1000 * rank, scale=args.scale)
     kernels = batch.kernels()
-    nbytes = algorithmic_bytes(batch.rt.n_used)
+    if args.kernel:
+        kernels = [(n, f) for n, f in kernels if n in args.kernel.split(",")]
+        if not kernels:
+            raise SystemExit(f"unknown --kernel {args.kernel}")
+    nbytes = algorithmic_bytes(batch.rt.n_used, args.scale)
+    nbytes = {n: nbytes[n] for n, _ in kernels}
+    rows = rows_per_launch(args.scale)
     bytes_per_step = sum(nbytes.values())
     stream = torch.cuda.current_stream(device)
 
@@ -366,8 +386,8 @@ def run_ours(args):
                             "bytes": nbytes[name], "gbs": round(gbs, 1),
                             "frac": round(gbs / peak, 4),
                             "share": None}
-        if ROWS[name]:
-            per_kernel[name]["rows_per_s"] = ROWS[name] / (avg_ms * 1e-3)
+        if rows[name]:
+            per_kernel[name]["rows_per_s"] = rows[name] / (avg_ms * 1e-3)
     total_kernel_ms = sum(v["us"] for v in per_kernel.values())
     for v in per_kernel.values():
         v["share"] = round(v["us"] / total_kernel_ms, 4)
@@ -375,11 +395,20 @@ def run_ours(args):
     d = per_kernel[dominant]
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.kernel:
         e2e = run_e2e(batch, kernels, nbytes, args, device)
 
-    sw_bytes = nbytes["swiglu_fwd"] + nbytes["swiglu_bwd"]
-    sw_us = per_kernel["swiglu_fwd"]["us"] + per_kernel["swiglu_bwd"]["us"]
+    sw = None
+    if "swiglu_fwd" in per_kernel and "swiglu_bwd" in per_kernel:
+        sw_bytes = nbytes["swiglu_fwd"] + nbytes["swiglu_bwd"]
+        sw_us = per_kernel["swiglu_fwd"]["us"] + per_kernel["swiglu_bwd"]["us"]
+        sw_gbs = sw_bytes / (sw_us * 1e-6) / 1e9
+        sw = {"gbs": round(sw_gbs, 1), "frac": round(sw_gbs / peak, 4),
+              "rows_per_s": rows["swiglu_fwd"] / (sw_us * 1e-6),
+              "fwd_frac": per_kernel["swiglu_fwd"]["frac"],
+              "bwd_frac": per_kernel["swiglu_bwd"]["frac"]}
+    workload = WORKLOAD_NAME if not args.kernel and args.scale == 1.0 else \
+        f"{args.kernel or 'all'} at scale {args.scale:g} of: {WORKLOAD_NAME}"
     line = {
         "metric": METRIC,
         "value": round(aggregate_value(bytes_per_step, K, world, max_ms * 1e-3), 1),
@@ -393,24 +422,21 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD_NAME, "bytes_per_step": bytes_per_step,
+        "config": {"workload": workload, "bytes_per_step": bytes_per_step,
                    "l2": "no flush: every kernel streams > 126 MB (inputs larger than L2)",
                    "parallelism": f"weak: {world} independent replica(s), one per GPU",
                    "n_used": batch.rt.n_used},
-        "swiglu_fwd_bwd": {"gbs": round(sw_bytes / (sw_us * 1e-6) / 1e9, 1),
-                           "frac": round(sw_bytes / (sw_us * 1e-6) / 1e9 / peak, 4),
-                           "rows_per_s": SWIGLU["rows"] / (sw_us * 1e-6),
-                           "fwd_frac": per_kernel["swiglu_fwd"]["frac"],
-                           "bwd_frac": per_kernel["swiglu_bwd"]["frac"]},
+        "swiglu_fwd_bwd": sw,
         "roofline": {"kernel": dominant, "bound": "hbm", "achieved": d["gbs"], "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": d["frac"],
-                     "algorithmic_bytes": d["bytes"], "traffic": ncu_traffic(dominant)},
+                     "algorithmic_bytes": d["bytes"],
+                     "traffic": ncu_traffic(dominant) if args.scale == 1.0 else None},
         "kernels": per_kernel,
         "gpu_launches": K * len(kernels),
         "clocks": clocks,
         "e2e": e2e,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.kernel:
         line["cpu_baseline"] = cpu_baseline(args.cpu_sample, steps=1)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -580,6 +606,10 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--kernel", default=None,
+                    help="comma-separated kernels to run alone (profiling); default: the whole step")
+    ap.add_argument("--scale", type=float, default=1.0,
+                    help="row-count scale of the workload (profiling captures); default 1")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")

@@ -10,7 +10,7 @@
 // p = probs[permutation_map[r]].  Rows r < *n_used with a negative map entry
 // are alignment padding: zero-filled when zero_padding is set, otherwise not
 // touched.  Rows r >= *n_used are neither read nor written.  The kernel is a
-// fixed persistent grid striding over (row, 8-column chunk) pairs up to the
+// fixed persistent grid whose warps stride over rows up to the
 // device-resident bound, so a captured graph stays valid as n_used changes,
 // and every output element is computed by the same instruction sequence
 // whatever the grid (batch invariance).
@@ -20,17 +20,19 @@
 namespace moe {
 namespace {
 
-constexpr int kUnroll = 2;
-
 template <int ACT>
-__device__ __forceinline__ float act_one(float a, float b, float p, float scale) {
+__device__ __forceinline__ float act_one(float a, float b, float p, float scale,
+                                        float inv_scale) {
   if constexpr (ACT == MOE_ACT_SQRELU) {
     const float rl = a < 0.0f ? 0.0f : a;                 // relu, NaN kept
     return round_to<BF16>(rl * rl) * p;
   } else if constexpr (ACT == MOE_ACT_SQRELU_CLAMP) {
-    const float z = scale * tanhf(__fdiv_rn(a, scale));
-    const float rl = z < 0.0f ? 0.0f : z;
-    return (rl * rl) * p;
+    // relu(s tanh(x/s)) = s tanh(relu(x/s)) for s > 0: the relu goes first, so
+    // tanh only sees y >= 0 (x/s to within an fp32 ulp via the reciprocal; a
+    // NaN x stays NaN through max.NaN).
+    const float y = max_nan(a * inv_scale, 0.0f);
+    const float z = scale * tanh_nonneg(y);
+    return (z * z) * p;
   } else {
     const float s = a * sigmoid(a);
     return (s * b) * p;
@@ -48,87 +50,101 @@ __device__ __forceinline__ int64_t live_rows(const int32_t* n_used, int64_t max_
   return n;
 }
 
-template <int ACT, bool VEC>
+// One warp owns one row at a time (warps stride over rows up to the
+// device-resident bound); lanes take 8-column chunks lane, lane + 32, ...
+// The next row's map entry is fetched while the current row streams, so the
+// row's data loads never wait on the map lookup.
+template <int ACT, bool VEC, int U>
 __global__ void __launch_bounds__(kThreads)
 act_permuted_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ out,
                     const int32_t* __restrict__ pmap, const int32_t* __restrict__ n_used,
                     const float* __restrict__ probs, int64_t num_probs, int64_t max_rows,
                     int64_t width, float scale, int zero_padding, int32_t* err) {
   const int64_t rows = live_rows(n_used, max_rows, err);
+  const float inv_scale = 1.0f / scale;
   constexpr int64_t unit = VEC ? kVec : 1;
   const int64_t upr = width / unit;                      // units per row
   const int64_t in_w = ACT == MOE_ACT_SWIGLU ? 2 * width : width;
-  const int64_t total = rows * upr;
-  const int64_t S = (int64_t)gridDim.x * kThreads;
-  int64_t q = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  if (q >= total) return;
-  RowCursor cur(q, S, upr);
-  constexpr int U = VEC ? kUnroll : 1;
-  for (; q < total; q += U * S) {
-    uint4 a[U], b[U];
-    float p[U];
-    int64_t r[U], c[U];
-    int state[U];  // 0: nothing, 1: compute, 2: write zeros
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
+  int64_t r = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  int32_t m_next = __ldg(pmap + r);
+  for (; r < rows; r += nwarps) {
+    const int32_t m = m_next;
+    if (r + nwarps < rows) m_next = __ldg(pmap + r + nwarps);
+    uint16_t* orow = out + r * width;
+    if (m < 0) {                                         // alignment padding row
+      if (zero_padding) {
+        for (int64_t c = lane; c < upr; c += 32) {
+          if constexpr (VEC) st_stream(orow + c * kVec, make_uint4(0u, 0u, 0u, 0u));
+          else orow[c] = 0;
+        }
+      }
+      continue;
+    }
+    if (m >= num_probs) {
+      if (lane == 0) flag_error(err, MOE_DEVERR_MAP);
+      continue;
+    }
+    const float p = __ldg(probs + m);
+    const uint16_t* xrow = x + r * in_w;
+    for (int64_t c0 = lane; c0 < upr; c0 += 32 * U) {
+      uint4 a[U], b[U];
 #pragma unroll
-    for (int k = 0; k < U; ++k) {
-      state[k] = 0;
-      r[k] = cur.r;
-      c[k] = cur.c;
-      if (q + k * S < total) {
-        const int32_t m = __ldg(pmap + cur.r);
-        if (m < 0) {
-          state[k] = zero_padding ? 2 : 0;
-        } else if (m >= num_probs) {
-          flag_error(err, MOE_DEVERR_MAP);
-        } else {
-          state[k] = 1;
-          p[k] = __ldg(probs + m);
-          const uint16_t* src = x + cur.r * in_w + cur.c * unit;
+      for (int k = 0; k < U; ++k) {
+        const int64_t c = c0 + 32 * k;
+        if (c < upr) {
           if constexpr (VEC) {
-            a[k] = ld_stream(src);
-            if constexpr (ACT == MOE_ACT_SWIGLU) b[k] = ld_stream(src + width);
+            a[k] = ld_stream(xrow + c * kVec);
+            if constexpr (ACT == MOE_ACT_SWIGLU) b[k] = ld_stream(xrow + width + c * kVec);
           } else {
-            a[k].x = __ldg(src);
-            if constexpr (ACT == MOE_ACT_SWIGLU) b[k].x = __ldg(src + width);
+            a[k].x = __ldg(xrow + c);
+            if constexpr (ACT == MOE_ACT_SWIGLU) b[k].x = __ldg(xrow + width + c);
           }
         }
       }
-      cur.advance();
-    }
 #pragma unroll
-    for (int k = 0; k < U; ++k) {
-      uint16_t* dst = out + r[k] * width + c[k] * unit;
-      if (state[k] == 2) {
-        if constexpr (VEC) st_stream(dst, make_uint4(0u, 0u, 0u, 0u));
-        else *dst = 0;
-      } else if (state[k] == 1) {
-        if constexpr (VEC) {
-          float av[8], bv[8], o[8];
-          unpack_bf16x8(a[k], av);
-          if constexpr (ACT == MOE_ACT_SWIGLU) unpack_bf16x8(b[k], bv);
+      for (int k = 0; k < U; ++k) {
+        const int64_t c = c0 + 32 * k;
+        if (c < upr) {
+          if constexpr (VEC) {
+            float av[8], bv[8], o[8];
+            unpack_bf16x8(a[k], av);
+            if constexpr (ACT == MOE_ACT_SWIGLU) unpack_bf16x8(b[k], bv);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            o[i] = act_one<ACT>(av[i], ACT == MOE_ACT_SWIGLU ? bv[i] : 0.0f, p[k], scale);
-          store8<BF16>(dst, o);
-        } else {
-          const float av = __uint_as_float(a[k].x << 16);
-          const float bv = ACT == MOE_ACT_SWIGLU ? __uint_as_float(b[k].x << 16) : 0.0f;
-          *dst = f32_to_bf16(act_one<ACT>(av, bv, p[k], scale));
+            for (int i = 0; i < 8; ++i)
+              o[i] = act_one<ACT>(av[i], ACT == MOE_ACT_SWIGLU ? bv[i] : 0.0f, p, scale,
+                                 inv_scale);
+            store8<BF16>(orow + c * kVec, o);
+          } else {
+            const float av = __uint_as_float(a[k].x << 16);
+            const float bv = ACT == MOE_ACT_SWIGLU ? __uint_as_float(b[k].x << 16) : 0.0f;
+            orow[c] = f32_to_bf16(act_one<ACT>(av, bv, p, scale, inv_scale));
+          }
         }
       }
     }
   }
 }
 
+// Chunks per lane loaded ahead: 6 single-stream loads, or 3 chunks of the
+// two-stream SwiGLU input.
+#ifndef MOE_ACT_LOADS_AHEAD
+#define MOE_ACT_LOADS_AHEAD 6
+#endif
+
 template <int ACT, bool VEC>
 int launch_act(const uint16_t* x, uint16_t* out, const int32_t* pmap, const int32_t* n_used,
                const float* probs, int64_t num_probs, int64_t max_rows, int64_t width,
                float scale, int zero_padding, int32_t* err, cudaStream_t stream) {
-  auto k = act_permuted_kernel<ACT, VEC>;
-  const int64_t units = max_rows * (VEC ? width / kVec : width);
-  const int64_t per_block = (int64_t)kThreads * (VEC ? kUnroll : 1);
+  constexpr int U = VEC ? (ACT == MOE_ACT_SWIGLU ? MOE_ACT_LOADS_AHEAD / 2 : MOE_ACT_LOADS_AHEAD)
+                        : 1;
+  auto k = act_permuted_kernel<ACT, VEC, U>;
+  const int64_t warps_per_block = kThreads / 32;
   int grid;
-  if (int rc = persistent_grid((const void*)k, 0, (units + per_block - 1) / per_block, &grid))
+  if (int rc = persistent_grid((const void*)k, 0, (max_rows + warps_per_block - 1) / warps_per_block,
+                               &grid))
     return rc;
   k<<<grid, kThreads, 0, stream>>>(x, out, pmap, n_used, probs, num_probs, max_rows, width,
                                    scale, zero_padding, err);

@@ -182,32 +182,67 @@ template <> __device__ __forceinline__ void store8<F32>(float* p, const float (&
 
 // ------------------------------------------------------------ math
 
-// e^x = 2^(x * log2 e), with the hardware base-2 exponential (PTX
-// ex2.approx.f32; subnormal results are kept) -- then the logistic function
-// 1 / (1 + e^-z) with the hardware reciprocal (PTX rcp.approx.f32).  Both
-// approximations are within a few fp32 ulp, far below half a bf16 ulp.
-__device__ __forceinline__ float ex2_approx(float x) {
+// Flush-to-zero hardware approximations (one MUFU instruction each):
+// ex2.approx.ftz.f32 = 2^x, rcp.approx.ftz.f32 = 1/x, tanh.approx.f32.
+__device__ __forceinline__ float ex2_ftz(float x) {
   float y;
-  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-__device__ __forceinline__ float rcp_approx(float x) {
+__device__ __forceinline__ float rcp_ftz(float x) {
   float y;
-  asm("rcp.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e): e^x = 2^(x log2 e)
+constexpr float kTwoM32 = 0x1p-32f;
 
+// The logistic function sigma(z) = 1 / (1 + e^-z), evaluated as
+//   e  = 2^(-z log2 e)                  (subnormal e, z > 87.3, flushes to 0:
+//                                        1 + e rounds to 1 either way)
+//   q  = 1 / ((1 + e) * 2^-32)          (scaled so the reciprocal stays a normal
+//                                        number for every z > -109, where the
+//                                        unscaled one would be subnormal and flush)
+//   sigma = q * 2^-32                   (a plain multiply: subnormal sigma kept)
+// (1 + e) * 2^-32 is one fused multiply-add, e * 2^-32 + 2^-32, exact up to the
+// same single rounding as 1 + e.  For z < -88.7, e = +inf and sigma = 0, as in
+// an fp32 evaluation of the definition.  Error: a few fp32 ulp, far below half
+// a bf16 ulp.
 __device__ __forceinline__ float sigmoid(float z) {
-  return rcp_approx(1.0f + ex2_approx(z * -kLog2e));
+  const float e = ex2_ftz(z * -kLog2e);
+  return rcp_ftz(fmaf(e, kTwoM32, kTwoM32)) * kTwoM32;
 }
 
-// torch.clamp semantics: a NaN input stays NaN (every comparison is false).
-__device__ __forceinline__ float clamp_max(float v, float hi) { return v > hi ? hi : v; }
+// torch.clamp semantics: a NaN input stays NaN.  PTX min/max with .NaN
+// return NaN when an operand is NaN (the limits never are).
+__device__ __forceinline__ float min_nan(float a, float b) {
+  float r;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float clamp_max(float v, float hi) { return min_nan(v, hi); }
 __device__ __forceinline__ float clamp_sym(float v, float lim) {
-  return v < -lim ? -lim : (v > lim ? lim : v);
+  return max_nan(min_nan(v, lim), -lim);
+}
+
+// tanh(y) for y >= 0 (or NaN), for the soft clamp.  Two published forms:
+//   y <  1/32: the Taylor series y (1 - y^2/3 + 2 y^4/15), truncation error
+//              below 17 y^6 / 315 < 6e-11 relative;
+//   y >= 1/32: tanh y = 1 - 2 / (1 + e^{2y}); the cancellation in 1 - ... costs
+//              at most ~1e-5 relative there (far below half a bf16 ulp).
+// For y > 44, e^{2y} = inf and the result is exactly 1.  NaN stays NaN.
+__device__ __forceinline__ float tanh_nonneg(float y) {
+  const float y2 = y * y;
+  const float poly = y * fmaf(y2, fmaf(y2, 2.0f / 15.0f, -1.0f / 3.0f), 1.0f);
+  const float big = 1.0f - 2.0f * rcp_ftz(1.0f + ex2_ftz(y * (2.0f * kLog2e)));
+  return y < 0.03125f ? poly : big;
 }
 
 // Fixed xor-butterfly sum over the 32 lanes of a warp: the same tree every

@@ -9,10 +9,12 @@
 //
 // Forward: a flat, persistent, grid-stride stream over 8-column chunks: per
 // chunk two 16-byte loads (gate, up) and one 16-byte store.  Backward: a
-// persistent loop over groups of rows; W threads own one row, walk its
-// chunks with a fixed column assignment, write d_gate / d_up straight into
-// the two halves of grad_x and reduce the row's probability gradient with a
-// fixed tree (per-thread partials, warp butterfly, warps in index order).
+// persistent loop over groups of rows; W threads own one row (one warp for the
+// vectorised path), walk its chunks with a fixed column assignment, write
+// d_gate / d_up straight into the two halves of grad_x and reduce the row's
+// probability gradient with a fixed tree (per-thread partials in column order,
+// warp butterfly, warps in index order).  No barrier is needed when W = 32, so
+// every warp streams independently with its next loads already in flight.
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -242,8 +244,23 @@ int launch_persistent(K kernel, int64_t useful_blocks, cudaStream_t stream, cons
 
 }  // namespace
 
-constexpr int kFwdUnroll = 2;
-constexpr int kBwdUnroll = 2;
+// Tuning knobs (compile-time).  kFwdUnroll: chunks whose loads a thread issues
+// before it computes any of them.  kBwdRowThreads: threads that own one row in
+// the backward (0: the smallest of 32/64/128/256 covering the row's chunks);
+// it fixes the grad_probs summation tree together with the row length.
+// kBwdUnroll: chunks per thread loaded ahead in the backward.
+#ifndef MOE_SWIGLU_FWD_UNROLL
+#define MOE_SWIGLU_FWD_UNROLL 2
+#endif
+#ifndef MOE_SWIGLU_BWD_ROW_THREADS
+#define MOE_SWIGLU_BWD_ROW_THREADS 32
+#endif
+#ifndef MOE_SWIGLU_BWD_UNROLL
+#define MOE_SWIGLU_BWD_UNROLL 2
+#endif
+constexpr int kFwdUnroll = MOE_SWIGLU_FWD_UNROLL;
+constexpr int kBwdRowThreads = MOE_SWIGLU_BWD_ROW_THREADS;
+constexpr int kBwdUnroll = MOE_SWIGLU_BWD_UNROLL;
 
 int launch_swiglu_clamped_fwd(const uint16_t* x, const float* probs, uint16_t* y, int64_t rows,
                               int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
@@ -276,7 +293,8 @@ int launch_swiglu_clamped_bwd(const uint16_t* x, const float* probs, const uint1
                               cudaStream_t stream) {
   const bool vec = inter % kVec == 0 && ld_x % kVec == 0 && ld_gy % kVec == 0 &&
                    ld_gx % kVec == 0 && aligned16(x) && aligned16(grad_y) && aligned16(grad_x);
-  const int W = threads_per_row(vec ? inter / kVec : inter);
+  const int W = (vec && kBwdRowThreads) ? kBwdRowThreads
+                                        : threads_per_row(vec ? inter / kVec : inter);
   const int64_t blocks = (rows + kThreads / W - 1) / (kThreads / W);
 #define MOE_BWD_ARGS stream, x, probs, grad_y, grad_x, grad_probs, rows, inter, ld_x, ld_gy, ld_gx, limit
   if (vec) {

@@ -48,35 +48,40 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def load(path: str) -> ctypes.CDLL:
+    """Load an oracle build at `path` and declare its C signatures."""
+    lib = ctypes.CDLL(path)
+    P, I64, I32, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
+    sig = {
+        "orc_bf16_from_f32": (ctypes.c_uint16, [F]),
+        "orc_f32_from_bf16": (F, [ctypes.c_uint16]),
+        "orc_f16_from_f32": (ctypes.c_uint16, [F]),
+        "orc_f32_from_f16": (F, [ctypes.c_uint16]),
+        "orc_swiglu_clamped_fwd": (None, [P, P, P, I64, I64, I64, I64, F]),
+        "orc_swiglu_clamped_bwd": (None, [P, P, P, P, P, P, I64, I64, I64, I64, I64, F]),
+        "orc_swiglu_clamped_fwd_f64": (None, [P, P, P, P, I64, ctypes.c_double]),
+        "orc_router_weight_fwd": (None, [P, ctypes.c_int, P, P, ctypes.c_int, I64, I64]),
+        "orc_router_weight_bwd": (None, [P, ctypes.c_int, P, ctypes.c_int, P, P, P, P,
+                                         I64, I64]),
+        "orc_act_with_probs_permuted": (ctypes.c_int, [ctypes.c_int, P, P, P, I32, P, I64,
+                                                       I64, I64, F, ctypes.c_int]),
+        "orc_unpermute_ordered": (ctypes.c_int, [P, ctypes.c_int, I64, P, I32, P,
+                                                 ctypes.c_int, I64, I64, I32]),
+        "orc_residual_add": (None, [P, P, P, P, I64, ctypes.c_int]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
 def _lib():
     global _LIB
     with _LOCK:
         if _LIB is None:
             build()
-            lib = ctypes.CDLL(_LIB_PATH)
-            P, I64, I32, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
-            sig = {
-                "orc_bf16_from_f32": (ctypes.c_uint16, [F]),
-                "orc_f32_from_bf16": (F, [ctypes.c_uint16]),
-                "orc_f16_from_f32": (ctypes.c_uint16, [F]),
-                "orc_f32_from_f16": (F, [ctypes.c_uint16]),
-                "orc_swiglu_clamped_fwd": (None, [P, P, P, I64, I64, I64, I64, F]),
-                "orc_swiglu_clamped_bwd": (None, [P, P, P, P, P, P, I64, I64, I64, I64, I64, F]),
-                "orc_swiglu_clamped_fwd_f64": (None, [P, P, P, P, I64, ctypes.c_double]),
-                "orc_router_weight_fwd": (None, [P, ctypes.c_int, P, P, ctypes.c_int, I64, I64]),
-                "orc_router_weight_bwd": (None, [P, ctypes.c_int, P, ctypes.c_int, P, P, P, P,
-                                                 I64, I64]),
-                "orc_act_with_probs_permuted": (ctypes.c_int, [ctypes.c_int, P, P, P, I32, P, I64,
-                                                               I64, I64, F, ctypes.c_int]),
-                "orc_unpermute_ordered": (ctypes.c_int, [P, ctypes.c_int, I64, P, I32, P,
-                                                         ctypes.c_int, I64, I64, I32]),
-                "orc_residual_add": (None, [P, P, P, P, I64, ctypes.c_int]),
-            }
-            for name, (res, args) in sig.items():
-                fn = getattr(lib, name)
-                fn.restype = res
-                fn.argtypes = args
-            _LIB = lib
+            _LIB = load(_LIB_PATH)
     return _LIB
 
 

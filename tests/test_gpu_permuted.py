@@ -174,3 +174,33 @@ def test_unpermute_batch_invariant(cuda_device):
                          rt.inverse_map[sub].contiguous(), rt.probs, rt.counts)
     part = _run_unpermute(cuda_device, rt2, eo, torch.bfloat16, 37)
     assert_bits_equal(part, full[sub.numpy()], "batch invariance")
+
+
+@pytest.mark.parametrize("act,oact,tol", ACTS)
+@pytest.mark.parametrize("scale", [1.0, 7.0, 30.0])
+def test_act_permuted_special_values(cuda_device, act, oact, tol, scale):
+    """NaN, +-inf, +-0, tiny and huge inputs, and values on both sides of the
+    switch between the two tanh forms (y = x/s around 1/32)."""
+    vals = [float("nan"), float("inf"), -float("inf"), 0.0, -0.0, 1e-30, -1e-30, 1e-39, 3e38,
+            -3e38, 1e30, scale / 32, scale / 32 * 1.01, scale / 32 * 0.99, -scale / 32, 0.5, -0.5,
+            2.0, 9.0, 44.0 * scale, 100.0 * scale, -88.5, -87.0, 20.0]
+    width = 8 * ((len(vals) + 7) // 8)
+    row = torch.tensor(vals + [1.0] * (width - len(vals)), dtype=torch.bfloat16)
+    rows = 4
+    cols = 2 * width if oact == oracle.SWIGLU else width
+    x = torch.zeros(rows, cols, dtype=torch.bfloat16)
+    for r in range(rows):
+        x[r, :width] = row.roll(r)
+        if cols > width:
+            x[r, width:] = row.roll(-r)
+    rt = inputs.Routing(rows, 1, 1, 1, rows, rows, torch.arange(rows, dtype=torch.int32),
+                        torch.arange(rows, dtype=torch.int32).reshape(rows, 1),
+                        torch.tensor([0.25, 1.0, 0.7, 3.0]), torch.tensor([rows]))
+    got = _run_act(cuda_device, act, rt, x, width, scale, True)
+    ref, _ = oracle.act_with_probs_permuted(oact, bits(x), np.zeros((rows, width), np.uint16),
+                                            bits(rt.permutation_map), rows, bits(rt.probs), width,
+                                            scale, True)
+    if tol == 0:
+        assert_bits_equal(got, ref, "act specials")
+    else:
+        assert_within_ulp16(got, ref, tol, what="act specials")
