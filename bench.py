@@ -106,88 +106,115 @@ KERNEL_SOURCES = {
 }
 
 
-class Batch:
-    """All inputs and outputs of one step, on one device."""
+GROUPS = {  # kernel -> the input group it needs
+    "swiglu_fwd": "swiglu", "swiglu_bwd": "swiglu",
+    "router_weight_fwd": "router", "router_weight_bwd": "router",
+    "act_sqrelu": "act", "act_sqrelu_clamp": "act", "act_swiglu": "act",
+    "unpermute": "unpermute", "residual_add": "residual",
+}
+ORDER = ["swiglu_fwd", "router_weight_fwd", "act_sqrelu", "act_sqrelu_clamp", "act_swiglu",
+         "unpermute", "residual_add", "router_weight_bwd", "swiglu_bwd"]
 
-    def __init__(self, device, seed, scale=1.0):
+
+class Batch:
+    """All inputs and outputs of one step (or of the selected kernels), on one device."""
+
+    def __init__(self, device, seed, scale=1.0, kernels=None):
         from moe_expert_epilogue_b200 import inputs
         self.scale = scale
+        self.names = [k for k in ORDER if kernels is None or k in kernels]
+        groups = {GROUPS[k] for k in self.names}
         w = scaled(scale)
         gen_dev = device if device.type == "cuda" else "cpu"
-        sw = inputs.swiglu_inputs(w["swiglu"]["rows"], SWIGLU["inter"], sigma=SWIGLU["sigma"],
-                                  probs="topk_softmax", seed=seed, device=gen_dev)
-        self.sw_x, self.sw_p, self.sw_gy = sw["x"], sw["probs"], sw["grad_y"]
-        rw = inputs.router_weight_inputs(w["router"]["rows"], ROUTER["hidden"], seed=seed + 1,
-                                         device=gen_dev)
-        self.rw_x, self.rw_p, self.rw_g = rw["x"], rw["probs"], rw["grad_out"]
+        z = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device=device)  # noqa: E731
+        self.inputs, self.outputs = [], []
+        W = PERMUTED["width"]
+        # routing metadata is always drawn: its n_used enters the byte count
         rt = inputs.routing(w["permuted"]["tokens"], PERMUTED["top_k"], PERMUTED["experts"],
                             PERMUTED["align"], seed=seed + 2, device=gen_dev)
         self.rt = rt
-        W = PERMUTED["width"]
-        self.act_x = inputs.permuted_activation_input(rt, W, swiglu=False, seed=seed + 3,
-                                                      device=gen_dev)
-        self.act_x2 = inputs.permuted_activation_input(rt, W, swiglu=True, seed=seed + 4,
-                                                       device=gen_dev)
-        self.pmap, self.probs = rt.permutation_map, rt.probs
-        self.n_used = torch.tensor([rt.n_used], dtype=torch.int32, device=gen_dev)
-        self.eo = inputs.expert_output_input(rt, PERMUTED["hidden"], seed=seed + 5, device=gen_dev)
-        self.inv = rt.inverse_map
-        self.valid = torch.tensor([rt.tokens], dtype=torch.int32, device=gen_dev)
-        res = inputs.residual_inputs((w["residual"]["rows"], RESIDUAL["hidden"]), torch.bfloat16,
-                                     seed=seed + 6, device=gen_dev)
-        self.res_e, self.res_s, self.res_r = (res["expert_output"], res["shared_expert_output"],
-                                              res["residual"])
-        self.to(device)
-        # outputs
-        z = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device=device)  # noqa: E731
-        R, I = w["swiglu"]["rows"], SWIGLU["inter"]
-        Rr = w["router"]["rows"]
-        self.sw_y, self.sw_gx, self.sw_gp = z(R, I), z(R, 2 * I), z(R, 1, dt=torch.float32)
-        self.rw_gx, self.rw_gp = z(Rr, ROUTER["hidden"]), z(Rr, 1, dt=torch.float32)
-        self.act_o1, self.act_o2, self.act_o3 = (z(rt.max_rows, W) for _ in range(3))
-        self.unp_out = z(w["permuted"]["tokens"], PERMUTED["hidden"])
-        self.res_out = z(w["residual"]["rows"], RESIDUAL["hidden"])
+        if "swiglu" in groups:
+            sw = inputs.swiglu_inputs(w["swiglu"]["rows"], SWIGLU["inter"], sigma=SWIGLU["sigma"],
+                                      probs="topk_softmax", seed=seed, device=gen_dev)
+            self.sw_x, self.sw_p, self.sw_gy = sw["x"], sw["probs"], sw["grad_y"]
+            R, I = w["swiglu"]["rows"], SWIGLU["inter"]
+            self.sw_y, self.sw_gx, self.sw_gp = z(R, I), z(R, 2 * I), z(R, 1, dt=torch.float32)
+            self.inputs += ["sw_x", "sw_p", "sw_gy"]
+            self.outputs += ["sw_y", "sw_gx", "sw_gp"]
+        if "router" in groups:
+            rw = inputs.router_weight_inputs(w["router"]["rows"], ROUTER["hidden"], seed=seed + 1,
+                                             device=gen_dev)
+            self.rw_x, self.rw_p, self.rw_g = rw["x"], rw["probs"], rw["grad_out"]
+            Rr = w["router"]["rows"]
+            self.rw_gx, self.rw_gp = z(Rr, ROUTER["hidden"]), z(Rr, 1, dt=torch.float32)
+            self.inputs += ["rw_x", "rw_p", "rw_g"]
+            self.outputs += ["rw_gx", "rw_gp"]
+        if "act" in groups:
+            self.act_x = inputs.permuted_activation_input(rt, W, swiglu=False, seed=seed + 3,
+                                                          device=gen_dev)
+            self.act_x2 = inputs.permuted_activation_input(rt, W, swiglu=True, seed=seed + 4,
+                                                           device=gen_dev)
+            self.act_o1, self.act_o2, self.act_o3 = (z(rt.max_rows, W) for _ in range(3))
+            self.inputs += ["act_x", "act_x2"]
+            self.outputs += ["act_o1", "act_o2", "act_o3"]
+        if "act" in groups or "unpermute" in groups:
+            self.pmap, self.probs = rt.permutation_map, rt.probs
+            self.n_used = torch.tensor([rt.n_used], dtype=torch.int32, device=gen_dev)
+            self.inv = rt.inverse_map
+            self.valid = torch.tensor([rt.tokens], dtype=torch.int32, device=gen_dev)
+            self.inputs += ["pmap", "probs", "n_used", "inv", "valid"]
+        if "unpermute" in groups:
+            self.eo = inputs.expert_output_input(rt, PERMUTED["hidden"], seed=seed + 5,
+                                                 device=gen_dev)
+            self.unp_out = z(w["permuted"]["tokens"], PERMUTED["hidden"])
+            self.inputs += ["eo"]
+            self.outputs += ["unp_out"]
+        if "residual" in groups:
+            res = inputs.residual_inputs((w["residual"]["rows"], RESIDUAL["hidden"]),
+                                         torch.bfloat16, seed=seed + 6, device=gen_dev)
+            self.res_e, self.res_s, self.res_r = (res["expert_output"],
+                                                  res["shared_expert_output"], res["residual"])
+            self.res_out = z(w["residual"]["rows"], RESIDUAL["hidden"])
+            self.inputs += ["res_e", "res_s", "res_r"]
+            self.outputs += ["res_out"]
+        if "router_weight_fwd" in self.names:
+            # chained epilogue: the router-weight forward writes the first rows of the
+            # residual's expert output (a tensor of its own when run alone)
+            n = self.rw_x.shape[0]
+            self.rw_out = self.res_e[:n] if "residual" in groups else z(n, ROUTER["hidden"])
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
-
-    INPUT_NAMES = ("sw_x", "sw_p", "sw_gy", "rw_x", "rw_p", "rw_g", "act_x", "act_x2", "pmap",
-                   "probs", "n_used", "eo", "inv", "valid", "res_e", "res_s", "res_r")
-    OUTPUT_NAMES = ("sw_y", "sw_gx", "sw_gp", "rw_gx", "rw_gp", "act_o1", "act_o2", "act_o3",
-                    "unp_out", "res_out")
-
-    def to(self, device):
-        for k in self.INPUT_NAMES:
+        for k in self.inputs:
             setattr(self, k, getattr(self, k).to(device))
 
     def kernels(self):
-        """(name, launch) pairs of one step, in MoE-layer order."""
+        """(name, launch) pairs, in MoE-layer order."""
         from moe_expert_epilogue_b200 import ops
         L = SWIGLU["limit"]
         P = PERMUTED
-        # the router-weight forward writes the first rows of the residual's expert output
-        rw_out = self.res_e[:self.rw_x.shape[0]]
-        return [
-            ("swiglu_fwd", lambda: ops.swiglu_clamped_fwd(self.sw_x, self.sw_p, L, out=self.sw_y)),
-            ("router_weight_fwd", lambda: ops.router_weight_mul_fwd(
-                self.rw_x, self.rw_p, torch.bfloat16, out=rw_out)),
-            ("act_sqrelu", lambda: ops.act_with_probs_permuted(
+        table = {
+            "swiglu_fwd": lambda: ops.swiglu_clamped_fwd(self.sw_x, self.sw_p, L, out=self.sw_y),
+            "router_weight_fwd": lambda: ops.router_weight_mul_fwd(
+                self.rw_x, self.rw_p, torch.bfloat16, out=self.rw_out),
+            "act_sqrelu": lambda: ops.act_with_probs_permuted(
                 ops.MOE_ACT_SQRELU, self.act_x, self.pmap, self.n_used, self.probs, 1.0, True,
-                out=self.act_o1, dev_err=self.dev_err)),
-            ("act_sqrelu_clamp", lambda: ops.act_with_probs_permuted(
+                out=self.act_o1, dev_err=self.dev_err),
+            "act_sqrelu_clamp": lambda: ops.act_with_probs_permuted(
                 ops.MOE_ACT_SQRELU_CLAMP, self.act_x, self.pmap, self.n_used, self.probs,
-                P["scale"], True, out=self.act_o2, dev_err=self.dev_err)),
-            ("act_swiglu", lambda: ops.act_with_probs_permuted(
+                P["scale"], True, out=self.act_o2, dev_err=self.dev_err),
+            "act_swiglu": lambda: ops.act_with_probs_permuted(
                 ops.MOE_ACT_SWIGLU, self.act_x2, self.pmap, self.n_used, self.probs, 1.0, True,
-                out=self.act_o3, dev_err=self.dev_err)),
-            ("unpermute", lambda: ops.unpermute_ordered(self.eo, self.inv, self.valid,
-                                                        self.unp_out, dev_err=self.dev_err)),
-            ("residual_add", lambda: ops.residual_add(self.res_e, self.res_s, self.res_r,
-                                                      out=self.res_out)),
-            ("router_weight_bwd", lambda: ops.router_weight_mul_bwd(
-                self.rw_g, self.rw_x, self.rw_p, grad_x=self.rw_gx, grad_probs=self.rw_gp)),
-            ("swiglu_bwd", lambda: ops.swiglu_clamped_bwd(self.sw_x, self.sw_p, self.sw_gy, L,
-                                                          grad_x=self.sw_gx,
-                                                          grad_probs=self.sw_gp)),
-        ]
+                out=self.act_o3, dev_err=self.dev_err),
+            "unpermute": lambda: ops.unpermute_ordered(self.eo, self.inv, self.valid,
+                                                       self.unp_out, dev_err=self.dev_err),
+            "residual_add": lambda: ops.residual_add(self.res_e, self.res_s, self.res_r,
+                                                     out=self.res_out),
+            "router_weight_bwd": lambda: ops.router_weight_mul_bwd(
+                self.rw_g, self.rw_x, self.rw_p, grad_x=self.rw_gx, grad_probs=self.rw_gp),
+            "swiglu_bwd": lambda: ops.swiglu_clamped_bwd(self.sw_x, self.sw_p, self.sw_gy, L,
+                                                         grad_x=self.sw_gx,
+                                                         grad_probs=self.sw_gp),
+        }
+        return [(n, table[n]) for n in self.names]
 
 
 # ---------------------------------------------------------------- distributed
@@ -338,12 +365,11 @@ def run_ours(args):
             mbuild.build()
         barrier(device)
 
-    batch = Batch(device, seed=1000 * rank, scale=args.scale)
+    only = set(args.kernel.split(",")) if args.kernel else None
+    if only and not only <= set(ORDER):
+        raise SystemExit(f"unknown --kernel {args.kernel}; choose from {ORDER}")
+    batch = Batch(device, seed=1000 * rank, scale=args.scale, kernels=only)
     kernels = batch.kernels()
-    if args.kernel:
-        kernels = [(n, f) for n, f in kernels if n in args.kernel.split(",")]
-        if not kernels:
-            raise SystemExit(f"unknown --kernel {args.kernel}")
     nbytes = algorithmic_bytes(batch.rt.n_used, args.scale)
     nbytes = {n: nbytes[n] for n, _ in kernels}
     rows = rows_per_launch(args.scale)
@@ -450,11 +476,11 @@ def run_e2e(batch, kernels, nbytes, args, device):
     host->device copies of every input, the kernels, and device->host copies
     of every output, all inside the timed region."""
     host_in = {k: torch.empty_like(getattr(batch, k), device="cpu").pin_memory()
-               for k in batch.INPUT_NAMES}
+               for k in batch.inputs}
     for k, h in host_in.items():
         h.copy_(getattr(batch, k))
     host_out = {k: torch.empty_like(getattr(batch, k), device="cpu").pin_memory()
-                for k in batch.OUTPUT_NAMES}
+                for k in batch.outputs}
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
     stream = torch.cuda.current_stream(device)

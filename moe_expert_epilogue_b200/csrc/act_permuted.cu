@@ -31,7 +31,7 @@ __device__ __forceinline__ float act_one(float a, float b, float p, float scale,
     // tanh only sees y >= 0 (x/s to within an fp32 ulp via the reciprocal; a
     // NaN x stays NaN through max.NaN).
     const float y = max_nan(a * inv_scale, 0.0f);
-    const float z = scale * tanh_nonneg(y);
+    const float z = scale * tanh_approx(y);
     return (z * z) * p;
   } else {
     const float s = a * sigmoid(a);
@@ -112,10 +112,23 @@ act_permuted_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ out,
             float av[8], bv[8], o[8];
             unpack_bf16x8(a[k], av);
             if constexpr (ACT == MOE_ACT_SWIGLU) unpack_bf16x8(b[k], bv);
+            if constexpr (ACT == MOE_ACT_SQRELU) {
+              // the squares are rounded to bf16 two at a time (packed conversion),
+              // then widened back for the fp32 probability multiply
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              o[i] = act_one<ACT>(av[i], ACT == MOE_ACT_SWIGLU ? bv[i] : 0.0f, p, scale,
-                                 inv_scale);
+              for (int i = 0; i < 8; i += 2) {
+                const float r0 = av[i] < 0.0f ? 0.0f : av[i];
+                const float r1 = av[i + 1] < 0.0f ? 0.0f : av[i + 1];
+                const uint32_t sq = pack_bf16x2(r0 * r0, r1 * r1);
+                o[i] = bf16_lo(sq) * p;
+                o[i + 1] = bf16_hi(sq) * p;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                o[i] = act_one<ACT>(av[i], ACT == MOE_ACT_SWIGLU ? bv[i] : 0.0f, p, scale,
+                                   inv_scale);
+            }
             store8<BF16>(orow + c * kVec, o);
           } else {
             const float av = __uint_as_float(a[k].x << 16);

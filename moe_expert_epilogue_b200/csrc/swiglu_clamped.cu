@@ -92,6 +92,49 @@ swiglu_fwd_vec(const uint16_t* __restrict__ x, const float* __restrict__ probs,
   }
 }
 
+// Warp-per-row forward for rows of at least 64 chunks: a warp owns one row at
+// a time, loads the row's probability once and streams its chunks lane,
+// lane + 32, ... with U chunks' loads in flight per lane.
+template <int U>
+__global__ void __launch_bounds__(kThreads)
+swiglu_fwd_rows(const uint16_t* __restrict__ x, const float* __restrict__ probs,
+                uint16_t* __restrict__ y, int64_t rows, int64_t inter, int64_t ld_x,
+                int64_t ld_y, float L) {
+  const int64_t cpr = inter / kVec;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
+  const FwdMath f{L};
+  for (int64_t r = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); r < rows;
+       r += nwarps) {
+    const float p = __ldg(probs + r);
+    const uint16_t* xr = x + r * ld_x;
+    uint16_t* yr = y + r * ld_y;
+    for (int64_t c0 = lane; c0 < cpr; c0 += 32 * U) {
+      uint4 gw[U], uw[U];
+#pragma unroll
+      for (int k = 0; k < U; ++k) {
+        const int64_t c = c0 + 32 * k;
+        if (c < cpr) {
+          gw[k] = ld_stream(xr + c * kVec);
+          uw[k] = ld_stream(xr + inter + c * kVec);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < U; ++k) {
+        const int64_t c = c0 + 32 * k;
+        if (c < cpr) {
+          float g[8], u[8], o[8];
+          unpack_bf16x8(gw[k], g);
+          unpack_bf16x8(uw[k], u);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o[i] = f(g[i], u[i], p);
+          store8<BF16>(yr + c * kVec, o);
+        }
+      }
+    }
+  }
+}
+
 // Element-granular forward: any inter, leading dimensions and alignment.
 __global__ void __launch_bounds__(kThreads)
 swiglu_fwd_scalar(const uint16_t* __restrict__ x, const float* __restrict__ probs,
@@ -132,8 +175,12 @@ __device__ __forceinline__ float row_reduce(float acc, float (*red)[kThreads / 3
   }
 }
 
+#ifndef MOE_SWIGLU_BWD_MIN_BLOCKS
+#define MOE_SWIGLU_BWD_MIN_BLOCKS 1
+#endif
+
 template <int W, int U>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, MOE_SWIGLU_BWD_MIN_BLOCKS)
 swiglu_bwd_vec(const uint16_t* __restrict__ x, const float* __restrict__ probs,
                const uint16_t* __restrict__ gy, uint16_t* __restrict__ gx,
                float* __restrict__ gp, int64_t rows, int64_t inter, int64_t ld_x,
@@ -252,13 +299,21 @@ int launch_persistent(K kernel, int64_t useful_blocks, cudaStream_t stream, cons
 #ifndef MOE_SWIGLU_FWD_UNROLL
 #define MOE_SWIGLU_FWD_UNROLL 2
 #endif
+#ifndef MOE_SWIGLU_FWD_ROW_UNROLL
+#define MOE_SWIGLU_FWD_ROW_UNROLL 8
+#endif
+#ifndef MOE_SWIGLU_FWD_ROWS
+#define MOE_SWIGLU_FWD_ROWS 1
+#endif
 #ifndef MOE_SWIGLU_BWD_ROW_THREADS
 #define MOE_SWIGLU_BWD_ROW_THREADS 32
 #endif
 #ifndef MOE_SWIGLU_BWD_UNROLL
-#define MOE_SWIGLU_BWD_UNROLL 2
+#define MOE_SWIGLU_BWD_UNROLL 4
 #endif
 constexpr int kFwdUnroll = MOE_SWIGLU_FWD_UNROLL;
+constexpr int kFwdRowUnroll = MOE_SWIGLU_FWD_ROW_UNROLL;
+constexpr bool kFwdRows = MOE_SWIGLU_FWD_ROWS != 0;
 constexpr int kBwdRowThreads = MOE_SWIGLU_BWD_ROW_THREADS;
 constexpr int kBwdUnroll = MOE_SWIGLU_BWD_UNROLL;
 
@@ -268,7 +323,13 @@ int launch_swiglu_clamped_fwd(const uint16_t* x, const float* probs, uint16_t* y
   const bool vec = inter % kVec == 0 && ld_x % kVec == 0 && ld_y % kVec == 0 && aligned16(x) &&
                    aligned16(y);
   int grid;
-  if (vec) {
+  if (vec && kFwdRows && inter / kVec >= 64) {
+    auto k = swiglu_fwd_rows<kFwdRowUnroll>;
+    if (int rc = persistent_grid((const void*)k, 0, (rows + kThreads / 32 - 1) / (kThreads / 32),
+                                 &grid))
+      return rc;
+    k<<<grid, kThreads, 0, stream>>>(x, probs, y, rows, inter, ld_x, ld_y, limit);
+  } else if (vec) {
     const int64_t units = rows * (inter / kVec);
     auto k = swiglu_fwd_vec<kFwdUnroll>;
     if (int rc = persistent_grid((const void*)k, 0,

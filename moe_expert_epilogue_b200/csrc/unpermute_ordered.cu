@@ -9,26 +9,68 @@
 // a token depend only on that token's rows, never on the grid or the batch.
 //
 // One CTA owns one token at a time (persistent loop up to the
-// device-resident valid_tokens).  Warp 0 compacts the token's inverse-map row
+// device-resident valid_tokens).  Warp 0 compacts a token's inverse-map row
 // into an ordered list of live rows in shared memory (ballot + popc keeps
-// the increasing-expert order); then every thread takes 8-column chunks of
-// the hidden dimension and issues the loads of up to 8 contributing rows
-// before it adds them in list order.
+// the increasing-expert order), one token ahead; every thread takes 8-column
+// chunks of the hidden dimension and issues the loads of up to 8 contributing
+// rows before it adds them in list order.
 #include "common.cuh"
 #include "launch.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kBatch = 8;  // contributing rows loaded before they are summed
+// contributing rows loaded before they are summed: 128 bytes per thread in flight
+template <class DI> constexpr int kBatch = DI::kBytes == 4 ? 4 : 8;
 
-template <class DI, class DO, bool VEC>
+// Compacts inverse_map row t (entries e = 0 .. E-1) into list[], keeping the
+// increasing-expert order: each 32-entry slice is one ballot, and a live
+// entry's position is the number of live entries before it.  Entries at or
+// past max_rows are reported and dropped.  Warp-wide; returns the count.
+__device__ __forceinline__ int compact_row(const int32_t* inv_row, int E, int64_t max_rows,
+                                           int32_t* list, int32_t* err, int lane) {
+  int count = 0;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    int32_t row = e < E ? __ldg(inv_row + e) : -1;
+    if (row >= max_rows) {
+      flag_error(err, MOE_DEVERR_INVERSE);
+      row = -1;
+    }
+    const unsigned live = __ballot_sync(0xffffffffu, row >= 0);
+    if (row >= 0) list[count + __popc(live & ((1u << lane) - 1u))] = row;
+    count += __popc(live);
+  }
+  return count;
+}
+
+// Same, for E <= 64, from two entries per lane already loaded into registers.
+__device__ __forceinline__ int compact_pair(int32_t r0, int32_t r1, int64_t max_rows,
+                                            int32_t* list, int32_t* err, int lane) {
+  if (r0 >= max_rows) { flag_error(err, MOE_DEVERR_INVERSE); r0 = -1; }
+  if (r1 >= max_rows) { flag_error(err, MOE_DEVERR_INVERSE); r1 = -1; }
+  const unsigned m0 = __ballot_sync(0xffffffffu, r0 >= 0);
+  const unsigned m1 = __ballot_sync(0xffffffffu, r1 >= 0);
+  const unsigned below = (1u << lane) - 1u;
+  if (r0 >= 0) list[__popc(m0 & below)] = r0;
+  if (r1 >= 0) list[__popc(m0) + __popc(m1 & below)] = r1;
+  return __popc(m0) + __popc(m1);
+}
+
+// The CTA walks tokens t = blockIdx.x, + gridDim.x, ...  Row lists are
+// double-buffered and built one token ahead by warp 0: at the top of an
+// iteration warp 0 issues the loads of the NEXT token's inverse-map row (for
+// E <= 64: two entries per lane, into registers), gathers its own share of the
+// current token, and only then compacts the next list, so the map latency hides
+// behind the gathers.  One barrier per token: it publishes the list built in
+// the previous iteration and retires the buffer about to be rebuilt.
+template <class DI, class DO, bool VEC, bool SMALL_E>
 __global__ void __launch_bounds__(kThreads)
 unpermute_kernel(const typename DI::T* __restrict__ eo, int64_t max_rows,
                  const int32_t* __restrict__ inv, const int32_t* __restrict__ valid_tokens,
                  typename DO::T* __restrict__ out, int64_t tokens, int64_t hidden, int E,
                  int32_t* err) {
-  extern __shared__ int32_t s_list[];  // [2][E]: double-buffered row lists
+  extern __shared__ int32_t s_list[];  // [2][E]
   __shared__ int s_count[2];
   int64_t n = __ldg(valid_tokens);
   if (n < 0 || n > tokens) {
@@ -36,39 +78,37 @@ unpermute_kernel(const typename DI::T* __restrict__ eo, int64_t max_rows,
     n = n < 0 ? 0 : tokens;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int parity = 0;
-  for (int64_t t = blockIdx.x; t < n; t += gridDim.x, parity ^= 1) {
-    int32_t* list = s_list + parity * E;
-    if (warp == 0) {
-      int count = 0;
-      for (int e0 = 0; e0 < E; e0 += 32) {
-        const int e = e0 + lane;
-        int32_t row = e < E ? __ldg(inv + t * E + e) : -1;
-        if (row >= max_rows) {
-          flag_error(err, MOE_DEVERR_INVERSE);
-          row = -1;
-        }
-        const unsigned live = __ballot_sync(0xffffffffu, row >= 0);
-        if (row >= 0) list[count + __popc(live & ((1u << lane) - 1u))] = row;
-        count += __popc(live);
-      }
-      if (lane == 0) s_count[parity] = count;
-    }
+  int64_t t = blockIdx.x;
+  if (t >= n) return;                                   // CTA-uniform
+  if (warp == 0) {
+    const int c = compact_row(inv + t * E, E, max_rows, s_list, err, lane);
+    if (lane == 0) s_count[0] = c;
+  }
+  for (int parity = 0; t < n; t += gridDim.x, parity ^= 1) {
     __syncthreads();
+    const int32_t* list = s_list + parity * E;
     const int count = s_count[parity];
+    const int64_t t_next = t + gridDim.x;
+    const bool build = warp == 0 && t_next < n;         // warp-uniform
+    int32_t p0 = -1, p1 = -1;
+    if (SMALL_E && build) {
+      const int32_t* nrow = inv + t_next * E;
+      if (lane < E) p0 = __ldg(nrow + lane);
+      if (lane + 32 < E) p1 = __ldg(nrow + lane + 32);
+    }
     if constexpr (VEC) {
       const int64_t cpr = hidden / kVec;
       for (int64_t c = threadIdx.x; c < cpr; c += kThreads) {
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-        for (int j0 = 0; j0 < count; j0 += kBatch) {
-          Raw8<DI> raw[kBatch];
+        for (int j0 = 0; j0 < count; j0 += kBatch<DI>) {
+          Raw8<DI> raw[kBatch<DI>];
 #pragma unroll
-          for (int j = 0; j < kBatch; ++j)
+          for (int j = 0; j < kBatch<DI>; ++j)
             if (j0 + j < count) raw[j] = load8<DI>(eo + (int64_t)list[j0 + j] * hidden + c * kVec);
 #pragma unroll
-          for (int j = 0; j < kBatch; ++j) {
+          for (int j = 0; j < kBatch<DI>; ++j) {
             if (j0 + j < count) {
               float v[8];
               widen8<DI>(raw[j], v);
@@ -86,6 +126,12 @@ unpermute_kernel(const typename DI::T* __restrict__ eo, int64_t max_rows,
         store1<DO>(out + t * hidden + h, acc);
       }
     }
+    if (build) {
+      int32_t* next = s_list + (parity ^ 1) * E;
+      const int c = SMALL_E ? compact_pair(p0, p1, max_rows, next, err, lane)
+                            : compact_row(inv + t_next * E, E, max_rows, next, err, lane);
+      if (lane == 0) s_count[parity ^ 1] = c;
+    }
   }
 }
 
@@ -95,7 +141,9 @@ int launch_unpermute(const void* eo, int64_t max_rows, const int32_t* inv,
                      int E, int32_t* err, cudaStream_t stream) {
   const bool vec = hidden % kVec == 0 && aligned16(eo) && aligned16(out);
   const size_t smem = 2 * (size_t)E * sizeof(int32_t);
-  auto k = vec ? unpermute_kernel<DI, DO, true> : unpermute_kernel<DI, DO, false>;
+  auto k = vec ? (E <= 64 ? unpermute_kernel<DI, DO, true, true> : unpermute_kernel<DI, DO, true, false>)
+              : (E <= 64 ? unpermute_kernel<DI, DO, false, true>
+                         : unpermute_kernel<DI, DO, false, false>);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute((const void*)k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);

@@ -121,7 +121,8 @@ def _run_unpermute(dev, rt, eo, out_dtype, valid, inv=None, err=None):
 @pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32, torch.float16])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32, torch.float16])
 @pytest.mark.parametrize("tokens,top_k,experts,align,hidden,valid", [
-    (50, 2, 4, 4, 72, 50), (300, 8, 64, 16, 1001, 290), (129, 6, 10, 128, 4096, 100)])
+    (50, 2, 4, 4, 72, 50), (300, 8, 64, 16, 1001, 290), (129, 6, 10, 128, 4096, 100),
+    (200, 4, 100, 8, 264, 200), (70, 2, 65, 4, 16, 69), (3000, 8, 64, 16, 512, 2999)])
 def test_unpermute_bitwise(cuda_device, in_dtype, out_dtype, tokens, top_k, experts, align, hidden,
                            valid):
     rt = inputs.routing(tokens, top_k, experts, align, seed=hidden)
