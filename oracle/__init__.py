@@ -68,6 +68,9 @@ def load(path: str) -> ctypes.CDLL:
         "orc_unpermute_ordered": (ctypes.c_int, [P, ctypes.c_int, I64, P, I32, P,
                                                  ctypes.c_int, I64, I64, I32]),
         "orc_residual_add": (None, [P, P, P, P, I64, ctypes.c_int]),
+        "orc_weighted_silu_mul_bounded": (ctypes.c_int, [P, P, P, I64, I64, I64]),
+        "orc_epilogue_chain": (ctypes.c_int, [P, P, I64, P, I32, P, P, P, I64, I64, I32,
+                                              ctypes.c_int, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -233,3 +236,38 @@ def residual_add(expert_output, shared_expert_output, residual, dt):
     out = np.empty_like(r)
     _lib().orc_residual_add(_p(e), _p(s), _p(r), _p(out), e.size, dt)
     return out
+
+
+def weighted_silu_mul_bounded(y, weights, out_init, bound_elems):
+    """y: uint16 [rows, 2*half_n]; weights float32 [rows]; out_init uint16
+    [rows, half_n] (prior contents).  Returns (out, error_bits)."""
+    y = _c(y, np.uint16)
+    rows, two_h = y.shape
+    half_n = two_h // 2
+    w = _c(np.asarray(weights, np.float32).ravel(), np.float32)
+    out = np.array(out_init, dtype=np.uint16, copy=True)
+    assert out.shape == (rows, half_n) and w.size == rows
+    err = _lib().orc_weighted_silu_mul_bounded(_p(y), _p(w), _p(out), int(bound_elems), rows,
+                                               half_n)
+    return out, err
+
+
+def epilogue_chain(expert_output, row_probs, inverse_map, valid_tokens, shared, residual,
+                   out_init, dt):
+    """The materialised chain router-weight multiply -> ordered unpermute ->
+    residual add.  Returns (out, error_bits)."""
+    st = _storage_np(dt)
+    eo = _c(expert_output, st)
+    max_rows, hidden = eo.shape
+    rp = _c(np.asarray(row_probs, np.float32).ravel(), np.float32)
+    inv = _c(inverse_map, np.int32)
+    tokens, n_exp = inv.shape
+    sh = _c(shared, st)
+    rs = _c(residual, st)
+    out = np.array(out_init, dtype=st, copy=True)
+    scratch = np.empty((max_rows, hidden), st)
+    routed = np.zeros((tokens, hidden), st)
+    err = _lib().orc_epilogue_chain(_p(eo), _p(rp), max_rows, _p(inv), int(valid_tokens), _p(sh),
+                                    _p(rs), _p(out), tokens, hidden, n_exp, dt, _p(scratch),
+                                    _p(routed))
+    return out, err

@@ -360,3 +360,54 @@ void orc_residual_add(const void *expert_output, const void *shared_expert_outpu
         store_rounded(out, dt, i, r + t);
     }
 }
+
+/* ------------------------------------- device-bounded weighted SwiGLU [BI] */
+
+/* [BI] _weighted_silu_mul_bounded_kernel, weighted_silu_mul_bounded: y is
+ * [rows, 2*half_n] (gate | up), out is [rows, half_n], weights [rows].  Every
+ * output element e = r * half_n + j below bound_elems gets
+ *     out[r, j] = bf16( silu(gate) * up * weights[r] )     (fp32, one rounding)
+ * and elements at or past the bound are neither read nor written.  A bound
+ * outside [0, rows*half_n] is clamped (ORC_ERR_COUNT).  Returns the error bits. */
+int orc_weighted_silu_mul_bounded(const uint16_t *y, const float *weights, uint16_t *out,
+                                  int64_t bound_elems, int64_t rows, int64_t half_n)
+{
+    int err = 0;
+    int64_t n = bound_elems;
+    if (n < 0) { n = 0; err |= ORC_ERR_COUNT; }
+    if (n > rows * half_n) { n = rows * half_n; err |= ORC_ERR_COUNT; }
+    for (int64_t e = 0; e < n; ++e) {
+        int64_t r = e / half_n, j = e % half_n;
+        float g = orc_f32_from_bf16(y[r * 2 * half_n + j]);
+        float u = orc_f32_from_bf16(y[r * 2 * half_n + half_n + j]);
+        float s = g * sigmoid_f32(g);
+        float v = (s * u) * weights[r];
+        out[r * half_n + j] = orc_bf16_from_f32(v);
+    }
+    return err;
+}
+
+/* ------------------------------------------- fused epilogue chain [OPT][BI][RES] */
+
+/* The epilogue chain as three materialised steps, each exactly as above:
+ *   1. router-weight multiply per expert-output row ([OPT] _rw_fwd_core with the
+ *      permuted probabilities): w[row, :] = round_dt(eo[row, :] * row_probs[row])
+ *   2. fixed-order unpermute ([BI]): routed[t, :] = round_dt(sum over e ascending
+ *      of w[inverse_map[t, e], :]), fp32 from +0
+ *   3. residual add ([RES]): out[t, :] = round_dt(residual + round_dt(routed + shared))
+ * for tokens t < valid_tokens; other tokens untouched.  `scratch` is a
+ * caller-provided [max_rows, hidden] buffer of dtype dt for step 1 and
+ * `routed` a [tokens, hidden] one for step 2.  Returns the unpermute's error bits. */
+int orc_epilogue_chain(const void *expert_output, const float *row_probs, int64_t max_rows,
+                       const int32_t *inverse_map, int32_t valid_tokens,
+                       const void *shared_expert_output, const void *residual, void *out,
+                       int64_t tokens, int64_t hidden, int32_t num_local_experts, int dt,
+                       void *scratch, void *routed)
+{
+    orc_router_weight_fwd(expert_output, dt, row_probs, scratch, dt, max_rows, hidden);
+    int err = orc_unpermute_ordered(scratch, dt, max_rows, inverse_map, valid_tokens, routed, dt,
+                                    tokens, hidden, num_local_experts);
+    int64_t n = valid_tokens < 0 ? 0 : (valid_tokens > tokens ? tokens : valid_tokens);
+    orc_residual_add(routed, shared_expert_output, residual, out, n * hidden, dt);
+    return err;
+}

@@ -50,6 +50,15 @@ MUTATIONS = [
     ("unpermute_descending", "for (int32_t e = 0; e < num_local_experts; ++e) {",
      "for (int32_t e = num_local_experts - 1; e >= 0; --e) {",
      ["test_unpermute_sums_in_increasing_expert_order"]),
+    ("bounded_drops_weight", "float v = (s * u) * weights[r];", "float v = s * u;",
+     ["test_weighted_silu_mul_bounded_vs_torch"]),
+    ("bounded_off_by_one", "for (int64_t e = 0; e < n; ++e) {\n        int64_t r = e / half_n",
+     "for (int64_t e = 0; e <= n && e < rows * half_n; ++e) {\n        int64_t r = e / half_n",
+     ["test_weighted_silu_mul_bounded_vs_torch"]),
+    ("chain_swaps_shared_and_residual",
+     "orc_residual_add(routed, shared_expert_output, residual, out, n * hidden, dt);",
+     "orc_residual_add(routed, residual, shared_expert_output, out, n * hidden, dt);",
+     ["test_epilogue_chain_is_the_composition_of_the_three_steps"]),
     ("residual_single_rounding", "float t = round_to_dtype(e + s, dt);", "float t = e + s;",
      ["test_residual_add_rounds_expert_sum_first",
       "test_residual_add_bitwise_equals_two_torch_adds"]),

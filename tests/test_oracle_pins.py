@@ -431,3 +431,82 @@ def test_routing_layout_invariants():
     rows = inv[inv >= 0]
     assert np.unique(rows).size == rows.size
     np.testing.assert_allclose(rt.probs.reshape(64, 4).sum(1).numpy(), 1.0, rtol=1e-6)
+
+
+# ------------------------------------------------------ bounded weighted SwiGLU
+
+@pytest.mark.parametrize("bound_rows,extra", [(37, 0), (20, 5), (0, 0), (50, 0)])
+def test_weighted_silu_mul_bounded_vs_torch(bound_rows, extra):
+    rows, half_n = 50, 24
+    g = torch.Generator().manual_seed(21)
+    y = (torch.randn(rows, 2 * half_n, generator=g) * 3).to(torch.bfloat16)
+    w = torch.rand(rows, generator=g)
+    bound = bound_rows * half_n + extra
+    canary = np.full((rows, half_n), 0x1234, np.uint16)
+    got, err = oracle.weighted_silu_mul_bounded(bits(y), bits(w), canary, bound)
+    assert err == 0
+    want = bits((F.silu(y[:, :half_n].float()) * y[:, half_n:].float() * w[:, None])
+                .to(torch.bfloat16))
+    flat_got, flat_want = got.reshape(-1), want.reshape(-1)
+    assert_within_ulp16(flat_got[:bound], flat_want[:bound], 1, what="bounded swiglu")
+    assert (flat_got[bound:] == 0x1234).all()
+
+
+def test_weighted_silu_mul_bounded_clamps_a_bad_bound():
+    y = torch.ones(4, 16, dtype=torch.bfloat16)
+    out0 = np.zeros((4, 8), np.uint16)
+    got, err = oracle.weighted_silu_mul_bounded(bits(y), np.ones(4, np.float32), out0, 10 ** 6)
+    assert err == oracle.ERR_COUNT and (got != 0).all()
+    _, err = oracle.weighted_silu_mul_bounded(bits(y), np.ones(4, np.float32), out0, -1)
+    assert err == oracle.ERR_COUNT
+
+
+# ------------------------------------------------------ fused epilogue chain
+
+def _chain_inputs(dtype, seed, tokens=30, top_k=3, experts=6, align=4, hidden=40):
+    rt = inputs.routing(tokens, top_k, experts, align, seed=seed)
+    eo = inputs.expert_output_input(rt, hidden, dtype=dtype, seed=seed + 1)
+    pm = rt.permutation_map
+    row_probs = torch.where(pm >= 0, rt.probs[pm.clamp(min=0).long()], torch.zeros(()))
+    res = inputs.residual_inputs((tokens, hidden), dtype, seed=seed + 2)
+    return rt, eo, row_probs.float(), res["shared_expert_output"], res["residual"]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32])
+def test_epilogue_chain_is_the_composition_of_the_three_steps(dtype):
+    """Step 1 and 3 by torch (the pages' definitions), step 2 by the pinned
+    unpermute oracle: the chain must equal their composition bit for bit."""
+    rt, eo, rp, sh, rs = _chain_inputs(dtype, 22)
+    dt = DT[dtype]
+    kind = "f16" if dtype == torch.float16 else "bf16"
+    init = bits(torch.full((rt.tokens, eo.shape[1]), 5.0, dtype=dtype))
+    got, err = oracle.epilogue_chain(bits(eo), bits(rp), bits(rt.inverse_map), rt.tokens - 3,
+                                     bits(sh), bits(rs), init, dt)
+    assert err == 0
+    w = (eo.float() * rp[:, None]).to(dtype)             # NaN sentinel rows stay NaN, unread
+    routed, _ = oracle.unpermute_ordered(bits(w), dt, bits(rt.inverse_map), rt.tokens - 3,
+                                         np.zeros_like(init), dt)
+    routed_t = from_bits(routed, dtype)
+    want = bits(rs + (routed_t + sh))
+    n = rt.tokens - 3
+    assert_bits_equal(got[:n], want[:n], "chain", kind=kind)
+    assert_bits_equal(got[n:], init[n:], "untouched tokens", kind=kind)
+
+
+def test_epilogue_chain_exact_integers():
+    """Expert rows of small integers with power-of-two probabilities: every
+    product and sum is exact, so the chain equals int64 arithmetic."""
+    tokens, top_k, experts, hidden = 16, 2, 4, 8
+    rt = inputs.routing(tokens, top_k, experts, 2, seed=23)
+    rng = np.random.default_rng(24)
+    vals = rng.integers(-40, 40, (rt.max_rows, hidden))
+    rp = np.where(bits(rt.permutation_map) >= 0, 0.5, 0.0).astype(np.float32)
+    sh = rng.integers(-10, 10, (tokens, hidden))
+    rs = rng.integers(-10, 10, (tokens, hidden))
+    f = lambda a: bits(torch.tensor(a, dtype=torch.float32))      # noqa: E731
+    got, _ = oracle.epilogue_chain(f(vals), rp, bits(rt.inverse_map), tokens, f(sh), f(rs),
+                                   np.zeros((tokens, hidden), np.float32), oracle.F32)
+    inv = bits(rt.inverse_map)
+    want = rs + sh + np.array([[sum(vals[inv[t, e], h] for e in range(experts) if inv[t, e] >= 0)
+                                for h in range(hidden)] for t in range(tokens)]) * 0.5
+    np.testing.assert_array_equal(got, want.astype(np.float32))
