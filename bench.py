@@ -217,6 +217,72 @@ class Batch:
         return [(n, table[n]) for n in self.names]
 
 
+# ---------------------------------------------------------------- next rows
+
+def time_launches(fn, reps, device):
+    """Mean device time (ms) of `reps` back-to-back calls of fn after 3 warm-ups."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize(device)
+    return a.elapsed_time(b) / reps
+
+
+def measure_next_rows(device, seed, reps, peak):
+    """The ops beyond the step: the device-bounded weighted SwiGLU and the fused
+    router-weight -> unpermute -> residual chain (against the same chain as
+    three launches).  Timed after the step, outside its timed region."""
+    from moe_expert_epilogue_b200 import inputs, ops
+    out = {}
+    T, K, E, A, H = (PERMUTED["tokens"], PERMUTED["top_k"], PERMUTED["experts"],
+                     PERMUTED["align"], PERMUTED["hidden"])
+    rows, half_n = T * K, PERMUTED["width"]
+    g = torch.Generator(device=device).manual_seed(seed + 7)
+    y = (torch.randn(rows, 2 * half_n, generator=g, device=device) * 3).to(torch.bfloat16)
+    w = torch.rand(rows, generator=g, device=device)
+    bound = torch.tensor([rows * half_n], dtype=torch.int64, device=device)
+    o = torch.empty(rows, half_n, dtype=torch.bfloat16, device=device)
+    ms = time_launches(lambda: ops.weighted_silu_mul_bounded(y, w, bound, out=o), reps, device)
+    nb = rows * (2 * half_n * 2 + 4 + half_n * 2)
+    out["weighted_silu_mul_bounded"] = {
+        "shape": f"rows {rows} (all live), half_n {half_n}", "us": round(ms * 1e3, 2),
+        "bytes": nb, "gbs": round(nb / ms / 1e6, 1), "frac": round(nb / ms / 1e6 / peak, 4)}
+    del y, w, o
+    rt = inputs.routing(T, K, E, A, seed=seed + 2, device=device)
+    eo = inputs.expert_output_input(rt, H, seed=seed + 5, device=device)
+    pm = rt.permutation_map
+    rp = torch.where(pm >= 0, rt.probs[pm.clamp(min=0).long()],
+                     torch.zeros((), device=device)).float()
+    res = inputs.residual_inputs((T, H), torch.bfloat16, seed=seed + 6, device=device)
+    sh, rs = res["shared_expert_output"], res["residual"]
+    vt = torch.tensor([T], dtype=torch.int32, device=device)
+    fo = torch.empty_like(rs)
+    ms_f = time_launches(lambda: ops.epilogue_fused(eo, rp, rt.inverse_map, vt, sh, rs, out=fo),
+                         reps, device)
+    wbuf, routed, co = torch.empty_like(eo), torch.empty_like(rs), torch.empty_like(rs)
+
+    def chained():
+        ops.router_weight_mul_fwd(eo, rp, torch.bfloat16, out=wbuf)
+        ops.unpermute_ordered(wbuf, rt.inverse_map, vt, routed)
+        ops.residual_add(routed, sh, rs, out=co)
+    ms_c = time_launches(chained, reps, device)
+    live = T * K
+    nb_f = live * H * 2 + live * 4 + T * E * 4 + 3 * T * H * 2
+    nb_c = (rt.max_rows * H * 2 * 2 + rt.max_rows * 4) + (live * H * 2 + T * E * 4 + T * H * 2) \
+        + 4 * T * H * 2
+    out["epilogue_fused"] = {
+        "shape": f"{T} tokens x top-{K} of {E}, hidden {H}, bf16", "us": round(ms_f * 1e3, 2),
+        "bytes": nb_f, "gbs": round(nb_f / ms_f / 1e6, 1), "frac": round(nb_f / ms_f / 1e6 / peak, 4),
+        "chained_three_launches_us": round(ms_c * 1e3, 2), "chained_bytes": nb_c,
+        "speedup_vs_chained": round(ms_c / ms_f, 3)}
+    return out
+
+
 # ---------------------------------------------------------------- distributed
 
 def dist_env():
@@ -423,6 +489,12 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e and not args.kernel:
         e2e = run_e2e(batch, kernels, nbytes, args, device)
+    n_used, n_kernels = batch.rt.n_used, len(kernels)
+    next_rows = None
+    if not args.kernel and not args.no_next_rows:
+        del batch, kernels
+        torch.cuda.empty_cache()
+        next_rows = measure_next_rows(device, 1000 * rank, 20, peak)
 
     sw = None
     if "swiglu_fwd" in per_kernel and "swiglu_bwd" in per_kernel:
@@ -451,16 +523,17 @@ def run_ours(args):
         "config": {"workload": workload, "bytes_per_step": bytes_per_step,
                    "l2": "no flush: every kernel streams > 126 MB (inputs larger than L2)",
                    "parallelism": f"weak: {world} independent replica(s), one per GPU",
-                   "n_used": batch.rt.n_used},
+                   "n_used": n_used},
         "swiglu_fwd_bwd": sw,
         "roofline": {"kernel": dominant, "bound": "hbm", "achieved": d["gbs"], "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": d["frac"],
                      "algorithmic_bytes": d["bytes"],
                      "traffic": ncu_traffic(dominant) if args.scale == 1.0 else None},
         "kernels": per_kernel,
-        "gpu_launches": K * len(kernels),
+        "gpu_launches": K * n_kernels,
         "clocks": clocks,
         "e2e": e2e,
+        "next_rows": next_rows,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.kernel:
         line["cpu_baseline"] = cpu_baseline(args.cpu_sample, steps=1)
@@ -632,6 +705,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the separately timed ops beyond the step")
     ap.add_argument("--kernel", default=None,
                     help="comma-separated kernels to run alone (profiling); default: the whole step")
     ap.add_argument("--scale", type=float, default=1.0,

@@ -231,6 +231,62 @@ MOE_API int moe_residual_add(const void* expert_output, const void* shared_exper
                      const void* residual, void* out, int64_t numel, moe_dtype dt,
                      cudaStream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Device-bounded weighted SwiGLU with routing weights applied at the
+ * activation.
+ * [BI] _weighted_silu_mul_bounded_kernel, weighted_silu_mul_bounded:
+ *   for every flat output element e = r * half_n + j with e < *bound_elems:
+ *     out[r, j] = bf16( silu(y[r, j]) * y[r, half_n + j] * weights[r] )
+ *   fp32 math, one rounding (the training fused weighted-SwiGLU rounding);
+ *   elements at or past the bound are neither read nor written.
+ * y             bf16 [rows, 2*half_n] contiguous (gate | up)
+ * weights       fp32 [rows] (routing probability of each row, flat)
+ * out           bf16 [rows, half_n] contiguous
+ * bound_elems   int64 (device): live_rows * half_n in normal use; a value
+ *               outside [0, rows*half_n] is clamped and MOE_DEVERR_COUNT set
+ * num_programs  persistent CTAs (<= 0: SMs x resident CTAs per SM).  The grid
+ *               size cannot change any output bit.
+ * dev_err       optional int32 (device)
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_weighted_silu_mul_bounded(const void* y, const float* weights, void* out,
+                                          const int64_t* bound_elems, int64_t rows,
+                                          int64_t half_n, int32_t num_programs,
+                                          int32_t* dev_err, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Fused epilogue chain: router-weight multiply -> fixed-order unpermute ->
+ * residual + (routed + shared) add, in one kernel.
+ * Composition of [OPT] _rw_fwd_core (per expert-output row, with that row's
+ * permuted probability), [BI] _unpermute_tokens_in_expert_order_kernel and
+ * [RES] fused_moe_residual_add; bit-identical to
+ *   moe_router_weight_mul_fwd(eo rows, dt -> dt)  then
+ *   moe_unpermute_ordered(dt -> dt)               then
+ *   moe_residual_add(dt)
+ * because every rounding of the chain is kept:
+ *   for each token t < *valid_tokens:
+ *     acc = +0;  for e ascending with row = inverse_map[t, e] >= 0:
+ *       acc += round_dt(expert_output[row, :] * row_probs[row])
+ *     out[t, :] = round_dt(residual[t, :] + round_dt(round_dt(acc) + shared[t, :]))
+ *   tokens t >= *valid_tokens are untouched.  The expert rows, the shared
+ *   output and the residual are read once and out is written once; nothing
+ *   else touches memory.
+ * expert_output  dt [max_rows, hidden] contiguous (expert-grouped FC2 output)
+ * row_probs      fp32 [max_rows]: routing probability of each expert-output
+ *                row (the permuted probabilities; unread for padding rows)
+ * inverse_map    int32 [tokens, num_local_experts] (device): row or < 0
+ * valid_tokens   int32 (device)
+ * shared_expert_output, residual, out   dt [tokens, hidden] contiguous;
+ *                out may equal residual (in place)
+ * dt             MOE_BF16, MOE_FP16 or MOE_FP32 (all tensors)
+ * dev_err        optional int32 (device): MOE_DEVERR_COUNT, MOE_DEVERR_INVERSE
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_epilogue_fused(const void* expert_output, const float* row_probs,
+                               int64_t max_rows, const int32_t* inverse_map,
+                               const int32_t* valid_tokens, const void* shared_expert_output,
+                               const void* residual, void* out, int64_t tokens, int64_t hidden,
+                               int32_t num_local_experts, moe_dtype dt, int32_t* dev_err,
+                               cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -34,6 +34,8 @@ SIGNATURES = {
     "moe_act_with_probs_permuted": [_I, _P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _I, _P, _P],
     "moe_unpermute_ordered": [_P, _I, _I64, _P, _P, _P, _I, _I64, _I64, _I32, _P, _P],
     "moe_residual_add": [_P, _P, _P, _P, _I64, _I, _P],
+    "moe_weighted_silu_mul_bounded": [_P, _P, _P, _P, _I64, _I64, _I32, _P, _P],
+    "moe_epilogue_fused": [_P, _P, _I64, _P, _P, _P, _P, _P, _I64, _I64, _I32, _I, _P, _P],
 }
 
 _lock = threading.Lock()
@@ -142,3 +144,17 @@ def moe_residual_add(expert_output, shared_expert_output, residual, out, numel, 
                      stream=None):
     _call("moe_residual_add", ptr(expert_output), ptr(shared_expert_output), ptr(residual),
           ptr(out), numel, dt, stream_handle(stream))
+
+
+def moe_weighted_silu_mul_bounded(y, weights, out, bound_elems, rows, half_n, num_programs=0,
+                                  dev_err=None, stream=None):
+    _call("moe_weighted_silu_mul_bounded", ptr(y), ptr(weights), ptr(out), ptr(bound_elems), rows,
+          half_n, num_programs, ptr(dev_err), stream_handle(stream))
+
+
+def moe_epilogue_fused(expert_output, row_probs, max_rows, inverse_map, valid_tokens,
+                       shared_expert_output, residual, out, tokens, hidden, num_local_experts,
+                       dt, dev_err=None, stream=None):
+    _call("moe_epilogue_fused", ptr(expert_output), ptr(row_probs), max_rows, ptr(inverse_map),
+          ptr(valid_tokens), ptr(shared_expert_output), ptr(residual), ptr(out), tokens, hidden,
+          num_local_experts, dt, ptr(dev_err), stream_handle(stream))

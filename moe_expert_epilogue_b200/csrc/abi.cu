@@ -244,4 +244,42 @@ int moe_residual_add(const void* expert_output, const void* shared_expert_output
                              stream);
 }
 
+int moe_weighted_silu_mul_bounded(const void* y, const float* weights, void* out,
+                                  const int64_t* bound_elems, int64_t rows, int64_t half_n,
+                                  int32_t num_programs, int32_t* dev_err, cudaStream_t stream) {
+  if (rows < 0 || half_n < 0 || !product_ok(rows, 2 * half_n)) return MOE_ERR_SHAPE;
+  if (rows == 0 || half_n == 0) return MOE_OK;
+  if (!y || !weights || !out || !bound_elems) return MOE_ERR_NULL;
+  if (!aligned_to(y, 2) || !aligned_to(out, 2) || !aligned_to(weights, 4) ||
+      !aligned_to(bound_elems, 8) || !aligned_to(dev_err, 4))
+    return MOE_ERR_ALIGN;
+  return launch_weighted_silu_mul_bounded(static_cast<const uint16_t*>(y), weights,
+                                          static_cast<uint16_t*>(out), bound_elems, rows, half_n,
+                                          num_programs, dev_err, stream);
+}
+
+int moe_epilogue_fused(const void* expert_output, const float* row_probs, int64_t max_rows,
+                       const int32_t* inverse_map, const int32_t* valid_tokens,
+                       const void* shared_expert_output, const void* residual, void* out,
+                       int64_t tokens, int64_t hidden, int32_t num_local_experts, moe_dtype dt,
+                       int32_t* dev_err, cudaStream_t stream) {
+  if (!dtype_ok(dt)) return MOE_ERR_DTYPE;
+  if (max_rows < 0 || tokens < 0 || hidden < 0 || num_local_experts < 1 ||
+      num_local_experts > 4096 || max_rows > INT32_MAX || !product_ok(max_rows, hidden) ||
+      !product_ok(tokens, hidden) || !product_ok(tokens, num_local_experts))
+    return MOE_ERR_SHAPE;
+  if (tokens == 0 || hidden == 0) return MOE_OK;
+  if (!inverse_map || !valid_tokens || !shared_expert_output || !residual || !out ||
+      (max_rows > 0 && (!expert_output || !row_probs)))
+    return MOE_ERR_NULL;
+  const int64_t es = dtype_size(dt);
+  if (!aligned_to(expert_output, es) || !aligned_to(shared_expert_output, es) ||
+      !aligned_to(residual, es) || !aligned_to(out, es) || !aligned_to(row_probs, 4) ||
+      !aligned_to(inverse_map, 4) || !aligned_to(valid_tokens, 4) || !aligned_to(dev_err, 4))
+    return MOE_ERR_ALIGN;
+  return launch_epilogue_fused(expert_output, row_probs, max_rows, inverse_map, valid_tokens,
+                               shared_expert_output, residual, out, tokens, hidden,
+                               num_local_experts, dt, dev_err, stream);
+}
+
 }  // extern "C"

@@ -1,0 +1,164 @@
+// epilogue_fused.cu -- the MoE epilogue chain in one pass:
+//   router-weight multiply (nemo_automodel.components.moe.optimized_ops,
+//     _rw_fwd_core, applied to the expert-grouped rows with their permuted
+//     probabilities),
+//   fixed-order unpermute (core.inference.moe.batch_invariant,
+//     _unpermute_tokens_in_expert_order_kernel),
+//   residual + (routed + shared) add (core.fusions.fused_moe_residual_add).
+//
+// Bit-identical to the three materialised steps, because every rounding of the
+// chain is kept in registers:
+//   w_j    = round_dt(eo[row_j, :] * row_probs[row_j])        step 1, per row
+//   routed = round_dt(((+0 + w_0) + w_1) + ...)               step 2, fp32, rows in
+//                                                              increasing expert order
+//   out    = round_dt(residual + round_dt(routed + shared))   step 3
+// The chain reads every expert row, the shared output and the residual once and
+// writes out once; the two [tokens, hidden] intermediates and the weighted copy
+// of the expert rows never reach memory.  The step-1 product is an explicitly
+// rounded multiply (__fmul_rn), so it is never fused into the step-2 add, for
+// fp32 as for the 16-bit types.
+//
+// Structure: the unpermute's -- one CTA per token at a time, row lists
+// compacted one token ahead by warp 0, one barrier per token; each thread
+// gathers up to 8 rows of an 8-column chunk (and the rows' probabilities,
+// which stay in L1) with the shared and residual chunks in flight beside them.
+#include "common.cuh"
+#include "launch.cuh"
+#include "rowlist.cuh"
+
+namespace moe {
+namespace {
+
+template <class D> constexpr int kRowsAhead = D::kBytes == 4 ? 4 : 8;
+
+template <class D, bool VEC, bool SMALL_E>
+__global__ void __launch_bounds__(kThreads)
+epilogue_fused_kernel(const typename D::T* __restrict__ eo, const float* __restrict__ row_probs,
+                      int64_t max_rows, const int32_t* __restrict__ inv,
+                      const int32_t* __restrict__ valid_tokens,
+                      const typename D::T* __restrict__ shared, const typename D::T* residual,
+                      typename D::T* out, int64_t tokens, int64_t hidden, int E, int32_t* err) {
+  extern __shared__ int32_t s_list[];  // [2][E]
+  __shared__ int s_count[2];
+  int64_t n = __ldg(valid_tokens);
+  if (n < 0 || n > tokens) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(err, MOE_DEVERR_COUNT);
+    n = n < 0 ? 0 : tokens;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int64_t t = blockIdx.x;
+  if (t >= n) return;                                   // CTA-uniform
+  if (warp == 0) {
+    const int c = compact_row(inv + t * E, E, max_rows, s_list, err, lane);
+    if (lane == 0) s_count[0] = c;
+  }
+  constexpr int B = kRowsAhead<D>;
+  for (int parity = 0; t < n; t += gridDim.x, parity ^= 1) {
+    __syncthreads();
+    const int32_t* list = s_list + parity * E;
+    const int count = s_count[parity];
+    const int64_t t_next = t + gridDim.x;
+    const bool build = warp == 0 && t_next < n;         // warp-uniform
+    int32_t p0 = -1, p1 = -1;
+    if (SMALL_E && build) {
+      const int32_t* nrow = inv + t_next * E;
+      if (lane < E) p0 = __ldg(nrow + lane);
+      if (lane + 32 < E) p1 = __ldg(nrow + lane + 32);
+    }
+    const int64_t base = t * hidden;
+    if constexpr (VEC) {
+      const int64_t cpr = hidden / kVec;
+      for (int64_t c = threadIdx.x; c < cpr; c += kThreads) {
+        const Raw8<D> rs = load8<D>(shared + base + c * kVec);
+        const Raw8<D> rr = load8<D, false>(residual + base + c * kVec);  // may alias out
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        for (int j0 = 0; j0 < count; j0 += B) {
+          Raw8<D> raw[B];
+          float p[B];
+#pragma unroll
+          for (int j = 0; j < B; ++j) {
+            if (j0 + j < count) {
+              const int64_t row = list[j0 + j];
+              raw[j] = load8<D>(eo + row * hidden + c * kVec);
+              p[j] = __ldg(row_probs + row);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < B; ++j) {
+            if (j0 + j < count) {
+              float v[8];
+              widen8<D>(raw[j], v);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc[i] = acc[i] + round_to<D>(__fmul_rn(v[i], p[j]));
+            }
+          }
+        }
+        float vs[8], vr[8];
+        widen8<D>(rs, vs);
+        widen8<D>(rr, vr);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = vr[i] + round_to<D>(round_to<D>(acc[i]) + vs[i]);
+        store8<D>(out + base + c * kVec, acc);
+      }
+    } else {
+      for (int64_t h = threadIdx.x; h < hidden; h += kThreads) {
+        float acc = 0.0f;
+        for (int j = 0; j < count; ++j) {
+          const int64_t row = list[j];
+          acc = acc + round_to<D>(__fmul_rn(load1<D>(eo + row * hidden + h), __ldg(row_probs + row)));
+        }
+        const float s = load1<D>(shared + base + h), r = load1c<D>(residual + base + h);
+        store1<D>(out + base + h, r + round_to<D>(round_to<D>(acc) + s));
+      }
+    }
+    if (build) {
+      int32_t* next = s_list + (parity ^ 1) * E;
+      const int c = SMALL_E ? compact_pair(p0, p1, max_rows, next, err, lane)
+                            : compact_row(inv + t_next * E, E, max_rows, next, err, lane);
+      if (lane == 0) s_count[parity ^ 1] = c;
+    }
+  }
+}
+
+template <class D>
+int launch(const void* eo, const float* row_probs, int64_t max_rows, const int32_t* inv,
+           const int32_t* valid_tokens, const void* shared, const void* residual, void* out,
+           int64_t tokens, int64_t hidden, int E, int32_t* err, cudaStream_t stream) {
+  using T = typename D::T;
+  const bool vec = hidden % kVec == 0 && aligned16(eo) && aligned16(shared) &&
+                   aligned16(residual) && aligned16(out);
+  const size_t smem = 2 * (size_t)E * sizeof(int32_t);
+  auto k = vec ? (E <= 64 ? epilogue_fused_kernel<D, true, true>
+                          : epilogue_fused_kernel<D, true, false>)
+               : (E <= 64 ? epilogue_fused_kernel<D, false, true>
+                          : epilogue_fused_kernel<D, false, false>);
+  int grid;
+  if (int rc = persistent_grid((const void*)k, smem, tokens > 0 ? tokens : 1, &grid)) return rc;
+  k<<<grid, kThreads, smem, stream>>>(static_cast<const T*>(eo), row_probs, max_rows, inv,
+                                      valid_tokens, static_cast<const T*>(shared),
+                                      static_cast<const T*>(residual), static_cast<T*>(out),
+                                      tokens, hidden, E, err);
+  return check_launch();
+}
+
+}  // namespace
+
+int launch_epilogue_fused(const void* expert_output, const float* row_probs, int64_t max_rows,
+                          const int32_t* inverse_map, const int32_t* valid_tokens,
+                          const void* shared_expert_output, const void* residual, void* out,
+                          int64_t tokens, int64_t hidden, int32_t num_local_experts,
+                          moe_dtype dt, int32_t* dev_err, cudaStream_t stream) {
+#define MOE_FUSED_ARGS expert_output, row_probs, max_rows, inverse_map, valid_tokens, \
+                       shared_expert_output, residual, out, tokens, hidden, num_local_experts, \
+                       dev_err, stream
+  switch (dt) {
+    case MOE_BF16: return launch<BF16>(MOE_FUSED_ARGS);
+    case MOE_FP16: return launch<F16>(MOE_FUSED_ARGS);
+    default: return launch<F32>(MOE_FUSED_ARGS);
+  }
+#undef MOE_FUSED_ARGS
+}
+
+}  // namespace moe

@@ -47,6 +47,15 @@ int launch_unpermute_ordered(const void* expert_output, moe_dtype in_dt, int64_t
                              void* out, moe_dtype out_dt, int64_t tokens, int64_t hidden,
                              int32_t num_local_experts, int32_t* dev_err,
                              cudaStream_t stream);
+int launch_weighted_silu_mul_bounded(const uint16_t* y, const float* weights, uint16_t* out,
+                                     const int64_t* bound_elems, int64_t rows, int64_t half_n,
+                                     int32_t num_programs, int32_t* dev_err,
+                                     cudaStream_t stream);
+int launch_epilogue_fused(const void* expert_output, const float* row_probs, int64_t max_rows,
+                          const int32_t* inverse_map, const int32_t* valid_tokens,
+                          const void* shared_expert_output, const void* residual, void* out,
+                          int64_t tokens, int64_t hidden, int32_t num_local_experts,
+                          moe_dtype dt, int32_t* dev_err, cudaStream_t stream);
 int launch_residual_add(const void* e, const void* s, const void* r, void* out, int64_t numel,
                         moe_dtype dt, cudaStream_t stream);
 

@@ -129,3 +129,35 @@ def residual_add(expert_output, shared_expert_output, residual, out=None, stream
     _abi.moe_residual_add(expert_output, shared_expert_output, residual, out, residual.numel(),
                           moe_dtype(residual.dtype), stream)
     return out
+
+
+def weighted_silu_mul_bounded(y, weights, bound_elems, num_programs=0, out=None, dev_err=None,
+                              stream=None):
+    """out[r, j] = bf16(silu(gate) * up * weights[r]) for flat elements below the
+    device-resident bound_elems (int64); y is [rows, 2*half_n] (gate | up)."""
+    _cuda(y, weights, bound_elems, dev_err)
+    rows, two_h = y.shape
+    half_n = two_h // 2
+    if bound_elems.dtype != torch.int64:
+        raise TypeError("bound_elems must be an int64 device tensor")
+    if out is None:
+        out = torch.empty(rows, half_n, dtype=y.dtype, device=y.device)
+    _abi.moe_weighted_silu_mul_bounded(y, _flat_probs(weights, rows), out, bound_elems, rows,
+                                       half_n, num_programs, dev_err, stream)
+    return out
+
+
+def epilogue_fused(expert_output, row_probs, inverse_map, valid_tokens, shared_expert_output,
+                   residual, out=None, dev_err=None, stream=None):
+    """residual + (unpermute(expert_output * row_probs) + shared), every rounding of
+    the three-step chain kept, in one kernel."""
+    _cuda(expert_output, row_probs, inverse_map, valid_tokens, shared_expert_output, residual,
+          dev_err)
+    max_rows, hidden = expert_output.shape
+    tokens, n_exp = inverse_map.shape
+    if out is None:
+        out = torch.empty_like(residual)
+    _abi.moe_epilogue_fused(expert_output, row_probs, max_rows, inverse_map, valid_tokens,
+                            shared_expert_output, residual, out, tokens, hidden, n_exp,
+                            moe_dtype(residual.dtype), dev_err, stream)
+    return out
