@@ -60,6 +60,9 @@ def load(path: str) -> ctypes.CDLL:
         "orc_swiglu_clamped_fwd": (None, [P, P, P, I64, I64, I64, I64, F]),
         "orc_swiglu_clamped_bwd": (None, [P, P, P, P, P, P, I64, I64, I64, I64, I64, F]),
         "orc_swiglu_clamped_fwd_f64": (None, [P, P, P, P, I64, ctypes.c_double]),
+        "orc_swiglu_clamped_fwd_dt": (None, [P, P, P, I64, I64, I64, I64, F, ctypes.c_int]),
+        "orc_swiglu_clamped_bwd_dt": (None, [P, P, P, P, P, P, I64, I64, I64, I64, I64, F,
+                                             ctypes.c_int]),
         "orc_router_weight_fwd": (None, [P, ctypes.c_int, P, P, ctypes.c_int, I64, I64]),
         "orc_router_weight_bwd": (None, [P, ctypes.c_int, P, ctypes.c_int, P, P, P, P,
                                          I64, I64]),
@@ -134,33 +137,33 @@ def f32_from_f16(bits) -> np.ndarray:
 
 # -------------------------------------------------------------- the ops
 
-def swiglu_clamped_fwd(x: np.ndarray, probs: np.ndarray, limit: float) -> np.ndarray:
-    """x: uint16 bf16 bits [rows, 2*inter]; probs: float32 [rows] or [rows, 1].
-    Returns y: uint16 bf16 bits [rows, inter]."""
-    x = _c(x, np.uint16)
+def swiglu_clamped_fwd(x: np.ndarray, probs: np.ndarray, limit: float, dt: int = BF16):
+    """x: [rows, 2*inter] in dtype dt (uint16 bits for bf16/fp16, float32 for fp32);
+    probs: float32 [rows] or [rows, 1].  Returns y [rows, inter] in dt."""
+    x = _c(x, _storage_np(dt))
     rows, two_i = x.shape
     inter = two_i // 2
     probs = _c(np.asarray(probs, np.float32).reshape(rows), np.float32)
-    y = np.empty((rows, inter), np.uint16)
-    _lib().orc_swiglu_clamped_fwd(_p(x), _p(probs), _p(y), rows, inter, two_i, inter,
-                                  float(limit))
+    y = np.empty((rows, inter), _storage_np(dt))
+    _lib().orc_swiglu_clamped_fwd_dt(_p(x), _p(probs), _p(y), rows, inter, two_i, inter,
+                                     float(limit), dt)
     return y
 
 
-def swiglu_clamped_bwd(x, probs, grad_y, limit):
-    """Returns (grad_x uint16 [rows, 2*inter], grad_probs float64 [rows],
+def swiglu_clamped_bwd(x, probs, grad_y, limit, dt: int = BF16):
+    """Returns (grad_x [rows, 2*inter] in dt, grad_probs float64 [rows],
     grad_probs_abs float64 [rows])."""
-    x = _c(x, np.uint16)
+    x = _c(x, _storage_np(dt))
     rows, two_i = x.shape
     inter = two_i // 2
     probs = _c(np.asarray(probs, np.float32).reshape(rows), np.float32)
-    grad_y = _c(grad_y, np.uint16)
+    grad_y = _c(grad_y, _storage_np(dt))
     assert grad_y.shape == (rows, inter)
-    gx = np.empty((rows, two_i), np.uint16)
+    gx = np.empty((rows, two_i), _storage_np(dt))
     gp = np.empty(rows, np.float64)
     ga = np.empty(rows, np.float64)
-    _lib().orc_swiglu_clamped_bwd(_p(x), _p(probs), _p(grad_y), _p(gx), _p(gp), _p(ga),
-                                  rows, inter, two_i, inter, two_i, float(limit))
+    _lib().orc_swiglu_clamped_bwd_dt(_p(x), _p(probs), _p(grad_y), _p(gx), _p(gp), _p(ga),
+                                     rows, inter, two_i, inter, two_i, float(limit), dt)
     return gx, gp, ga
 
 

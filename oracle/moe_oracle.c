@@ -138,24 +138,31 @@ static float clamp_f32(float v, float lo, float hi)
 /* [SWI] module docstring and forward kernel: for every row r and column
  * j < inter, with gate g = x[r, j] and up u = x[r, inter + j],
  *     y[r, j] = silu(clamp(g, max=L)) * clamp(u, -L, L) * probs[r]
- * in fp32, rounded once to x's dtype (bf16).  silu(z) = z * sigmoid(z). */
-void orc_swiglu_clamped_fwd(const uint16_t *x, const float *probs, uint16_t *y,
-                            int64_t rows, int64_t inter, int64_t ld_x, int64_t ld_y,
-                            float limit)
+ * in fp32, rounded once to x's dtype (bf16, fp16 or fp32: the page's
+ * _SUPPORTED_DTYPES).  silu(z) = z * sigmoid(z). */
+void orc_swiglu_clamped_fwd_dt(const void *x, const float *probs, void *y, int64_t rows,
+                               int64_t inter, int64_t ld_x, int64_t ld_y, float limit, int dt)
 {
     for (int64_t r = 0; r < rows; ++r) {
         float p = probs[r];
         for (int64_t j = 0; j < inter; ++j) {
-            float g = orc_f32_from_bf16(x[r * ld_x + j]);
-            float u = orc_f32_from_bf16(x[r * ld_x + inter + j]);
+            float g = load_as_f32(x, dt, r * ld_x + j);
+            float u = load_as_f32(x, dt, r * ld_x + inter + j);
             float gc = clamp_max_f32(g, limit);
             float uc = clamp_f32(u, -limit, limit);
             float s = gc * sigmoid_f32(gc);
             float v = s * uc;
             v = v * p;
-            y[r * ld_y + j] = orc_bf16_from_f32(v);
+            store_rounded(y, dt, r * ld_y + j, v);
         }
     }
+}
+
+void orc_swiglu_clamped_fwd(const uint16_t *x, const float *probs, uint16_t *y,
+                            int64_t rows, int64_t inter, int64_t ld_x, int64_t ld_y,
+                            float limit)
+{
+    orc_swiglu_clamped_fwd_dt(x, probs, y, rows, inter, ld_x, ld_y, limit, ORC_BF16);
 }
 
 /* [SWI] backward kernel: the chain rule of the forward above.
@@ -164,21 +171,21 @@ void orc_swiglu_clamped_fwd(const uint16_t *x, const float *probs, uint16_t *y,
  *   d_up   = a * silu(gc)         where -L <= u <= L, else 0
  * with silu'(z) = sigmoid(z) * (1 + z * (1 - sigmoid(z))).  The masks are
  * torch.clamp's: inclusive ranges tested on the input values.  d_gate goes to
- * grad_x[r, j] and d_up to grad_x[r, inter + j], each rounded once to bf16.
- * grad_probs[r] = sum_j dy * (silu(gc) * uc), each term in fp32, summed here
- * in float64; grad_probs_abs[r] is the float64 sum of the absolute terms. */
-void orc_swiglu_clamped_bwd(const uint16_t *x, const float *probs, const uint16_t *grad_y,
-                            uint16_t *grad_x, double *grad_probs, double *grad_probs_abs,
-                            int64_t rows, int64_t inter, int64_t ld_x, int64_t ld_gy,
-                            int64_t ld_gx, float limit)
+ * grad_x[r, j] and d_up to grad_x[r, inter + j], each rounded once to x's
+ * dtype.  grad_probs[r] = sum_j dy * (silu(gc) * uc), each term in fp32, summed
+ * here in float64; grad_probs_abs[r] is the float64 sum of the absolute terms. */
+void orc_swiglu_clamped_bwd_dt(const void *x, const float *probs, const void *grad_y,
+                               void *grad_x, double *grad_probs, double *grad_probs_abs,
+                               int64_t rows, int64_t inter, int64_t ld_x, int64_t ld_gy,
+                               int64_t ld_gx, float limit, int dt)
 {
     for (int64_t r = 0; r < rows; ++r) {
         float p = probs[r];
         double acc = 0.0, acc_abs = 0.0;
         for (int64_t j = 0; j < inter; ++j) {
-            float g = orc_f32_from_bf16(x[r * ld_x + j]);
-            float u = orc_f32_from_bf16(x[r * ld_x + inter + j]);
-            float dy = orc_f32_from_bf16(grad_y[r * ld_gy + j]);
+            float g = load_as_f32(x, dt, r * ld_x + j);
+            float u = load_as_f32(x, dt, r * ld_x + inter + j);
+            float dy = load_as_f32(grad_y, dt, r * ld_gy + j);
             float gc = clamp_max_f32(g, limit);
             float uc = clamp_f32(u, -limit, limit);
             float sg = sigmoid_f32(gc);
@@ -189,8 +196,8 @@ void orc_swiglu_clamped_bwd(const uint16_t *x, const float *probs, const uint16_
             float d_up = a * s;
             int gate_in = (g <= limit);
             int up_in = (u >= -limit) && (u <= limit);
-            grad_x[r * ld_gx + j] = gate_in ? orc_bf16_from_f32(d_gate) : (uint16_t)0;
-            grad_x[r * ld_gx + inter + j] = up_in ? orc_bf16_from_f32(d_up) : (uint16_t)0;
+            store_rounded(grad_x, dt, r * ld_gx + j, gate_in ? d_gate : 0.0f);
+            store_rounded(grad_x, dt, r * ld_gx + inter + j, up_in ? d_up : 0.0f);
             float t = dy * (s * uc);
             acc += (double)t;
             acc_abs += fabs((double)t);
@@ -198,6 +205,15 @@ void orc_swiglu_clamped_bwd(const uint16_t *x, const float *probs, const uint16_
         grad_probs[r] = acc;
         grad_probs_abs[r] = acc_abs;
     }
+}
+
+void orc_swiglu_clamped_bwd(const uint16_t *x, const float *probs, const uint16_t *grad_y,
+                            uint16_t *grad_x, double *grad_probs, double *grad_probs_abs,
+                            int64_t rows, int64_t inter, int64_t ld_x, int64_t ld_gy,
+                            int64_t ld_gx, float limit)
+{
+    orc_swiglu_clamped_bwd_dt(x, probs, grad_y, grad_x, grad_probs, grad_probs_abs, rows, inter,
+                              ld_x, ld_gy, ld_gx, limit, ORC_BF16);
 }
 
 /* float64 twin of the forward, unrounded, for finite-difference checks of the

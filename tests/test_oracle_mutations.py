@@ -17,12 +17,12 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "moe_oracle.c")
 
 # (id, text in the source, replacement, pins expected to fail)
 MUTATIONS = [
-    ("swap_gate_up", "float g = orc_f32_from_bf16(x[r * ld_x + j]);\n            float u = "
-     "orc_f32_from_bf16(x[r * ld_x + inter + j]);\n            float gc = clamp_max_f32(g, limit);"
+    ("swap_gate_up", "float g = load_as_f32(x, dt, r * ld_x + j);\n            float u = "
+     "load_as_f32(x, dt, r * ld_x + inter + j);\n            float gc = clamp_max_f32(g, limit);"
      "\n            float uc = clamp_f32(u, -limit, limit);\n            float s = gc * sigmoid_f32(gc);"
      "\n            float v = s * uc;",
-     "float u = orc_f32_from_bf16(x[r * ld_x + j]);\n            float g = "
-     "orc_f32_from_bf16(x[r * ld_x + inter + j]);\n            float gc = clamp_max_f32(g, limit);"
+     "float u = load_as_f32(x, dt, r * ld_x + j);\n            float g = "
+     "load_as_f32(x, dt, r * ld_x + inter + j);\n            float gc = clamp_max_f32(g, limit);"
      "\n            float uc = clamp_f32(u, -limit, limit);\n            float s = gc * sigmoid_f32(gc);"
      "\n            float v = s * uc;",
      ["test_swiglu_fwd_vs_float64_library_chain"]),

@@ -510,3 +510,70 @@ def test_epilogue_chain_exact_integers():
     want = rs + sh + np.array([[sum(vals[inv[t, e], h] for e in range(experts) if inv[t, e] >= 0)
                                 for h in range(hidden)] for t in range(tokens)]) * 0.5
     np.testing.assert_array_equal(got, want.astype(np.float32))
+
+
+# ------------------------------------------------ SwiGLU in fp16 and fp32
+
+def _swiglu_f64_parts(x64, p64, limit):
+    inter = x64.shape[1] // 2
+    g, u = x64[:, :inter], x64[:, inter:]
+    gc = torch.clamp(g, max=limit)
+    uc = torch.clamp(u, -limit, limit)
+    sg = torch.sigmoid(gc)
+    return g, u, gc, uc, sg
+
+
+@pytest.mark.parametrize("limit", [7.0, float("inf")])
+def test_swiglu_fp16_vs_float64_autograd(limit):
+    """fp16 storage: forward and grad_x within one fp16 ulp of the float64
+    library chain rounded once to fp16; grad_probs within the sum tolerance."""
+    d = inputs.swiglu_inputs(40, 72, sigma=3.0, limit=7.0, plant_ties=True, seed=25)
+    x16 = d["x"].to(torch.float16)
+    gy16 = d["grad_y"].to(torch.float16)
+    p = bits(d["probs"])
+    y = oracle.swiglu_clamped_fwd(bits(x16), p, limit, oracle.F16)
+    assert_within_ulp16(y, bits(_swiglu_ref64_any(x16, p, limit, torch.float16)), 1, kind="f16",
+                        what="fp16 fwd")
+    gx, gp, gabs = oracle.swiglu_clamped_bwd(bits(x16), p, bits(gy16), limit, oracle.F16)
+    xg = x16.double().requires_grad_(True)
+    pg = torch.from_numpy(p).double().reshape(-1, 1).requires_grad_(True)
+    g_, u_, gc, uc, _ = _swiglu_f64_parts(xg, pg, limit)
+    (F.silu(gc) * uc * pg).backward(gy16.double())
+    assert_within_ulp16(gx, bits(xg.grad.to(torch.float16)), 1, kind="f16", what="fp16 grad_x")
+    assert_sum_close(gp, pg.grad.reshape(-1).numpy(), gabs, 1e-6, "fp16 grad_probs")
+
+
+def _swiglu_ref64_any(x, p, limit, dtype):
+    x64 = x.double()
+    inter = x64.shape[1] // 2
+    y = F.silu(torch.clamp(x64[:, :inter], max=limit)) * torch.clamp(x64[:, inter:], -limit, limit)
+    return (y * torch.from_numpy(np.asarray(p)).double().reshape(-1, 1)).to(dtype)
+
+
+def test_swiglu_fp32_vs_float64_autograd():
+    """fp32 storage: every output within 2^-20 of the float64 value relative to
+    the magnitude of its terms (for d_gate: |dy p uc| sigma (1 + |gc| (1 - sigma)),
+    which bounds the cancellation in silu')."""
+    limit = 7.0
+    g = torch.Generator().manual_seed(26)
+    x = torch.randn(30, 2 * 50, generator=g) * 4
+    x[0, 0], x[1, 50] = limit, -limit                                  # ties stay inclusive
+    dy = torch.randn(30, 50, generator=g)
+    p = torch.rand(30, generator=g)
+    y = oracle.swiglu_clamped_fwd(x.numpy(), p.numpy(), limit, oracle.F32)
+    ref = _swiglu_ref64_any(x, p.numpy(), limit, torch.float64).numpy()
+    assert (np.abs(y - ref) <= 2 ** -20 * np.abs(ref) + 1e-30).all()
+    gx, gp, gabs = oracle.swiglu_clamped_bwd(x.numpy(), p.numpy(), dy.numpy(), limit, oracle.F32)
+    xg = x.double().requires_grad_(True)
+    pg = p.double().reshape(-1, 1).requires_grad_(True)
+    _, _, gc, uc, sg = _swiglu_f64_parts(xg, pg, limit)
+    (F.silu(gc) * uc * pg).backward(dy.double())
+    with torch.no_grad():
+        a = (dy.double() * pg).abs()
+        scale_g = a * uc.abs() * sg * (1 + gc.abs() * (1 - sg))
+        scale_u = a * (gc * sg).abs()
+    err = np.abs(gx - xg.grad.numpy())
+    scale = np.concatenate([scale_g.numpy(), scale_u.numpy()], 1)
+    assert (err <= 2 ** -20 * scale + 1e-30).all()
+    assert gx[0, 0] != 0 and gx[1, 50] != 0
+    assert_sum_close(gp, pg.grad.reshape(-1).numpy(), gabs, 1e-6, "fp32 grad_probs")
