@@ -101,12 +101,13 @@ MOE_API int moe_abi_version(void);
  * [SWI] module docstring and the forward kernel (_swiglu_clamped_fwd_kernel):
  *   y[r, j] = silu(clamp(g, max=L)) * clamp(u, -L, L) * probs[r]
  *   with g = x[r, j], u = x[r, inter + j], silu(z) = z * sigmoid(z);
- *   fp32 math, one rounding to bf16.  clamp is torch.clamp (NaN propagates).
- * x      bf16 [rows, ld_x], columns [0, inter) gate, [inter, 2*inter) up; ld_x >= 2*inter
+ *   fp32 math, one rounding to dt.  clamp is torch.clamp (NaN propagates).
+ * x      dt [rows, ld_x], columns [0, inter) gate, [inter, 2*inter) up; ld_x >= 2*inter
  * probs  fp32 [rows] (one routing probability per row, i.e. [rows, 1])
- * y      bf16 [rows, ld_y], ld_y >= inter; columns >= inter are not written
+ * y      dt [rows, ld_y], ld_y >= inter; columns >= inter are not written
  * limit  L > 0, may be +inf (no clamping); NaN or <= 0 -> MOE_ERR_LIMIT
- * dt     MOE_BF16 (others -> MOE_ERR_DTYPE)
+ * dt     storage dtype of x and y: MOE_BF16, MOE_FP16 or MOE_FP32 (the page's
+ *        _SUPPORTED_DTYPES)
  * ---------------------------------------------------------------------- */
 MOE_API int moe_swiglu_clamped_fwd(const void* x, const float* probs, void* y, int64_t rows,
                            int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
@@ -121,14 +122,15 @@ MOE_API int moe_swiglu_clamped_fwd(const void* x, const float* probs, void* y, i
  *   grad_probs[r]        = sum_j dy * s * uc   (fp32, reduced per row)
  *   silu'(z) = sigmoid(z) * (1 + z * (1 - sigmoid(z))); the masks are
  *   torch.clamp's inclusive ranges on the input values; grad_x is rounded
- *   once to bf16.  grad_probs is reduced in a fixed order (per-thread
+ *   once to dt.  grad_probs is reduced in a fixed order (per-thread
  *   partials over a fixed column assignment, a fixed warp butterfly, warps
  *   in index order), independent of the grid and of the batch.
- * x           bf16 [rows, ld_x]   (the forward's input, recomputed from)
+ * x           dt [rows, ld_x]   (the forward's input, recomputed from)
  * probs       fp32 [rows]
- * grad_y      bf16 [rows, ld_gy], ld_gy >= inter
- * grad_x      bf16 [rows, ld_gx], ld_gx >= 2*inter  (output)
- * grad_probs  fp32 [rows]                           (output)
+ * grad_y      dt [rows, ld_gy], ld_gy >= inter
+ * grad_x      dt [rows, ld_gx], ld_gx >= 2*inter  (output)
+ * grad_probs  fp32 [rows]                         (output)
+ * dt          MOE_BF16, MOE_FP16 or MOE_FP32
  * ---------------------------------------------------------------------- */
 MOE_API int moe_swiglu_clamped_bwd(const void* x, const float* probs, const void* grad_y,
                            void* grad_x, float* grad_probs, int64_t rows, int64_t inter,

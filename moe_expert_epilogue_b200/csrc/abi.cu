@@ -120,23 +120,22 @@ int moe_abi_version(void) { return 1; }
 int moe_swiglu_clamped_fwd(const void* x, const float* probs, void* y, int64_t rows,
                            int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
                            moe_dtype dt, cudaStream_t stream) {
-  if (dt != MOE_BF16) return MOE_ERR_DTYPE;
+  if (!dtype_ok(dt)) return MOE_ERR_DTYPE;
   if (rows < 0 || inter < 0 || ld_x < 2 * inter || ld_y < inter) return MOE_ERR_SHAPE;
   if (!product_ok(rows, ld_x) || !product_ok(rows, ld_y)) return MOE_ERR_SHAPE;
   if (!limit_ok(limit)) return MOE_ERR_LIMIT;
   if (rows == 0 || inter == 0) return MOE_OK;
   if (!x || !probs || !y) return MOE_ERR_NULL;
-  if (!aligned_to(x, 2) || !aligned_to(y, 2) || !aligned_to(probs, 4)) return MOE_ERR_ALIGN;
-  return launch_swiglu_clamped_fwd(static_cast<const uint16_t*>(x), probs,
-                                   static_cast<uint16_t*>(y), rows, inter, ld_x, ld_y, limit,
-                                   stream);
+  const int64_t es = dtype_size(dt);
+  if (!aligned_to(x, es) || !aligned_to(y, es) || !aligned_to(probs, 4)) return MOE_ERR_ALIGN;
+  return launch_swiglu_clamped_fwd(x, probs, y, rows, inter, ld_x, ld_y, limit, dt, stream);
 }
 
 int moe_swiglu_clamped_bwd(const void* x, const float* probs, const void* grad_y,
                            void* grad_x, float* grad_probs, int64_t rows, int64_t inter,
                            int64_t ld_x, int64_t ld_gy, int64_t ld_gx, float limit,
                            moe_dtype dt, cudaStream_t stream) {
-  if (dt != MOE_BF16) return MOE_ERR_DTYPE;
+  if (!dtype_ok(dt)) return MOE_ERR_DTYPE;
   if (rows < 0 || inter < 0 || ld_x < 2 * inter || ld_gy < inter || ld_gx < 2 * inter)
     return MOE_ERR_SHAPE;
   if (!product_ok(rows, ld_x) || !product_ok(rows, ld_gy) || !product_ok(rows, ld_gx))
@@ -145,13 +144,12 @@ int moe_swiglu_clamped_bwd(const void* x, const float* probs, const void* grad_y
   if (rows == 0) return MOE_OK;
   if (!probs || !grad_probs) return MOE_ERR_NULL;
   if (inter > 0 && (!x || !grad_y || !grad_x)) return MOE_ERR_NULL;
-  if (!aligned_to(x, 2) || !aligned_to(grad_y, 2) || !aligned_to(grad_x, 2) ||
+  const int64_t es = dtype_size(dt);
+  if (!aligned_to(x, es) || !aligned_to(grad_y, es) || !aligned_to(grad_x, es) ||
       !aligned_to(probs, 4) || !aligned_to(grad_probs, 4))
     return MOE_ERR_ALIGN;
-  return launch_swiglu_clamped_bwd(static_cast<const uint16_t*>(x), probs,
-                                   static_cast<const uint16_t*>(grad_y),
-                                   static_cast<uint16_t*>(grad_x), grad_probs, rows, inter,
-                                   ld_x, ld_gy, ld_gx, limit, stream);
+  return launch_swiglu_clamped_bwd(x, probs, grad_y, grad_x, grad_probs, rows, inter, ld_x,
+                                   ld_gy, ld_gx, limit, dt, stream);
 }
 
 int moe_router_weight_mul_fwd(const void* x, moe_dtype x_dt, const float* probs, void* out,

@@ -23,13 +23,13 @@ int check_launch();
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Launchers (one per op family); arguments already validated.
-int launch_swiglu_clamped_fwd(const uint16_t* x, const float* probs, uint16_t* y, int64_t rows,
+int launch_swiglu_clamped_fwd(const void* x, const float* probs, void* y, int64_t rows,
                               int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
-                              cudaStream_t stream);
-int launch_swiglu_clamped_bwd(const uint16_t* x, const float* probs, const uint16_t* grad_y,
-                              uint16_t* grad_x, float* grad_probs, int64_t rows, int64_t inter,
+                              moe_dtype dt, cudaStream_t stream);
+int launch_swiglu_clamped_bwd(const void* x, const float* probs, const void* grad_y,
+                              void* grad_x, float* grad_probs, int64_t rows, int64_t inter,
                               int64_t ld_x, int64_t ld_gy, int64_t ld_gx, float limit,
-                              cudaStream_t stream);
+                              moe_dtype dt, cudaStream_t stream);
 int launch_router_weight_fwd(const void* x, moe_dtype x_dt, const float* probs, void* out,
                              moe_dtype out_dt, int64_t rows, int64_t hidden,
                              cudaStream_t stream);

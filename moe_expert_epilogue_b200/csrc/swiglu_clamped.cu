@@ -1,20 +1,23 @@
 // swiglu_clamped.cu -- clamped, probability-weighted SwiGLU, forward and
 // one-pass backward (nemo_automodel.components.moe.swiglu_triton: module
-// docstring, _swiglu_clamped_fwd_kernel, _swiglu_clamped_bwd_kernel).
+// docstring, _swiglu_clamped_fwd_kernel, _swiglu_clamped_bwd_kernel,
+// _SUPPORTED_DTYPES = bf16, fp16, fp32).
 //
-//   y      = silu(clamp(g, max=L)) * clamp(u, -L, L) * p          fp32, one bf16 rounding
+//   y      = silu(clamp(g, max=L)) * clamp(u, -L, L) * p          fp32, one rounding to x.dtype
 //   d_gate = dy * p * uc * silu'(gc)  on g <= L        (torch.clamp's inclusive masks)
 //   d_up   = dy * p * silu(gc)        on -L <= u <= L
 //   d_p    = sum_j dy * silu(gc) * uc
 //
-// Forward: a flat, persistent, grid-stride stream over 8-column chunks: per
-// chunk two 16-byte loads (gate, up) and one 16-byte store.  Backward: a
-// persistent loop over groups of rows; W threads own one row (one warp for the
-// vectorised path), walk its chunks with a fixed column assignment, write
-// d_gate / d_up straight into the two halves of grad_x and reduce the row's
-// probability gradient with a fixed tree (per-thread partials in column order,
-// warp butterfly, warps in index order).  No barrier is needed when W = 32, so
-// every warp streams independently with its next loads already in flight.
+// Forward: one warp per row (warps stride over the rows), the row's
+// probability loaded once, U chunks of 8 columns per lane in flight (two
+// loads each: gate, up), one 16-byte store per chunk (two for fp32); a flat
+// grid-stride variant serves rows shorter than 64 chunks.  Backward: W threads
+// own one row (one warp for the vectorised path), walk its chunks with a fixed
+// column assignment, write d_gate / d_up straight into the two halves of
+// grad_x and reduce the row's probability gradient with a fixed tree
+// (per-thread partials in column order, warp butterfly, warps in index
+// order).  No barrier is needed when W = 32, so every warp streams
+// independently with its next loads already in flight.
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -51,10 +54,51 @@ __device__ __forceinline__ BwdOut bwd_math(float g, float u, float dy, float p, 
 
 // ------------------------------------------------------------------ forward
 
-template <int U>
+template <class D, int U>
 __global__ void __launch_bounds__(kThreads)
-swiglu_fwd_vec(const uint16_t* __restrict__ x, const float* __restrict__ probs,
-               uint16_t* __restrict__ y, int64_t rows, int64_t inter, int64_t ld_x,
+swiglu_fwd_rows(const typename D::T* __restrict__ x, const float* __restrict__ probs,
+                typename D::T* __restrict__ y, int64_t rows, int64_t inter, int64_t ld_x,
+                int64_t ld_y, float L) {
+  const int64_t cpr = inter / kVec;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
+  const FwdMath f{L};
+  for (int64_t r = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); r < rows;
+       r += nwarps) {
+    const float p = __ldg(probs + r);
+    const typename D::T* xr = x + r * ld_x;
+    typename D::T* yr = y + r * ld_y;
+    for (int64_t c0 = lane; c0 < cpr; c0 += 32 * U) {
+      Raw8<D> gw[U], uw[U];
+#pragma unroll
+      for (int k = 0; k < U; ++k) {
+        const int64_t c = c0 + 32 * k;
+        if (c < cpr) {
+          gw[k] = load8<D>(xr + c * kVec);
+          uw[k] = load8<D>(xr + inter + c * kVec);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < U; ++k) {
+        const int64_t c = c0 + 32 * k;
+        if (c < cpr) {
+          float g[8], u[8], o[8];
+          widen8<D>(gw[k], g);
+          widen8<D>(uw[k], u);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o[i] = f(g[i], u[i], p);
+          store8<D>(yr + c * kVec, o);
+        }
+      }
+    }
+  }
+}
+
+// Flat grid-stride forward over (row, chunk) pairs, for short rows.
+template <class D, int U>
+__global__ void __launch_bounds__(kThreads)
+swiglu_fwd_vec(const typename D::T* __restrict__ x, const float* __restrict__ probs,
+               typename D::T* __restrict__ y, int64_t rows, int64_t inter, int64_t ld_x,
                int64_t ld_y, float L) {
   const int64_t cpr = inter / kVec;
   const int64_t total = rows * cpr;
@@ -64,15 +108,15 @@ swiglu_fwd_vec(const uint16_t* __restrict__ x, const float* __restrict__ probs,
   RowCursor cur(q, S, cpr);
   const FwdMath f{L};
   for (; q < total; q += U * S) {
-    uint4 gw[U], uw[U];
+    Raw8<D> gw[U], uw[U];
     float p[U];
-    uint16_t* dst[U];
+    typename D::T* dst[U];
 #pragma unroll
     for (int k = 0; k < U; ++k) {
       if (q + k * S < total) {
-        const uint16_t* src = x + cur.r * ld_x + cur.c * kVec;
-        gw[k] = ld_stream(src);
-        uw[k] = ld_stream(src + inter);
+        const typename D::T* src = x + cur.r * ld_x + cur.c * kVec;
+        gw[k] = load8<D>(src);
+        uw[k] = load8<D>(src + inter);
         p[k] = __ldg(probs + cur.r);
         dst[k] = y + cur.r * ld_y + cur.c * kVec;
       }
@@ -82,63 +126,21 @@ swiglu_fwd_vec(const uint16_t* __restrict__ x, const float* __restrict__ probs,
     for (int k = 0; k < U; ++k) {
       if (q + k * S < total) {
         float g[8], u[8], o[8];
-        unpack_bf16x8(gw[k], g);
-        unpack_bf16x8(uw[k], u);
+        widen8<D>(gw[k], g);
+        widen8<D>(uw[k], u);
 #pragma unroll
         for (int i = 0; i < 8; ++i) o[i] = f(g[i], u[i], p[k]);
-        store8<BF16>(dst[k], o);
-      }
-    }
-  }
-}
-
-// Warp-per-row forward for rows of at least 64 chunks: a warp owns one row at
-// a time, loads the row's probability once and streams its chunks lane,
-// lane + 32, ... with U chunks' loads in flight per lane.
-template <int U>
-__global__ void __launch_bounds__(kThreads)
-swiglu_fwd_rows(const uint16_t* __restrict__ x, const float* __restrict__ probs,
-                uint16_t* __restrict__ y, int64_t rows, int64_t inter, int64_t ld_x,
-                int64_t ld_y, float L) {
-  const int64_t cpr = inter / kVec;
-  const int lane = threadIdx.x & 31;
-  const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
-  const FwdMath f{L};
-  for (int64_t r = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); r < rows;
-       r += nwarps) {
-    const float p = __ldg(probs + r);
-    const uint16_t* xr = x + r * ld_x;
-    uint16_t* yr = y + r * ld_y;
-    for (int64_t c0 = lane; c0 < cpr; c0 += 32 * U) {
-      uint4 gw[U], uw[U];
-#pragma unroll
-      for (int k = 0; k < U; ++k) {
-        const int64_t c = c0 + 32 * k;
-        if (c < cpr) {
-          gw[k] = ld_stream(xr + c * kVec);
-          uw[k] = ld_stream(xr + inter + c * kVec);
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < U; ++k) {
-        const int64_t c = c0 + 32 * k;
-        if (c < cpr) {
-          float g[8], u[8], o[8];
-          unpack_bf16x8(gw[k], g);
-          unpack_bf16x8(uw[k], u);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) o[i] = f(g[i], u[i], p);
-          store8<BF16>(yr + c * kVec, o);
-        }
+        store8<D>(dst[k], o);
       }
     }
   }
 }
 
 // Element-granular forward: any inter, leading dimensions and alignment.
+template <class D>
 __global__ void __launch_bounds__(kThreads)
-swiglu_fwd_scalar(const uint16_t* __restrict__ x, const float* __restrict__ probs,
-                  uint16_t* __restrict__ y, int64_t rows, int64_t inter, int64_t ld_x,
+swiglu_fwd_scalar(const typename D::T* __restrict__ x, const float* __restrict__ probs,
+                  typename D::T* __restrict__ y, int64_t rows, int64_t inter, int64_t ld_x,
                   int64_t ld_y, float L) {
   const int64_t total = rows * inter;
   const int64_t S = (int64_t)gridDim.x * kThreads;
@@ -147,9 +149,9 @@ swiglu_fwd_scalar(const uint16_t* __restrict__ x, const float* __restrict__ prob
   RowCursor cur(q, S, inter);
   const FwdMath f{L};
   for (; q < total; q += S, cur.advance()) {
-    const uint16_t* src = x + cur.r * ld_x + cur.c;
-    const float g = load1<BF16>(src), u = load1<BF16>(src + inter);
-    store1<BF16>(y + cur.r * ld_y + cur.c, f(g, u, __ldg(probs + cur.r)));
+    const typename D::T* src = x + cur.r * ld_x + cur.c;
+    const float g = load1<D>(src), u = load1<D>(src + inter);
+    store1<D>(y + cur.r * ld_y + cur.c, f(g, u, __ldg(probs + cur.r)));
   }
 }
 
@@ -175,14 +177,10 @@ __device__ __forceinline__ float row_reduce(float acc, float (*red)[kThreads / 3
   }
 }
 
-#ifndef MOE_SWIGLU_BWD_MIN_BLOCKS
-#define MOE_SWIGLU_BWD_MIN_BLOCKS 1
-#endif
-
-template <int W, int U>
-__global__ void __launch_bounds__(kThreads, MOE_SWIGLU_BWD_MIN_BLOCKS)
-swiglu_bwd_vec(const uint16_t* __restrict__ x, const float* __restrict__ probs,
-               const uint16_t* __restrict__ gy, uint16_t* __restrict__ gx,
+template <class D, int W, int U>
+__global__ void __launch_bounds__(kThreads)
+swiglu_bwd_vec(const typename D::T* __restrict__ x, const float* __restrict__ probs,
+               const typename D::T* __restrict__ gy, typename D::T* __restrict__ gx,
                float* __restrict__ gp, int64_t rows, int64_t inter, int64_t ld_x,
                int64_t ld_gy, int64_t ld_gx, float L) {
   constexpr int G = kThreads / W;
@@ -195,18 +193,18 @@ swiglu_bwd_vec(const uint16_t* __restrict__ x, const float* __restrict__ probs,
     float acc = 0.0f;
     if (r < rows) {
       const float p = __ldg(probs + r);
-      const uint16_t* xr = x + r * ld_x;
-      const uint16_t* gyr = gy + r * ld_gy;
-      uint16_t* gxr = gx + r * ld_gx;
+      const typename D::T* xr = x + r * ld_x;
+      const typename D::T* gyr = gy + r * ld_gy;
+      typename D::T* gxr = gx + r * ld_gx;
       for (int64_t c0 = lane; c0 < cpr; c0 += (int64_t)U * W) {
-        uint4 gw[U], uw[U], dw[U];
+        Raw8<D> gw[U], uw[U], dw[U];
 #pragma unroll
         for (int k = 0; k < U; ++k) {
           const int64_t c = c0 + (int64_t)k * W;
           if (c < cpr) {
-            gw[k] = ld_stream(xr + c * kVec);
-            uw[k] = ld_stream(xr + inter + c * kVec);
-            dw[k] = ld_stream(gyr + c * kVec);
+            gw[k] = load8<D>(xr + c * kVec);
+            uw[k] = load8<D>(xr + inter + c * kVec);
+            dw[k] = load8<D>(gyr + c * kVec);
           }
         }
 #pragma unroll
@@ -214,9 +212,9 @@ swiglu_bwd_vec(const uint16_t* __restrict__ x, const float* __restrict__ probs,
           const int64_t c = c0 + (int64_t)k * W;
           if (c < cpr) {
             float g[8], u[8], d[8], og[8], ou[8];
-            unpack_bf16x8(gw[k], g);
-            unpack_bf16x8(uw[k], u);
-            unpack_bf16x8(dw[k], d);
+            widen8<D>(gw[k], g);
+            widen8<D>(uw[k], u);
+            widen8<D>(dw[k], d);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const BwdOut o = bwd_math(g[i], u[i], d[i], p, L);
@@ -224,8 +222,8 @@ swiglu_bwd_vec(const uint16_t* __restrict__ x, const float* __restrict__ probs,
               ou[i] = o.d_up;
               acc += o.t;
             }
-            store8<BF16>(gxr + c * kVec, og);
-            store8<BF16>(gxr + inter + c * kVec, ou);
+            store8<D>(gxr + c * kVec, og);
+            store8<D>(gxr + inter + c * kVec, ou);
           }
         }
       }
@@ -236,10 +234,10 @@ swiglu_bwd_vec(const uint16_t* __restrict__ x, const float* __restrict__ probs,
   }
 }
 
-template <int W>
+template <class D, int W>
 __global__ void __launch_bounds__(kThreads)
-swiglu_bwd_scalar(const uint16_t* __restrict__ x, const float* __restrict__ probs,
-                  const uint16_t* __restrict__ gy, uint16_t* __restrict__ gx,
+swiglu_bwd_scalar(const typename D::T* __restrict__ x, const float* __restrict__ probs,
+                  const typename D::T* __restrict__ gy, typename D::T* __restrict__ gx,
                   float* __restrict__ gp, int64_t rows, int64_t inter, int64_t ld_x,
                   int64_t ld_gy, int64_t ld_gx, float L) {
   constexpr int G = kThreads / W;
@@ -252,12 +250,12 @@ swiglu_bwd_scalar(const uint16_t* __restrict__ x, const float* __restrict__ prob
     if (r < rows) {
       const float p = __ldg(probs + r);
       for (int64_t j = lane; j < inter; j += W) {
-        const float g = load1<BF16>(x + r * ld_x + j);
-        const float u = load1<BF16>(x + r * ld_x + inter + j);
-        const float d = load1<BF16>(gy + r * ld_gy + j);
+        const float g = load1<D>(x + r * ld_x + j);
+        const float u = load1<D>(x + r * ld_x + inter + j);
+        const float d = load1<D>(gy + r * ld_gy + j);
         const BwdOut o = bwd_math(g, u, d, p, L);
-        store1<BF16>(gx + r * ld_gx + j, o.d_gate);
-        store1<BF16>(gx + r * ld_gx + inter + j, o.d_up);
+        store1<D>(gx + r * ld_gx + j, o.d_gate);
+        store1<D>(gx + r * ld_gx + inter + j, o.d_up);
         acc += o.t;
       }
     }
@@ -277,33 +275,17 @@ inline int threads_per_row(int64_t units) {
   return 256;
 }
 
-template <class K>
-int launch_persistent(K kernel, int64_t useful_blocks, cudaStream_t stream, const uint16_t* x,
-                      const float* probs, const uint16_t* gy, uint16_t* gx, float* gp,
-                      int64_t rows, int64_t inter, int64_t ld_x, int64_t ld_gy, int64_t ld_gx,
-                      float L) {
-  int grid;
-  if (int rc = persistent_grid((const void*)kernel, 0, useful_blocks, &grid)) return rc;
-  kernel<<<grid, kThreads, 0, stream>>>(x, probs, gy, gx, gp, rows, inter, ld_x, ld_gy, ld_gx,
-                                        L);
-  return check_launch();
-}
-
-}  // namespace
-
-// Tuning knobs (compile-time).  kFwdUnroll: chunks whose loads a thread issues
-// before it computes any of them.  kBwdRowThreads: threads that own one row in
-// the backward (0: the smallest of 32/64/128/256 covering the row's chunks);
-// it fixes the grad_probs summation tree together with the row length.
-// kBwdUnroll: chunks per thread loaded ahead in the backward.
+// Tuning knobs (compile-time).  Unrolls are chunks whose loads a thread issues
+// before it computes any of them, given for 16-bit types (fp32 chunks are twice
+// the bytes and use half).  MOE_SWIGLU_BWD_ROW_THREADS: threads that own one
+// row in the vectorised backward (0: as the element-wise path, the smallest of
+// 32/64/128/256 covering the row); with the row length it fixes the grad_probs
+// summation tree.
 #ifndef MOE_SWIGLU_FWD_UNROLL
 #define MOE_SWIGLU_FWD_UNROLL 2
 #endif
 #ifndef MOE_SWIGLU_FWD_ROW_UNROLL
 #define MOE_SWIGLU_FWD_ROW_UNROLL 8
-#endif
-#ifndef MOE_SWIGLU_FWD_ROWS
-#define MOE_SWIGLU_FWD_ROWS 1
 #endif
 #ifndef MOE_SWIGLU_BWD_ROW_THREADS
 #define MOE_SWIGLU_BWD_ROW_THREADS 32
@@ -311,68 +293,112 @@ int launch_persistent(K kernel, int64_t useful_blocks, cudaStream_t stream, cons
 #ifndef MOE_SWIGLU_BWD_UNROLL
 #define MOE_SWIGLU_BWD_UNROLL 4
 #endif
-constexpr int kFwdUnroll = MOE_SWIGLU_FWD_UNROLL;
-constexpr int kFwdRowUnroll = MOE_SWIGLU_FWD_ROW_UNROLL;
-constexpr bool kFwdRows = MOE_SWIGLU_FWD_ROWS != 0;
+template <class D>
+constexpr int unroll_for(int u16) { return D::kBytes == 4 ? (u16 + 1) / 2 : u16; }
 constexpr int kBwdRowThreads = MOE_SWIGLU_BWD_ROW_THREADS;
-constexpr int kBwdUnroll = MOE_SWIGLU_BWD_UNROLL;
 
-int launch_swiglu_clamped_fwd(const uint16_t* x, const float* probs, uint16_t* y, int64_t rows,
-                              int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
-                              cudaStream_t stream) {
+template <class D>
+int fwd(const void* xv, const float* probs, void* yv, int64_t rows, int64_t inter, int64_t ld_x,
+        int64_t ld_y, float limit, cudaStream_t stream) {
+  using T = typename D::T;
+  const T* x = static_cast<const T*>(xv);
+  T* y = static_cast<T*>(yv);
   const bool vec = inter % kVec == 0 && ld_x % kVec == 0 && ld_y % kVec == 0 && aligned16(x) &&
                    aligned16(y);
   int grid;
-  if (vec && kFwdRows && inter / kVec >= 64) {
-    auto k = swiglu_fwd_rows<kFwdRowUnroll>;
+  if (vec && inter / kVec >= 64) {
+    auto k = swiglu_fwd_rows<D, unroll_for<D>(MOE_SWIGLU_FWD_ROW_UNROLL)>;
     if (int rc = persistent_grid((const void*)k, 0, (rows + kThreads / 32 - 1) / (kThreads / 32),
                                  &grid))
       return rc;
     k<<<grid, kThreads, 0, stream>>>(x, probs, y, rows, inter, ld_x, ld_y, limit);
   } else if (vec) {
+    constexpr int U = unroll_for<D>(MOE_SWIGLU_FWD_UNROLL);
+    auto k = swiglu_fwd_vec<D, U>;
     const int64_t units = rows * (inter / kVec);
-    auto k = swiglu_fwd_vec<kFwdUnroll>;
-    if (int rc = persistent_grid((const void*)k, 0,
-                                 (units + kThreads * kFwdUnroll - 1) / (kThreads * kFwdUnroll),
+    if (int rc = persistent_grid((const void*)k, 0, (units + kThreads * U - 1) / (kThreads * U),
                                  &grid))
       return rc;
     k<<<grid, kThreads, 0, stream>>>(x, probs, y, rows, inter, ld_x, ld_y, limit);
   } else {
-    const int64_t units = rows * inter;
-    if (int rc = persistent_grid((const void*)swiglu_fwd_scalar, 0,
-                                 (units + kThreads - 1) / kThreads, &grid))
+    auto k = swiglu_fwd_scalar<D>;
+    if (int rc = persistent_grid((const void*)k, 0, (rows * inter + kThreads - 1) / kThreads,
+                                 &grid))
       return rc;
-    swiglu_fwd_scalar<<<grid, kThreads, 0, stream>>>(x, probs, y, rows, inter, ld_x, ld_y,
-                                                     limit);
+    k<<<grid, kThreads, 0, stream>>>(x, probs, y, rows, inter, ld_x, ld_y, limit);
   }
   return check_launch();
 }
 
-int launch_swiglu_clamped_bwd(const uint16_t* x, const float* probs, const uint16_t* grad_y,
-                              uint16_t* grad_x, float* grad_probs, int64_t rows, int64_t inter,
-                              int64_t ld_x, int64_t ld_gy, int64_t ld_gx, float limit,
-                              cudaStream_t stream) {
+template <class K, class T>
+int launch_bwd(K kernel, int W, cudaStream_t stream, const T* x, const float* probs, const T* gy,
+               T* gx, float* gp, int64_t rows, int64_t inter, int64_t ld_x, int64_t ld_gy,
+               int64_t ld_gx, float L) {
+  int grid;
+  const int64_t blocks = (rows + kThreads / W - 1) / (kThreads / W);
+  if (int rc = persistent_grid((const void*)kernel, 0, blocks, &grid)) return rc;
+  kernel<<<grid, kThreads, 0, stream>>>(x, probs, gy, gx, gp, rows, inter, ld_x, ld_gy, ld_gx, L);
+  return check_launch();
+}
+
+template <class D>
+int bwd(const void* xv, const float* probs, const void* gyv, void* gxv, float* gp, int64_t rows,
+        int64_t inter, int64_t ld_x, int64_t ld_gy, int64_t ld_gx, float limit,
+        cudaStream_t stream) {
+  using T = typename D::T;
+  const T* x = static_cast<const T*>(xv);
+  const T* gy = static_cast<const T*>(gyv);
+  T* gx = static_cast<T*>(gxv);
   const bool vec = inter % kVec == 0 && ld_x % kVec == 0 && ld_gy % kVec == 0 &&
-                   ld_gx % kVec == 0 && aligned16(x) && aligned16(grad_y) && aligned16(grad_x);
+                   ld_gx % kVec == 0 && aligned16(x) && aligned16(gy) && aligned16(gx);
   const int W = (vec && kBwdRowThreads) ? kBwdRowThreads
                                         : threads_per_row(vec ? inter / kVec : inter);
-  const int64_t blocks = (rows + kThreads / W - 1) / (kThreads / W);
-#define MOE_BWD_ARGS stream, x, probs, grad_y, grad_x, grad_probs, rows, inter, ld_x, ld_gy, ld_gx, limit
+  constexpr int U = unroll_for<D>(MOE_SWIGLU_BWD_UNROLL);
+#define MOE_BWD_ARGS stream, x, probs, gy, gx, gp, rows, inter, ld_x, ld_gy, ld_gx, limit
   if (vec) {
     switch (W) {
-      case 32: return launch_persistent(swiglu_bwd_vec<32, kBwdUnroll>, blocks, MOE_BWD_ARGS);
-      case 64: return launch_persistent(swiglu_bwd_vec<64, kBwdUnroll>, blocks, MOE_BWD_ARGS);
-      case 128: return launch_persistent(swiglu_bwd_vec<128, kBwdUnroll>, blocks, MOE_BWD_ARGS);
-      default: return launch_persistent(swiglu_bwd_vec<256, kBwdUnroll>, blocks, MOE_BWD_ARGS);
+      case 32: return launch_bwd(swiglu_bwd_vec<D, 32, U>, 32, MOE_BWD_ARGS);
+      case 64: return launch_bwd(swiglu_bwd_vec<D, 64, U>, 64, MOE_BWD_ARGS);
+      case 128: return launch_bwd(swiglu_bwd_vec<D, 128, U>, 128, MOE_BWD_ARGS);
+      default: return launch_bwd(swiglu_bwd_vec<D, 256, U>, 256, MOE_BWD_ARGS);
     }
   }
   switch (W) {
-    case 32: return launch_persistent(swiglu_bwd_scalar<32>, blocks, MOE_BWD_ARGS);
-    case 64: return launch_persistent(swiglu_bwd_scalar<64>, blocks, MOE_BWD_ARGS);
-    case 128: return launch_persistent(swiglu_bwd_scalar<128>, blocks, MOE_BWD_ARGS);
-    default: return launch_persistent(swiglu_bwd_scalar<256>, blocks, MOE_BWD_ARGS);
+    case 32: return launch_bwd(swiglu_bwd_scalar<D, 32>, 32, MOE_BWD_ARGS);
+    case 64: return launch_bwd(swiglu_bwd_scalar<D, 64>, 64, MOE_BWD_ARGS);
+    case 128: return launch_bwd(swiglu_bwd_scalar<D, 128>, 128, MOE_BWD_ARGS);
+    default: return launch_bwd(swiglu_bwd_scalar<D, 256>, 256, MOE_BWD_ARGS);
   }
 #undef MOE_BWD_ARGS
+}
+
+}  // namespace
+
+int launch_swiglu_clamped_fwd(const void* x, const float* probs, void* y, int64_t rows,
+                              int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
+                              moe_dtype dt, cudaStream_t stream) {
+  switch (dt) {
+    case MOE_BF16: return fwd<BF16>(x, probs, y, rows, inter, ld_x, ld_y, limit, stream);
+    case MOE_FP16: return fwd<F16>(x, probs, y, rows, inter, ld_x, ld_y, limit, stream);
+    default: return fwd<F32>(x, probs, y, rows, inter, ld_x, ld_y, limit, stream);
+  }
+}
+
+int launch_swiglu_clamped_bwd(const void* x, const float* probs, const void* grad_y,
+                              void* grad_x, float* grad_probs, int64_t rows, int64_t inter,
+                              int64_t ld_x, int64_t ld_gy, int64_t ld_gx, float limit,
+                              moe_dtype dt, cudaStream_t stream) {
+  switch (dt) {
+    case MOE_BF16:
+      return bwd<BF16>(x, probs, grad_y, grad_x, grad_probs, rows, inter, ld_x, ld_gy, ld_gx,
+                       limit, stream);
+    case MOE_FP16:
+      return bwd<F16>(x, probs, grad_y, grad_x, grad_probs, rows, inter, ld_x, ld_gy, ld_gx,
+                      limit, stream);
+    default:
+      return bwd<F32>(x, probs, grad_y, grad_x, grad_probs, rows, inter, ld_x, ld_gy, ld_gx,
+                      limit, stream);
+  }
 }
 
 }  // namespace moe

@@ -171,3 +171,52 @@ def test_swiglu_large_workload_sampled_rows(cuda_device, sigma):
     assert bool((gx[:, :inter][gate > L] == 0).all())
     assert bool((gx[:, inter:][(up > L) | (up < -L)] == 0).all())
     assert bool(torch.isfinite(y.float()).all()) and bool(torch.isfinite(gp).all())
+
+
+# ------------------------------------------------------- fp16 / fp32 storage
+
+ODT = {torch.float16: oracle.F16, torch.float32: oracle.F32}
+
+
+def _f32_bwd_scale(x, p, dy, limit):
+    """Magnitude of the terms of each grad_x element (float64), which bounds
+    the rounding error of an fp32 evaluation including the cancellation in
+    silu'(gc) = sigma (1 + gc (1 - sigma))."""
+    x = x.double()
+    inter = x.shape[1] // 2
+    gc = torch.clamp(x[:, :inter], max=limit)
+    uc = torch.clamp(x[:, inter:], -limit, limit)
+    sg = torch.sigmoid(gc)
+    a = (dy.double() * p.double().reshape(-1, 1)).abs()
+    return torch.cat([a * uc.abs() * sg * (1 + gc.abs() * (1 - sg)), a * (gc * sg).abs()], 1)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.float32])
+@pytest.mark.parametrize("rows,inter,limit", [(256, 512, 7.0), (300, 2048, 10.0),
+                                              (97, 1001, 7.0), (64, 40, float("inf"))])
+def test_swiglu_fp16_fp32_parity(cuda_device, dtype, rows, inter, limit):
+    d = inputs.swiglu_inputs(rows, inter, sigma=3.0, limit=7.0, plant_ties=True, seed=rows)
+    if dtype == torch.float32:
+        g = torch.Generator().manual_seed(inter)
+        x = torch.randn(rows, 2 * inter, generator=g) * 3.0
+        x[0, 0], x[1, inter] = limit if limit != INF else 1.0, -limit if limit != INF else 1.0
+        gy = torch.randn(rows, inter, generator=g)
+    else:
+        x, gy = d["x"].to(dtype), d["grad_y"].to(dtype)
+    p = d["probs"]
+    xd, pd, gyd = x.to(cuda_device), p.to(cuda_device), gy.to(cuda_device)
+    y = ops.swiglu_clamped_fwd(xd, pd, limit)
+    gx, gp = ops.swiglu_clamped_bwd(xd, pd, gyd, limit)
+    torch.cuda.synchronize()
+    dt = ODT[dtype]
+    y_ref = oracle.swiglu_clamped_fwd(bits(x), bits(p), limit, dt)
+    gx_ref, gp_ref, gabs = oracle.swiglu_clamped_bwd(bits(x), bits(p), bits(gy), limit, dt)
+    if dtype == torch.float16:
+        assert_within_ulp16(bits(y), y_ref, 1, kind="f16", what="fp16 y")
+        assert_within_ulp16(bits(gx), gx_ref, 1, kind="f16", what="fp16 grad_x")
+    else:
+        yg = bits(y)
+        assert (np.abs(yg - y_ref) <= 2 ** -18 * np.abs(y_ref) + 1e-35).all(), "fp32 y"
+        scale = _f32_bwd_scale(x, p, gy, limit).numpy()
+        assert (np.abs(bits(gx) - gx_ref) <= 2 ** -17 * scale + 1e-35).all(), "fp32 grad_x"
+    assert_sum_close(bits(gp).ravel(), gp_ref, gabs, 1e-5, "grad_probs")
