@@ -51,13 +51,14 @@ def _status(fn, *args):
 
 def test_swiglu_validation(lib):
     f = _abi.moe_swiglu_clamped_fwd
-    assert _status(f, FAKE, FAKE, FAKE, 4, 8, 16, 8, 7.0, _abi.MOE_FP16, 0) == _abi.MOE_ERR_DTYPE
+    assert _status(f, FAKE, FAKE, FAKE, 4, 8, 16, 8, 7.0, 7, 0) == _abi.MOE_ERR_DTYPE
     assert _status(f, FAKE, FAKE, FAKE, 4, 8, 15, 8, 7.0, _abi.MOE_BF16, 0) == _abi.MOE_ERR_SHAPE
     assert _status(f, FAKE, FAKE, FAKE, -1, 8, 16, 8, 7.0, _abi.MOE_BF16, 0) == _abi.MOE_ERR_SHAPE
     for bad in (0.0, -1.0, float("nan")):
         assert _status(f, FAKE, FAKE, FAKE, 4, 8, 16, 8, bad, _abi.MOE_BF16, 0) == _abi.MOE_ERR_LIMIT
     assert _status(f, None, FAKE, FAKE, 4, 8, 16, 8, 7.0, _abi.MOE_BF16, 0) == _abi.MOE_ERR_NULL
     assert _status(f, FAKE + 1, FAKE, FAKE, 4, 8, 16, 8, 7.0, _abi.MOE_BF16, 0) == _abi.MOE_ERR_ALIGN
+    assert _status(f, FAKE + 2, FAKE, FAKE, 4, 8, 16, 8, 7.0, _abi.MOE_FP32, 0) == _abi.MOE_ERR_ALIGN
     f(None, None, None, 0, 8, 16, 8, 7.0, _abi.MOE_BF16, 0)      # empty: a no-op
     b = _abi.moe_swiglu_clamped_bwd
     assert _status(b, FAKE, FAKE, FAKE, FAKE, None, 4, 8, 16, 8, 16, 7.0, 0, 0) == _abi.MOE_ERR_NULL
