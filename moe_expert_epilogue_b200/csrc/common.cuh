@@ -142,6 +142,21 @@ template <> __device__ __forceinline__ float round_to<F16>(float v) {
 }
 template <> __device__ __forceinline__ float round_to<F32>(float v) { return v; }
 
+// Round two fp32 values to the storage dtype and widen them back, with one
+// packed conversion (RNE) for the two.
+template <class D> __device__ __forceinline__ void round2(float& a, float& b);
+template <> __device__ __forceinline__ void round2<BF16>(float& a, float& b) {
+  const uint32_t w = pack_bf16x2(a, b);
+  a = bf16_lo(w);
+  b = bf16_hi(w);
+}
+template <> __device__ __forceinline__ void round2<F16>(float& a, float& b) {
+  const uint32_t w = pack_f16x2(a, b);
+  a = f16_to_f32((uint16_t)(w & 0xffffu));
+  b = f16_to_f32((uint16_t)(w >> 16));
+}
+template <> __device__ __forceinline__ void round2<F32>(float&, float&) {}
+
 // ------------------------------------------------- 8-element vector units
 
 // A chunk of 8 elements in registers as raw bits: one 16-byte word for the

@@ -91,7 +91,12 @@ epilogue_fused_kernel(const typename D::T* __restrict__ eo, const float* __restr
               float v[8];
               widen8<D>(raw[j], v);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) acc[i] = acc[i] + round_to<D>(__fmul_rn(v[i], p[j]));
+              for (int i = 0; i < 8; i += 2) {
+                float w0 = __fmul_rn(v[i], p[j]), w1 = __fmul_rn(v[i + 1], p[j]);
+                round2<D>(w0, w1);                      // step 1's rounding, two at a time
+                acc[i] = acc[i] + w0;
+                acc[i + 1] = acc[i + 1] + w1;
+              }
             }
           }
         }
@@ -99,7 +104,13 @@ epilogue_fused_kernel(const typename D::T* __restrict__ eo, const float* __restr
         widen8<D>(rs, vs);
         widen8<D>(rr, vr);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = vr[i] + round_to<D>(round_to<D>(acc[i]) + vs[i]);
+        for (int i = 0; i < 8; i += 2) {
+          round2<D>(acc[i], acc[i + 1]);                // step 2's rounding
+          float t0 = acc[i] + vs[i], t1 = acc[i + 1] + vs[i + 1];
+          round2<D>(t0, t1);                            // step 3's first rounding
+          acc[i] = vr[i] + t0;
+          acc[i + 1] = vr[i + 1] + t1;
+        }
         store8<D>(out + base + c * kVec, acc);
       }
     } else {
@@ -122,6 +133,105 @@ epilogue_fused_kernel(const typename D::T* __restrict__ eo, const float* __restr
   }
 }
 
+// Barrier-free variant for E <= 64: a warp owns one work item -- a token and
+// one of SPLIT equal column ranges of its hidden dimension -- at a time.  The
+// warp compacts the token's inverse-map row itself (two entries per lane,
+// already loaded during the previous item) into its own shared-memory list,
+// so warps never wait for each other; items = tokens * SPLIT keep the load
+// balanced across the persistent grid.
+template <class D, int SPLIT>
+__global__ void __launch_bounds__(kThreads)
+epilogue_fused_warp(const typename D::T* __restrict__ eo, const float* __restrict__ row_probs,
+                    int64_t max_rows, const int32_t* __restrict__ inv,
+                    const int32_t* __restrict__ valid_tokens,
+                    const typename D::T* __restrict__ shared, const typename D::T* residual,
+                    typename D::T* out, int64_t tokens, int64_t hidden, int E, int32_t* err) {
+  __shared__ int32_t s_list[kThreads / 32][64];
+  int64_t n = __ldg(valid_tokens);
+  if (n < 0 || n > tokens) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(err, MOE_DEVERR_COUNT);
+    n = n < 0 ? 0 : tokens;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
+  const int64_t items = n * SPLIT;
+  const int64_t cpr = hidden / kVec;
+  const int64_t cpi = (cpr + SPLIT - 1) / SPLIT;          // chunks per item
+  int32_t* list = s_list[warp];
+  int64_t it = (int64_t)blockIdx.x * (kThreads / 32) + warp;
+  if (it >= items) return;                                 // warp-uniform
+  int32_t p0, p1;
+  {
+    const int32_t* row = inv + (it / SPLIT) * E;
+    p0 = lane < E ? __ldg(row + lane) : -1;
+    p1 = lane + 32 < E ? __ldg(row + lane + 32) : -1;
+  }
+  constexpr int B = kRowsAhead<D>;
+  for (; it < items; it += nwarps) {
+    const int64_t t = it / SPLIT;
+    __syncwarp();                                          // the previous list is consumed
+    const int count = compact_pair(p0, p1, max_rows, list, err, lane);
+    __syncwarp();
+    const int64_t itn = it + nwarps;
+    if (itn < items) {                                     // next item's entries, in flight
+      const int32_t* row = inv + (itn / SPLIT) * E;
+      p0 = lane < E ? __ldg(row + lane) : -1;
+      p1 = lane + 32 < E ? __ldg(row + lane + 32) : -1;
+    }
+    const int64_t base = t * hidden;
+    const int64_t c_end = min(cpr, (it % SPLIT + 1) * cpi);
+    for (int64_t c = (it % SPLIT) * cpi + lane; c < c_end; c += 32) {
+      const Raw8<D> rs = load8<D>(shared + base + c * kVec);
+      const Raw8<D> rr = load8<D, false>(residual + base + c * kVec);  // may alias out
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+      for (int j0 = 0; j0 < count; j0 += B) {
+        Raw8<D> raw[B];
+        float p[B];
+#pragma unroll
+        for (int j = 0; j < B; ++j) {
+          if (j0 + j < count) {
+            const int64_t row = list[j0 + j];
+            raw[j] = load8<D>(eo + row * hidden + c * kVec);
+            p[j] = __ldg(row_probs + row);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < B; ++j) {
+          if (j0 + j < count) {
+            float v[8];
+            widen8<D>(raw[j], v);
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+              float w0 = __fmul_rn(v[i], p[j]), w1 = __fmul_rn(v[i + 1], p[j]);
+              round2<D>(w0, w1);
+              acc[i] = acc[i] + w0;
+              acc[i + 1] = acc[i + 1] + w1;
+            }
+          }
+        }
+      }
+      float vs[8], vr[8];
+      widen8<D>(rs, vs);
+      widen8<D>(rr, vr);
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        round2<D>(acc[i], acc[i + 1]);
+        float t0 = acc[i] + vs[i], t1 = acc[i + 1] + vs[i + 1];
+        round2<D>(t0, t1);
+        acc[i] = vr[i] + t0;
+        acc[i + 1] = vr[i + 1] + t1;
+      }
+      store8<D>(out + base + c * kVec, acc);
+    }
+  }
+}
+
+#ifndef MOE_FUSED_WARP_ITEMS
+#define MOE_FUSED_WARP_ITEMS 1
+#endif
+
 template <class D>
 int launch(const void* eo, const float* row_probs, int64_t max_rows, const int32_t* inv,
            const int32_t* valid_tokens, const void* shared, const void* residual, void* out,
@@ -129,6 +239,23 @@ int launch(const void* eo, const float* row_probs, int64_t max_rows, const int32
   using T = typename D::T;
   const bool vec = hidden % kVec == 0 && aligned16(eo) && aligned16(shared) &&
                    aligned16(residual) && aligned16(out);
+  if (MOE_FUSED_WARP_ITEMS && vec && E <= 64) {
+    // SPLIT: items per token, the largest power of two <= chunks per row / 128
+    const int64_t cpr = hidden / kVec;
+    const int split = cpr >= 1024 ? 8 : cpr >= 512 ? 4 : cpr >= 256 ? 2 : 1;
+    auto k = split == 8 ? epilogue_fused_warp<D, 8> : split == 4 ? epilogue_fused_warp<D, 4>
+           : split == 2 ? epilogue_fused_warp<D, 2> : epilogue_fused_warp<D, 1>;
+    int grid;
+    const int64_t warps = tokens * split;
+    if (int rc = persistent_grid((const void*)k, 0, (warps + kThreads / 32 - 1) / (kThreads / 32),
+                                 &grid))
+      return rc;
+    k<<<grid, kThreads, 0, stream>>>(static_cast<const T*>(eo), row_probs, max_rows, inv,
+                                     valid_tokens, static_cast<const T*>(shared),
+                                     static_cast<const T*>(residual), static_cast<T*>(out),
+                                     tokens, hidden, E, err);
+    return check_launch();
+  }
   const size_t smem = 2 * (size_t)E * sizeof(int32_t);
   auto k = vec ? (E <= 64 ? epilogue_fused_kernel<D, true, true>
                           : epilogue_fused_kernel<D, true, false>)

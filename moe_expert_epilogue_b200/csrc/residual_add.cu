@@ -50,7 +50,12 @@ residual_add_vec(const typename D::T* e, const typename D::T* s, const typename 
         widen8<D>(rs[k], vs);
         widen8<D>(rr[k], vr);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = add_pair<D>(ve[i], vs[i], vr[i]);
+        for (int i = 0; i < 8; i += 2) {
+          float t0 = ve[i] + vs[i], t1 = ve[i + 1] + vs[i + 1];
+          round2<D>(t0, t1);                            // the expert sum, rounded to D
+          o[i] = vr[i] + t0;
+          o[i + 1] = vr[i + 1] + t1;
+        }
         store8<D>(out + c * kVec, o);
       }
     }
