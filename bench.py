@@ -233,15 +233,28 @@ def time_launches(fn, reps, device):
     return a.elapsed_time(b) / reps
 
 
-def measure_next_rows(device, seed, reps, peak):
+NEXT_ROWS = ("weighted_silu_mul_bounded", "epilogue_fused")
+
+
+def measure_next_rows(device, seed, reps, peak, scale=1.0, only=None):
     """The ops beyond the step: the device-bounded weighted SwiGLU and the fused
     router-weight -> unpermute -> residual chain (against the same chain as
     three launches).  Timed after the step, outside its timed region."""
     from moe_expert_epilogue_b200 import inputs, ops
     out = {}
-    T, K, E, A, H = (PERMUTED["tokens"], PERMUTED["top_k"], PERMUTED["experts"],
-                     PERMUTED["align"], PERMUTED["hidden"])
+    T = scaled(scale)["permuted"]["tokens"]
+    K, E, A, H = PERMUTED["top_k"], PERMUTED["experts"], PERMUTED["align"], PERMUTED["hidden"]
     rows, half_n = T * K, PERMUTED["width"]
+    if only in (None, "weighted_silu_mul_bounded"):
+        out.update(_measure_bounded(device, seed, reps, peak, rows, half_n))
+    if only in (None, "epilogue_fused"):
+        out.update(_measure_fused(device, seed, reps, peak, T, K, E, A, H))
+    return out
+
+
+def _measure_bounded(device, seed, reps, peak, rows, half_n):
+    from moe_expert_epilogue_b200 import ops
+    out = {}
     g = torch.Generator(device=device).manual_seed(seed + 7)
     y = (torch.randn(rows, 2 * half_n, generator=g, device=device) * 3).to(torch.bfloat16)
     w = torch.rand(rows, generator=g, device=device)
@@ -252,7 +265,12 @@ def measure_next_rows(device, seed, reps, peak):
     out["weighted_silu_mul_bounded"] = {
         "shape": f"rows {rows} (all live), half_n {half_n}", "us": round(ms * 1e3, 2),
         "bytes": nb, "gbs": round(nb / ms / 1e6, 1), "frac": round(nb / ms / 1e6 / peak, 4)}
-    del y, w, o
+    return out
+
+
+def _measure_fused(device, seed, reps, peak, T, K, E, A, H):
+    from moe_expert_epilogue_b200 import inputs, ops
+    out = {}
     rt = inputs.routing(T, K, E, A, seed=seed + 2, device=device)
     eo = inputs.expert_output_input(rt, H, seed=seed + 5, device=device)
     pm = rt.permutation_map
@@ -432,8 +450,17 @@ def run_ours(args):
         barrier(device)
 
     only = set(args.kernel.split(",")) if args.kernel else None
+    if only and len(only) == 1 and next(iter(only)) in NEXT_ROWS:
+        # a next-row op alone (profiling captures): warm-ups, then --steps launches
+        peak, _ = hbm_peak()
+        res = measure_next_rows(device, 1000 * rank, args.steps, peak, args.scale,
+                                only=next(iter(only)))
+        if rank == 0:
+            print(json.dumps({"kernel": args.kernel, "scale": args.scale, "result": res}),
+                  flush=True)
+        return
     if only and not only <= set(ORDER):
-        raise SystemExit(f"unknown --kernel {args.kernel}; choose from {ORDER}")
+        raise SystemExit(f"unknown --kernel {args.kernel}; choose from {ORDER + list(NEXT_ROWS)}")
     batch = Batch(device, seed=1000 * rank, scale=args.scale, kernels=only)
     kernels = batch.kernels()
     nbytes = algorithmic_bytes(batch.rt.n_used, args.scale)
@@ -488,7 +515,7 @@ def run_ours(args):
 
     e2e = None
     if not args.no_e2e and not args.kernel:
-        e2e = run_e2e(batch, kernels, nbytes, args, device)
+        e2e = run_e2e(batch, nbytes, args, device, 1000 * rank)
     n_used, n_kernels = batch.rt.n_used, len(kernels)
     next_rows = None
     if not args.kernel and not args.no_next_rows:
@@ -544,10 +571,16 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_e2e(batch, kernels, nbytes, args, device):
+def run_e2e(batch, nbytes, args, device, seed):
     """The same step through the public API with inputs in pinned host memory:
-    host->device copies of every input, the kernels, and device->host copies
-    of every output, all inside the timed region."""
+    every step copies all of its inputs host -> device, runs the kernels and
+    copies all of its outputs device -> host, all inside the timed region.
+    Steps are pipelined as a user would drive them: two device buffer sets,
+    a copy-in stream, the compute stream and a copy-out stream, so step k's
+    kernels overlap step k+1's inputs and step k-1's outputs on the host link.
+    Events order every reuse of a buffer set."""
+    sets = [batch, Batch(device, seed=seed + 7, scale=args.scale)]
+    kernel_sets = [b.kernels() for b in sets]
     host_in = {k: torch.empty_like(getattr(batch, k), device="cpu").pin_memory()
                for k in batch.inputs}
     for k, h in host_in.items():
@@ -556,34 +589,51 @@ def run_e2e(batch, kernels, nbytes, args, device):
                 for k in batch.outputs}
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    stream = torch.cuda.current_stream(device)
+    s_cmp = torch.cuda.current_stream(device)
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = {name: [torch.cuda.Event(), torch.cuda.Event()] for name in ("in", "cmp", "out")}
+    for i in range(2):                     # every buffer set starts free
+        ev["cmp"][i].record(s_cmp)
+        ev["out"][i].record(s_cmp)
 
-    def step():
-        for k, h in host_in.items():
-            getattr(batch, k).copy_(h, non_blocking=True)
-        for _, fn in kernels:
-            fn()
-        for k, h in host_out.items():
-            h.copy_(getattr(batch, k), non_blocking=True)
+    def step(k):
+        i, b = k % 2, sets[k % 2]
+        s_in.wait_event(ev["cmp"][i])      # step k-2's kernels are done with set i's inputs
+        with torch.cuda.stream(s_in):
+            for name, h in host_in.items():
+                getattr(b, name).copy_(h, non_blocking=True)
+        ev["in"][i].record(s_in)
+        s_cmp.wait_event(ev["in"][i])
+        s_cmp.wait_event(ev["out"][i])     # step k-2's outputs of set i have left
+        with torch.cuda.stream(s_cmp):
+            for _, fn in kernel_sets[i]:
+                fn()
+        ev["cmp"][i].record(s_cmp)
+        s_out.wait_event(ev["cmp"][i])
+        with torch.cuda.stream(s_out):
+            for name, h in host_out.items():
+                h.copy_(getattr(b, name), non_blocking=True)
+        ev["out"][i].record(s_out)
 
-    for _ in range(max(1, min(args.warmup, 2))):
-        step()
+    for k in range(2):
+        step(k)
     torch.cuda.synchronize(device)
     n = args.e2e_steps
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(device)
     torch.cuda.synchronize(device)
-    a.record(stream)
-    for _ in range(n):
-        step()
-    b.record(stream)
+    a.record(s_in)
+    for k in range(n):
+        step(k)
+    z.record(s_out)
     torch.cuda.synchronize(device)
     barrier(device)
-    ms = max_over_ranks(a.elapsed_time(b), device)
+    ms = max_over_ranks(a.elapsed_time(z), device)
     _, _, world = dist_env()
     return {"value": round(aggregate_value(sum(nbytes.values()), n, world, ms * 1e-3), 2),
             "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": n, "ms_per_step": round(ms / n, 3)}
+            "steps": n, "ms_per_step": round(ms / n, 3),
+            "pipeline": "2 device buffer sets; copy-in, compute and copy-out streams"}
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -699,7 +749,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--cpu-sample", type=float, default=0.25,
                     help="fraction of the rows of every op the CPU oracle runs")
     ap.add_argument("--no-e2e", action="store_true")
