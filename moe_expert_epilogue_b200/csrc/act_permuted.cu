@@ -60,6 +60,7 @@ act_permuted_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ out,
                     const int32_t* __restrict__ pmap, const int32_t* __restrict__ n_used,
                     const float* __restrict__ probs, int64_t num_probs, int64_t max_rows,
                     int64_t width, float scale, int zero_padding, int32_t* err) {
+  pdl_prologue();
   const int64_t rows = live_rows(n_used, max_rows, err);
   const float inv_scale = 1.0f / scale;
   constexpr int64_t unit = VEC ? kVec : 1;
@@ -159,7 +160,7 @@ int launch_act(const uint16_t* x, uint16_t* out, const int32_t* pmap, const int3
   if (int rc = persistent_grid((const void*)k, 0, (max_rows + warps_per_block - 1) / warps_per_block,
                                &grid))
     return rc;
-  k<<<grid, kThreads, 0, stream>>>(x, out, pmap, n_used, probs, num_probs, max_rows, width,
+  launch_kernel(k, grid, 0, stream, x, out, pmap, n_used, probs, num_probs, max_rows, width,
                                    scale, zero_padding, err);
   return check_launch();
 }

@@ -302,6 +302,24 @@ struct RowCursor {
   }
 };
 
+// Programmatic dependent launch (PDL).  Every kernel of the library is
+// launched with programmatic stream serialisation allowed and begins with
+// this prologue: griddepcontrol.wait blocks until the grids this one depends
+// on (the previous work in the stream) have completed and their memory is
+// visible -- so nothing is read early -- and launch_dependents lets the next
+// kernel's CTAs be scheduled onto SMs as this kernel's CTAs retire, hiding
+// the launch latency and the tail of each kernel boundary.  Without a
+// programmatic dependency both instructions are no-ops.
+#ifndef MOE_PDL
+#define MOE_PDL 1
+#endif
+__device__ __forceinline__ void pdl_prologue() {
+#if MOE_PDL
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
+}
+
 // Device-side error word: set bits, never trap.
 __device__ __forceinline__ void flag_error(int32_t* err, int32_t bits) {
   if (err) atomicOr(err, bits);

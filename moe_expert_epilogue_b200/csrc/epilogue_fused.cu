@@ -38,6 +38,7 @@ epilogue_fused_kernel(const typename D::T* __restrict__ eo, const float* __restr
                       const int32_t* __restrict__ valid_tokens,
                       const typename D::T* __restrict__ shared, const typename D::T* residual,
                       typename D::T* out, int64_t tokens, int64_t hidden, int E, int32_t* err) {
+  pdl_prologue();
   extern __shared__ int32_t s_list[];  // [2][E]
   __shared__ int s_count[2];
   int64_t n = __ldg(valid_tokens);
@@ -146,6 +147,7 @@ epilogue_fused_warp(const typename D::T* __restrict__ eo, const float* __restric
                     const int32_t* __restrict__ valid_tokens,
                     const typename D::T* __restrict__ shared, const typename D::T* residual,
                     typename D::T* out, int64_t tokens, int64_t hidden, int E, int32_t* err) {
+  pdl_prologue();
   __shared__ int32_t s_list[kThreads / 32][64];
   int64_t n = __ldg(valid_tokens);
   if (n < 0 || n > tokens) {
@@ -250,7 +252,7 @@ int launch(const void* eo, const float* row_probs, int64_t max_rows, const int32
     if (int rc = persistent_grid((const void*)k, 0, (warps + kThreads / 32 - 1) / (kThreads / 32),
                                  &grid))
       return rc;
-    k<<<grid, kThreads, 0, stream>>>(static_cast<const T*>(eo), row_probs, max_rows, inv,
+    launch_kernel(k, grid, 0, stream, static_cast<const T*>(eo), row_probs, max_rows, inv,
                                      valid_tokens, static_cast<const T*>(shared),
                                      static_cast<const T*>(residual), static_cast<T*>(out),
                                      tokens, hidden, E, err);
@@ -263,7 +265,7 @@ int launch(const void* eo, const float* row_probs, int64_t max_rows, const int32
                           : epilogue_fused_kernel<D, false, false>);
   int grid;
   if (int rc = persistent_grid((const void*)k, smem, tokens > 0 ? tokens : 1, &grid)) return rc;
-  k<<<grid, kThreads, smem, stream>>>(static_cast<const T*>(eo), row_probs, max_rows, inv,
+  launch_kernel(k, grid, smem, stream, static_cast<const T*>(eo), row_probs, max_rows, inv,
                                       valid_tokens, static_cast<const T*>(shared),
                                       static_cast<const T*>(residual), static_cast<T*>(out),
                                       tokens, hidden, E, err);

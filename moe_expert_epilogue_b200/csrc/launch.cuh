@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "common.cuh"
 #include "moe_epilogue.h"
 
 namespace moe {
@@ -19,6 +20,25 @@ int persistent_grid(const void* kernel, size_t smem, int64_t useful_blocks, int*
 
 // MOE_ERR_CUDA if the launch just issued failed.
 int check_launch();
+
+// Enqueue kernel<<<grid, kThreads, smem, stream>>>(args...) with programmatic
+// stream serialisation allowed (see pdl_prologue); a failure is left in the
+// runtime's error state for check_launch().
+template <typename... KArgs, typename... Args>
+inline void launch_kernel(void (*kernel)(KArgs...), int grid, size_t smem, cudaStream_t stream,
+                          Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = MOE_PDL;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  (void)cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

@@ -27,6 +27,7 @@ template <class D>
 __global__ void __launch_bounds__(kThreads)
 residual_add_vec(const typename D::T* e, const typename D::T* s, const typename D::T* r,
                  typename D::T* out, int64_t numel) {
+  pdl_prologue();
   const int64_t chunks = numel / kVec;
   const int64_t S = (int64_t)gridDim.x * kThreads;
   const int64_t t0 = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -70,6 +71,7 @@ template <class D>
 __global__ void __launch_bounds__(kThreads)
 residual_add_scalar(const typename D::T* e, const typename D::T* s, const typename D::T* r,
                     typename D::T* out, int64_t numel) {
+  pdl_prologue();
   const int64_t S = (int64_t)gridDim.x * kThreads;
   for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < numel; i += S)
     store1<D>(out + i, add_pair<D>(load1<D>(e + i), load1<D>(s + i), load1c<D>(r + i)));
@@ -88,13 +90,13 @@ int launch(const void* e, const void* s, const void* r, void* out, int64_t numel
     if (int rc = persistent_grid((const void*)k, 0, chunks > 0 ? (chunks + per_block - 1) / per_block : 1,
                                  &grid))
       return rc;
-    k<<<grid, kThreads, 0, stream>>>(static_cast<const T*>(e), static_cast<const T*>(s),
+    launch_kernel(k, grid, 0, stream, static_cast<const T*>(e), static_cast<const T*>(s),
                                      static_cast<const T*>(r), static_cast<T*>(out), numel);
   } else {
     auto k = residual_add_scalar<D>;
     if (int rc = persistent_grid((const void*)k, 0, (numel + kThreads - 1) / kThreads, &grid))
       return rc;
-    k<<<grid, kThreads, 0, stream>>>(static_cast<const T*>(e), static_cast<const T*>(s),
+    launch_kernel(k, grid, 0, stream, static_cast<const T*>(e), static_cast<const T*>(s),
                                      static_cast<const T*>(r), static_cast<T*>(out), numel);
   }
   return check_launch();

@@ -23,6 +23,7 @@ template <class DI, class DO>
 __global__ void __launch_bounds__(kThreads)
 scale_rows_vec(const typename DI::T* __restrict__ in, const float* __restrict__ probs,
                typename DO::T* __restrict__ out, int64_t rows, int64_t hidden) {
+  pdl_prologue();
   const int64_t cpr = hidden / kVec;
   const int64_t total = rows * cpr;
   const int64_t S = (int64_t)gridDim.x * kThreads;
@@ -59,6 +60,7 @@ template <class DI, class DO>
 __global__ void __launch_bounds__(kThreads)
 scale_rows_scalar(const typename DI::T* __restrict__ in, const float* __restrict__ probs,
                   typename DO::T* __restrict__ out, int64_t rows, int64_t hidden) {
+  pdl_prologue();
   const int64_t total = rows * hidden;
   const int64_t S = (int64_t)gridDim.x * kThreads;
   int64_t q = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -91,6 +93,7 @@ __global__ void __launch_bounds__(kThreads)
 rw_bwd_rows(const typename DG::T* __restrict__ g, const typename DX::T* __restrict__ x,
             const float* __restrict__ probs, typename DX::T* __restrict__ gx,
             float* __restrict__ gp, int64_t rows, int64_t hidden) {
+  pdl_prologue();
   constexpr int G = kThreads / W;
   __shared__ float red[2][kThreads / 32];
   const int sub = threadIdx.x / W, lane = threadIdx.x % W;
@@ -163,13 +166,13 @@ int launch_scale(const void* in, const float* probs, void* out, int64_t rows, in
     if (int rc = persistent_grid((const void*)k, 0,
                                  (units + kThreads * kUnroll - 1) / (kThreads * kUnroll), &grid))
       return rc;
-    k<<<grid, kThreads, 0, stream>>>(i, probs, o, rows, hidden);
+    launch_kernel(k, grid, 0, stream, i, probs, o, rows, hidden);
   } else {
     auto k = scale_rows_scalar<DI, DO>;
     if (int rc = persistent_grid((const void*)k, 0, (rows * hidden + kThreads - 1) / kThreads,
                                  &grid))
       return rc;
-    k<<<grid, kThreads, 0, stream>>>(i, probs, o, rows, hidden);
+    launch_kernel(k, grid, 0, stream, i, probs, o, rows, hidden);
   }
   return check_launch();
 }
@@ -181,7 +184,7 @@ int launch_rows(const void* g, const void* x, const float* probs, void* gx, floa
   int grid;
   const int64_t blocks = (rows + kThreads / W - 1) / (kThreads / W);
   if (int rc = persistent_grid((const void*)k, 0, blocks, &grid)) return rc;
-  k<<<grid, kThreads, 0, stream>>>(static_cast<const typename DG::T*>(g),
+  launch_kernel(k, grid, 0, stream, static_cast<const typename DG::T*>(g),
                                    static_cast<const typename DX::T*>(x), probs,
                                    static_cast<typename DX::T*>(gx), gp, rows, hidden);
   return check_launch();

@@ -59,6 +59,7 @@ __global__ void __launch_bounds__(kThreads)
 swiglu_fwd_rows(const typename D::T* __restrict__ x, const float* __restrict__ probs,
                 typename D::T* __restrict__ y, int64_t rows, int64_t inter, int64_t ld_x,
                 int64_t ld_y, float L) {
+  pdl_prologue();
   const int64_t cpr = inter / kVec;
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
@@ -100,6 +101,7 @@ __global__ void __launch_bounds__(kThreads)
 swiglu_fwd_vec(const typename D::T* __restrict__ x, const float* __restrict__ probs,
                typename D::T* __restrict__ y, int64_t rows, int64_t inter, int64_t ld_x,
                int64_t ld_y, float L) {
+  pdl_prologue();
   const int64_t cpr = inter / kVec;
   const int64_t total = rows * cpr;
   const int64_t S = (int64_t)gridDim.x * kThreads;
@@ -142,6 +144,7 @@ __global__ void __launch_bounds__(kThreads)
 swiglu_fwd_scalar(const typename D::T* __restrict__ x, const float* __restrict__ probs,
                   typename D::T* __restrict__ y, int64_t rows, int64_t inter, int64_t ld_x,
                   int64_t ld_y, float L) {
+  pdl_prologue();
   const int64_t total = rows * inter;
   const int64_t S = (int64_t)gridDim.x * kThreads;
   int64_t q = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -183,6 +186,7 @@ swiglu_bwd_vec(const typename D::T* __restrict__ x, const float* __restrict__ pr
                const typename D::T* __restrict__ gy, typename D::T* __restrict__ gx,
                float* __restrict__ gp, int64_t rows, int64_t inter, int64_t ld_x,
                int64_t ld_gy, int64_t ld_gx, float L) {
+  pdl_prologue();
   constexpr int G = kThreads / W;
   __shared__ float red[2][kThreads / 32];
   const int sub = threadIdx.x / W, lane = threadIdx.x % W;
@@ -240,6 +244,7 @@ swiglu_bwd_scalar(const typename D::T* __restrict__ x, const float* __restrict__
                   const typename D::T* __restrict__ gy, typename D::T* __restrict__ gx,
                   float* __restrict__ gp, int64_t rows, int64_t inter, int64_t ld_x,
                   int64_t ld_gy, int64_t ld_gx, float L) {
+  pdl_prologue();
   constexpr int G = kThreads / W;
   __shared__ float red[2][kThreads / 32];
   const int sub = threadIdx.x / W, lane = threadIdx.x % W;
@@ -311,7 +316,7 @@ int fwd(const void* xv, const float* probs, void* yv, int64_t rows, int64_t inte
     if (int rc = persistent_grid((const void*)k, 0, (rows + kThreads / 32 - 1) / (kThreads / 32),
                                  &grid))
       return rc;
-    k<<<grid, kThreads, 0, stream>>>(x, probs, y, rows, inter, ld_x, ld_y, limit);
+    launch_kernel(k, grid, 0, stream, x, probs, y, rows, inter, ld_x, ld_y, limit);
   } else if (vec) {
     constexpr int U = unroll_for<D>(MOE_SWIGLU_FWD_UNROLL);
     auto k = swiglu_fwd_vec<D, U>;
@@ -319,13 +324,13 @@ int fwd(const void* xv, const float* probs, void* yv, int64_t rows, int64_t inte
     if (int rc = persistent_grid((const void*)k, 0, (units + kThreads * U - 1) / (kThreads * U),
                                  &grid))
       return rc;
-    k<<<grid, kThreads, 0, stream>>>(x, probs, y, rows, inter, ld_x, ld_y, limit);
+    launch_kernel(k, grid, 0, stream, x, probs, y, rows, inter, ld_x, ld_y, limit);
   } else {
     auto k = swiglu_fwd_scalar<D>;
     if (int rc = persistent_grid((const void*)k, 0, (rows * inter + kThreads - 1) / kThreads,
                                  &grid))
       return rc;
-    k<<<grid, kThreads, 0, stream>>>(x, probs, y, rows, inter, ld_x, ld_y, limit);
+    launch_kernel(k, grid, 0, stream, x, probs, y, rows, inter, ld_x, ld_y, limit);
   }
   return check_launch();
 }
@@ -337,7 +342,7 @@ int launch_bwd(K kernel, int W, cudaStream_t stream, const T* x, const float* pr
   int grid;
   const int64_t blocks = (rows + kThreads / W - 1) / (kThreads / W);
   if (int rc = persistent_grid((const void*)kernel, 0, blocks, &grid)) return rc;
-  kernel<<<grid, kThreads, 0, stream>>>(x, probs, gy, gx, gp, rows, inter, ld_x, ld_gy, ld_gx, L);
+  launch_kernel(kernel, grid, 0, stream, x, probs, gy, gx, gp, rows, inter, ld_x, ld_gy, ld_gx, L);
   return check_launch();
 }
 

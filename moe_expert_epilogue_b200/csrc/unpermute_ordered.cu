@@ -37,6 +37,7 @@ unpermute_kernel(const typename DI::T* __restrict__ eo, int64_t max_rows,
                  const int32_t* __restrict__ inv, const int32_t* __restrict__ valid_tokens,
                  typename DO::T* __restrict__ out, int64_t tokens, int64_t hidden, int E,
                  int32_t* err) {
+  pdl_prologue();
   extern __shared__ int32_t s_list[];  // [2][E]
   __shared__ int s_count[2];
   int64_t n = __ldg(valid_tokens);
@@ -118,7 +119,7 @@ int launch_unpermute(const void* eo, int64_t max_rows, const int32_t* inv,
   }
   int grid;
   if (int rc = persistent_grid((const void*)k, smem, tokens > 0 ? tokens : 1, &grid)) return rc;
-  k<<<grid, kThreads, smem, stream>>>(static_cast<const typename DI::T*>(eo), max_rows, inv,
+  launch_kernel(k, grid, smem, stream, static_cast<const typename DI::T*>(eo), max_rows, inv,
                                       valid_tokens, static_cast<typename DO::T*>(out), tokens,
                                       hidden, E, err);
   return check_launch();

@@ -26,6 +26,7 @@ __global__ void __launch_bounds__(kThreads)
 weighted_silu_bounded_kernel(const uint16_t* __restrict__ y, const float* __restrict__ w,
                              uint16_t* __restrict__ out, const int64_t* __restrict__ bound_p,
                              int64_t rows, int64_t half_n, int32_t* err) {
+  pdl_prologue();
   int64_t bound = __ldg(bound_p);
   const int64_t total = rows * half_n;
   if (bound < 0 || bound > total) {
@@ -93,7 +94,7 @@ int launch_weighted_silu_mul_bounded(const uint16_t* y, const float* weights, ui
                                       &grid)) {
     return rc;
   }
-  k<<<grid, kThreads, 0, stream>>>(y, weights, out, bound_elems, rows, half_n, dev_err);
+  launch_kernel(k, grid, 0, stream, y, weights, out, bound_elems, rows, half_n, dev_err);
   return check_launch();
 }
 
