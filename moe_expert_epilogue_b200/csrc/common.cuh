@@ -313,10 +313,15 @@ struct RowCursor {
 #ifndef MOE_PDL
 #define MOE_PDL 1
 #endif
+#ifndef MOE_PDL_TRIGGER
+#define MOE_PDL_TRIGGER 1
+#endif
 __device__ __forceinline__ void pdl_prologue() {
 #if MOE_PDL
   asm volatile("griddepcontrol.wait;" ::: "memory");
+#if MOE_PDL_TRIGGER
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
 #endif
 }
 

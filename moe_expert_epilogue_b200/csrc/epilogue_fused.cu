@@ -140,8 +140,15 @@ epilogue_fused_kernel(const typename D::T* __restrict__ eo, const float* __restr
 // already loaded during the previous item) into its own shared-memory list,
 // so warps never wait for each other; items = tokens * SPLIT keep the load
 // balanced across the persistent grid.
+// Three resident CTAs per SM (at most 85 registers a thread): more warps to
+// hide the gather latency; measured 126 us against 138 us with the compiler's
+// own choice (102 registers, two CTAs) at 8192 tokens x top-8, hidden 4096.
+#ifndef MOE_FUSED_MIN_BLOCKS
+#define MOE_FUSED_MIN_BLOCKS 3
+#endif
+
 template <class D, int SPLIT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, MOE_FUSED_MIN_BLOCKS)
 epilogue_fused_warp(const typename D::T* __restrict__ eo, const float* __restrict__ row_probs,
                     int64_t max_rows, const int32_t* __restrict__ inv,
                     const int32_t* __restrict__ valid_tokens,

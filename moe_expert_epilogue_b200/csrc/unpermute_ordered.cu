@@ -103,11 +103,98 @@ unpermute_kernel(const typename DI::T* __restrict__ eo, int64_t max_rows,
   }
 }
 
+// Barrier-free variant for E <= 64 (the unpermute counterpart of the fused
+// epilogue's): a warp owns one work item -- a token and one of SPLIT equal
+// column ranges of its hidden dimension -- compacts the token's inverse-map
+// row itself (entries loaded during the previous item) into its own list, and
+// never waits for the other warps.
+template <class DI, class DO, int SPLIT>
+__global__ void __launch_bounds__(kThreads)
+unpermute_warp(const typename DI::T* __restrict__ eo, int64_t max_rows,
+               const int32_t* __restrict__ inv, const int32_t* __restrict__ valid_tokens,
+               typename DO::T* __restrict__ out, int64_t tokens, int64_t hidden, int E,
+               int32_t* err) {
+  pdl_prologue();
+  __shared__ int32_t s_list[kThreads / 32][64];
+  int64_t n = __ldg(valid_tokens);
+  if (n < 0 || n > tokens) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(err, MOE_DEVERR_COUNT);
+    n = n < 0 ? 0 : tokens;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
+  const int64_t items = n * SPLIT;
+  const int64_t cpr = hidden / kVec;
+  const int64_t cpi = (cpr + SPLIT - 1) / SPLIT;
+  int32_t* list = s_list[warp];
+  int64_t it = (int64_t)blockIdx.x * (kThreads / 32) + warp;
+  if (it >= items) return;                                 // warp-uniform
+  int32_t p0, p1;
+  {
+    const int32_t* row = inv + (it / SPLIT) * E;
+    p0 = lane < E ? __ldg(row + lane) : -1;
+    p1 = lane + 32 < E ? __ldg(row + lane + 32) : -1;
+  }
+  constexpr int B = kBatch<DI>;
+  for (; it < items; it += nwarps) {
+    const int64_t t = it / SPLIT;
+    __syncwarp();
+    const int count = compact_pair(p0, p1, max_rows, list, err, lane);
+    __syncwarp();
+    const int64_t itn = it + nwarps;
+    if (itn < items) {
+      const int32_t* row = inv + (itn / SPLIT) * E;
+      p0 = lane < E ? __ldg(row + lane) : -1;
+      p1 = lane + 32 < E ? __ldg(row + lane + 32) : -1;
+    }
+    const int64_t c_end = min(cpr, (it % SPLIT + 1) * cpi);
+    for (int64_t c = (it % SPLIT) * cpi + lane; c < c_end; c += 32) {
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+      for (int j0 = 0; j0 < count; j0 += B) {
+        Raw8<DI> raw[B];
+#pragma unroll
+        for (int j = 0; j < B; ++j)
+          if (j0 + j < count) raw[j] = load8<DI>(eo + (int64_t)list[j0 + j] * hidden + c * kVec);
+#pragma unroll
+        for (int j = 0; j < B; ++j) {
+          if (j0 + j < count) {
+            float v[8];
+            widen8<DI>(raw[j], v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = acc[i] + v[i];
+          }
+        }
+      }
+      store8<DO>(out + t * hidden + c * kVec, acc);
+    }
+  }
+}
+
+#ifndef MOE_UNPERMUTE_WARP_ITEMS
+#define MOE_UNPERMUTE_WARP_ITEMS 1
+#endif
+
 template <class DI, class DO>
 int launch_unpermute(const void* eo, int64_t max_rows, const int32_t* inv,
                      const int32_t* valid_tokens, void* out, int64_t tokens, int64_t hidden,
                      int E, int32_t* err, cudaStream_t stream) {
   const bool vec = hidden % kVec == 0 && aligned16(eo) && aligned16(out);
+  if (MOE_UNPERMUTE_WARP_ITEMS && vec && E <= 64) {
+    const int64_t cpr = hidden / kVec;
+    const int split = cpr >= 1024 ? 8 : cpr >= 512 ? 4 : cpr >= 256 ? 2 : 1;
+    auto k = split == 8 ? unpermute_warp<DI, DO, 8> : split == 4 ? unpermute_warp<DI, DO, 4>
+           : split == 2 ? unpermute_warp<DI, DO, 2> : unpermute_warp<DI, DO, 1>;
+    int grid;
+    const int64_t warps = tokens * split;
+    if (int rc = persistent_grid((const void*)k, 0, (warps + kThreads / 32 - 1) / (kThreads / 32),
+                                 &grid))
+      return rc;
+    launch_kernel(k, grid, 0, stream, static_cast<const typename DI::T*>(eo), max_rows, inv,
+                  valid_tokens, static_cast<typename DO::T*>(out), tokens, hidden, E, err);
+    return check_launch();
+  }
   const size_t smem = 2 * (size_t)E * sizeof(int32_t);
   auto k = vec ? (E <= 64 ? unpermute_kernel<DI, DO, true, true> : unpermute_kernel<DI, DO, true, false>)
               : (E <= 64 ? unpermute_kernel<DI, DO, false, true>
