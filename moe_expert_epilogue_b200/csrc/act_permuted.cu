@@ -54,8 +54,17 @@ __device__ __forceinline__ int64_t live_rows(const int32_t* n_used, int64_t max_
 // device-resident bound); lanes take 8-column chunks lane, lane + 32, ...
 // The next row's map entry is fetched while the current row streams, so the
 // row's data loads never wait on the map lookup.
+#ifndef MOE_ACT_MIN_BLOCKS
+#define MOE_ACT_MIN_BLOCKS 0
+#endif
+#if MOE_ACT_MIN_BLOCKS > 0
+#define MOE_ACT_MIN_BLOCKS_ATTR __launch_bounds__(kThreads, MOE_ACT_MIN_BLOCKS)
+#else
+#define MOE_ACT_MIN_BLOCKS_ATTR __launch_bounds__(kThreads)
+#endif
+
 template <int ACT, bool VEC, int U>
-__global__ void __launch_bounds__(kThreads)
+__global__ void MOE_ACT_MIN_BLOCKS_ATTR
 act_permuted_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ out,
                     const int32_t* __restrict__ pmap, const int32_t* __restrict__ n_used,
                     const float* __restrict__ probs, int64_t num_probs, int64_t max_rows,

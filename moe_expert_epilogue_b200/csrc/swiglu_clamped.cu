@@ -54,8 +54,17 @@ __device__ __forceinline__ BwdOut bwd_math(float g, float u, float dy, float p, 
 
 // ------------------------------------------------------------------ forward
 
+#ifndef MOE_SWIGLU_FWD_MIN_BLOCKS
+#define MOE_SWIGLU_FWD_MIN_BLOCKS 0
+#endif
+#if MOE_SWIGLU_FWD_MIN_BLOCKS > 0
+#define MOE_SWIGLU_FWD_MIN_BLOCKS_ATTR __launch_bounds__(kThreads, MOE_SWIGLU_FWD_MIN_BLOCKS)
+#else
+#define MOE_SWIGLU_FWD_MIN_BLOCKS_ATTR __launch_bounds__(kThreads)
+#endif
+
 template <class D, int U>
-__global__ void __launch_bounds__(kThreads)
+__global__ void MOE_SWIGLU_FWD_MIN_BLOCKS_ATTR
 swiglu_fwd_rows(const typename D::T* __restrict__ x, const float* __restrict__ probs,
                 typename D::T* __restrict__ y, int64_t rows, int64_t inter, int64_t ld_x,
                 int64_t ld_y, float L) {
@@ -180,8 +189,17 @@ __device__ __forceinline__ float row_reduce(float acc, float (*red)[kThreads / 3
   }
 }
 
+#ifndef MOE_SWIGLU_BWD_MIN_BLOCKS
+#define MOE_SWIGLU_BWD_MIN_BLOCKS 0
+#endif
+#if MOE_SWIGLU_BWD_MIN_BLOCKS > 0
+#define MOE_SWIGLU_BWD_MIN_BLOCKS_ATTR __launch_bounds__(kThreads, MOE_SWIGLU_BWD_MIN_BLOCKS)
+#else
+#define MOE_SWIGLU_BWD_MIN_BLOCKS_ATTR __launch_bounds__(kThreads)
+#endif
+
 template <class D, int W, int U>
-__global__ void __launch_bounds__(kThreads)
+__global__ void MOE_SWIGLU_BWD_MIN_BLOCKS_ATTR
 swiglu_bwd_vec(const typename D::T* __restrict__ x, const float* __restrict__ probs,
                const typename D::T* __restrict__ gy, typename D::T* __restrict__ gx,
                float* __restrict__ gp, int64_t rows, int64_t inter, int64_t ld_x,

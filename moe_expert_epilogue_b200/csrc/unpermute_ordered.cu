@@ -108,8 +108,17 @@ unpermute_kernel(const typename DI::T* __restrict__ eo, int64_t max_rows,
 // column ranges of its hidden dimension -- compacts the token's inverse-map
 // row itself (entries loaded during the previous item) into its own list, and
 // never waits for the other warps.
+#ifndef MOE_UNPERMUTE_MIN_BLOCKS
+#define MOE_UNPERMUTE_MIN_BLOCKS 0
+#endif
+#if MOE_UNPERMUTE_MIN_BLOCKS > 0
+#define MOE_UNPERMUTE_MIN_BLOCKS_ATTR __launch_bounds__(kThreads, MOE_UNPERMUTE_MIN_BLOCKS)
+#else
+#define MOE_UNPERMUTE_MIN_BLOCKS_ATTR __launch_bounds__(kThreads)
+#endif
+
 template <class DI, class DO, int SPLIT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void MOE_UNPERMUTE_MIN_BLOCKS_ATTR
 unpermute_warp(const typename DI::T* __restrict__ eo, int64_t max_rows,
                const int32_t* __restrict__ inv, const int32_t* __restrict__ valid_tokens,
                typename DO::T* __restrict__ out, int64_t tokens, int64_t hidden, int E,
