@@ -573,7 +573,7 @@ def run_ours(args):
         "next_rows": next_rows,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.kernel:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_sample, steps=1)
+        line["cpu_baseline"] = cpu_baseline(args.cpu_sample or 0.25, steps=1)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -726,10 +726,20 @@ def _cpu_model():
     return None
 
 
+def reference_fraction(args) -> float:
+    """Row fraction of every op the oracle runs per step in the reference arm:
+    --cpu-sample if given, else sized so that the warm-up and timed steps take
+    about two minutes on a ~17 s-per-full-step host (capped at a quarter)."""
+    if args.cpu_sample is not None:
+        return args.cpu_sample
+    return max(0.005, min(0.25, 120.0 / (17.0 * max(1, args.steps + args.warmup))))
+
+
 def run_reference(args):
     rank, _, world = dist_env()
     if rank != 0:
         return
+    args.cpu_sample = reference_fraction(args)
     w = cpu_sample_workload(args.cpu_sample)
     for _ in range(args.warmup):
         oracle_step(w)
@@ -760,8 +770,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--e2e-steps", type=int, default=6)
-    ap.add_argument("--cpu-sample", type=float, default=0.25,
-                    help="fraction of the rows of every op the CPU oracle runs")
+    ap.add_argument("--cpu-sample", type=float, default=None,
+                    help="fraction of the rows of every op the CPU oracle runs (default: "
+                         "0.25 for the cpu_baseline; sized to the step count for the "
+                         "reference arm)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")

@@ -59,3 +59,27 @@ def test_single_process_is_identity():
     import bench
     assert bench.max_over_ranks(3.5, torch.device("cpu")) == 3.5
     assert bench.aggregate_value(2 * 10 ** 9, 10, 1, 2.0) == pytest.approx(10.0)
+
+
+def test_algorithmic_bytes_match_the_closed_forms():
+    """Byte model of the step against hand-counted sizes of the workload."""
+    import bench
+    n_used = 69760
+    b = bench.algorithmic_bytes(n_used)
+    assert b["swiglu_fwd"] == 805_568_512 and b["swiglu_bwd"] == 1_342_701_568
+    assert b["router_weight_fwd"] == 469_827_584 and b["router_weight_bwd"] == 704_774_144
+    assert b["unpermute"] == 606_076_928 and b["residual_add"] == 1_879_048_192
+    assert b["act_sqrelu"] == 65536 * 1536 * 2 + n_used * 1536 * 2 + 4 * n_used + 4 * 65536
+    assert b["act_swiglu"] == 65536 * 3072 * 2 + n_used * 1536 * 2 + 4 * n_used + 4 * 65536
+    half = bench.algorithmic_bytes(n_used // 2, scale=0.5)
+    assert half["residual_add"] == b["residual_add"] // 2
+
+
+def test_reference_arm_runs_on_the_host(capsys):
+    """The reference arm (the CPU oracle on a bounded sample) prints one JSON line."""
+    import json
+    import bench
+    bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0", "--cpu-sample", "0.01"])
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "GB/s"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
