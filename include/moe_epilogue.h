@@ -84,7 +84,9 @@ enum {
 enum {
   MOE_DEVERR_COUNT = 1,  /* *n_used / *valid_tokens outside [0, max]: clamped    */
   MOE_DEVERR_MAP = 2,    /* permutation_map entry >= num_probs: row skipped       */
-  MOE_DEVERR_INVERSE = 4 /* inverse_map entry >= max_rows: contribution skipped   */
+  MOE_DEVERR_INVERSE = 4, /* inverse_map entry >= max_rows: contribution skipped  */
+  MOE_DEVERR_TIMEOUT = 8  /* a kernel's barrier wait gave up after ~1 s (a copy that
+                             never completed); the affected rows were not written  */
 };
 
 /* Human-readable name of a status code (static storage). */
@@ -95,6 +97,12 @@ MOE_API int moe_last_cuda_error(void);
 
 /* Library ABI version, currently 1. */
 MOE_API int moe_abi_version(void);
+
+/* Error bits recorded on the current device by kernels that have no dev_err
+ * argument (today: the TMA-staged clamped-SwiGLU forward, MOE_DEVERR_TIMEOUT).
+ * Synchronous: waits for the device, copies the word into *bits and, if
+ * `clear`, resets it.  Returns MOE_OK, MOE_ERR_NULL or MOE_ERR_CUDA. */
+MOE_API int moe_device_errors(int32_t* bits, int clear);
 
 /* ------------------------------------------------------------------------
  * Clamped, probability-weighted SwiGLU, forward.

@@ -20,7 +20,7 @@ MOE_BF16, MOE_FP16, MOE_FP32 = 0, 1, 2
 MOE_ACT_SQRELU, MOE_ACT_SQRELU_CLAMP, MOE_ACT_SWIGLU = 0, 1, 2
 (MOE_OK, MOE_ERR_NULL, MOE_ERR_SHAPE, MOE_ERR_DTYPE, MOE_ERR_ALIGN, MOE_ERR_LIMIT,
  MOE_ERR_CUDA) = range(7)
-MOE_DEVERR_COUNT, MOE_DEVERR_MAP, MOE_DEVERR_INVERSE = 1, 2, 4
+MOE_DEVERR_COUNT, MOE_DEVERR_MAP, MOE_DEVERR_INVERSE, MOE_DEVERR_TIMEOUT = 1, 2, 4, 8
 
 _P, _I64, _I32, _F, _I = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float,
                           ctypes.c_int)
@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
             L.moe_last_cuda_error.argtypes = []
             L.moe_abi_version.restype = _I
             L.moe_abi_version.argtypes = []
+            L.moe_device_errors.restype = _I
+            L.moe_device_errors.argtypes = [ctypes.POINTER(_I32), _I]
             for name, args in SIGNATURES.items():
                 fn = getattr(L, name)
                 fn.restype = _I
@@ -158,3 +160,11 @@ def moe_epilogue_fused(expert_output, row_probs, max_rows, inverse_map, valid_to
     _call("moe_epilogue_fused", ptr(expert_output), ptr(row_probs), max_rows, ptr(inverse_map),
           ptr(valid_tokens), ptr(shared_expert_output), ptr(residual), ptr(out), tokens, hidden,
           num_local_experts, dt, ptr(dev_err), stream_handle(stream))
+
+
+def moe_device_errors(clear=True) -> int:
+    """Error bits recorded on the current device by kernels without a dev_err
+    argument (MOE_DEVERR_TIMEOUT); synchronous."""
+    v = _I32(0)
+    _call("moe_device_errors", ctypes.byref(v), int(bool(clear)))
+    return int(v.value)

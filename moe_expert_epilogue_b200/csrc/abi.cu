@@ -48,6 +48,23 @@ int device_sms(int* sms) {
 
 }  // namespace
 
+int device_sm_count(int* sms) { return device_sms(sms); }
+
+int ensure_smem_limit(const void* kernel, size_t smem) {
+  static std::mutex mu;
+  static std::unordered_map<const void*, uint64_t> done;  // kernel -> bitmask of devices
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (bit && (done[kernel] & bit)) return MOE_OK;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return cuda_fail(e);
+  done[kernel] |= bit;
+  return MOE_OK;
+}
+
 int cuda_fail(cudaError_t e) {
   g_last_cuda_error = (int)e;
   return MOE_ERR_CUDA;

@@ -25,11 +25,11 @@ int check_launch();
 // stream serialisation allowed (see pdl_prologue); a failure is left in the
 // runtime's error state for check_launch().
 template <typename... KArgs, typename... Args>
-inline void launch_kernel(void (*kernel)(KArgs...), int grid, size_t smem, cudaStream_t stream,
-                          Args... args) {
+inline void launch_kernel_block(void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                                cudaStream_t stream, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3((unsigned)block);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -39,6 +39,18 @@ inline void launch_kernel(void (*kernel)(KArgs...), int grid, size_t smem, cudaS
   cfg.numAttrs = 1;
   (void)cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
+
+template <typename... KArgs, typename... Args>
+inline void launch_kernel(void (*kernel)(KArgs...), int grid, size_t smem, cudaStream_t stream,
+                          Args... args) {
+  launch_kernel_block(kernel, grid, kThreads, smem, stream, args...);
+}
+
+// SM count of the current device (cached per device).
+int device_sm_count(int* sms);
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+int ensure_smem_limit(const void* kernel, size_t smem);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

@@ -8,10 +8,16 @@
 //   d_up   = dy * p * silu(gc)        on -L <= u <= L
 //   d_p    = sum_j dy * silu(gc) * uc
 //
-// Forward: one warp per row (warps stride over the rows), the row's
-// probability loaded once, U chunks of 8 columns per lane in flight (two
-// loads each: gate, up), one 16-byte store per chunk (two for fp32); a flat
-// grid-stride variant serves rows shorter than 64 chunks.  Backward: W threads
+// Forward, 16-bit types: TMA-staged.  One CTA per SM; a producer thread
+// copies whole rows (gate | up, one cp.async.bulk each) into a ring of S
+// shared-memory stages, and 8 consumer warps compute rows out of shared
+// memory, writing y straight to global memory -- S rows (up to ~200 KB) in
+// flight per SM without holding them in registers (measured 4 % faster than
+// the register-staged kernel at rows 65536, inter 2048).  Otherwise (fp32,
+// rows too long for the ring): one warp per row (warps stride over the rows),
+// the row's probability loaded once, U chunks of 8 columns per lane in flight
+// (two loads each: gate, up), one 16-byte store per chunk (two for fp32); a
+// flat grid-stride variant serves rows shorter than 64 chunks.  Backward: W threads
 // own one row (one warp for the vectorised path), walk its chunks with a fixed
 // column assignment, write d_gate / d_up straight into the two halves of
 // grad_x and reduce the row's probability gradient with a fixed tree
@@ -20,6 +26,7 @@
 // independently with its next loads already in flight.
 #include "common.cuh"
 #include "launch.cuh"
+#include "tma.cuh"
 
 namespace moe {
 namespace {
@@ -101,6 +108,91 @@ swiglu_fwd_rows(const typename D::T* __restrict__ x, const float* __restrict__ p
         }
       }
     }
+  }
+}
+
+// Errors recorded by the kernels of this file that wait on barriers (bits
+// MOE_DEVERR_*), per device; read and cleared by moe_device_errors().
+__device__ int32_t g_device_errors;
+
+constexpr int kTmaConsumers = 8;
+constexpr int kTmaThreads = 32 * (kTmaConsumers + 1);
+constexpr size_t kTmaSmemMax = 200 * 1024;
+
+// TMA-staged forward.  Row k of the CTA (r = blockIdx.x + k * gridDim.x) goes
+// to stage k % S and to consumer warp k % C; since C divides S, every stage is
+// filled and emptied by one consumer in order, so a stage has at most one fill
+// outstanding and the barrier parities are unambiguous.  full[s] completes a
+// phase when the producer's arrival and the row's bytes are in; empty[s] when
+// the consumer has read the row.  Every wait is bounded: on a timeout the
+// waiting warp records MOE_DEVERR_TIMEOUT and stops; the producer then waits
+// (bounded again) for every copy it issued before its CTA exits.
+template <class D, int S>
+__global__ void __launch_bounds__(kTmaThreads, 1)
+swiglu_fwd_tma(const typename D::T* __restrict__ x, const float* __restrict__ probs,
+               typename D::T* __restrict__ y, int64_t rows, int64_t inter, int64_t ld_x,
+               int64_t ld_y, float L) {
+  static_assert(S % kTmaConsumers == 0, "each stage must belong to one consumer warp");
+  pdl_prologue();
+  using T = typename D::T;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t stage_bytes = (uint32_t)(2 * inter * sizeof(T));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * stage_bytes);
+  uint64_t* empty = full + S;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      tma::mbar_init(&full[s], 1);
+      tma::mbar_init(&empty[s], 1);
+    }
+    tma::mbar_init_fence();
+  }
+  __syncthreads();
+  const int64_t my_rows = rows > blockIdx.x ? (rows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (warp == 0) {                                        // producer
+    if (lane != 0) return;
+    int64_t k = 0;
+    for (; k < my_rows; ++k) {
+      const int s = (int)(k % S);
+      const uint32_t n = (uint32_t)(k / S);
+      if (n > 0 && !tma::mbar_wait(&empty[s], (n - 1) & 1)) {
+        atomicOr(&g_device_errors, MOE_DEVERR_TIMEOUT);
+        break;
+      }
+      const int64_t r = blockIdx.x + k * gridDim.x;
+      tma::mbar_arrive_expect_tx(&full[s], stage_bytes);
+      tma::bulk_load(smem + (size_t)s * stage_bytes, x + r * ld_x, stage_bytes, &full[s]);
+    }
+    for (int s = 0; s < S && s < k; ++s) {                // drain every issued copy
+      const int64_t last = s + ((k - 1 - s) / S) * S;
+      if (!tma::mbar_wait(&full[s], (uint32_t)(last / S) & 1))
+        atomicOr(&g_device_errors, MOE_DEVERR_TIMEOUT);
+    }
+    return;
+  }
+  const int cw = warp - 1;                                // consumers
+  const int64_t cpr = inter / kVec;
+  const FwdMath f{L};
+  for (int64_t k = cw; k < my_rows; k += kTmaConsumers) {
+    const int s = (int)(k % S);
+    if (!tma::mbar_wait(&full[s], (uint32_t)(k / S) & 1)) {
+      if (lane == 0) atomicOr(&g_device_errors, MOE_DEVERR_TIMEOUT);
+      return;
+    }
+    const int64_t r = blockIdx.x + k * gridDim.x;
+    const float p = __ldg(probs + r);
+    const T* st = reinterpret_cast<const T*>(smem + (size_t)s * stage_bytes);
+    T* yr = y + r * ld_y;
+    for (int64_t c = lane; c < cpr; c += 32) {
+      float g[8], u[8], o[8];
+      widen8<D>(tma::lds8<D>(st + c * kVec), g);
+      widen8<D>(tma::lds8<D>(st + inter + c * kVec), u);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = f(g[i], u[i], p);
+      store8<D>(yr + c * kVec, o);
+    }
+    __syncwarp();                                          // every lane has read the stage
+    if (lane == 0) tma::mbar_arrive(&empty[s]);
   }
 }
 
@@ -307,6 +399,9 @@ inline int threads_per_row(int64_t units) {
 #ifndef MOE_SWIGLU_FWD_UNROLL
 #define MOE_SWIGLU_FWD_UNROLL 2
 #endif
+#ifndef MOE_SWIGLU_FWD_TMA
+#define MOE_SWIGLU_FWD_TMA 1
+#endif
 #ifndef MOE_SWIGLU_FWD_ROW_UNROLL
 #define MOE_SWIGLU_FWD_ROW_UNROLL 8
 #endif
@@ -329,6 +424,22 @@ int fwd(const void* xv, const float* probs, void* yv, int64_t rows, int64_t inte
   const bool vec = inter % kVec == 0 && ld_x % kVec == 0 && ld_y % kVec == 0 && aligned16(x) &&
                    aligned16(y);
   int grid;
+  if constexpr (D::kBytes == 2) {
+    // TMA ring: 16 stages of one row, or 8 for longer rows, if it fits
+    const size_t stage = (size_t)2 * inter * sizeof(T);
+    const int S = 16 * stage + 256 <= kTmaSmemMax ? 16 : 8 * stage + 128 <= kTmaSmemMax ? 8 : 0;
+    if (MOE_SWIGLU_FWD_TMA && vec && inter / kVec >= 64 && S > 0) {
+      auto k = S == 16 ? swiglu_fwd_tma<D, 16> : swiglu_fwd_tma<D, 8>;
+      const size_t smem = (size_t)S * stage + 2 * (size_t)S * sizeof(uint64_t);
+      if (int rc = ensure_smem_limit((const void*)k, kTmaSmemMax)) return rc;
+      int sms = 0;
+      if (int rc = device_sm_count(&sms)) return rc;
+      grid = (int)(rows < sms ? rows : sms);
+      launch_kernel_block(k, grid, kTmaThreads, smem, stream, x, probs, y, rows, inter, ld_x,
+                          ld_y, limit);
+      return check_launch();
+    }
+  }
   if (vec && inter / kVec >= 64) {
     auto k = swiglu_fwd_rows<D, unroll_for<D>(MOE_SWIGLU_FWD_ROW_UNROLL)>;
     if (int rc = persistent_grid((const void*)k, 0, (rows + kThreads / 32 - 1) / (kThreads / 32),
@@ -425,3 +536,15 @@ int launch_swiglu_clamped_bwd(const void* x, const float* probs, const void* gra
 }
 
 }  // namespace moe
+
+extern "C" int moe_device_errors(int32_t* bits, int clear) {
+  if (!bits) return MOE_ERR_NULL;
+  cudaError_t e = cudaMemcpyFromSymbol(bits, moe::g_device_errors, sizeof(int32_t));
+  if (e != cudaSuccess) return moe::cuda_fail(e);
+  if (clear) {
+    const int32_t zero = 0;
+    e = cudaMemcpyToSymbol(moe::g_device_errors, &zero, sizeof(int32_t));
+    if (e != cudaSuccess) return moe::cuda_fail(e);
+  }
+  return MOE_OK;
+}
