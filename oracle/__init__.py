@@ -64,6 +64,10 @@ def load(path: str) -> ctypes.CDLL:
         "orc_swiglu_clamped_bwd_dt": (None, [P, P, P, P, P, P, I64, I64, I64, I64, I64, F,
                                              ctypes.c_int]),
         "orc_router_weight_fwd": (None, [P, ctypes.c_int, P, P, ctypes.c_int, I64, I64]),
+        "orc_router_weight_fwd_p": (None, [P, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int,
+                                           I64, I64]),
+        "orc_router_weight_bwd_p": (None, [P, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int, P,
+                                           P, P, I64, I64]),
         "orc_router_weight_bwd": (None, [P, ctypes.c_int, P, ctypes.c_int, P, P, P, P,
                                          I64, I64]),
         "orc_act_with_probs_permuted": (ctypes.c_int, [ctypes.c_int, P, P, P, I32, P, I64,
@@ -176,27 +180,28 @@ def swiglu_clamped_fwd_f64(g, u, p, limit) -> np.ndarray:
     return y
 
 
-def router_weight_fwd(x, x_dt, probs, out_dt):
+def router_weight_fwd(x, x_dt, probs, out_dt, p_dt=F32):
+    """probs: [rows] or [rows, 1] in dtype p_dt (uint16 bits for bf16/fp16)."""
     x = _c(x, _storage_np(x_dt))
     rows, hidden = x.shape
-    probs = _c(np.asarray(probs, np.float32).reshape(rows), np.float32)
+    probs = _c(np.asarray(probs).reshape(rows), _storage_np(p_dt))
     out = np.empty((rows, hidden), _storage_np(out_dt))
-    _lib().orc_router_weight_fwd(_p(x), x_dt, _p(probs), _p(out), out_dt, rows, hidden)
+    _lib().orc_router_weight_fwd_p(_p(x), x_dt, _p(probs), p_dt, _p(out), out_dt, rows, hidden)
     return out
 
 
-def router_weight_bwd(grad_out, g_dt, x, x_dt, probs):
+def router_weight_bwd(grad_out, g_dt, x, x_dt, probs, p_dt=F32):
     """x may be None (forward did not save x).  Returns (grad_x, grad_probs f64
-    or None, grad_probs_abs f64 or None)."""
+    or None, grad_probs_abs f64 or None); grad_probs is the unrounded sum."""
     grad_out = _c(grad_out, _storage_np(g_dt))
     rows, hidden = grad_out.shape
     x = _c(x, _storage_np(x_dt))
-    probs = _c(np.asarray(probs, np.float32).reshape(rows), np.float32)
+    probs = _c(np.asarray(probs).reshape(rows), _storage_np(p_dt))
     gx = np.empty((rows, hidden), _storage_np(x_dt))
     gp = np.empty(rows, np.float64) if x is not None else None
     ga = np.empty(rows, np.float64) if x is not None else None
-    _lib().orc_router_weight_bwd(_p(grad_out), g_dt, _p(x), x_dt, _p(probs), _p(gx),
-                                 _p(gp), _p(ga), rows, hidden)
+    _lib().orc_router_weight_bwd_p(_p(grad_out), g_dt, _p(x), x_dt, _p(probs), p_dt, _p(gx),
+                                   _p(gp), _p(ga), rows, hidden)
     return gx, gp, ga
 
 

@@ -232,31 +232,42 @@ void orc_swiglu_clamped_fwd_f64(const double *g, const double *u, const double *
 /* ------------------------------------------------ router-weight multiply [OPT] */
 
 /* [OPT] _rw_fwd_core: out = (x.float() * probs.float()).to(out_dtype), one
- * fp32 multiply per element and one rounding. */
+ * fp32 multiply per element and one rounding.  probs has dtype p_dt (widened
+ * exactly to fp32). */
+void orc_router_weight_fwd_p(const void *x, int x_dt, const void *probs, int p_dt, void *out,
+                             int out_dt, int64_t rows, int64_t hidden)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        float p = load_as_f32(probs, p_dt, r);
+        for (int64_t h = 0; h < hidden; ++h) {
+            float v = load_as_f32(x, x_dt, r * hidden + h) * p;
+            store_rounded(out, out_dt, r * hidden + h, v);
+        }
+    }
+}
+
 void orc_router_weight_fwd(const void *x, int x_dt, const float *probs, void *out,
                            int out_dt, int64_t rows, int64_t hidden)
 {
-    for (int64_t r = 0; r < rows; ++r)
-        for (int64_t h = 0; h < hidden; ++h) {
-            float v = load_as_f32(x, x_dt, r * hidden + h) * probs[r];
-            store_rounded(out, out_dt, r * hidden + h, v);
-        }
+    orc_router_weight_fwd_p(x, x_dt, probs, ORC_F32, out, out_dt, rows, hidden);
 }
 
 /* [OPT] _rw_bwd_x_core and _rw_bwd_probs_core:
  *   grad_x = (g_f32 * probs_f32).to(x.dtype)
- *   grad_probs = (g_f32 * x_f32).sum(-1)   (fp32 terms, summed here in float64)
+ *   grad_probs = (g_f32 * x_f32).sum(-1)   (fp32 terms, summed here in float64;
+ *                                           the caller rounds to probs.dtype)
  * x == NULL means the forward did not save x (save_x false): the probability
  * gradient is not computed. */
-void orc_router_weight_bwd(const void *grad_out, int g_dt, const void *x, int x_dt,
-                           const float *probs, void *grad_x, double *grad_probs,
-                           double *grad_probs_abs, int64_t rows, int64_t hidden)
+void orc_router_weight_bwd_p(const void *grad_out, int g_dt, const void *x, int x_dt,
+                             const void *probs, int p_dt, void *grad_x, double *grad_probs,
+                             double *grad_probs_abs, int64_t rows, int64_t hidden)
 {
     for (int64_t r = 0; r < rows; ++r) {
+        float p = load_as_f32(probs, p_dt, r);
         double acc = 0.0, acc_abs = 0.0;
         for (int64_t h = 0; h < hidden; ++h) {
             float g = load_as_f32(grad_out, g_dt, r * hidden + h);
-            store_rounded(grad_x, x_dt, r * hidden + h, g * probs[r]);
+            store_rounded(grad_x, x_dt, r * hidden + h, g * p);
             if (x) {
                 float t = g * load_as_f32(x, x_dt, r * hidden + h);
                 acc += (double)t;
@@ -268,6 +279,14 @@ void orc_router_weight_bwd(const void *grad_out, int g_dt, const void *x, int x_
             grad_probs_abs[r] = acc_abs;
         }
     }
+}
+
+void orc_router_weight_bwd(const void *grad_out, int g_dt, const void *x, int x_dt,
+                           const float *probs, void *grad_x, double *grad_probs,
+                           double *grad_probs_abs, int64_t rows, int64_t hidden)
+{
+    orc_router_weight_bwd_p(grad_out, g_dt, x, x_dt, probs, ORC_F32, grad_x, grad_probs,
+                            grad_probs_abs, rows, hidden);
 }
 
 /* ------------------------------------ batch-invariant permuted activation [BI] */

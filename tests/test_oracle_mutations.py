@@ -42,7 +42,7 @@ MUTATIONS = [
     ("f16_ties_away", "if (rem > 0x1000u || (rem == 0x1000u && (q & 1u))) q++;",
      "if (rem >= 0x1000u) q++;", ["test_f16_rounding_matches_numpy"]),
     ("rw_grad_probs_uses_p", "float t = g * load_as_f32(x, x_dt, r * hidden + h);",
-     "float t = g * probs[r];", ["test_router_weight_bwd_vs_torch_autograd"]),
+     "float t = g * p;", ["test_router_weight_bwd_vs_torch_autograd"]),
     ("sqrelu_single_rounding", "float sq = round_to_dtype(rl * rl, ORC_BF16);",
      "float sq = rl * rl;", ["test_sqrelu_rounding_witness"]),
     ("clamp_scale_dropped", "float z = clamp_scale * tanhf(xv / clamp_scale);",

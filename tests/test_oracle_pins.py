@@ -577,3 +577,27 @@ def test_swiglu_fp32_vs_float64_autograd():
     assert (err <= 2 ** -20 * scale + 1e-30).all()
     assert gx[0, 0] != 0 and gx[1, 50] != 0
     assert_sum_close(gp, pg.grad.reshape(-1).numpy(), gabs, 1e-6, "fp32 grad_probs")
+
+
+@pytest.mark.parametrize("p_dtype", [torch.bfloat16, torch.float16])
+def test_router_weight_low_precision_probs_vs_torch(p_dtype):
+    """bf16 / fp16 routing probabilities: the forward widens them exactly
+    (probs.float()) -- bitwise equal to torch; the backward's grad_x likewise
+    and grad_probs is torch autograd's fp32 sum (cast to the probs dtype by
+    the caller of the oracle)."""
+    d = inputs.router_weight_inputs(24, 200, seed=27)
+    probs = d["probs"].to(p_dtype)
+    x = d["x"].clone().requires_grad_(True)
+    p = probs.clone().requires_grad_(True)
+    out = (x.float() * p.float()).to(torch.bfloat16)
+    got = oracle.router_weight_fwd(bits(d["x"]), oracle.BF16, bits(probs), oracle.BF16,
+                                   DT[p_dtype])
+    assert_bits_equal(got, bits(out), "fwd with low-precision probs")
+    out.backward(d["grad_out"])
+    gx, gp, gabs = oracle.router_weight_bwd(bits(d["grad_out"]), oracle.BF16, bits(d["x"]),
+                                            oracle.BF16, bits(probs), DT[p_dtype])
+    assert_bits_equal(gx, bits(x.grad), "grad_x")
+    # torch rounds its fp32 sum to the probs dtype: within one ulp of that dtype
+    want = p.grad.reshape(-1).double().numpy()
+    rel = 2.0 ** -7 if p_dtype == torch.bfloat16 else 2.0 ** -10
+    assert (np.abs(gp - want) <= rel * np.abs(want) + 1e-5 * gabs).all()
