@@ -177,6 +177,22 @@ MOE_API int moe_router_weight_mul_bwd(const void* grad_out, moe_dtype g_dt, cons
                               cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * The router-weight multiply with routing probabilities of any dtype.
+ * [OPT] _rw_fwd_core (probs.float()) and _rw_bwd_probs_core (the sum "cast to
+ * probs_dtype"): as moe_router_weight_mul_fwd / _bwd, with probs of dtype
+ * probs_dt (bf16, fp16 or fp32; widened exactly to fp32) and grad_probs
+ * rounded once (RNE) to probs_dt.  probs and grad_probs are [rows] in
+ * probs_dt.  The fp32 entry points above are these with probs_dt = MOE_FP32.
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_router_weight_mul_fwd_ex(const void* x, moe_dtype x_dt, const void* probs,
+                                         moe_dtype probs_dt, void* out, moe_dtype out_dt,
+                                         int64_t rows, int64_t hidden, cudaStream_t stream);
+MOE_API int moe_router_weight_mul_bwd_ex(const void* grad_out, moe_dtype g_dt, const void* x,
+                                         moe_dtype x_dt, const void* probs, moe_dtype probs_dt,
+                                         void* grad_x, void* grad_probs, int64_t rows,
+                                         int64_t hidden, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Batch-invariant activation with router probabilities over a padded,
  * expert-grouped row layout.
  * [BI] _squared_relu_with_probs_kernel, squared_relu_with_probs,

@@ -31,6 +31,8 @@ SIGNATURES = {
     "moe_swiglu_clamped_bwd": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _F, _I, _P],
     "moe_router_weight_mul_fwd": [_P, _I, _P, _P, _I, _I64, _I64, _P],
     "moe_router_weight_mul_bwd": [_P, _I, _P, _I, _P, _P, _P, _I64, _I64, _P],
+    "moe_router_weight_mul_fwd_ex": [_P, _I, _P, _I, _P, _I, _I64, _I64, _P],
+    "moe_router_weight_mul_bwd_ex": [_P, _I, _P, _I, _P, _I, _P, _P, _I64, _I64, _P],
     "moe_act_with_probs_permuted": [_I, _P, _P, _P, _P, _P, _I64, _I64, _I64, _F, _I, _P, _P],
     "moe_unpermute_ordered": [_P, _I, _I64, _P, _P, _P, _I, _I64, _I64, _I32, _P, _P],
     "moe_residual_add": [_P, _P, _P, _P, _I64, _I, _P],
@@ -123,6 +125,18 @@ def moe_router_weight_mul_fwd(x, x_dt, probs, out, out_dt, rows, hidden, stream=
 def moe_router_weight_mul_bwd(grad_out, g_dt, x, x_dt, probs, grad_x, grad_probs, rows, hidden,
                               stream=None):
     _call("moe_router_weight_mul_bwd", ptr(grad_out), g_dt, ptr(x), x_dt, ptr(probs),
+          ptr(grad_x), ptr(grad_probs), rows, hidden, stream_handle(stream))
+
+
+def moe_router_weight_mul_fwd_ex(x, x_dt, probs, probs_dt, out, out_dt, rows, hidden,
+                                 stream=None):
+    _call("moe_router_weight_mul_fwd_ex", ptr(x), x_dt, ptr(probs), probs_dt, ptr(out), out_dt,
+          rows, hidden, stream_handle(stream))
+
+
+def moe_router_weight_mul_bwd_ex(grad_out, g_dt, x, x_dt, probs, probs_dt, grad_x, grad_probs,
+                                 rows, hidden, stream=None):
+    _call("moe_router_weight_mul_bwd_ex", ptr(grad_out), g_dt, ptr(x), x_dt, ptr(probs), probs_dt,
           ptr(grad_x), ptr(grad_probs), rows, hidden, stream_handle(stream))
 
 

@@ -169,36 +169,51 @@ int moe_swiglu_clamped_bwd(const void* x, const float* probs, const void* grad_y
                                    ld_gy, ld_gx, limit, dt, stream);
 }
 
-int moe_router_weight_mul_fwd(const void* x, moe_dtype x_dt, const float* probs, void* out,
-                              moe_dtype out_dt, int64_t rows, int64_t hidden,
-                              cudaStream_t stream) {
-  if (!dtype_ok(x_dt) || !dtype_ok(out_dt)) return MOE_ERR_DTYPE;
+int moe_router_weight_mul_fwd_ex(const void* x, moe_dtype x_dt, const void* probs,
+                                 moe_dtype probs_dt, void* out, moe_dtype out_dt, int64_t rows,
+                                 int64_t hidden, cudaStream_t stream) {
+  if (!dtype_ok(x_dt) || !dtype_ok(out_dt) || !dtype_ok(probs_dt)) return MOE_ERR_DTYPE;
   if (rows < 0 || hidden < 0 || !product_ok(rows, hidden)) return MOE_ERR_SHAPE;
   if (rows == 0 || hidden == 0) return MOE_OK;
   if (!x || !probs || !out) return MOE_ERR_NULL;
   if (!aligned_to(x, dtype_size(x_dt)) || !aligned_to(out, dtype_size(out_dt)) ||
-      !aligned_to(probs, 4))
+      !aligned_to(probs, dtype_size(probs_dt)))
     return MOE_ERR_ALIGN;
-  return launch_router_weight_fwd(x, x_dt, probs, out, out_dt, rows, hidden, stream);
+  return launch_router_weight_fwd(x, x_dt, probs, probs_dt, out, out_dt, rows, hidden, stream);
 }
 
-int moe_router_weight_mul_bwd(const void* grad_out, moe_dtype g_dt, const void* x,
-                              moe_dtype x_dt, const float* probs, void* grad_x,
-                              float* grad_probs, int64_t rows, int64_t hidden,
+int moe_router_weight_mul_fwd(const void* x, moe_dtype x_dt, const float* probs, void* out,
+                              moe_dtype out_dt, int64_t rows, int64_t hidden,
                               cudaStream_t stream) {
-  if (!dtype_ok(g_dt) || !dtype_ok(x_dt)) return MOE_ERR_DTYPE;
+  return moe_router_weight_mul_fwd_ex(x, x_dt, probs, MOE_FP32, out, out_dt, rows, hidden,
+                                      stream);
+}
+
+int moe_router_weight_mul_bwd_ex(const void* grad_out, moe_dtype g_dt, const void* x,
+                                 moe_dtype x_dt, const void* probs, moe_dtype probs_dt,
+                                 void* grad_x, void* grad_probs, int64_t rows, int64_t hidden,
+                                 cudaStream_t stream) {
+  if (!dtype_ok(g_dt) || !dtype_ok(x_dt) || !dtype_ok(probs_dt)) return MOE_ERR_DTYPE;
   if (rows < 0 || hidden < 0 || !product_ok(rows, hidden)) return MOE_ERR_SHAPE;
   if ((x == nullptr) != (grad_probs == nullptr)) return MOE_ERR_NULL;
   if (rows == 0) return MOE_OK;
   if (!probs) return MOE_ERR_NULL;
   if (hidden > 0 && (!grad_out || !grad_x)) return MOE_ERR_NULL;
   if (!aligned_to(grad_out, dtype_size(g_dt)) || !aligned_to(x, dtype_size(x_dt)) ||
-      !aligned_to(grad_x, dtype_size(x_dt)) || !aligned_to(probs, 4) ||
-      !aligned_to(grad_probs, 4))
+      !aligned_to(grad_x, dtype_size(x_dt)) || !aligned_to(probs, dtype_size(probs_dt)) ||
+      !aligned_to(grad_probs, dtype_size(probs_dt)))
     return MOE_ERR_ALIGN;
   if (hidden == 0 && grad_probs == nullptr) return MOE_OK;
-  return launch_router_weight_bwd(grad_out, g_dt, x, x_dt, probs, grad_x, grad_probs, rows,
-                                  hidden, stream);
+  return launch_router_weight_bwd(grad_out, g_dt, x, x_dt, probs, probs_dt, grad_x, grad_probs,
+                                  rows, hidden, stream);
+}
+
+int moe_router_weight_mul_bwd(const void* grad_out, moe_dtype g_dt, const void* x,
+                              moe_dtype x_dt, const float* probs, void* grad_x,
+                              float* grad_probs, int64_t rows, int64_t hidden,
+                              cudaStream_t stream) {
+  return moe_router_weight_mul_bwd_ex(grad_out, g_dt, x, x_dt, probs, MOE_FP32, grad_x,
+                                      grad_probs, rows, hidden, stream);
 }
 
 int moe_act_with_probs_permuted(moe_act act, const void* x, void* out,

@@ -62,12 +62,12 @@ int launch_swiglu_clamped_bwd(const void* x, const float* probs, const void* gra
                               void* grad_x, float* grad_probs, int64_t rows, int64_t inter,
                               int64_t ld_x, int64_t ld_gy, int64_t ld_gx, float limit,
                               moe_dtype dt, cudaStream_t stream);
-int launch_router_weight_fwd(const void* x, moe_dtype x_dt, const float* probs, void* out,
-                             moe_dtype out_dt, int64_t rows, int64_t hidden,
+int launch_router_weight_fwd(const void* x, moe_dtype x_dt, const void* probs, moe_dtype p_dt,
+                             void* out, moe_dtype out_dt, int64_t rows, int64_t hidden,
                              cudaStream_t stream);
 int launch_router_weight_bwd(const void* grad_out, moe_dtype g_dt, const void* x,
-                             moe_dtype x_dt, const float* probs, void* grad_x,
-                             float* grad_probs, int64_t rows, int64_t hidden,
+                             moe_dtype x_dt, const void* probs, moe_dtype p_dt, void* grad_x,
+                             void* grad_probs, int64_t rows, int64_t hidden,
                              cudaStream_t stream);
 int launch_act_with_probs_permuted(moe_act act, const uint16_t* x, uint16_t* out,
                                    const int32_t* permutation_map, const int32_t* n_used,

@@ -18,10 +18,24 @@ namespace {
 
 constexpr int kUnroll = 2;
 
+// Routing probabilities may be bf16, fp16 or fp32 (widened exactly); the
+// probability gradient is rounded to their dtype.  Once per row, so a runtime
+// switch is free.
+__device__ __forceinline__ float load_prob(const void* p, int dt, int64_t i) {
+  if (dt == MOE_BF16) return __uint_as_float((uint32_t)__ldg(static_cast<const uint16_t*>(p) + i) << 16);
+  if (dt == MOE_FP16) return f16_to_f32(__ldg(static_cast<const uint16_t*>(p) + i));
+  return __ldg(static_cast<const float*>(p) + i);
+}
+__device__ __forceinline__ void store_prob(void* p, int dt, int64_t i, float v) {
+  if (dt == MOE_BF16) static_cast<uint16_t*>(p)[i] = f32_to_bf16(v);
+  else if (dt == MOE_FP16) static_cast<uint16_t*>(p)[i] = f32_to_f16(v);
+  else static_cast<float*>(p)[i] = v;
+}
+
 // out[r, :] = cast(in[r, :] * p[r]) over a [rows, cpr] chunk grid.
 template <class DI, class DO>
 __global__ void __launch_bounds__(kThreads)
-scale_rows_vec(const typename DI::T* __restrict__ in, const float* __restrict__ probs,
+scale_rows_vec(const typename DI::T* __restrict__ in, const void* __restrict__ probs, int p_dt,
                typename DO::T* __restrict__ out, int64_t rows, int64_t hidden) {
   pdl_prologue();
   const int64_t cpr = hidden / kVec;
@@ -39,7 +53,7 @@ scale_rows_vec(const typename DI::T* __restrict__ in, const float* __restrict__ 
       if (q + k * S < total) {
         off[k] = cur.r * hidden + cur.c * kVec;
         raw[k] = load8<DI>(in + off[k]);
-        p[k] = __ldg(probs + cur.r);
+        p[k] = load_prob(probs, p_dt, cur.r);
       }
       cur.advance();
     }
@@ -58,8 +72,8 @@ scale_rows_vec(const typename DI::T* __restrict__ in, const float* __restrict__ 
 
 template <class DI, class DO>
 __global__ void __launch_bounds__(kThreads)
-scale_rows_scalar(const typename DI::T* __restrict__ in, const float* __restrict__ probs,
-                  typename DO::T* __restrict__ out, int64_t rows, int64_t hidden) {
+scale_rows_scalar(const typename DI::T* __restrict__ in, const void* __restrict__ probs,
+                  int p_dt, typename DO::T* __restrict__ out, int64_t rows, int64_t hidden) {
   pdl_prologue();
   const int64_t total = rows * hidden;
   const int64_t S = (int64_t)gridDim.x * kThreads;
@@ -67,7 +81,7 @@ scale_rows_scalar(const typename DI::T* __restrict__ in, const float* __restrict
   if (q >= total) return;
   RowCursor cur(q, S, hidden);
   for (; q < total; q += S, cur.advance())
-    store1<DO>(out + q, load1<DI>(in + q) * __ldg(probs + cur.r));
+    store1<DO>(out + q, load1<DI>(in + q) * load_prob(probs, p_dt, cur.r));
 }
 
 template <int W>
@@ -91,8 +105,8 @@ __device__ __forceinline__ float row_reduce(float acc, float (*red)[kThreads / 3
 template <class DG, class DX, int W, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 rw_bwd_rows(const typename DG::T* __restrict__ g, const typename DX::T* __restrict__ x,
-            const float* __restrict__ probs, typename DX::T* __restrict__ gx,
-            float* __restrict__ gp, int64_t rows, int64_t hidden) {
+            const void* __restrict__ probs, int p_dt, typename DX::T* __restrict__ gx,
+            void* __restrict__ gp, int64_t rows, int64_t hidden) {
   pdl_prologue();
   constexpr int G = kThreads / W;
   __shared__ float red[2][kThreads / 32];
@@ -102,7 +116,7 @@ rw_bwd_rows(const typename DG::T* __restrict__ g, const typename DX::T* __restri
     const int64_t r = r0 + sub;
     float acc = 0.0f;
     if (r < rows) {
-      const float p = __ldg(probs + r);
+      const float p = load_prob(probs, p_dt, r);
       const int64_t base = r * hidden;
       if constexpr (VEC) {
         const int64_t cpr = hidden / kVec;
@@ -142,7 +156,7 @@ rw_bwd_rows(const typename DG::T* __restrict__ g, const typename DX::T* __restri
       }
     }
     const float s = row_reduce<W>(acc, red, parity);
-    if (r < rows && lane == 0) gp[r] = s;
+    if (r < rows && lane == 0) store_prob(gp, p_dt, r, s);
     parity ^= 1;
   }
 }
@@ -155,8 +169,8 @@ inline int threads_per_row(int64_t units) {
 }
 
 template <class DI, class DO>
-int launch_scale(const void* in, const float* probs, void* out, int64_t rows, int64_t hidden,
-                 cudaStream_t stream) {
+int launch_scale(const void* in, const void* probs, int p_dt, void* out, int64_t rows,
+                 int64_t hidden, cudaStream_t stream) {
   const auto* i = static_cast<const typename DI::T*>(in);
   auto* o = static_cast<typename DO::T*>(out);
   int grid;
@@ -166,36 +180,36 @@ int launch_scale(const void* in, const float* probs, void* out, int64_t rows, in
     if (int rc = persistent_grid((const void*)k, 0,
                                  (units + kThreads * kUnroll - 1) / (kThreads * kUnroll), &grid))
       return rc;
-    launch_kernel(k, grid, 0, stream, i, probs, o, rows, hidden);
+    launch_kernel(k, grid, 0, stream, i, probs, p_dt, o, rows, hidden);
   } else {
     auto k = scale_rows_scalar<DI, DO>;
     if (int rc = persistent_grid((const void*)k, 0, (rows * hidden + kThreads - 1) / kThreads,
                                  &grid))
       return rc;
-    launch_kernel(k, grid, 0, stream, i, probs, o, rows, hidden);
+    launch_kernel(k, grid, 0, stream, i, probs, p_dt, o, rows, hidden);
   }
   return check_launch();
 }
 
 template <class DG, class DX, int W, bool VEC>
-int launch_rows(const void* g, const void* x, const float* probs, void* gx, float* gp,
+int launch_rows(const void* g, const void* x, const void* probs, int p_dt, void* gx, void* gp,
                 int64_t rows, int64_t hidden, cudaStream_t stream) {
   auto k = rw_bwd_rows<DG, DX, W, VEC>;
   int grid;
   const int64_t blocks = (rows + kThreads / W - 1) / (kThreads / W);
   if (int rc = persistent_grid((const void*)k, 0, blocks, &grid)) return rc;
   launch_kernel(k, grid, 0, stream, static_cast<const typename DG::T*>(g),
-                                   static_cast<const typename DX::T*>(x), probs,
+                                   static_cast<const typename DX::T*>(x), probs, p_dt,
                                    static_cast<typename DX::T*>(gx), gp, rows, hidden);
   return check_launch();
 }
 
 template <class DG, class DX>
-int launch_bwd_with_probs(const void* g, const void* x, const float* probs, void* gx, float* gp,
-                          int64_t rows, int64_t hidden, cudaStream_t stream) {
+int launch_bwd_with_probs(const void* g, const void* x, const void* probs, int p_dt, void* gx,
+                          void* gp, int64_t rows, int64_t hidden, cudaStream_t stream) {
   const bool vec = hidden % kVec == 0 && aligned16(g) && aligned16(x) && aligned16(gx);
   const int W = threads_per_row(vec ? hidden / kVec : hidden);
-#define MOE_RW_ARGS g, x, probs, gx, gp, rows, hidden, stream
+#define MOE_RW_ARGS g, x, probs, p_dt, gx, gp, rows, hidden, stream
   if (vec) {
     switch (W) {
       case 32: return launch_rows<DG, DX, 32, true>(MOE_RW_ARGS);
@@ -231,34 +245,34 @@ int dispatch2(moe_dtype a, moe_dtype b, A... args) {
 }
 
 template <class DI, class DO> struct Fwd {
-  static int run(const void* x, const float* p, void* out, int64_t rows, int64_t hidden,
+  static int run(const void* x, const void* p, int p_dt, void* out, int64_t rows, int64_t hidden,
                  cudaStream_t s) {
-    return launch_scale<DI, DO>(x, p, out, rows, hidden, s);
+    return launch_scale<DI, DO>(x, p, p_dt, out, rows, hidden, s);
   }
 };
 
 template <class DG, class DX> struct Bwd {
-  static int run(const void* g, const void* x, const float* p, void* gx, float* gp, int64_t rows,
-                 int64_t hidden, cudaStream_t s) {
-    if (x == nullptr) return launch_scale<DG, DX>(g, p, gx, rows, hidden, s);
-    return launch_bwd_with_probs<DG, DX>(g, x, p, gx, gp, rows, hidden, s);
+  static int run(const void* g, const void* x, const void* p, int p_dt, void* gx, void* gp,
+                 int64_t rows, int64_t hidden, cudaStream_t s) {
+    if (x == nullptr) return launch_scale<DG, DX>(g, p, p_dt, gx, rows, hidden, s);
+    return launch_bwd_with_probs<DG, DX>(g, x, p, p_dt, gx, gp, rows, hidden, s);
   }
 };
 
 }  // namespace
 
-int launch_router_weight_fwd(const void* x, moe_dtype x_dt, const float* probs, void* out,
-                             moe_dtype out_dt, int64_t rows, int64_t hidden,
+int launch_router_weight_fwd(const void* x, moe_dtype x_dt, const void* probs, moe_dtype p_dt,
+                             void* out, moe_dtype out_dt, int64_t rows, int64_t hidden,
                              cudaStream_t stream) {
-  return dispatch2<Fwd>(x_dt, out_dt, x, probs, out, rows, hidden, stream);
+  return dispatch2<Fwd>(x_dt, out_dt, x, probs, (int)p_dt, out, rows, hidden, stream);
 }
 
 int launch_router_weight_bwd(const void* grad_out, moe_dtype g_dt, const void* x,
-                             moe_dtype x_dt, const float* probs, void* grad_x,
-                             float* grad_probs, int64_t rows, int64_t hidden,
+                             moe_dtype x_dt, const void* probs, moe_dtype p_dt, void* grad_x,
+                             void* grad_probs, int64_t rows, int64_t hidden,
                              cudaStream_t stream) {
-  return dispatch2<Bwd>(g_dt, x_dt, grad_out, x, probs, grad_x, grad_probs, rows, hidden,
-                        stream);
+  return dispatch2<Bwd>(g_dt, x_dt, grad_out, x, probs, (int)p_dt, grad_x, grad_probs, rows,
+                        hidden, stream);
 }
 
 }  // namespace moe

@@ -65,8 +65,14 @@ def swiglu_clamped_bwd(x, probs, grad_y, limit, grad_x=None, grad_probs=None, st
     return grad_x, grad_probs
 
 
+def _row_probs(probs: torch.Tensor, rows: int) -> torch.Tensor:
+    if probs.numel() != rows or not probs.is_contiguous():
+        raise ValueError("probs must be contiguous with one value per row")
+    return probs
+
+
 def router_weight_mul_fwd(x, probs, out_dtype=None, out=None, stream=None):
-    """out = (x.float() * probs.float()).to(out_dtype)."""
+    """out = (x.float() * probs.float()).to(out_dtype); probs bf16, fp16 or fp32."""
     _cuda(x, probs)
     rows, hidden = x.shape
     if not x.is_contiguous():
@@ -74,25 +80,26 @@ def router_weight_mul_fwd(x, probs, out_dtype=None, out=None, stream=None):
     out_dtype = out_dtype or x.dtype
     if out is None:
         out = torch.empty(rows, hidden, dtype=out_dtype, device=x.device)
-    _abi.moe_router_weight_mul_fwd(x, moe_dtype(x.dtype), _flat_probs(probs, rows), out,
-                                   moe_dtype(out.dtype), rows, hidden, stream)
+    _abi.moe_router_weight_mul_fwd_ex(x, moe_dtype(x.dtype), _row_probs(probs, rows),
+                                      moe_dtype(probs.dtype), out, moe_dtype(out.dtype), rows,
+                                      hidden, stream)
     return out
 
 
 def router_weight_mul_bwd(grad_out, x, probs, x_dtype=None, grad_x=None, grad_probs=None,
                           stream=None):
-    """Returns (grad_x, grad_probs or None).  Pass x=None when the forward did
-    not save x: then only grad_x is computed."""
+    """Returns (grad_x, grad_probs or None); grad_probs has probs' dtype.  Pass
+    x=None when the forward did not save x: then only grad_x is computed."""
     _cuda(grad_out, x, probs)
     rows, hidden = grad_out.shape
     x_dtype = x.dtype if x is not None else (x_dtype or grad_out.dtype)
     if grad_x is None:
         grad_x = torch.empty(rows, hidden, dtype=x_dtype, device=grad_out.device)
     if x is not None and grad_probs is None:
-        grad_probs = torch.empty(rows, 1, dtype=torch.float32, device=grad_out.device)
-    _abi.moe_router_weight_mul_bwd(grad_out, moe_dtype(grad_out.dtype), x, moe_dtype(x_dtype),
-                                   _flat_probs(probs, rows), grad_x,
-                                   grad_probs if x is not None else None, rows, hidden, stream)
+        grad_probs = torch.empty(rows, 1, dtype=probs.dtype, device=grad_out.device)
+    _abi.moe_router_weight_mul_bwd_ex(grad_out, moe_dtype(grad_out.dtype), x, moe_dtype(x_dtype),
+                                      _row_probs(probs, rows), moe_dtype(probs.dtype), grad_x,
+                                      grad_probs if x is not None else None, rows, hidden, stream)
     return grad_x, (grad_probs if x is not None else None)
 
 

@@ -73,6 +73,16 @@ def test_router_weight_validation(lib):
     # x and grad_probs must be given together
     assert _status(b, FAKE, 0, FAKE, 0, FAKE, FAKE, None, 4, 8, 0) == _abi.MOE_ERR_NULL
     assert _status(b, FAKE, 0, None, 0, FAKE, FAKE, FAKE, 4, 8, 0) == _abi.MOE_ERR_NULL
+    fx = _abi.moe_router_weight_mul_fwd_ex
+    assert _status(fx, FAKE, 0, FAKE, 9, FAKE, 0, 4, 8, 0) == _abi.MOE_ERR_DTYPE
+    # 16-bit probabilities need 2-byte alignment, fp32 ones 4
+    assert _status(fx, FAKE, 0, FAKE + 1, _abi.MOE_BF16, FAKE, 0, 4, 8, 0) == _abi.MOE_ERR_ALIGN
+    assert _status(fx, FAKE, 0, FAKE + 2, _abi.MOE_FP32, FAKE, 0, 4, 8, 0) == _abi.MOE_ERR_ALIGN
+    bx = _abi.moe_router_weight_mul_bwd_ex
+    assert _status(bx, FAKE, 0, FAKE, 0, FAKE, _abi.MOE_FP16, FAKE, FAKE + 1, 4, 8,
+                   0) == _abi.MOE_ERR_ALIGN
+    assert _status(bx, FAKE, 0, FAKE, 0, None, _abi.MOE_FP16, FAKE, FAKE, 4, 8,
+                   0) == _abi.MOE_ERR_NULL
 
 
 def test_permuted_and_unpermute_validation(lib):

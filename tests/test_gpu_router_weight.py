@@ -93,3 +93,39 @@ def test_router_weight_full_workload_sampled_rows(cuda_device, out_dtype):
     assert torch.equal((x.float() * p).to(out_dtype).view(torch.int8 if out_dtype != torch.float32
                                                           else torch.int32).cpu()[ti],
                        out.view(torch.int8 if out_dtype != torch.float32 else torch.int32).cpu()[ti])
+
+
+# Unit roundoff of the probabilities' dtype: grad_probs is the fp32 row sum
+# rounded once (RNE) to that dtype.
+UNIT_ROUNDOFF = {torch.bfloat16: 2.0 ** -8, torch.float16: 2.0 ** -11}
+
+
+@pytest.mark.parametrize("p_dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("rows,hidden", [(129, 7176), (300, 1001), (1, 8), (3000, 40)])
+@pytest.mark.parametrize("x_dtype", [torch.bfloat16, torch.float32])
+def test_router_weight_low_precision_probs(cuda_device, p_dtype, rows, hidden, x_dtype):
+    """Routing probabilities stored in bf16/fp16: out and grad_x bit-exact
+    against the oracle; grad_probs in the probabilities' dtype within one
+    rounding of it plus the reduction tolerance."""
+    d = inputs.router_weight_inputs(rows, hidden, seed=rows + 7 * hidden)
+    x = d["x"].to(x_dtype)
+    p = d["probs"].to(p_dtype)
+    xd, pd, gd = x.to(cuda_device), p.to(cuda_device), d["grad_out"].to(cuda_device)
+    out = ops.router_weight_mul_fwd(xd, pd, torch.bfloat16)
+    gx, gp = ops.router_weight_mul_bwd(gd, xd, pd)
+    gx2, gp2 = ops.router_weight_mul_bwd(gd, None, pd, x_dtype=x_dtype)
+    torch.cuda.synchronize()
+    assert gp.dtype == p_dtype and gp2 is None
+    assert_bits_equal(bits(out), oracle.router_weight_fwd(bits(x), ODT[x_dtype], bits(p),
+                                                          oracle.BF16, ODT[p_dtype]), "fwd")
+    gx_ref, gp_ref, gabs = oracle.router_weight_bwd(bits(d["grad_out"]), oracle.BF16, bits(x),
+                                                    ODT[x_dtype], bits(p), ODT[p_dtype])
+    assert_bits_equal(bits(gx), gx_ref, "grad_x")
+    assert_bits_equal(bits(gx2), gx_ref, "grad_x (x not saved)")
+    got = gp.float().cpu().numpy().ravel().astype(np.float64)
+    bound = UNIT_ROUNDOFF[p_dtype] * np.abs(gp_ref) + 1.01e-5 * np.maximum(np.abs(gp_ref), gabs)
+    assert (np.abs(got - gp_ref) <= bound).all(), "grad_probs"
+    # the 16-bit probabilities widen exactly: same bits as fp32 probabilities of equal value
+    out32 = ops.router_weight_mul_fwd(xd, pd.float(), torch.bfloat16)
+    torch.cuda.synchronize()
+    assert_bits_equal(bits(out32), bits(out), "fwd vs widened fp32 probs")
