@@ -14,7 +14,10 @@ The shapes and value distributions are those of the pages' workloads:
 * batch-invariant permuted activation and unpermute
   (core.inference.moe.batch_invariant): top-k routing over E experts, rows
   grouped by expert and padded to the grouped-GEMM alignment;
-* residual add (core.fusions.fused_moe_residual_add): three same-shape tensors.
+* residual add (core.fusions.fused_moe_residual_add): three same-shape tensors;
+* rank-order reduce-scatter (core.inference.moe.batch_invariant,
+  ordered_reduce_scatter_v): every EP rank's partial outputs for the tokens of
+  all ranks, each rank owning a ragged, contiguous block of token rows.
 """
 from __future__ import annotations
 
@@ -179,6 +182,38 @@ def residual_inputs(shape, dtype, *, seed=0, device="cpu"):
 
 
 # --------------------------------------------------- raw-bit views (numpy)
+
+@dataclasses.dataclass
+class ReduceScatterCase:
+    """world buffers [capacity_rows, hidden] (rank order); rank q's tokens are
+    rows [rank_token_offset[q], rank_token_offset[q] + counts[q]); ep_tokens =
+    sum(counts) rows hold data, the rest of each buffer is NaN ("never read")."""
+    buffers: list
+    rank_token_offset: torch.Tensor   # int32 [world]
+    counts: list
+    ep_tokens: int
+
+
+def reduce_scatter_inputs(world, tokens, hidden, *, dtype=torch.bfloat16, spare_rows=0,
+                          sigma=1.0, seed=0, device="cpu") -> ReduceScatterCase:
+    """`tokens` token rows split over `world` ranks by a uniform multinomial
+    draw (ragged counts, some possibly zero); partials ~ N(0, sigma^2) drawn in
+    fp32 and stored in `dtype`; `spare_rows` NaN rows past the data."""
+    g = _gen(seed, device)
+    owner = torch.randint(0, world, (tokens,), generator=g, device=device)
+    counts = torch.bincount(owner, minlength=world).tolist()
+    offsets = [0]
+    for c in counts[:-1]:
+        offsets.append(offsets[-1] + c)
+    cap = tokens + spare_rows
+    bufs = []
+    for _ in range(world):
+        b = torch.full((cap, hidden), float("nan"), dtype=dtype, device=device)
+        b[:tokens] = (torch.randn(tokens, hidden, generator=g, device=device) * sigma).to(dtype)
+        bufs.append(b)
+    return ReduceScatterCase(bufs, torch.tensor(offsets, dtype=torch.int32, device=device),
+                             counts, tokens)
+
 
 def bits(t: torch.Tensor):
     """numpy view of a CPU tensor: uint16 bits for 16-bit floats, else as is."""

@@ -78,6 +78,8 @@ def load(path: str) -> ctypes.CDLL:
         "orc_weighted_silu_mul_bounded": (ctypes.c_int, [P, P, P, I64, I64, I64]),
         "orc_epilogue_chain": (ctypes.c_int, [P, P, I64, P, I32, P, P, P, I64, I64, I32,
                                               ctypes.c_int, P, P]),
+        "orc_ordered_reduce_scatter_v": (ctypes.c_int, [P, I32, I32, P, I32, I64, I64, I64,
+                                                        ctypes.c_int, P, ctypes.c_int]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -278,4 +280,27 @@ def epilogue_chain(expert_output, row_probs, inverse_map, valid_tokens, shared, 
     err = _lib().orc_epilogue_chain(_p(eo), _p(rp), max_rows, _p(inv), int(valid_tokens), _p(sh),
                                     _p(rs), _p(out), tokens, hidden, n_exp, dt, _p(scratch),
                                     _p(routed))
+    return out, err
+
+
+def ordered_reduce_scatter_v(inputs, in_dt, rank, rank_token_offset, ep_tokens, out_init,
+                             out_dt):
+    """inputs: list of `world` [capacity_rows, hidden] arrays (uint16 bits for
+    bf16/fp16), one per rank in rank order; out_init: [local_tokens, hidden]
+    (its contents stand for the output buffer before the call).
+    Returns (out, error_bits)."""
+    st = _storage_np(in_dt)
+    ins = [_c(a, st) for a in inputs]
+    capacity, hidden = ins[0].shape
+    if any(a.shape != (capacity, hidden) for a in ins):
+        raise ValueError("every rank's buffer must have the same shape")
+    ptrs = (ctypes.c_void_p * len(ins))(*[a.ctypes.data for a in ins])
+    offs = _c(np.asarray(rank_token_offset, np.int32).ravel(), np.int32)
+    if offs.size != len(ins):
+        raise ValueError("one token offset per rank")
+    out = np.array(out_init, dtype=_storage_np(out_dt), copy=True)
+    local_tokens = out.shape[0]
+    err = _lib().orc_ordered_reduce_scatter_v(ctypes.cast(ptrs, ctypes.c_void_p), len(ins),
+                                              int(rank), _p(offs), int(ep_tokens), capacity,
+                                              local_tokens, hidden, in_dt, _p(out), out_dt)
     return out, err

@@ -446,3 +446,40 @@ int orc_epilogue_chain(const void *expert_output, const float *row_probs, int64_
     orc_residual_add(routed, shared_expert_output, residual, out, n * hidden, dt);
     return err;
 }
+
+/* ------------------------------------- rank-order reduce-scatter [BI] */
+
+/* [BI] ordered_reduce_scatter_v, _ordered_reduce_scatter_v_kernel ("reduce peer
+ * rows with an explicit rank-order FP32 sum"): each of `world` ranks holds a
+ * [capacity_rows, hidden] buffer (dtype in_dt) of partial results for the
+ * tokens of every rank; rank q's tokens are the rows starting at
+ * rank_token_offset[q].  Rank `rank` receives its local_tokens rows:
+ *     out[t, h] = out_dt( ((x_0 + x_1) + x_2) + ... + x_{world-1} ),
+ *     x_q = f32(inputs[q][rank_token_offset[rank] + t, h]),
+ * each add in fp32 in rank order, one rounding at the end.  Only the first
+ * ep_tokens rows of the buffers hold data (the page's ep_max_tokens); an
+ * ep_tokens outside [0, capacity_rows] is clamped, and an output row whose
+ * source row falls outside the data is neither read nor written; both set
+ * ORC_ERR_COUNT.  Returns the error bits. */
+int orc_ordered_reduce_scatter_v(const void *const *inputs, int32_t world, int32_t rank,
+                                 const int32_t *rank_token_offset, int32_t ep_tokens,
+                                 int64_t capacity_rows, int64_t local_tokens, int64_t hidden,
+                                 int in_dt, void *out, int out_dt)
+{
+    int err = 0;
+    int64_t rows = ep_tokens;
+    if (rows < 0) { rows = 0; err |= ORC_ERR_COUNT; }
+    if (rows > capacity_rows) { rows = capacity_rows; err |= ORC_ERR_COUNT; }
+    const int64_t first = rank_token_offset[rank];
+    for (int64_t t = 0; t < local_tokens; ++t) {
+        const int64_t g = first + t;
+        if (g < 0 || g >= rows) { err |= ORC_ERR_COUNT; continue; }
+        for (int64_t h = 0; h < hidden; ++h) {
+            float acc = load_as_f32(inputs[0], in_dt, g * hidden + h);
+            for (int32_t q = 1; q < world; ++q)
+                acc = acc + load_as_f32(inputs[q], in_dt, g * hidden + h);
+            store_rounded(out, out_dt, t * hidden + h, acc);
+        }
+    }
+    return err;
+}

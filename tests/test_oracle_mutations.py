@@ -55,6 +55,24 @@ MUTATIONS = [
     ("bounded_off_by_one", "for (int64_t e = 0; e < n; ++e) {\n        int64_t r = e / half_n",
      "for (int64_t e = 0; e <= n && e < rows * half_n; ++e) {\n        int64_t r = e / half_n",
      ["test_weighted_silu_mul_bounded_vs_torch"]),
+    ("rs_reverse_rank_order",
+     "float acc = load_as_f32(inputs[0], in_dt, g * hidden + h);\n"
+     "            for (int32_t q = 1; q < world; ++q)\n"
+     "                acc = acc + load_as_f32(inputs[q], in_dt, g * hidden + h);",
+     "float acc = load_as_f32(inputs[world - 1], in_dt, g * hidden + h);\n"
+     "            for (int32_t q = world - 2; q >= 0; --q)\n"
+     "                acc = acc + load_as_f32(inputs[q], in_dt, g * hidden + h);",
+     ["test_reduce_scatter_adds_in_rank_order"]),
+    ("rs_first_rank_offset", "const int64_t first = rank_token_offset[rank];",
+     "const int64_t first = rank_token_offset[0];",
+     ["test_reduce_scatter_exact_integers_pick_the_rank_rows"]),
+    ("rs_drops_last_rank", "for (int32_t q = 1; q < world; ++q)",
+     "for (int32_t q = 1; q < world - 1; ++q)",
+     ["test_reduce_scatter_exact_integers_pick_the_rank_rows"]),
+    ("rs_rounds_each_add",
+     "acc = acc + load_as_f32(inputs[q], in_dt, g * hidden + h);",
+     "acc = round_to_dtype(acc + load_as_f32(inputs[q], in_dt, g * hidden + h), out_dt);",
+     ["test_reduce_scatter_rounds_once_at_the_end"]),
     ("chain_swaps_shared_and_residual",
      "orc_residual_add(routed, shared_expert_output, residual, out, n * hidden, dt);",
      "orc_residual_add(routed, residual, shared_expert_output, out, n * hidden, dt);",

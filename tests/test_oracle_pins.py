@@ -601,3 +601,97 @@ def test_router_weight_low_precision_probs_vs_torch(p_dtype):
     want = p.grad.reshape(-1).double().numpy()
     rel = 2.0 ** -7 if p_dtype == torch.bfloat16 else 2.0 ** -10
     assert (np.abs(gp - want) <= rel * np.abs(want) + 1e-5 * gabs).all()
+
+
+# ------------------------------------------------- rank-order reduce-scatter
+
+def _rs(inputs_list, in_dt, rank, offsets, ep_tokens, local, hidden, out_dt, init=0):
+    out0 = np.full((local, hidden), init, oracle._storage_np(out_dt))
+    return oracle.ordered_reduce_scatter_v(inputs_list, in_dt, rank, offsets, ep_tokens, out0,
+                                           out_dt)
+
+
+def test_reduce_scatter_exact_integers_pick_the_rank_rows():
+    """fp32 buffers x_q[g, h] = (q + 1) * (g * hidden + h + 1): every partial
+    sum is an integer below 2^24, so the exact sum is (1 + ... + W) * (g*H + h
+    + 1) for whichever rows g were read.  A wrong offset, a dropped or repeated
+    rank, or a transposed index changes it."""
+    world, hidden, counts = 4, 6, [3, 0, 5, 2]
+    offsets = np.concatenate([[0], np.cumsum(counts)[:-1]]).astype(np.int32)
+    total = int(sum(counts))
+    cap = total + 3
+    g = np.arange(cap, dtype=np.float64)[:, None] * hidden + np.arange(hidden) + 1
+    bufs = [((q + 1) * g).astype(np.float32) for q in range(world)]
+    for rank in range(world):
+        out, err = _rs(bufs, oracle.F32, rank, offsets, total, counts[rank], hidden, oracle.F32)
+        assert err == 0
+        rows = offsets[rank] + np.arange(counts[rank])
+        want = world * (world + 1) // 2 * g[rows]
+        assert np.array_equal(out.astype(np.float64), want), rank
+
+
+def test_reduce_scatter_adds_in_rank_order():
+    """fp32 witness of the order: 2^24 + 1 rounds back to 2^24 (ties to even),
+    so ((2^24 + 1) + 1) = 2^24 while ((1 + 1) + 2^24) = 2^24 + 2."""
+    big, one = np.float32(2.0 ** 24), np.float32(1.0)
+    cols = [np.array([[big, one]], np.float32), np.array([[one, one]], np.float32),
+            np.array([[one, big]], np.float32)]
+    out, err = _rs(cols, oracle.F32, 0, [0, 0, 0], 1, 1, 2, oracle.F32)
+    assert err == 0
+    assert out[0, 0] == 2.0 ** 24 and out[0, 1] == 2.0 ** 24 + 2
+
+
+def test_reduce_scatter_rounds_once_at_the_end():
+    """bf16 witness: 1 + 2^-8 + 2^-8 = 1 + 2^-7 is a bf16 value (0x3F81), but
+    rounding after each add (1 + 2^-8 is a tie -> 1) would give 1.0 (0x3F80)."""
+    vals = [1.0, 2.0 ** -8, 2.0 ** -8]
+    bufs = [oracle.bf16_from_f32(np.array([v], np.float32)).reshape(1, 1) for v in vals]
+    out, _ = _rs(bufs, oracle.BF16, 0, [0, 0, 0], 1, 1, 1, oracle.BF16)
+    assert int(out[0, 0]) == 0x3F81
+
+
+@pytest.mark.parametrize("in_dtype,out_dtype", [(torch.bfloat16, torch.bfloat16),
+                                                (torch.float16, torch.float32),
+                                                (torch.float32, torch.bfloat16)])
+def test_reduce_scatter_two_ranks_vs_torch(in_dtype, out_dtype):
+    """W = 2: one fp32 add and one rounding, which torch computes as
+    (a.float() + b.float()).to(out); W = 1: a plain dtype conversion."""
+    odt = {torch.bfloat16: oracle.BF16, torch.float16: oracle.F16, torch.float32: oracle.F32}
+    gen = torch.Generator().manual_seed(11)
+    a = (torch.randn(40, 24, generator=gen) * 3).to(in_dtype)
+    b = (torch.randn(40, 24, generator=gen) * 3).to(in_dtype)
+    out, err = _rs([bits(a), bits(b)], odt[in_dtype], 1, [0, 17], 40, 20, 24, odt[out_dtype])
+    assert err == 0
+    assert_bits_equal(out, bits((a.float() + b.float()).to(out_dtype)[17:37]), "W=2")
+    one, _ = _rs([bits(a)], odt[in_dtype], 0, [5], 40, 30, 24, odt[out_dtype])
+    assert_bits_equal(one, bits(a.to(out_dtype)[5:35]), "W=1")
+
+
+def test_reduce_scatter_within_the_fp32_error_bound():
+    """Random bf16 partials, W = 8: the result is within the textbook bound of a
+    recursive fp32 sum, (W - 1) u32 sum|x| (u32 = 2^-24), of the exact float64
+    sum -- before the final rounding, here to fp32 so none is added."""
+    world, cap, hidden = 8, 64, 33
+    gen = torch.Generator().manual_seed(12)
+    ts = [(torch.randn(cap, hidden, generator=gen) * 10.0 ** (q % 3)).to(torch.bfloat16)
+          for q in range(world)]
+    out, err = _rs([bits(t) for t in ts], oracle.BF16, 3, [0, 8, 16, 24, 32, 40, 48, 56], 64, 8,
+                   hidden, oracle.F32)
+    assert err == 0
+    x = np.stack([t.double().numpy()[24:32] for t in ts])
+    exact, mag = x.sum(0), np.abs(x).sum(0)
+    assert (np.abs(out - exact) <= (world - 1) * 2.0 ** -24 * mag + 1e-300).all()
+
+
+def test_reduce_scatter_bounds():
+    """Rows past ep_tokens are neither read nor written; an ep_tokens beyond
+    the buffers is clamped to them; both set the count error."""
+    cap, hidden = 10, 4
+    bufs = [np.full((cap, hidden), q + 1.0, np.float32) for q in range(2)]
+    out, err = _rs(bufs, oracle.F32, 1, [0, 6], 8, 4, hidden, oracle.F32, init=-7.0)
+    assert err == oracle.ERR_COUNT
+    assert (out[:2] == 3.0).all() and (out[2:] == -7.0).all()
+    out, err = _rs(bufs, oracle.F32, 1, [0, 6], 12, 4, hidden, oracle.F32, init=-7.0)
+    assert err == oracle.ERR_COUNT and (out == 3.0).all()
+    out, err = _rs(bufs, oracle.F32, 0, [-1, 6], 10, 2, hidden, oracle.F32, init=-7.0)
+    assert err == oracle.ERR_COUNT and (out[0] == -7.0).all() and (out[1] == 3.0).all()
