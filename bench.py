@@ -235,13 +235,15 @@ def time_launches(fn, reps, device):
     return a.elapsed_time(b) / reps
 
 
-NEXT_ROWS = ("weighted_silu_mul_bounded", "epilogue_fused")
+NEXT_ROWS = ("weighted_silu_mul_bounded", "epilogue_fused", "ordered_reduce_scatter_v")
+RS_WORLD = 8  # EP ranks of the rank-order reduce-scatter, all blocks on this GPU
 
 
 def measure_next_rows(device, seed, reps, peak, scale=1.0, only=None):
-    """The ops beyond the step: the device-bounded weighted SwiGLU and the fused
+    """The ops beyond the step: the device-bounded weighted SwiGLU, the fused
     router-weight -> unpermute -> residual chain (against the same chain as
-    three launches).  Timed after the step, outside its timed region."""
+    three launches) and the rank-order reduce-scatter.  Timed after the step,
+    outside its timed region."""
     from moe_expert_epilogue_b200 import inputs, ops
     out = {}
     T = scaled(scale)["permuted"]["tokens"]
@@ -251,7 +253,41 @@ def measure_next_rows(device, seed, reps, peak, scale=1.0, only=None):
         out.update(_measure_bounded(device, seed, reps, peak, rows, half_n))
     if only in (None, "epilogue_fused"):
         out.update(_measure_fused(device, seed, reps, peak, T, K, E, A, H))
+    if only in (None, "ordered_reduce_scatter_v"):
+        out.update(_measure_reduce_scatter(device, seed, reps, peak, T, H))
     return out
+
+
+def _measure_reduce_scatter(device, seed, reps, peak, T, H, world=RS_WORLD):
+    """The rank-order reduce-scatter with every EP rank's [T, H] block on this
+    GPU: one pass = the world's launches (one per rank) back to back, together
+    reading every block once and writing T rows.  On several GPUs the same
+    kernel reads (world-1)/world of these bytes over NVLink instead."""
+    from moe_expert_epilogue_b200 import inputs, ops
+    case = inputs.reduce_scatter_inputs(world, T, H, seed=seed + 8, device=device)
+    table = ops.pointer_table(case.buffers)
+    offs = case.rank_token_offset
+    ep = torch.tensor([case.ep_tokens], dtype=torch.int32, device=device)
+    outs = [torch.empty(c, H, dtype=torch.bfloat16, device=device) for c in case.counts]
+
+    def one_pass():
+        for r in range(world):
+            ops.ordered_reduce_scatter_v(table, r, offs, ep, T, H, torch.bfloat16, out=outs[r])
+    # each launch is ~10 us of device time: replay the pass as a CUDA graph so
+    # that host launch overhead does not show in the device time
+    one_pass()
+    torch.cuda.synchronize(device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        one_pass()
+    ms = time_launches(graph.replay, reps, device)
+    del graph
+    nb = world * T * H * 2 + T * H * 2
+    return {"ordered_reduce_scatter_v": {
+        "shape": f"{world} ranks' bf16 blocks of {T} tokens x hidden {H} on one GPU, "
+                 f"{world} launches (ragged per-rank rows)",
+        "us": round(ms * 1e3, 2), "bytes": nb, "gbs": round(nb / ms / 1e6, 1),
+        "frac": round(nb / ms / 1e6 / peak, 4)}}
 
 
 def _measure_bounded(device, seed, reps, peak, rows, half_n):

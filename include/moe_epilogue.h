@@ -48,6 +48,7 @@
 #ifndef MOE_EPILOGUE_H
 #define MOE_EPILOGUE_H
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
@@ -312,6 +313,65 @@ MOE_API int moe_epilogue_fused(const void* expert_output, const float* row_probs
                                const void* residual, void* out, int64_t tokens, int64_t hidden,
                                int32_t num_local_experts, moe_dtype dt, int32_t* dev_err,
                                cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Rank-order reduce-scatter of variable token rows.
+ * [BI] ordered_reduce_scatter_v, _ordered_reduce_scatter_v_kernel (reduce
+ * peer rows with an explicit rank-order fp32 sum).  Every rank q holds at
+ * buffers[q] + input_byte_offset a row-major [capacity_rows, hidden] block
+ * (in_dt) of partial results for the tokens of all ranks; rank q's tokens are
+ * the rows starting at rank_token_offset[q].  This call writes this rank's
+ *   out[t, h] = out_dt( ((x_0 + x_1) + ...) + x_{world-1} ),
+ *   x_q = f32(input_q[rank_token_offset[rank] + t, h]),  t < local_tokens,
+ * each add in fp32 in rank order and one rounding, so the bits depend on
+ * nothing but the inputs.  Only the first *ep_tokens rows of each block hold
+ * data (the page's ep_max_tokens): an *ep_tokens outside [0, capacity_rows]
+ * is clamped, and an output row whose source row lies outside the data is
+ * neither read nor written; both set MOE_DEVERR_COUNT.
+ * buffers            DEVICE array of `world` pointers, rank order, each
+ *                    addressable from this GPU: its own memory, or a peer's
+ *                    mapped into this process (moe_ipc_open).  Read with plain
+ *                    loads (no bulk copies, no multicast).
+ * input_byte_offset  >= 0, a multiple of in_dt's size
+ * world              1..64;  rank in [0, world)
+ * rank_token_offset  int32 [world] (device)
+ * ep_tokens          int32 (device)
+ * out                out_dt [local_tokens, hidden] contiguous, this GPU
+ * dev_err            optional int32 (device)
+ * Ordering is the caller's: the launch must follow the completion of every
+ * rank's input block, and no rank may overwrite its block until every rank's
+ * launch has completed (e.g. a stream-ordered barrier -- a one-element
+ * all-reduce -- before and after).  The kernel waits on nothing.  Fast path:
+ * hidden % 8 == 0, out, input_byte_offset and every buffer 16-byte aligned.
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_ordered_reduce_scatter_v(const void* const* buffers, int64_t input_byte_offset,
+                                         int32_t world, int32_t rank,
+                                         const int32_t* rank_token_offset,
+                                         const int32_t* ep_tokens, int64_t capacity_rows,
+                                         void* out, int64_t local_tokens, int64_t hidden,
+                                         moe_dtype in_dt, moe_dtype out_dt, int32_t* dev_err,
+                                         cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Buffers shared between the processes of one node (CUDA IPC): the plumbing
+ * under moe_ordered_reduce_scatter_v's `buffers` (the pages use a symmetric-
+ * memory handle; this library maps plain device allocations instead).
+ * moe_symm_alloc  cudaMalloc of `bytes` on the current device, zero-filled;
+ *                 *ptr owned by the caller, released with moe_symm_free.
+ * moe_ipc_export  writes the MOE_IPC_HANDLE_BYTES-byte handle of an allocation
+ *                 made by moe_symm_alloc (host memory) for other processes.
+ * moe_ipc_open    maps another process's allocation into this one (peer access
+ *                 enabled as needed); *ptr is valid until moe_ipc_close.  A
+ *                 process cannot open its own handle (MOE_ERR_CUDA).
+ * Errors: MOE_ERR_NULL for NULL arguments, MOE_ERR_CUDA with
+ * moe_last_cuda_error() set otherwise.
+ * ---------------------------------------------------------------------- */
+#define MOE_IPC_HANDLE_BYTES 64
+MOE_API int moe_symm_alloc(size_t bytes, void** ptr);
+MOE_API int moe_symm_free(void* ptr);
+MOE_API int moe_ipc_export(const void* ptr, void* handle);
+MOE_API int moe_ipc_open(const void* handle, void** ptr);
+MOE_API int moe_ipc_close(void* ptr);
 
 #ifdef __cplusplus
 }

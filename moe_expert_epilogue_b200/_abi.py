@@ -38,7 +38,16 @@ SIGNATURES = {
     "moe_residual_add": [_P, _P, _P, _P, _I64, _I, _P],
     "moe_weighted_silu_mul_bounded": [_P, _P, _P, _P, _I64, _I64, _I32, _P, _P],
     "moe_epilogue_fused": [_P, _P, _I64, _P, _P, _P, _P, _P, _I64, _I64, _I32, _I, _P, _P],
+    "moe_ordered_reduce_scatter_v": [_P, _I64, _I32, _I32, _P, _P, _I64, _P, _I64, _I64, _I, _I,
+                                     _P, _P],
+    "moe_symm_alloc": [ctypes.c_size_t, ctypes.POINTER(_P)],
+    "moe_symm_free": [_P],
+    "moe_ipc_export": [_P, ctypes.c_char_p],
+    "moe_ipc_open": [ctypes.c_char_p, ctypes.POINTER(_P)],
+    "moe_ipc_close": [_P],
 }
+
+MOE_IPC_HANDLE_BYTES = 64
 
 _lock = threading.Lock()
 _lib = None
@@ -174,6 +183,45 @@ def moe_epilogue_fused(expert_output, row_probs, max_rows, inverse_map, valid_to
     _call("moe_epilogue_fused", ptr(expert_output), ptr(row_probs), max_rows, ptr(inverse_map),
           ptr(valid_tokens), ptr(shared_expert_output), ptr(residual), ptr(out), tokens, hidden,
           num_local_experts, dt, ptr(dev_err), stream_handle(stream))
+
+
+def moe_ordered_reduce_scatter_v(buffers, input_byte_offset, world, rank, rank_token_offset,
+                                 ep_tokens, capacity_rows, out, local_tokens, hidden, in_dt,
+                                 out_dt, dev_err=None, stream=None):
+    _call("moe_ordered_reduce_scatter_v", ptr(buffers), input_byte_offset, world, rank,
+          ptr(rank_token_offset), ptr(ep_tokens), capacity_rows, ptr(out), local_tokens, hidden,
+          in_dt, out_dt, ptr(dev_err), stream_handle(stream))
+
+
+def moe_symm_alloc(nbytes: int) -> int:
+    """A zero-filled device allocation of `nbytes` on the current device."""
+    p = _P(0)
+    _call("moe_symm_alloc", nbytes, ctypes.byref(p))
+    return int(p.value)
+
+
+def moe_symm_free(p: int) -> None:
+    _call("moe_symm_free", p)
+
+
+def moe_ipc_export(p: int) -> bytes:
+    """The MOE_IPC_HANDLE_BYTES-byte IPC handle of an moe_symm_alloc allocation."""
+    buf = ctypes.create_string_buffer(MOE_IPC_HANDLE_BYTES)
+    _call("moe_ipc_export", p, buf)
+    return buf.raw
+
+
+def moe_ipc_open(handle: bytes) -> int:
+    """Maps another process's allocation into this one; returns its pointer."""
+    if len(handle) != MOE_IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle has MOE_IPC_HANDLE_BYTES bytes")
+    p = _P(0)
+    _call("moe_ipc_open", handle, ctypes.byref(p))
+    return int(p.value)
+
+
+def moe_ipc_close(p: int) -> None:
+    _call("moe_ipc_close", p)
 
 
 def moe_device_errors(clear=True) -> int:

@@ -312,4 +312,25 @@ int moe_epilogue_fused(const void* expert_output, const float* row_probs, int64_
                                num_local_experts, dt, dev_err, stream);
 }
 
+int moe_ordered_reduce_scatter_v(const void* const* buffers, int64_t input_byte_offset,
+                                 int32_t world, int32_t rank, const int32_t* rank_token_offset,
+                                 const int32_t* ep_tokens, int64_t capacity_rows, void* out,
+                                 int64_t local_tokens, int64_t hidden, moe_dtype in_dt,
+                                 moe_dtype out_dt, int32_t* dev_err, cudaStream_t stream) {
+  if (!dtype_ok(in_dt) || !dtype_ok(out_dt)) return MOE_ERR_DTYPE;
+  if (world < 1 || world > max_reduce_scatter_world() || rank < 0 || rank >= world ||
+      local_tokens < 0 || hidden < 0 || capacity_rows < 0 || input_byte_offset < 0 ||
+      !product_ok(local_tokens, hidden) || !product_ok(capacity_rows, hidden))
+    return MOE_ERR_SHAPE;
+  if (local_tokens == 0 || hidden == 0) return MOE_OK;
+  if (!buffers || !rank_token_offset || !ep_tokens || !out) return MOE_ERR_NULL;
+  if (!aligned_to(buffers, sizeof(void*)) || !aligned_to(rank_token_offset, 4) ||
+      !aligned_to(ep_tokens, 4) || !aligned_to(out, dtype_size(out_dt)) ||
+      !aligned_to(dev_err, 4) || input_byte_offset % dtype_size(in_dt) != 0)
+    return MOE_ERR_ALIGN;
+  return launch_ordered_reduce_scatter_v(buffers, input_byte_offset, world, rank,
+                                         rank_token_offset, ep_tokens, capacity_rows, out,
+                                         local_tokens, hidden, in_dt, out_dt, dev_err, stream);
+}
+
 }  // extern "C"

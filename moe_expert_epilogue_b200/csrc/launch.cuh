@@ -62,6 +62,12 @@ int launch_swiglu_clamped_bwd(const void* x, const float* probs, const void* gra
                               void* grad_x, float* grad_probs, int64_t rows, int64_t inter,
                               int64_t ld_x, int64_t ld_gy, int64_t ld_gx, float limit,
                               moe_dtype dt, cudaStream_t stream);
+int max_reduce_scatter_world();
+int launch_ordered_reduce_scatter_v(const void* const* bufs, int64_t byte_off, int world, int rank,
+                                    const int32_t* offs, const int32_t* ep_tokens,
+                                    int64_t capacity, void* out, int64_t local, int64_t hidden,
+                                    moe_dtype in_dt, moe_dtype out_dt, int32_t* err,
+                                    cudaStream_t stream);
 int launch_router_weight_fwd(const void* x, moe_dtype x_dt, const void* probs, moe_dtype p_dt,
                              void* out, moe_dtype out_dt, int64_t rows, int64_t hidden,
                              cudaStream_t stream);

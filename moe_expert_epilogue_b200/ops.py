@@ -168,3 +168,39 @@ def epilogue_fused(expert_output, row_probs, inverse_map, valid_tokens, shared_e
                             shared_expert_output, residual, out, tokens, hidden, n_exp,
                             moe_dtype(residual.dtype), dev_err, stream)
     return out
+
+
+def pointer_table(tensors, device=None) -> torch.Tensor:
+    """int64 [len(tensors)] device array of the tensors' data pointers, in order
+    (the `buffers` argument of ordered_reduce_scatter_v for buffers that this
+    GPU holds itself)."""
+    device = device or tensors[0].device
+    return torch.tensor([t.data_ptr() for t in tensors], dtype=torch.int64, device=device)
+
+
+def ordered_reduce_scatter_v(buffers, rank, rank_token_offset, ep_tokens, capacity_rows, hidden,
+                             in_dtype, local_tokens=None, out=None, out_dtype=None,
+                             input_byte_offset=0, dev_err=None, stream=None):
+    """This rank's rows of the rank-order fp32 reduce-scatter.
+
+    buffers: int64 device tensor [world] of pointers (rank order) to each rank's
+    [capacity_rows, hidden] block of `in_dtype` at `input_byte_offset`;
+    rank_token_offset int32 [world] and ep_tokens int32 [1] on the device.
+    Returns out [local_tokens, hidden] (`out_dtype`, default in_dtype).  The
+    caller orders the launch against the other ranks' writes."""
+    _cuda(buffers, rank_token_offset, ep_tokens, out, dev_err)
+    if buffers.dtype != torch.int64 or buffers.dim() != 1:
+        raise ValueError("buffers must be an int64 vector of device pointers")
+    world = buffers.numel()
+    if out is None:
+        if local_tokens is None:
+            raise ValueError("give local_tokens or out")
+        out = torch.empty(local_tokens, hidden, dtype=out_dtype or in_dtype,
+                          device=buffers.device)
+    elif not out.is_contiguous() or out.dim() != 2 or out.shape[1] != hidden:
+        raise ValueError("out must be a contiguous [local_tokens, hidden] tensor")
+    _abi.moe_ordered_reduce_scatter_v(buffers, int(input_byte_offset), world, int(rank),
+                                      rank_token_offset, ep_tokens, int(capacity_rows), out,
+                                      out.shape[0], hidden, moe_dtype(in_dtype),
+                                      moe_dtype(out.dtype), dev_err, stream)
+    return out

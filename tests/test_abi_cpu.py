@@ -98,6 +98,36 @@ def test_permuted_and_unpermute_validation(lib):
     assert _status(u, FAKE, 0, 4, FAKE, FAKE + 2, FAKE, 0, 4, 8, 4, None, 0) == _abi.MOE_ERR_ALIGN
 
 
+def test_reduce_scatter_validation(lib):
+    f = _abi.moe_ordered_reduce_scatter_v
+    ok = dict(buffers=FAKE, input_byte_offset=0, world=4, rank=1, rank_token_offset=FAKE,
+              ep_tokens=FAKE, capacity_rows=100, out=FAKE, local_tokens=10, hidden=64,
+              in_dt=_abi.MOE_BF16, out_dt=_abi.MOE_BF16)
+
+    def st(**kw):
+        return _status(f, *dict(ok, **kw).values())
+    assert st(in_dt=5) == _abi.MOE_ERR_DTYPE
+    assert st(world=0) == _abi.MOE_ERR_SHAPE and st(world=65) == _abi.MOE_ERR_SHAPE
+    assert st(rank=4) == _abi.MOE_ERR_SHAPE and st(rank=-1) == _abi.MOE_ERR_SHAPE
+    assert st(input_byte_offset=-16) == _abi.MOE_ERR_SHAPE
+    assert st(buffers=None) == _abi.MOE_ERR_NULL and st(ep_tokens=None) == _abi.MOE_ERR_NULL
+    assert st(input_byte_offset=1) == _abi.MOE_ERR_ALIGN
+    assert st(buffers=FAKE + 4) == _abi.MOE_ERR_ALIGN
+    assert st(out=FAKE + 2, out_dt=_abi.MOE_FP32) == _abi.MOE_ERR_ALIGN
+    f(*dict(ok, local_tokens=0, buffers=None).values())          # nothing to do: a no-op
+
+
+def test_ipc_argument_checks(lib):
+    import ctypes
+    assert lib.moe_symm_alloc(16, None) == _abi.MOE_ERR_NULL
+    assert lib.moe_ipc_export(None, ctypes.create_string_buffer(64)) == _abi.MOE_ERR_NULL
+    assert lib.moe_ipc_open(None, None) == _abi.MOE_ERR_NULL
+    assert lib.moe_ipc_close(None) == _abi.MOE_ERR_NULL
+    assert lib.moe_symm_free(None) == _abi.MOE_OK
+    with pytest.raises(ValueError):
+        _abi.moe_ipc_open(b"short")
+
+
 def test_residual_validation(lib):
     r = _abi.moe_residual_add
     assert _status(r, FAKE, FAKE, FAKE, FAKE, 16, 3, 0) == _abi.MOE_ERR_DTYPE
