@@ -21,68 +21,110 @@ def moe_dtype(dtype: torch.dtype) -> int:
 
 
 def _cuda(*ts):
+    """Every given tensor on one CUDA device (checked after the shape checks,
+    just before the library call)."""
+    dev = None
     for t in ts:
-        if t is not None and not t.is_cuda:
+        if t is None:
+            continue
+        if not t.is_cuda:
             raise ValueError("tensors must live on a CUDA device")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors on different devices: {dev} and {t.device}")
 
 
-def _rows_stride(t: torch.Tensor) -> int:
-    if t.dim() != 2 or t.stride(1) != 1:
-        raise ValueError("expected a 2-D tensor with unit column stride")
+def _check(t, name, dtype=None, shape=None, numel=None, contiguous=True):
+    """Dtype, shape (or element count) and contiguity of one argument; the C ABI
+    trusts the sizes it is given, so a mismatch must stop here."""
+    if t is None:
+        return
+    if dtype is not None:
+        allowed = dtype if isinstance(dtype, tuple) else (dtype,)
+        if t.dtype not in allowed:
+            raise TypeError(f"{name}: dtype {t.dtype}, expected {' or '.join(map(str, allowed))}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name}: {t.numel()} elements, expected {numel}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+_FLOATS = (torch.bfloat16, torch.float16, torch.float32)
+
+
+def _rows_stride(t: torch.Tensor, name="tensor") -> int:
+    if t.dim() != 2 or t.stride(1) != 1 or (t.shape[0] > 1 and t.stride(0) < t.shape[1]):
+        raise ValueError(f"{name}: expected a 2-D tensor with unit column stride and "
+                         "non-overlapping rows")
     return t.stride(0)
 
 
-def _flat_probs(probs: torch.Tensor, rows: int) -> torch.Tensor:
-    if probs.dtype != torch.float32 or probs.numel() != rows or not probs.is_contiguous():
-        raise ValueError("probs must be a contiguous fp32 tensor with one value per row")
+def _flat_probs(probs: torch.Tensor, rows: int, name="probs") -> torch.Tensor:
+    _check(probs, name, dtype=torch.float32, numel=rows)
     return probs
 
 
+def _two_d(t, name):
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D, got shape {tuple(t.shape)}")
+    return t.shape
+
+
 def swiglu_clamped_fwd(x, probs, limit, out=None, stream=None):
-    """y = silu(clamp(gate, max=L)) * clamp(up, -L, L) * probs (bf16)."""
-    _cuda(x, probs)
-    rows, two_i = x.shape
+    """y = silu(clamp(gate, max=L)) * clamp(up, -L, L) * probs, in x's dtype."""
+    rows, two_i = _two_d(x, "x")
+    if two_i % 2:
+        raise ValueError("x must hold [gate | up]: an even number of columns")
     inter = two_i // 2
+    _check(x, "x", dtype=_FLOATS, contiguous=False)
     if out is None:
         out = torch.empty(rows, inter, dtype=x.dtype, device=x.device)
-    _abi.moe_swiglu_clamped_fwd(x, _flat_probs(probs, rows), out, rows, inter, _rows_stride(x),
-                                _rows_stride(out), limit, moe_dtype(x.dtype), stream)
+    _check(out, "out", dtype=x.dtype, shape=(rows, inter), contiguous=False)
+    ld_x, ld_y = _rows_stride(x, "x"), _rows_stride(out, "out")
+    _flat_probs(probs, rows)
+    _cuda(x, probs, out)
+    _abi.moe_swiglu_clamped_fwd(x, probs, out, rows, inter, ld_x, ld_y, limit,
+                                moe_dtype(x.dtype), stream)
     return out
 
 
 def swiglu_clamped_bwd(x, probs, grad_y, limit, grad_x=None, grad_probs=None, stream=None):
-    """Returns (grad_x [rows, 2*inter] bf16, grad_probs [rows, 1] fp32)."""
-    _cuda(x, probs, grad_y)
-    rows, two_i = x.shape
+    """Returns (grad_x [rows, 2*inter] in x's dtype, grad_probs [rows, 1] fp32)."""
+    rows, two_i = _two_d(x, "x")
+    if two_i % 2:
+        raise ValueError("x must hold [gate | up]: an even number of columns")
     inter = two_i // 2
+    _check(x, "x", dtype=_FLOATS, contiguous=False)
+    _check(grad_y, "grad_y", dtype=x.dtype, shape=(rows, inter), contiguous=False)
     if grad_x is None:
-        grad_x = torch.empty_like(x)
+        grad_x = torch.empty_like(x, memory_format=torch.contiguous_format)
     if grad_probs is None:
         grad_probs = torch.empty(rows, 1, dtype=torch.float32, device=x.device)
-    _abi.moe_swiglu_clamped_bwd(x, _flat_probs(probs, rows), grad_y, grad_x, grad_probs, rows,
-                                inter, _rows_stride(x), _rows_stride(grad_y),
-                                _rows_stride(grad_x), limit, moe_dtype(x.dtype), stream)
+    _check(grad_x, "grad_x", dtype=x.dtype, shape=(rows, two_i), contiguous=False)
+    _check(grad_probs, "grad_probs", dtype=torch.float32, numel=rows)
+    ld_x, ld_gy, ld_gx = (_rows_stride(x, "x"), _rows_stride(grad_y, "grad_y"),
+                          _rows_stride(grad_x, "grad_x"))
+    _flat_probs(probs, rows)
+    _cuda(x, probs, grad_y, grad_x, grad_probs)
+    _abi.moe_swiglu_clamped_bwd(x, probs, grad_y, grad_x, grad_probs, rows, inter, ld_x, ld_gy,
+                                ld_gx, limit, moe_dtype(x.dtype), stream)
     return grad_x, grad_probs
-
-
-def _row_probs(probs: torch.Tensor, rows: int) -> torch.Tensor:
-    if probs.numel() != rows or not probs.is_contiguous():
-        raise ValueError("probs must be contiguous with one value per row")
-    return probs
 
 
 def router_weight_mul_fwd(x, probs, out_dtype=None, out=None, stream=None):
     """out = (x.float() * probs.float()).to(out_dtype); probs bf16, fp16 or fp32."""
-    _cuda(x, probs)
-    rows, hidden = x.shape
-    if not x.is_contiguous():
-        raise ValueError("x must be contiguous")
-    out_dtype = out_dtype or x.dtype
+    rows, hidden = _two_d(x, "x")
+    _check(x, "x", dtype=_FLOATS)
+    _check(probs, "probs", dtype=_FLOATS, numel=rows)
     if out is None:
-        out = torch.empty(rows, hidden, dtype=out_dtype, device=x.device)
-    _abi.moe_router_weight_mul_fwd_ex(x, moe_dtype(x.dtype), _row_probs(probs, rows),
-                                      moe_dtype(probs.dtype), out, moe_dtype(out.dtype), rows,
-                                      hidden, stream)
+        out = torch.empty(rows, hidden, dtype=out_dtype or x.dtype, device=x.device)
+    _check(out, "out", dtype=_FLOATS, shape=(rows, hidden))
+    _cuda(x, probs, out)
+    _abi.moe_router_weight_mul_fwd_ex(x, moe_dtype(x.dtype), probs, moe_dtype(probs.dtype), out,
+                                      moe_dtype(out.dtype), rows, hidden, stream)
     return out
 
 
@@ -90,28 +132,43 @@ def router_weight_mul_bwd(grad_out, x, probs, x_dtype=None, grad_x=None, grad_pr
                           stream=None):
     """Returns (grad_x, grad_probs or None); grad_probs has probs' dtype.  Pass
     x=None when the forward did not save x: then only grad_x is computed."""
-    _cuda(grad_out, x, probs)
-    rows, hidden = grad_out.shape
+    rows, hidden = _two_d(grad_out, "grad_out")
+    _check(grad_out, "grad_out", dtype=_FLOATS)
+    _check(x, "x", dtype=_FLOATS, shape=(rows, hidden))
+    _check(probs, "probs", dtype=_FLOATS, numel=rows)
     x_dtype = x.dtype if x is not None else (x_dtype or grad_out.dtype)
     if grad_x is None:
         grad_x = torch.empty(rows, hidden, dtype=x_dtype, device=grad_out.device)
-    if x is not None and grad_probs is None:
+    _check(grad_x, "grad_x", dtype=x_dtype, shape=(rows, hidden))
+    if x is None:
+        grad_probs = None
+    elif grad_probs is None:
         grad_probs = torch.empty(rows, 1, dtype=probs.dtype, device=grad_out.device)
+    _check(grad_probs, "grad_probs", dtype=probs.dtype, numel=rows)
+    _cuda(grad_out, x, probs, grad_x, grad_probs)
     _abi.moe_router_weight_mul_bwd_ex(grad_out, moe_dtype(grad_out.dtype), x, moe_dtype(x_dtype),
-                                      _row_probs(probs, rows), moe_dtype(probs.dtype), grad_x,
-                                      grad_probs if x is not None else None, rows, hidden, stream)
-    return grad_x, (grad_probs if x is not None else None)
+                                      probs, moe_dtype(probs.dtype), grad_x, grad_probs, rows,
+                                      hidden, stream)
+    return grad_x, grad_probs
 
 
 def act_with_probs_permuted(act, x, permutation_map, n_used, probs, clamp_scale=1.0,
                             zero_padding=False, out=None, dev_err=None, stream=None):
     """Activation with router probabilities over the padded, expert-grouped
-    layout; act is MOE_ACT_SQRELU, MOE_ACT_SQRELU_CLAMP or MOE_ACT_SWIGLU."""
-    _cuda(x, permutation_map, n_used, probs, dev_err)
-    max_rows, cols = x.shape
+    layout (bf16); act is MOE_ACT_SQRELU, MOE_ACT_SQRELU_CLAMP or MOE_ACT_SWIGLU."""
+    max_rows, cols = _two_d(x, "x")
+    if act == MOE_ACT_SWIGLU and cols % 2:
+        raise ValueError("SwiGLU input must hold [gate | up]: an even number of columns")
     width = cols // 2 if act == MOE_ACT_SWIGLU else cols
+    _check(x, "x", dtype=torch.bfloat16)
+    _check(permutation_map, "permutation_map", dtype=torch.int32, numel=max_rows)
+    _check(n_used, "n_used", dtype=torch.int32, numel=1)
+    _check(probs, "probs", dtype=torch.float32)
+    _check(dev_err, "dev_err", dtype=torch.int32, numel=1)
     if out is None:
         out = torch.empty(max_rows, width, dtype=x.dtype, device=x.device)
+    _check(out, "out", dtype=torch.bfloat16, shape=(max_rows, width))
+    _cuda(x, permutation_map, n_used, probs, out, dev_err)
     _abi.moe_act_with_probs_permuted(act, x, out, permutation_map, n_used, probs, probs.numel(),
                                      max_rows, width, clamp_scale, zero_padding, dev_err, stream)
     return out
@@ -119,9 +176,14 @@ def act_with_probs_permuted(act, x, permutation_map, n_used, probs, clamp_scale=
 
 def unpermute_ordered(expert_output, inverse_map, valid_tokens, out, dev_err=None, stream=None):
     """out[t] = sum over increasing local expert e of expert_output[inverse_map[t, e]]."""
+    max_rows, hidden = _two_d(expert_output, "expert_output")
+    tokens, n_exp = _two_d(inverse_map, "inverse_map")
+    _check(expert_output, "expert_output", dtype=_FLOATS)
+    _check(inverse_map, "inverse_map", dtype=torch.int32)
+    _check(valid_tokens, "valid_tokens", dtype=torch.int32, numel=1)
+    _check(out, "out", dtype=_FLOATS, shape=(tokens, hidden))
+    _check(dev_err, "dev_err", dtype=torch.int32, numel=1)
     _cuda(expert_output, inverse_map, valid_tokens, out, dev_err)
-    max_rows, hidden = expert_output.shape
-    tokens, n_exp = inverse_map.shape
     _abi.moe_unpermute_ordered(expert_output, moe_dtype(expert_output.dtype), max_rows,
                                inverse_map, valid_tokens, out, moe_dtype(out.dtype), tokens,
                                hidden, n_exp, dev_err, stream)
@@ -129,10 +191,16 @@ def unpermute_ordered(expert_output, inverse_map, valid_tokens, out, dev_err=Non
 
 
 def residual_add(expert_output, shared_expert_output, residual, out=None, stream=None):
-    """out = residual + (expert_output + shared_expert_output), two roundings."""
-    _cuda(expert_output, shared_expert_output, residual)
+    """out = residual + (expert_output + shared_expert_output), two roundings;
+    out may be residual itself (in place)."""
+    _check(residual, "residual", dtype=_FLOATS)
+    for t, name in ((expert_output, "expert_output"),
+                    (shared_expert_output, "shared_expert_output")):
+        _check(t, name, dtype=residual.dtype, shape=residual.shape)
     if out is None:
         out = torch.empty_like(residual)
+    _check(out, "out", dtype=residual.dtype, shape=residual.shape)
+    _cuda(expert_output, shared_expert_output, residual, out)
     _abi.moe_residual_add(expert_output, shared_expert_output, residual, out, residual.numel(),
                           moe_dtype(residual.dtype), stream)
     return out
@@ -142,31 +210,45 @@ def weighted_silu_mul_bounded(y, weights, bound_elems, num_programs=0, out=None,
                               stream=None):
     """out[r, j] = bf16(silu(gate) * up * weights[r]) for flat elements below the
     device-resident bound_elems (int64); y is [rows, 2*half_n] (gate | up)."""
-    _cuda(y, weights, bound_elems, dev_err)
-    rows, two_h = y.shape
+    rows, two_h = _two_d(y, "y")
+    if two_h % 2:
+        raise ValueError("y must hold [gate | up]: an even number of columns")
     half_n = two_h // 2
-    if bound_elems.dtype != torch.int64:
-        raise TypeError("bound_elems must be an int64 device tensor")
+    _check(y, "y", dtype=torch.bfloat16)
+    _check(bound_elems, "bound_elems", dtype=torch.int64, numel=1)
+    _check(dev_err, "dev_err", dtype=torch.int32, numel=1)
+    _flat_probs(weights, rows, "weights")
     if out is None:
         out = torch.empty(rows, half_n, dtype=y.dtype, device=y.device)
-    _abi.moe_weighted_silu_mul_bounded(y, _flat_probs(weights, rows), out, bound_elems, rows,
-                                       half_n, num_programs, dev_err, stream)
+    _check(out, "out", dtype=torch.bfloat16, shape=(rows, half_n))
+    _cuda(y, weights, bound_elems, out, dev_err)
+    _abi.moe_weighted_silu_mul_bounded(y, weights, out, bound_elems, rows, half_n, num_programs,
+                                       dev_err, stream)
     return out
 
 
 def epilogue_fused(expert_output, row_probs, inverse_map, valid_tokens, shared_expert_output,
                    residual, out=None, dev_err=None, stream=None):
     """residual + (unpermute(expert_output * row_probs) + shared), every rounding of
-    the three-step chain kept, in one kernel."""
-    _cuda(expert_output, row_probs, inverse_map, valid_tokens, shared_expert_output, residual,
-          dev_err)
-    max_rows, hidden = expert_output.shape
-    tokens, n_exp = inverse_map.shape
+    the three-step chain kept, in one kernel; out may be residual (in place)."""
+    max_rows, hidden = _two_d(expert_output, "expert_output")
+    tokens, n_exp = _two_d(inverse_map, "inverse_map")
+    _check(residual, "residual", dtype=_FLOATS, shape=(tokens, hidden))
+    dt = residual.dtype
+    _check(expert_output, "expert_output", dtype=dt)
+    _check(shared_expert_output, "shared_expert_output", dtype=dt, shape=(tokens, hidden))
+    _flat_probs(row_probs, max_rows, "row_probs")
+    _check(inverse_map, "inverse_map", dtype=torch.int32)
+    _check(valid_tokens, "valid_tokens", dtype=torch.int32, numel=1)
+    _check(dev_err, "dev_err", dtype=torch.int32, numel=1)
     if out is None:
         out = torch.empty_like(residual)
+    _check(out, "out", dtype=dt, shape=(tokens, hidden))
+    _cuda(expert_output, row_probs, inverse_map, valid_tokens, shared_expert_output, residual,
+          out, dev_err)
     _abi.moe_epilogue_fused(expert_output, row_probs, max_rows, inverse_map, valid_tokens,
                             shared_expert_output, residual, out, tokens, hidden, n_exp,
-                            moe_dtype(residual.dtype), dev_err, stream)
+                            moe_dtype(dt), dev_err, stream)
     return out
 
 
@@ -188,17 +270,21 @@ def ordered_reduce_scatter_v(buffers, rank, rank_token_offset, ep_tokens, capaci
     rank_token_offset int32 [world] and ep_tokens int32 [1] on the device.
     Returns out [local_tokens, hidden] (`out_dtype`, default in_dtype).  The
     caller orders the launch against the other ranks' writes."""
-    _cuda(buffers, rank_token_offset, ep_tokens, out, dev_err)
-    if buffers.dtype != torch.int64 or buffers.dim() != 1:
-        raise ValueError("buffers must be an int64 vector of device pointers")
+    if buffers.dim() != 1:
+        raise ValueError("buffers must be a vector of device pointers")
+    _check(buffers, "buffers", dtype=torch.int64)
     world = buffers.numel()
+    _check(rank_token_offset, "rank_token_offset", dtype=torch.int32, numel=world)
+    _check(ep_tokens, "ep_tokens", dtype=torch.int32, numel=1)
+    _check(dev_err, "dev_err", dtype=torch.int32, numel=1)
     if out is None:
         if local_tokens is None:
             raise ValueError("give local_tokens or out")
         out = torch.empty(local_tokens, hidden, dtype=out_dtype or in_dtype,
                           device=buffers.device)
-    elif not out.is_contiguous() or out.dim() != 2 or out.shape[1] != hidden:
-        raise ValueError("out must be a contiguous [local_tokens, hidden] tensor")
+    _two_d(out, "out")
+    _check(out, "out", dtype=_FLOATS, shape=(out.shape[0], hidden))
+    _cuda(buffers, rank_token_offset, ep_tokens, out, dev_err)
     _abi.moe_ordered_reduce_scatter_v(buffers, int(input_byte_offset), world, int(rank),
                                       rank_token_offset, ep_tokens, int(capacity_rows), out,
                                       out.shape[0], hidden, moe_dtype(in_dtype),
