@@ -138,7 +138,7 @@ MOE_API int moe_swiglu_clamped_fwd(const void* x, const float* probs, void* y, i
  * probs       fp32 [rows]
  * grad_y      dt [rows, ld_gy], ld_gy >= inter
  * grad_x      dt [rows, ld_gx], ld_gx >= 2*inter  (output)
- * grad_probs  fp32 [rows]                         (output)
+ * grad_probs  fp32 [rows]                         (output; +0 when inter == 0)
  * dt          MOE_BF16, MOE_FP16 or MOE_FP32
  * ---------------------------------------------------------------------- */
 MOE_API int moe_swiglu_clamped_bwd(const void* x, const float* probs, const void* grad_y,
@@ -167,10 +167,12 @@ MOE_API int moe_router_weight_mul_fwd(const void* x, moe_dtype x_dt, const float
  * grad_out    g_dt [rows, hidden] contiguous (the forward output's dtype)
  * x           x_dt [rows, hidden] contiguous, or NULL when the forward did
  *             not save x (save_x false): then grad_probs must be NULL too and
- *             only grad_x is computed (x is never read).
+ *             only grad_x is computed (x is never read).  With hidden == 0, x
+ *             has no elements and may be NULL either way.
  * probs       fp32 [rows]
  * grad_x      x_dt [rows, hidden]  (output)
- * grad_probs  fp32 [rows] or NULL  (output; fixed-order row reduction)
+ * grad_probs  fp32 [rows] or NULL  (output; fixed-order row reduction; the
+ *             empty sum +0 when hidden == 0)
  * ---------------------------------------------------------------------- */
 MOE_API int moe_router_weight_mul_bwd(const void* grad_out, moe_dtype g_dt, const void* x,
                               moe_dtype x_dt, const float* probs, void* grad_x,

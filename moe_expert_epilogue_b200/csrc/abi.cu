@@ -6,7 +6,9 @@
 // row-major x with one probability per row;
 // core.fusions.fused_moe_residual_add.can_use_fused_moe_residual_add: same
 // shape and dtype in {BF16, FP16, FP32}) and the swiglu_limit > 0 contract of
-// the clamped SwiGLU.  Sizes of zero return MOE_OK without a launch.
+// the clamped SwiGLU.  Sizes of zero return MOE_OK without a launch; the one
+// output an empty size still defines, a probability-gradient sum over no
+// terms, is written as +0 by a memset.
 #include <atomic>
 #include <cmath>
 #include <mutex>
@@ -68,6 +70,13 @@ int ensure_smem_limit(const void* kernel, size_t smem) {
 int cuda_fail(cudaError_t e) {
   g_last_cuda_error = (int)e;
   return MOE_ERR_CUDA;
+}
+
+// The sum over no terms is +0: all-zero bits in every dtype of the library.
+int zero_fill(void* p, int64_t bytes, cudaStream_t stream) {
+  if (!p || bytes <= 0) return MOE_OK;
+  const cudaError_t e = cudaMemsetAsync(p, 0, (size_t)bytes, stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
 int check_launch() {
@@ -165,6 +174,7 @@ int moe_swiglu_clamped_bwd(const void* x, const float* probs, const void* grad_y
   if (!aligned_to(x, es) || !aligned_to(grad_y, es) || !aligned_to(grad_x, es) ||
       !aligned_to(probs, 4) || !aligned_to(grad_probs, 4))
     return MOE_ERR_ALIGN;
+  if (inter == 0) return zero_fill(grad_probs, rows * 4, stream);   // empty sums: +0
   return launch_swiglu_clamped_bwd(x, probs, grad_y, grad_x, grad_probs, rows, inter, ld_x,
                                    ld_gy, ld_gx, limit, dt, stream);
 }
@@ -195,7 +205,9 @@ int moe_router_weight_mul_bwd_ex(const void* grad_out, moe_dtype g_dt, const voi
                                  cudaStream_t stream) {
   if (!dtype_ok(g_dt) || !dtype_ok(x_dt) || !dtype_ok(probs_dt)) return MOE_ERR_DTYPE;
   if (rows < 0 || hidden < 0 || !product_ok(rows, hidden)) return MOE_ERR_SHAPE;
-  if ((x == nullptr) != (grad_probs == nullptr)) return MOE_ERR_NULL;
+  // x and grad_probs come together (save_x); with hidden == 0 x has no
+  // elements and may be NULL, and grad_probs alone asks for the empty sums.
+  if (hidden > 0 && (x == nullptr) != (grad_probs == nullptr)) return MOE_ERR_NULL;
   if (rows == 0) return MOE_OK;
   if (!probs) return MOE_ERR_NULL;
   if (hidden > 0 && (!grad_out || !grad_x)) return MOE_ERR_NULL;
@@ -203,7 +215,7 @@ int moe_router_weight_mul_bwd_ex(const void* grad_out, moe_dtype g_dt, const voi
       !aligned_to(grad_x, dtype_size(x_dt)) || !aligned_to(probs, dtype_size(probs_dt)) ||
       !aligned_to(grad_probs, dtype_size(probs_dt)))
     return MOE_ERR_ALIGN;
-  if (hidden == 0 && grad_probs == nullptr) return MOE_OK;
+  if (hidden == 0) return zero_fill(grad_probs, rows * dtype_size(probs_dt), stream);
   return launch_router_weight_bwd(grad_out, g_dt, x, x_dt, probs, probs_dt, grad_x, grad_probs,
                                   rows, hidden, stream);
 }
