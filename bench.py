@@ -738,18 +738,77 @@ def oracle_step(w):
             + 4 * Rs * RESIDUAL["hidden"] * 2)
 
 
-def cpu_baseline(frac, steps=1):
+def cpu_baseline(frac, steps=1, all_cores=True):
+    """The oracle on the host: single-threaded on the first `frac` of every
+    op's rows, and (all_cores) the same fraction split over one process per
+    host core."""
     w = cpu_sample_workload(frac)
     t0 = time.perf_counter()
     b = 0
     for _ in range(steps):
         b += oracle_step(w)
     dt = time.perf_counter() - t0
-    return {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "seconds": round(dt, 2), "host_cpu": _cpu_model(), "host_nproc": os.cpu_count(),
-            "sample": f"first {frac:g} of the rows/tokens of every op of the step "
-                      f"(swiglu rows {w['R']}, router rows {w['Rr']}, tokens {w['T']}, "
-                      f"residual rows {w['Rs']}); single-threaded C oracle, -O2"}
+    out = {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "seconds": round(dt, 2), "host_cpu": _cpu_model(), "host_nproc": os.cpu_count(),
+           "sample": f"first {frac:g} of the rows/tokens of every op of the step "
+                     f"(swiglu rows {w['R']}, router rows {w['Rr']}, tokens {w['T']}, "
+                     f"residual rows {w['Rs']}); single-threaded C oracle, -O2"}
+    del w
+    if all_cores and (os.cpu_count() or 1) > 1:
+        out["all_cores"] = oracle_pool(frac, os.cpu_count(), warmup=1, steps=4 * max(1, steps))
+    return out
+
+
+def _oracle_worker(frac, seed, warmup, steps, barrier_, q):
+    """One process of the host pool: its own sample, warm-up passes, then the
+    timed passes started together with the other processes."""
+    try:
+        w = cpu_sample_workload(frac, seed)
+        for _ in range(warmup):
+            oracle_step(w)
+        barrier_.wait(timeout=600)
+        t0 = time.perf_counter()
+        b = 0
+        for _ in range(steps):
+            b += oracle_step(w)
+        q.put((b, time.perf_counter() - t0, None))
+    except Exception as e:  # reported to the parent, which raises
+        q.put((0, 0.0, repr(e)))
+
+
+def oracle_pool(frac_total, n, warmup=1, steps=1):
+    """The oracle as it stands on `n` host processes (spawned), each on its own
+    seeded sample of frac_total / n of every op's rows: aggregate GB/s = all
+    processes' algorithmic bytes / the slowest process's time."""
+    import multiprocessing as mp
+    import oracle
+    oracle.build()                       # built once here, loaded by every process
+    ctx = mp.get_context("spawn")
+    barrier_ = ctx.Barrier(n + 1)
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_oracle_worker,
+                         args=(frac_total / n, 7919 * (i + 1), warmup, steps, barrier_, q))
+             for i in range(n)]
+    for p in procs:
+        p.start()
+    try:
+        barrier_.wait(timeout=600)
+        res = [q.get(timeout=1200) for _ in range(n)]
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    errs = [e for _, _, e in res if e]
+    if errs:
+        raise RuntimeError(f"oracle pool: {errs[0]}")
+    b = sum(r[0] for r in res)
+    dt = max(r[1] for r in res)
+    return {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": n, "kind": "oracle",
+            "seconds": round(dt, 2),
+            "sample": f"{n} processes, each its own seeded sample of {frac_total / n:.4g} of the "
+                      f"rows/tokens of every op ({frac_total:g} in total), {steps} timed "
+                      "pass(es) after a warm-up; single-threaded C oracle in each"}
 
 
 def _cpu_model():
@@ -762,38 +821,33 @@ def _cpu_model():
     return None
 
 
-def reference_fraction(args) -> float:
-    """Row fraction of every op the oracle runs per step in the reference arm:
-    --cpu-sample if given, else sized so that the warm-up and timed steps take
-    about two minutes on a ~17 s-per-full-step host (capped at a quarter)."""
+def reference_fraction(args, cores=1) -> float:
+    """Row fraction of every op the oracle runs per step in the reference arm
+    (split over `cores` processes): --cpu-sample if given, else sized so that
+    the warm-up and timed steps take about two minutes on a host that needs
+    ~17 s of one core per full step, capped at half the workload (host memory)."""
     if args.cpu_sample is not None:
         return args.cpu_sample
-    return max(0.005, min(0.25, 120.0 / (17.0 * max(1, args.steps + args.warmup))))
+    return max(0.005, min(0.5, 120.0 * cores / (17.0 * max(1, args.steps + args.warmup))))
 
 
 def run_reference(args):
+    """The reference arm: the CPU oracle, as it stands, on every host core (one
+    process per core, each on its share of the sampled rows)."""
     rank, _, world = dist_env()
     if rank != 0:
         return
-    args.cpu_sample = reference_fraction(args)
-    w = cpu_sample_workload(args.cpu_sample)
-    for _ in range(args.warmup):
-        oracle_step(w)
-    t0 = time.perf_counter()
-    b = 0
-    for _ in range(args.steps):
-        b += oracle_step(w)
-    dt = time.perf_counter() - t0
-    value = round(b / dt / 1e9, 4)
+    n = max(1, os.cpu_count() or 1)
+    args.cpu_sample = reference_fraction(args, n)
+    pool = oracle_pool(args.cpu_sample, n, warmup=args.warmup, steps=args.steps)
+    value = pool["value"]
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(dt / args.steps * 1e3, 2), "higher_is_better": True,
+        "ms_per_step": round(pool["seconds"] / args.steps * 1e3, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD_NAME, "sample_fraction": args.cpu_sample},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"first {args.cpu_sample:g} of the rows/tokens of every op per "
-                                   "step; single-threaded C oracle"},
+        "cpu_baseline": pool,
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
