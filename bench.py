@@ -859,7 +859,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--e2e-steps", type=int, default=20,
+                    help="pipelined end-to-end steps (fill and drain of the copy pipeline "
+                         "are amortised over them)")
     ap.add_argument("--cpu-sample", type=float, default=None,
                     help="fraction of the rows of every op the CPU oracle runs (default: "
                          "0.25 for the cpu_baseline; sized to the step count for the "
