@@ -20,9 +20,16 @@ time (CUDA events on the launching stream, barrier + synchronize on both
 sides).  Per-kernel durations come from CUDA events around each launch on
 every 10th timed step (event records between kernels would stop the
 programmatic launch overlap on every step).  Every kernel's working set
-exceeds the 126 MB L2, so no flush is needed between steps.  Multi-GPU runs (torchrun) are weak scaling: each rank
-runs the full step on its own inputs; the only collectives are the barrier and
-the max of the timings.
+exceeds the 126 MB L2, so no flush is needed between steps.  Multi-GPU runs
+(torchrun) are weak scaling: each rank runs the full step on its own inputs;
+the only collectives are the barrier and the max of the timings.
+
+The line also carries `e2e` (the same step through the public API with every
+input copied from pinned host memory and every output copied back inside the
+timed region, pipelined), `next_rows` (the bounded SwiGLU, the fused chain and
+the rank-order reduce-scatter, timed after the step), `clocks`, `roofline` and
+`cpu_baseline` (the CPU oracle, one core and all cores).  `--impl reference`
+times the CPU oracle alone on every host core.
 """
 from __future__ import annotations
 
