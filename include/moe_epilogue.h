@@ -1,41 +1,50 @@
 /*
  * moe_epilogue.h -- C ABI of the B200 (sm_100a) MoE expert-epilogue library.
  *
- * Seven memory-bound ops that sit between the grouped GEMMs of a
- * Mixture-of-Experts layer and the residual stream.  Each entry point takes
- * caller-owned DEVICE pointers, sizes and a CUDA stream, validates its
- * arguments on the host, enqueues exactly one kernel on `stream` and returns.
+ * The memory-bound ops that sit between the grouped GEMMs of a
+ * Mixture-of-Experts layer and the residual stream (the seven of the hot path,
+ * their dtype variants, the bounded SwiGLU, the fused epilogue chain and the
+ * rank-order reduce-scatter), plus the IPC helpers under the reduce-scatter.
+ * Each op entry point takes caller-owned DEVICE pointers, sizes and a CUDA
+ * stream, validates its arguments on the host, enqueues exactly one kernel on
+ * `stream` and returns.
  *
  * Common contract
  *   - Ownership: every pointer is owned by the caller and must stay valid
- *     until the enqueued kernel has finished.  The library allocates nothing,
- *     keeps no per-call state and never synchronises, so calls may be captured
- *     in a CUDA graph.
+ *     until the enqueued kernel has finished.  The op entry points allocate
+ *     nothing, keep no per-call state and never synchronise, so calls may be
+ *     captured in a CUDA graph.  (Only moe_symm_alloc and moe_ipc_open create
+ *     anything; the caller releases it with moe_symm_free / moe_ipc_close.)
  *   - Layout: 2-D tensors are row-major.  `ld_*` arguments are leading
  *     dimensions in ELEMENTS (the distance between the starts of two rows);
  *     where no leading dimension is taken, rows are contiguous.
- *   - Counts that change at run time (n_used, valid_tokens) are int32 values
- *     in DEVICE memory, read by the kernel, so a captured graph stays valid as
- *     they change.  The matching maximum sizes are host arguments.
+ *   - Counts that change at run time (n_used, valid_tokens, bound_elems,
+ *     ep_tokens, rank offsets) live in DEVICE memory, read by the kernel, so
+ *     a captured graph stays valid as they change.  The matching maximum sizes
+ *     are host arguments.
  *   - Alignment: every pointer must be aligned to its element size
  *     (MOE_ERR_ALIGN otherwise).  16-byte aligned pointers and leading
  *     dimensions / widths that are multiples of 8 elements take the
  *     vectorised path; anything else takes an element-wise path inside the
  *     same kernel family with identical results.
  *   - Aliasing: outputs must not overlap inputs, except that
- *     moe_residual_add may run in place (out == residual).
+ *     moe_residual_add and moe_epilogue_fused may run in place
+ *     (out == residual).
  *   - Errors: the return value is MOE_OK or one of the MOE_ERR_* codes below.
  *     Argument errors are detected before anything is enqueued.  MOE_ERR_CUDA
  *     means a CUDA runtime call failed (moe_last_cuda_error() gives the
  *     cudaError_t); note that an asynchronous error left pending by earlier
- *     work on the device can surface here too.  Sizes of zero are valid no-ops.
- *   - Device error word: the two ops that read routing metadata from device
- *     memory take an optional `int32_t* dev_err` (device memory, may be
- *     NULL).  Out-of-range metadata never causes an out-of-bounds access:
+ *     work on the device can surface here too.  Sizes of zero are valid
+ *     no-ops, except that a probability gradient over zero columns is still
+ *     written: the empty sum, +0.
+ *   - Device error word: the ops that read counts or routing metadata from
+ *     device memory take an optional `int32_t* dev_err` (device memory, may
+ *     be NULL).  Out-of-range metadata never causes an out-of-bounds access:
  *     the kernel clamps or skips and ORs MOE_DEVERR_* bits into *dev_err.
  *   - Numerics: inputs are widened to fp32, the documented formula is
  *     evaluated in fp32 and each output is rounded once to its dtype with
- *     round-to-nearest-even.  Every result is independent of the grid size,
+ *     round-to-nearest-even (the fused chain keeps each rounding of the
+ *     three steps it fuses).  Every result is independent of the grid size,
  *     of the other rows / tokens in the batch and of the run (no atomics in
  *     any reduction).
  *
