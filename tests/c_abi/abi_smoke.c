@@ -6,7 +6,10 @@
  * values computed here in plain C on exactly representable inputs:
  *   residual add: e = i, s = 0.5, r = 2  (all exact in fp32)  -> out = i + 2.5
  *   clamped SwiGLU with gate = 0: silu(0) = 0 -> y = +0 whatever up and p are
- * It also checks that a bad argument returns MOE_ERR_LIMIT without a launch.
+ * It also checks that a bad argument returns MOE_ERR_LIMIT without a launch, and
+ * runs the rank-order reduce-scatter over three buffers from moe_symm_alloc
+ * (exact integers: block q holds (q + 1) * (row * 16 + col + 1), so rank 1's
+ * rows 4..7 sum to 6 * (row * 16 + col + 1)), after exporting an IPC handle.
  * Exit status 0 on success.
  */
 #include <stdio.h>
@@ -71,6 +74,43 @@ int main(void) {
       MOE_ERR_LIMIT) {
     fprintf(stderr, "a negative limit was not rejected\n");
     return 1;
+  }
+  /* rank-order reduce-scatter over three library-allocated buffers */
+  {
+    enum { W = 3, CAP = 10, HID = 16, LOCAL = 4 };
+    void* blocks[W];
+    float hb[CAP * HID];
+    for (int q = 0; q < W; ++q) {
+      CHECK(moe_symm_alloc(CAP * HID * sizeof(float), &blocks[q]));
+      for (int i = 0; i < CAP * HID; ++i) hb[i] = (float)((q + 1) * (i + 1));
+      CHECK(cudaMemcpy(blocks[q], hb, sizeof(hb), cudaMemcpyHostToDevice));
+    }
+    unsigned char handle[MOE_IPC_HANDLE_BYTES];
+    CHECK(moe_ipc_export(blocks[0], handle));
+    void** table;
+    int32_t *offs, *ep;
+    float* out;
+    const int32_t h_offs[W] = {0, 4, 8}, h_ep = CAP;
+    CHECK(cudaMalloc((void**)&table, sizeof(blocks)));
+    CHECK(cudaMemcpy(table, blocks, sizeof(blocks), cudaMemcpyHostToDevice));
+    CHECK(cudaMalloc((void**)&offs, sizeof(h_offs)));
+    CHECK(cudaMemcpy(offs, h_offs, sizeof(h_offs), cudaMemcpyHostToDevice));
+    CHECK(cudaMalloc((void**)&ep, sizeof(h_ep)));
+    CHECK(cudaMemcpy(ep, &h_ep, sizeof(h_ep), cudaMemcpyHostToDevice));
+    CHECK(cudaMalloc((void**)&out, LOCAL * HID * sizeof(float)));
+    CHECK(moe_ordered_reduce_scatter_v((const void* const*)table, 0, W, 1, offs, ep, CAP, out,
+                                       LOCAL, HID, MOE_FP32, MOE_FP32, NULL, 0));
+    CHECK(cudaMemcpy(hb, out, LOCAL * HID * sizeof(float), cudaMemcpyDeviceToHost));
+    for (int i = 0; i < LOCAL * HID; ++i)
+      if (hb[i] != (float)(6 * (4 * HID + i + 1))) {
+        fprintf(stderr, "reduce-scatter: element %d is %g\n", i, hb[i]);
+        return 1;
+      }
+    for (int q = 0; q < W; ++q) CHECK(moe_symm_free(blocks[q]));
+    CHECK(cudaFree(table));
+    CHECK(cudaFree(offs));
+    CHECK(cudaFree(ep));
+    CHECK(cudaFree(out));
   }
   CHECK(cudaDeviceSynchronize());
   printf("abi_smoke: ok (%s)\n", moe_status_string(MOE_OK));
