@@ -129,23 +129,17 @@ def stream_barrier(group=None, device=None):
 def ordered_reduce_scatter_v(output: torch.Tensor, symm: SymmetricBuffer,
                              rank_token_offset: torch.Tensor, ep_tokens: torch.Tensor,
                              capacity_rows: int, hidden: int, in_dtype: torch.dtype,
-                             input_byte_offset: int = 0, dev_err=None,
-                             launch=None) -> torch.Tensor:
+                             input_byte_offset: int = 0, dev_err=None) -> torch.Tensor:
     """Collective over symm.group: this rank's `output` [local_tokens, hidden]
     = the rank-order fp32 sum of its token rows over every rank's block
     ([capacity_rows, hidden] of in_dtype at input_byte_offset in the symmetric
-    buffer), launched on the current stream.  `launch` replaces the kernel
-    call (host-side tests only)."""
+    buffer), launched on the current stream between two stream barriers."""
     esize = torch.empty((), dtype=in_dtype).element_size()
     if input_byte_offset + capacity_rows * hidden * esize > symm.nbytes:
         raise ValueError("the input block does not fit in the symmetric buffer")
     stream_barrier(symm.group, symm.device)
-    if launch is None:
-        ops.ordered_reduce_scatter_v(symm.table, symm.rank, rank_token_offset, ep_tokens,
-                                     capacity_rows, hidden, in_dtype, out=output,
-                                     input_byte_offset=input_byte_offset, dev_err=dev_err)
-    else:
-        launch(symm, output, rank_token_offset, ep_tokens, capacity_rows, hidden, in_dtype,
-               input_byte_offset)
+    ops.ordered_reduce_scatter_v(symm.table, symm.rank, rank_token_offset, ep_tokens,
+                                 capacity_rows, hidden, in_dtype, out=output,
+                                 input_byte_offset=input_byte_offset, dev_err=dev_err)
     stream_barrier(symm.group, symm.device)
     return output

@@ -6,7 +6,8 @@ by the "IPC handle"), so the real exchange protocol of SymmetricBuffer runs:
 allocate, export, all-gather the handles, open the peers' buffers, build the
 rank-ordered pointer table, barrier, reduce, barrier, unmap, free.  The
 reduction itself is the CPU oracle reading the peers' buffers through the
-table -- the CUDA kernel behind it is covered by the gpu tests.  Each rank
+table, patched in for the kernel call inside the spawned CPU processes -- the
+CUDA kernel itself is covered by the gpu tests.  Each rank
 checks its rows bit for bit against the oracle run on all ranks' seeded
 partials regenerated locally."""
 import os
@@ -73,19 +74,24 @@ class ShmIpc:
         return torch.tensor(ptrs, dtype=torch.int64)
 
 
-def _oracle_launch(symm, out, offsets, ep_tokens, cap, hidden, in_dtype, byte_offset):
-    """Reads every rank's block through symm's pointer table, rank order."""
-    import oracle
-    from moe_expert_epilogue_b200.inputs import bits
-    ins = []
-    for p in symm.table.tolist():
-        raw = symm.backend.view(p, symm.nbytes, None)
-        blk = raw[byte_offset:byte_offset + cap * hidden * 2].view(in_dtype).view(cap, hidden)
-        ins.append(bits(blk.clone()))
-    res, err = oracle.ordered_reduce_scatter_v(ins, oracle.BF16, symm.rank, offsets.numpy(),
-                                               int(ep_tokens), bits(out), oracle.F32)
-    assert err == 0
-    out.copy_(torch.from_numpy(res))
+def _oracle_kernel(backend):
+    """Stands in for the kernel call inside the spawned CPU workers: the oracle
+    reading every rank's block through the pointer table, rank order."""
+    def launch(table, rank, offsets, ep_tokens, cap, hidden, in_dtype, out=None,
+               input_byte_offset=0, dev_err=None):
+        import oracle
+        from moe_expert_epilogue_b200.inputs import bits
+        ins = []
+        for p in table.tolist():
+            raw = backend.view(p, backend.segs[p].size, None)
+            blk = raw[input_byte_offset:input_byte_offset + cap * hidden * 2]
+            ins.append(bits(blk.view(in_dtype).view(cap, hidden).clone()))
+        res, err = oracle.ordered_reduce_scatter_v(ins, oracle.BF16, rank, offsets.numpy(),
+                                                   int(ep_tokens), bits(out), oracle.F32)
+        assert err == 0
+        out.copy_(torch.from_numpy(res))
+        return out
+    return launch
 
 
 def _worker(rank, world, port, q):
@@ -95,10 +101,11 @@ def _worker(rank, world, port, q):
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     try:
-        from moe_expert_epilogue_b200 import inputs, symmetric
+        from moe_expert_epilogue_b200 import inputs, ops, symmetric
         case = inputs.reduce_scatter_inputs(world, TOKENS, HIDDEN, spare_rows=CAP_SPARE, seed=7)
         cap = TOKENS + CAP_SPARE
         backend = ShmIpc()
+        ops.ordered_reduce_scatter_v = _oracle_kernel(backend)     # this CPU process only
         nbytes = BYTE_OFFSET + cap * HIDDEN * 2
         symm = symmetric.SymmetricBuffer(nbytes, device=torch.device("cpu"), backend=backend)
         assert symm.ptrs[rank] == symm.local and len(symm.ptrs) == world
@@ -106,8 +113,7 @@ def _worker(rank, world, port, q):
         out = torch.full((case.counts[rank], HIDDEN), -1.0)
         symmetric.ordered_reduce_scatter_v(out, symm, case.rank_token_offset,
                                            torch.tensor([case.ep_tokens]), cap, HIDDEN,
-                                           torch.bfloat16, input_byte_offset=BYTE_OFFSET,
-                                           launch=_oracle_launch)
+                                           torch.bfloat16, input_byte_offset=BYTE_OFFSET)
         symm.close()
         q.put((rank, out.numpy().copy(), backend.log))
     finally:
