@@ -173,6 +173,16 @@ int launch(const void* const* bufs, int64_t byte_off, int world, int rank, const
     const int64_t per_block = (int64_t)kThreads * kUnroll * kVec;
     if (int rc = persistent_grid((const void*)k, 0, (n + per_block - 1) / per_block, &grid))
       return rc;
+    {
+      // the fewest CTAs that keep every thread's iteration count the same: no
+      // partial last round of a few threads (one launch per rank is short, so
+      // that round is a visible share of it; measured 65.8 -> 63.4 us for 8
+      // ranks' blocks of 4096 tokens x 4096, neutral at larger sizes)
+      const int64_t units = n / kVec, per = (int64_t)grid * kThreads * kUnroll;
+      const int64_t iters = (units + per - 1) / per;
+      const int64_t g = (units + iters * kThreads * kUnroll - 1) / (iters * kThreads * kUnroll);
+      grid = (int)(g < 1 ? 1 : g);
+    }
     launch_kernel(k, grid, 0, stream, bufs, byte_off, world, rank, offs, ep_tokens, capacity,
                   static_cast<TO*>(out), local, hidden, err);
   } else {
