@@ -17,7 +17,10 @@ The shapes and value distributions are those of the pages' workloads:
 * residual add (core.fusions.fused_moe_residual_add): three same-shape tensors;
 * rank-order reduce-scatter (core.inference.moe.batch_invariant,
   ordered_reduce_scatter_v): every EP rank's partial outputs for the tokens of
-  all ranks, each rank owning a ragged, contiguous block of token rows.
+  all ranks, each rank owning a ragged, contiguous block of token rows;
+* EP combine (the same page's unpermute followed by the reduce-scatter): the
+  top-k routing of the tokens of all ranks over world x experts-per-rank
+  experts, each rank holding its own experts' expert-grouped rows.
 """
 from __future__ import annotations
 
@@ -213,6 +216,55 @@ def reduce_scatter_inputs(world, tokens, hidden, *, dtype=torch.bfloat16, spare_
         bufs.append(b)
     return ReduceScatterCase(bufs, torch.tensor(offsets, dtype=torch.int32, device=device),
                              counts, tokens)
+
+
+@dataclasses.dataclass
+class EpCombineCase:
+    """Per rank q (rank order): expert_outputs[q] [max_rows, hidden], the rows of
+    its experts (expert-grouped, padded; NaN past its rows), and inverse_maps[q]
+    int32 [tokens, experts_per_rank] over the tokens of all ranks (row in
+    expert_outputs[q], or -1).  Rank q owns tokens [rank_token_offset[q],
+    + counts[q])."""
+    expert_outputs: list
+    inverse_maps: list
+    rank_token_offset: torch.Tensor
+    counts: list
+    tokens: int
+    max_rows: int
+    routing: Routing
+
+
+def ep_combine_inputs(world, tokens, top_k, experts_per_rank, align, hidden, *,
+                      dtype=torch.bfloat16, seed=0, device="cpu") -> EpCombineCase:
+    """Expert parallelism over `world` ranks: uniform top-k routing over
+    world * experts_per_rank experts (distinct per token); rank q hosts experts
+    [q * experts_per_rank, (q + 1) * experts_per_rank); expert outputs ~ N(0,1);
+    tokens split over the ranks by a uniform multinomial draw."""
+    E = world * experts_per_rank
+    rt = routing(tokens, top_k, E, align, seed=seed, device=device)
+    eo = expert_output_input(rt, hidden, dtype=dtype, seed=seed + 1, device=device)
+    padded = (rt.counts + align - 1) // align * align
+    starts = torch.cumsum(padded, 0) - padded
+    bounds = []
+    for q in range(world):
+        e0, e1 = q * experts_per_rank, (q + 1) * experts_per_rank
+        bounds.append((int(starts[e0]), int(starts[e1 - 1] + padded[e1 - 1])))
+    max_rows = max(1, max(r1 - r0 for r0, r1 in bounds))
+    eos, invs = [], []
+    for q, (r0, r1) in enumerate(bounds):
+        blk = torch.full((max_rows, hidden), float("nan"), dtype=dtype, device=device)
+        blk[:r1 - r0] = eo[r0:r1]
+        eos.append(blk)
+        inv = rt.inverse_map[:, q * experts_per_rank:(q + 1) * experts_per_rank]
+        invs.append(torch.where(inv >= 0, inv - r0, torch.full_like(inv, -1)).contiguous())
+    g = _gen(seed + 2, device)
+    owner = torch.randint(0, world, (tokens,), generator=g, device=device)
+    counts = torch.bincount(owner, minlength=world).tolist()
+    offsets = [0]
+    for c in counts[:-1]:
+        offsets.append(offsets[-1] + c)
+    return EpCombineCase(eos, invs, torch.tensor(offsets, dtype=torch.int32, device=device),
+                         counts, tokens, max_rows, rt)
 
 
 def bits(t: torch.Tensor):

@@ -80,6 +80,9 @@ def load(path: str) -> ctypes.CDLL:
                                               ctypes.c_int, P, P]),
         "orc_ordered_reduce_scatter_v": (ctypes.c_int, [P, I32, I32, P, I32, I64, I64, I64,
                                                         ctypes.c_int, P, ctypes.c_int]),
+        "orc_unpermute_reduce_scatter": (ctypes.c_int, [P, ctypes.c_int, I64, P, I32, I64, I32,
+                                                        I32, I32, P, ctypes.c_int, P, P,
+                                                        ctypes.c_int, I64, I64]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -303,4 +306,31 @@ def ordered_reduce_scatter_v(inputs, in_dt, rank, rank_token_offset, ep_tokens, 
     err = _lib().orc_ordered_reduce_scatter_v(ctypes.cast(ptrs, ctypes.c_void_p), len(ins),
                                               int(rank), _p(offs), int(ep_tokens), capacity,
                                               local_tokens, hidden, in_dt, _p(out), out_dt)
+    return out, err
+
+
+def unpermute_reduce_scatter(expert_outputs, eo_dt, inverse_maps, ep_tokens, rank,
+                             rank_token_offset, partial_dt, out_init, out_dt):
+    """expert_outputs: list of `world` [max_rows, hidden] arrays (one per rank,
+    rank order); inverse_maps: list of int32 [capacity_rows, E] arrays over the
+    token rows of all ranks; out_init: [local_tokens, hidden] (prior contents).
+    Returns (out, error_bits)."""
+    st = _storage_np(eo_dt)
+    eos = [_c(a, st) for a in expert_outputs]
+    max_rows, hidden = eos[0].shape
+    invs = [_c(a, np.int32) for a in inverse_maps]
+    capacity, n_exp = invs[0].shape
+    if any(a.shape != (max_rows, hidden) for a in eos) or \
+            any(a.shape != (capacity, n_exp) for a in invs) or len(eos) != len(invs):
+        raise ValueError("one [max_rows, hidden] block and one [capacity, E] map per rank")
+    world = len(eos)
+    eo_ptrs = (ctypes.c_void_p * world)(*[a.ctypes.data for a in eos])
+    inv_ptrs = (ctypes.c_void_p * world)(*[a.ctypes.data for a in invs])
+    offs = _c(np.asarray(rank_token_offset, np.int32).ravel(), np.int32)
+    out = np.array(out_init, dtype=_storage_np(out_dt), copy=True)
+    partials = np.zeros(world * capacity * hidden, _storage_np(partial_dt))
+    err = _lib().orc_unpermute_reduce_scatter(
+        ctypes.cast(eo_ptrs, ctypes.c_void_p), eo_dt, max_rows,
+        ctypes.cast(inv_ptrs, ctypes.c_void_p), n_exp, capacity, int(ep_tokens), world,
+        int(rank), _p(offs), partial_dt, _p(partials), _p(out), out_dt, out.shape[0], hidden)
     return out, err

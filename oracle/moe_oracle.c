@@ -483,3 +483,38 @@ int orc_ordered_reduce_scatter_v(const void *const *inputs, int32_t world, int32
     }
     return err;
 }
+
+/* --------------- EP combine: unpermute, then rank-order reduce-scatter [BI] */
+
+/* [BI] _unpermute_tokens_in_expert_order_kernel followed by
+ * ordered_reduce_scatter_v, materialised as the pages run them: every rank q
+ * unpermutes its own expert outputs (expert_outputs[q], rows of its
+ * num_local_experts experts, inverse_maps[q] over the capacity_rows token rows
+ * of all ranks) for the first ep_tokens tokens into a block of partial sums of
+ * dtype partial_dt; rank `rank` then sums its token rows over the ranks'
+ * blocks in rank order and rounds once to out_dt.  `partials` is a
+ * caller-provided buffer of world * capacity_rows * hidden elements of
+ * partial_dt (the symmetric buffers).  Returns the error bits of both steps. */
+int orc_unpermute_reduce_scatter(const void *const *expert_outputs, int eo_dt, int64_t max_rows,
+                                 const int32_t *const *inverse_maps, int32_t num_local_experts,
+                                 int64_t capacity_rows, int32_t ep_tokens, int32_t world,
+                                 int32_t rank, const int32_t *rank_token_offset, int partial_dt,
+                                 void *partials, void *out, int out_dt, int64_t local_tokens,
+                                 int64_t hidden)
+{
+    int err = 0;
+    const int64_t esize = partial_dt == ORC_F32 ? 4 : 2;
+    const void *blocks[64];
+    if (world < 1 || world > 64) return ORC_ERR_COUNT;
+    for (int32_t q = 0; q < world; ++q) {
+        void *block = (char *)partials + (int64_t)q * capacity_rows * hidden * esize;
+        err |= orc_unpermute_ordered(expert_outputs[q], eo_dt, max_rows, inverse_maps[q],
+                                     ep_tokens, block, partial_dt, capacity_rows, hidden,
+                                     num_local_experts);
+        blocks[q] = block;
+    }
+    err |= orc_ordered_reduce_scatter_v(blocks, world, rank, rank_token_offset, ep_tokens,
+                                        capacity_rows, local_tokens, hidden, partial_dt, out,
+                                        out_dt);
+    return err;
+}

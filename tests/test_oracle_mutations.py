@@ -73,6 +73,10 @@ MUTATIONS = [
      "acc = acc + load_as_f32(inputs[q], in_dt, g * hidden + h);",
      "acc = round_to_dtype(acc + load_as_f32(inputs[q], in_dt, g * hidden + h), out_dt);",
      ["test_reduce_scatter_rounds_once_at_the_end"]),
+    ("combine_first_rank_map_for_all",
+     "err |= orc_unpermute_ordered(expert_outputs[q], eo_dt, max_rows, inverse_maps[q],",
+     "err |= orc_unpermute_ordered(expert_outputs[q], eo_dt, max_rows, inverse_maps[0],",
+     ["test_ep_combine_exact_integers"]),
     ("chain_swaps_shared_and_residual",
      "orc_residual_add(routed, shared_expert_output, residual, out, n * hidden, dt);",
      "orc_residual_add(routed, residual, shared_expert_output, out, n * hidden, dt);",

@@ -695,3 +695,76 @@ def test_reduce_scatter_bounds():
     assert err == oracle.ERR_COUNT and (out == 3.0).all()
     out, err = _rs(bufs, oracle.F32, 0, [-1, 6], 10, 2, hidden, oracle.F32, init=-7.0)
     assert err == oracle.ERR_COUNT and (out[0] == -7.0).all() and (out[1] == 3.0).all()
+
+
+# ------------------------------------------------ EP combine (unpermute + RS)
+
+@pytest.mark.parametrize("partial_dtype,out_dtype", [(torch.bfloat16, torch.bfloat16),
+                                                     (torch.float32, torch.bfloat16),
+                                                     (torch.float32, torch.float32)])
+def test_ep_combine_is_the_composition_of_the_two_steps(partial_dtype, out_dtype):
+    """Per rank, the oracle's unpermute into a partial block, then its
+    rank-order reduce-scatter (both pinned above) -- called one after another
+    here -- give the combined function's bits."""
+    odt = {torch.bfloat16: oracle.BF16, torch.float32: oracle.F32}
+    case = inputs.ep_combine_inputs(3, 40, 3, 4, 4, 24, seed=21)
+    eos = [bits(e) for e in case.expert_outputs]
+    invs = [bits(i) for i in case.inverse_maps]
+    blocks = []
+    for q in range(3):
+        blk, err = oracle.unpermute_ordered(eos[q], oracle.BF16, invs[q], case.tokens,
+                                            np.zeros((case.tokens, 24),
+                                                     oracle._storage_np(odt[partial_dtype])),
+                                            odt[partial_dtype])
+        assert err == 0
+        blocks.append(blk)
+    offs = case.rank_token_offset.numpy()
+    for rank in range(3):
+        init = np.zeros((case.counts[rank], 24), oracle._storage_np(odt[out_dtype]))
+        want, err = oracle.ordered_reduce_scatter_v(blocks, odt[partial_dtype], rank, offs,
+                                                    case.tokens, init, odt[out_dtype])
+        got, err2 = oracle.unpermute_reduce_scatter(eos, oracle.BF16, invs, case.tokens, rank,
+                                                    offs, odt[partial_dtype], init, odt[out_dtype])
+        assert err == err2 == 0
+        assert_bits_equal(got, want, f"rank {rank}")
+
+
+def test_ep_combine_exact_integers():
+    """fp32 expert rows holding small integers: every sum is exact, so the
+    result is the integer sum over all ranks' experts of the token's rows,
+    computed here by brute force in int64 from the routing."""
+    world, tokens, top_k, epr, H = 4, 30, 3, 2, 5
+    case = inputs.ep_combine_inputs(world, tokens, top_k, epr, 2, H, dtype=torch.float32,
+                                    seed=22)
+    rng = np.random.default_rng(0)
+    eos = [rng.integers(-50, 50, (case.max_rows, H)).astype(np.float32) for _ in range(world)]
+    invs = [bits(i) for i in case.inverse_maps]
+    offs = case.rank_token_offset.numpy()
+    for rank in range(world):
+        got, err = oracle.unpermute_reduce_scatter(
+            eos, oracle.F32, invs, tokens, rank, offs, oracle.F32,
+            np.zeros((case.counts[rank], H), np.float32), oracle.F32)
+        assert err == 0
+        for t in range(case.counts[rank]):
+            g = offs[rank] + t
+            want = np.zeros(H, np.int64)
+            for q in range(world):
+                for e in range(epr):
+                    r = invs[q][g, e]
+                    if r >= 0:
+                        want += eos[q][r].astype(np.int64)
+            assert np.array_equal(got[t].astype(np.int64), want), (rank, t)
+
+
+def test_ep_combine_rounds_each_rank_partial():
+    """bf16 partials: rank 0's experts give 1 + 2^-8 (a tie: rounds to 1), rank 1
+    gives 2^-8, so the combined fp32 result is 1 + 2^-8; with fp32 partials it
+    is 1 + 2^-7.  One token, one column."""
+    vals = [[1.0, 2.0 ** -8], [2.0 ** -8, 0.0]]
+    eos = [np.array([[v] for v in vals[q]], np.float32) for q in range(2)]
+    invs = [np.array([[0, 1]], np.int32), np.array([[0, -1]], np.int32)]
+    out_b, _ = oracle.unpermute_reduce_scatter(eos, oracle.F32, invs, 1, 0, [0, 1], oracle.BF16,
+                                               np.zeros((1, 1), np.float32), oracle.F32)
+    out_f, _ = oracle.unpermute_reduce_scatter(eos, oracle.F32, invs, 1, 0, [0, 1], oracle.F32,
+                                               np.zeros((1, 1), np.float32), oracle.F32)
+    assert out_b[0, 0] == 1.0 + 2.0 ** -8 and out_f[0, 0] == 1.0 + 2.0 ** -7
