@@ -242,7 +242,8 @@ def time_launches(fn, reps, device):
     return a.elapsed_time(b) / reps
 
 
-NEXT_ROWS = ("weighted_silu_mul_bounded", "epilogue_fused", "ordered_reduce_scatter_v")
+NEXT_ROWS = ("weighted_silu_mul_bounded", "epilogue_fused", "ordered_reduce_scatter_v",
+             "unpermute_reduce_scatter")
 RS_WORLD = 8  # EP ranks of the rank-order reduce-scatter, all blocks on this GPU
 
 
@@ -262,7 +263,62 @@ def measure_next_rows(device, seed, reps, peak, scale=1.0, only=None):
         out.update(_measure_fused(device, seed, reps, peak, T, K, E, A, H))
     if only in (None, "ordered_reduce_scatter_v"):
         out.update(_measure_reduce_scatter(device, seed, reps, peak, T, H))
+    if only in (None, "unpermute_reduce_scatter"):
+        out.update(_measure_ep_combine(device, seed, reps, peak, T, K, E, A, H))
     return out
+
+
+def _graph_time(fn, reps, device):
+    """Mean device time of fn replayed as one CUDA graph (fn issues several
+    short launches whose host overhead would otherwise show)."""
+    fn()
+    torch.cuda.synchronize(device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fn()
+    ms = time_launches(graph.replay, reps, device)
+    del graph
+    return ms
+
+
+def _measure_ep_combine(device, seed, reps, peak, T, K, E, A, H, world=RS_WORLD):
+    """EP combine with every rank's expert rows on this GPU: the fused kernel
+    (one launch per rank) against the pages' two steps with the library's own
+    kernels (each rank's unpermute into a partial block, then one
+    reduce-scatter launch per rank)."""
+    from moe_expert_epilogue_b200 import inputs, ops
+    case = inputs.ep_combine_inputs(world, T, K, E // world, A, H, seed=seed + 9, device=device)
+    eo_t = ops.pointer_table(case.expert_outputs)
+    inv_t = ops.pointer_table(case.inverse_maps)
+    offs = case.rank_token_offset
+    ep = torch.tensor([T], dtype=torch.int32, device=device)
+    outs = [torch.empty(c, H, dtype=torch.bfloat16, device=device) for c in case.counts]
+
+    def fused():
+        for r in range(world):
+            ops.unpermute_reduce_scatter(eo_t, torch.bfloat16, case.max_rows, inv_t, E // world, T,
+                                         ep, r, offs, H, out=outs[r])
+    blocks = [torch.empty(T, H, dtype=torch.bfloat16, device=device) for _ in range(world)]
+    blk_t = ops.pointer_table(blocks)
+
+    def two_step():
+        for q in range(world):
+            ops.unpermute_ordered(case.expert_outputs[q], case.inverse_maps[q], ep, blocks[q])
+        for r in range(world):
+            ops.ordered_reduce_scatter_v(blk_t, r, offs, ep, T, H, torch.bfloat16, out=outs[r])
+    ms_f = _graph_time(fused, reps, device)
+    ms_2 = _graph_time(two_step, reps, device)
+    live = T * K
+    nb_f = live * H * 2 + world * T * (E // world) * 4 + T * H * 2
+    nb_2 = (live * H * 2 + world * T * (E // world) * 4 + world * T * H * 2) \
+        + (world * T * H * 2 + T * H * 2)
+    return {"unpermute_reduce_scatter": {
+        "shape": f"{world} ranks x {E // world} experts, {T} tokens top-{K}, hidden {H}, bf16, "
+                 f"all ranks' expert rows on one GPU, one launch per rank",
+        "us": round(ms_f * 1e3, 2), "bytes": nb_f, "gbs": round(nb_f / ms_f / 1e6, 1),
+        "frac": round(nb_f / ms_f / 1e6 / peak, 4),
+        "two_step_us": round(ms_2 * 1e3, 2), "two_step_bytes": nb_2,
+        "speedup_vs_two_step": round(ms_2 / ms_f, 3)}}
 
 
 def _measure_reduce_scatter(device, seed, reps, peak, T, H, world=RS_WORLD):
@@ -282,13 +338,7 @@ def _measure_reduce_scatter(device, seed, reps, peak, T, H, world=RS_WORLD):
             ops.ordered_reduce_scatter_v(table, r, offs, ep, T, H, torch.bfloat16, out=outs[r])
     # each launch is ~10 us of device time: replay the pass as a CUDA graph so
     # that host launch overhead does not show in the device time
-    one_pass()
-    torch.cuda.synchronize(device)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        one_pass()
-    ms = time_launches(graph.replay, reps, device)
-    del graph
+    ms = _graph_time(one_pass, reps, device)
     nb = world * T * H * 2 + T * H * 2
     return {"ordered_reduce_scatter_v": {
         "shape": f"{world} ranks' bf16 blocks of {T} tokens x hidden {H} on one GPU, "

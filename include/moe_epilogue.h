@@ -364,6 +364,49 @@ MOE_API int moe_ordered_reduce_scatter_v(const void* const* buffers, int64_t inp
                                          cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * EP combine: every rank's fixed-order unpermute and the rank-order
+ * reduce-scatter of the results, in one kernel over peer memory.
+ * [BI] _unpermute_tokens_in_expert_order_kernel followed by
+ * ordered_reduce_scatter_v, with the same bits as running them one after the
+ * other through blocks of partial sums of dtype partial_dt -- but no partial
+ * block is written or read:
+ *   for t < local_tokens, g = rank_token_offset[rank] + t:
+ *     for q = 0 .. world-1 (rank order):
+ *       part_q = partial_dt( +0 + sum over e ascending, row = inverse_maps[q][g, e]
+ *                            >= 0, of f32(expert_outputs[q][row, :]) )
+ *       acc = (q == 0) ? part_q : acc + part_q                          (fp32)
+ *     out[t, :] = out_dt(acc)
+ * expert_outputs     DEVICE array of `world` pointers (rank order) to each
+ *                    rank's expert-grouped rows, eo_dt [max_rows, hidden]
+ *                    contiguous, addressable from this GPU (own memory, or a
+ *                    peer's mapped with moe_ipc_open); read with plain loads
+ * inverse_maps       DEVICE array of `world` pointers to each rank's int32
+ *                    [capacity_rows, num_local_experts] inverse map over the
+ *                    token rows of all ranks (row in that rank's expert
+ *                    outputs, or < 0); num_local_experts <= 64
+ * ep_tokens          int32 (device): token rows that hold data (the pages'
+ *                    ep_max_tokens); clamped to capacity_rows
+ * world <= 64, rank, rank_token_offset int32 [world] (device): as for
+ *                    moe_ordered_reduce_scatter_v
+ * partial_dt         the partial blocks' dtype: eo_dt or MOE_FP32
+ * out                out_dt [local_tokens, hidden] contiguous; out_dt is eo_dt
+ *                    or MOE_FP32
+ * dev_err            optional int32 (device): MOE_DEVERR_COUNT (rows outside
+ *                    the data: not written), MOE_DEVERR_INVERSE (an entry of
+ *                    this rank's tokens >= max_rows: skipped)
+ * Ordering is the caller's: the launch must follow the completion of every
+ * rank's expert outputs, and no rank may overwrite them until every rank's
+ * launch has completed.  The kernel waits on nothing.
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_unpermute_reduce_scatter(const void* const* expert_outputs, moe_dtype eo_dt,
+                                         int64_t max_rows, const int32_t* const* inverse_maps,
+                                         int32_t num_local_experts, int64_t capacity_rows,
+                                         const int32_t* ep_tokens, int32_t world, int32_t rank,
+                                         const int32_t* rank_token_offset, moe_dtype partial_dt,
+                                         void* out, moe_dtype out_dt, int64_t local_tokens,
+                                         int64_t hidden, int32_t* dev_err, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Buffers shared between the processes of one node (CUDA IPC): the plumbing
  * under moe_ordered_reduce_scatter_v's `buffers` (the pages use a symmetric-
  * memory handle; this library maps plain device allocations instead).

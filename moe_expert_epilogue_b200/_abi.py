@@ -40,6 +40,8 @@ SIGNATURES = {
     "moe_epilogue_fused": [_P, _P, _I64, _P, _P, _P, _P, _P, _I64, _I64, _I32, _I, _P, _P],
     "moe_ordered_reduce_scatter_v": [_P, _I64, _I32, _I32, _P, _P, _I64, _P, _I64, _I64, _I, _I,
                                      _P, _P],
+    "moe_unpermute_reduce_scatter": [_P, _I, _I64, _P, _I32, _I64, _P, _I32, _I32, _P, _I, _P,
+                                     _I, _I64, _I64, _P, _P],
     "moe_symm_alloc": [ctypes.c_size_t, ctypes.POINTER(_P)],
     "moe_symm_free": [_P],
     "moe_ipc_export": [_P, ctypes.c_char_p],
@@ -191,6 +193,15 @@ def moe_ordered_reduce_scatter_v(buffers, input_byte_offset, world, rank, rank_t
     _call("moe_ordered_reduce_scatter_v", ptr(buffers), input_byte_offset, world, rank,
           ptr(rank_token_offset), ptr(ep_tokens), capacity_rows, ptr(out), local_tokens, hidden,
           in_dt, out_dt, ptr(dev_err), stream_handle(stream))
+
+
+def moe_unpermute_reduce_scatter(expert_outputs, eo_dt, max_rows, inverse_maps,
+                                 num_local_experts, capacity_rows, ep_tokens, world, rank,
+                                 rank_token_offset, partial_dt, out, out_dt, local_tokens, hidden,
+                                 dev_err=None, stream=None):
+    _call("moe_unpermute_reduce_scatter", ptr(expert_outputs), eo_dt, max_rows, ptr(inverse_maps),
+          num_local_experts, capacity_rows, ptr(ep_tokens), world, rank, ptr(rank_token_offset),
+          partial_dt, ptr(out), out_dt, local_tokens, hidden, ptr(dev_err), stream_handle(stream))
 
 
 def moe_symm_alloc(nbytes: int) -> int:

@@ -345,4 +345,33 @@ int moe_ordered_reduce_scatter_v(const void* const* buffers, int64_t input_byte_
                                          local_tokens, hidden, in_dt, out_dt, dev_err, stream);
 }
 
+int moe_unpermute_reduce_scatter(const void* const* expert_outputs, moe_dtype eo_dt,
+                                 int64_t max_rows, const int32_t* const* inverse_maps,
+                                 int32_t num_local_experts, int64_t capacity_rows,
+                                 const int32_t* ep_tokens, int32_t world, int32_t rank,
+                                 const int32_t* rank_token_offset, moe_dtype partial_dt,
+                                 void* out, moe_dtype out_dt, int64_t local_tokens,
+                                 int64_t hidden, int32_t* dev_err, cudaStream_t stream) {
+  if (!dtype_ok(eo_dt) || !dtype_ok(partial_dt) || !dtype_ok(out_dt)) return MOE_ERR_DTYPE;
+  if ((partial_dt != eo_dt && partial_dt != MOE_FP32) || (out_dt != eo_dt && out_dt != MOE_FP32))
+    return MOE_ERR_DTYPE;
+  if (world < 1 || world > max_ep_combine_world() || rank < 0 || rank >= world ||
+      num_local_experts < 1 || num_local_experts > max_ep_combine_experts() || max_rows < 0 ||
+      max_rows > INT32_MAX || capacity_rows < 0 || local_tokens < 0 || hidden < 0 ||
+      !product_ok(max_rows, hidden) || !product_ok(local_tokens, hidden) ||
+      !product_ok(capacity_rows, num_local_experts))
+    return MOE_ERR_SHAPE;
+  if (local_tokens == 0 || hidden == 0) return MOE_OK;
+  if (!expert_outputs || !inverse_maps || !ep_tokens || !rank_token_offset || !out)
+    return MOE_ERR_NULL;
+  if (!aligned_to(expert_outputs, sizeof(void*)) || !aligned_to(inverse_maps, sizeof(void*)) ||
+      !aligned_to(ep_tokens, 4) || !aligned_to(rank_token_offset, 4) ||
+      !aligned_to(out, dtype_size(out_dt)) || !aligned_to(dev_err, 4))
+    return MOE_ERR_ALIGN;
+  return launch_unpermute_reduce_scatter(
+      expert_outputs, eo_dt, max_rows, reinterpret_cast<const void* const*>(inverse_maps),
+      num_local_experts, capacity_rows, ep_tokens, world, rank, rank_token_offset, partial_dt,
+      out, out_dt, local_tokens, hidden, dev_err, stream);
+}
+
 }  // extern "C"

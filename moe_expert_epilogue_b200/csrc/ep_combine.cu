@@ -1,0 +1,314 @@
+// ep_combine.cu -- EP combine: every rank's token-local unpermute and the
+// rank-order reduce-scatter of its results, in one kernel over peer memory
+// (core.inference.moe.batch_invariant: _unpermute_tokens_in_expert_order_kernel
+// followed by ordered_reduce_scatter_v).
+//
+// On the pages each rank q first unpermutes its own experts' outputs into a
+// block of partial sums for the tokens of all ranks (in symmetric memory),
+// and every rank then sums its own tokens' rows of those blocks in rank order.
+// Here rank `rank` computes, for each of its tokens t (global row
+// g = rank_token_offset[rank] + t), straight from every rank's expert rows:
+//   for q = 0, 1, ..., world-1:
+//     part_q = partial_dt( +0 + sum over q's local experts e ascending with
+//                          inverse_maps[q][g, e] >= 0 of f32(expert_outputs[q][row, :]) )
+//     acc    = (q == 0) ? part_q : acc + part_q                         (fp32)
+//   out[t, :] = out_dt(acc)
+// -- the bits of the two-step form, with no partial blocks written or read:
+// each partial lives in registers, and the peers' expert rows and
+// inverse-map rows are read once, directly (plain loads; no bulk copies, no
+// multicast).  The kernel never waits on another rank: the caller orders the
+// launch after every rank's expert outputs are complete.
+//
+// One warp per item = (token, 1/split of the row).  For a group of up to 8
+// ranks the warp loads the token's inverse-map rows of all of them at once
+// (the first group of the next item is prefetched), compacts them into one
+// rank-ordered list of rows in shared memory, and then, per 16-byte unit of
+// the row, keeps up to 8 expert rows' loads in flight, closing each rank's
+// partial in rank order (ranks without rows contribute +0, as their partial
+// block row would).
+#include "common.cuh"
+#include "launch.cuh"
+#include "rowlist.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kMaxWorld = 64;    // ranks (their table entries live in shared memory)
+constexpr int kGroupRanks = 8;   // ranks whose inverse-map rows a warp stages at once
+constexpr int kMaxE = 64;        // local experts per rank (two inverse entries per lane)
+constexpr int kMaxUPL = 4;       // units per lane per item: split keeps items <= 128 units
+constexpr int kRowsInFlight = 8;
+
+// A unit of a row: 8 elements (16-byte loads) or 1 element.
+template <class D, bool VEC> struct Unit;
+template <class D> struct Unit<D, true> {
+  static constexpr int V = kVec;
+  using Raw = Raw8<D>;
+  __device__ __forceinline__ static Raw load(const typename D::T* p, bool aligned) {
+    if (aligned) return load8<D>(p);
+    Raw r;                                             // element loads, same bits
+    typename D::T* dst = reinterpret_cast<typename D::T*>(&r);
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) dst[i] = p[i];
+    return r;
+  }
+  __device__ __forceinline__ static void widen(const Raw& r, float (&v)[kVec]) { widen8<D>(r, v); }
+};
+template <class D> struct Unit<D, false> {
+  static constexpr int V = 1;
+  struct Raw { float v; };
+  __device__ __forceinline__ static Raw load(const typename D::T* p, bool) { return {load1<D>(p)}; }
+  __device__ __forceinline__ static void widen(const Raw& r, float (&v)[1]) { v[0] = r.v; }
+};
+
+template <class DP, int V>
+__device__ __forceinline__ void round_partial(float (&p)[V]) {
+  if constexpr (V == 1) {
+    p[0] = round_to<DP>(p[0]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < V; i += 2) round2<DP>(p[i], p[i + 1]);
+  }
+}
+
+// Folds the partials of ranks q0 .. q0+nq-1 for one unit into acc, rank order.
+// rows[0 .. ends[nq-1]) are the ranks' compacted expert rows, rank by rank.
+template <class DI, class DP, bool VEC>
+__device__ __forceinline__ void fold_group(const typename DI::T* const* eo, int q0, int nq,
+                                           const int32_t* rows, const int32_t* ends,
+                                           int64_t hidden, int64_t u, bool aligned,
+                                           float (&acc)[Unit<DI, VEC>::V]) {
+  using U = Unit<DI, VEC>;
+  constexpr int V = U::V;
+  float part[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) part[i] = 0.0f;
+  const int F = ends[nq - 1];
+  int q = 0;        // rank (within the group) whose partial is open
+  int kq = 0;       // rank of the next row to load
+  for (int f0 = 0; f0 < F; f0 += kRowsInFlight) {
+    typename U::Raw raw[kRowsInFlight];
+    int rk[kRowsInFlight];
+#pragma unroll
+    for (int j = 0; j < kRowsInFlight; ++j) {
+      const int f = f0 + j;
+      rk[j] = nq;
+      if (f < F) {                                       // warp-uniform
+        while (f >= ends[kq]) ++kq;
+        rk[j] = kq;
+        raw[j] = U::load(eo[q0 + kq] + (int64_t)rows[f] * hidden + u * V, aligned);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kRowsInFlight; ++j) {
+      if (f0 + j < F) {
+        for (; q < rk[j]; ++q) {                         // close the ranks before this row's
+          round_partial<DP, V>(part);
+#pragma unroll
+          for (int i = 0; i < V; ++i) {
+            acc[i] = (q0 + q == 0) ? part[i] : acc[i] + part[i];
+            part[i] = 0.0f;
+          }
+        }
+        float v[V];
+        U::widen(raw[j], v);
+#pragma unroll
+        for (int i = 0; i < V; ++i) part[i] = part[i] + v[i];
+      }
+    }
+  }
+  for (; q < nq; ++q) {                                  // the rest, empty ones included
+    round_partial<DP, V>(part);
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      acc[i] = (q0 + q == 0) ? part[i] : acc[i] + part[i];
+      part[i] = 0.0f;
+    }
+  }
+}
+
+template <class DI, class DP, class DO, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+ep_combine_warp(const void* const* __restrict__ eo_tab, const void* const* __restrict__ inv_tab,
+                int world, int rank, const int32_t* __restrict__ offs,
+                const int32_t* __restrict__ ep_tokens, int64_t capacity, int64_t max_rows,
+                int E, typename DO::T* __restrict__ out, int64_t local, int64_t hidden,
+                int split, int32_t* err) {
+  using TI = typename DI::T;
+  using U = Unit<DI, VEC>;
+  constexpr int V = U::V;
+  __shared__ const TI* s_eo[kMaxWorld];
+  __shared__ const int32_t* s_inv[kMaxWorld];
+  __shared__ int32_t s_rows[kThreads / 32][kGroupRanks * kMaxE];
+  __shared__ int32_t s_ends[kThreads / 32][kGroupRanks];
+  pdl_prologue();
+  // this rank's rows whose token lies inside the data (as the reduce-scatter)
+  const int64_t first = __ldg(offs + rank);
+  const int64_t ep = __ldg(ep_tokens);
+  const int64_t avail = ep < 0 ? 0 : (ep > capacity ? capacity : ep);
+  int64_t t_lo = first < 0 ? -first : 0;
+  int64_t t_hi = avail - first < local ? avail - first : local;
+  if (t_lo > local) t_lo = local;
+  if (t_hi < t_lo) t_hi = t_lo;
+  if ((ep < 0 || ep > capacity || t_lo > 0 || t_hi < local) && blockIdx.x == 0 &&
+      threadIdx.x == 0)
+    flag_error(err, MOE_DEVERR_COUNT);
+  int misaligned = 0;
+  for (int q = threadIdx.x; q < world; q += blockDim.x) {
+    s_eo[q] = static_cast<const TI*>(eo_tab[q]);
+    s_inv[q] = static_cast<const int32_t*>(inv_tab[q]);
+    misaligned |= (int)(reinterpret_cast<uintptr_t>(eo_tab[q]) & 15);
+  }
+  const bool aligned = __syncthreads_or(misaligned) == 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int32_t* rows = s_rows[warp];
+  int32_t* ends = s_ends[warp];
+  const int64_t units = hidden / V;
+  const int64_t upi = (units + split - 1) / split;       // units per item, <= 32 * kMaxUPL
+  const int64_t items = (t_hi - t_lo) * split;
+  const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
+  const int nq0 = world < kGroupRanks ? world : kGroupRanks;
+  int64_t it = (int64_t)blockIdx.x * (kThreads / 32) + warp;
+  if (it >= items) return;                               // warp-uniform; no barrier follows
+  int32_t p0[kGroupRanks], p1[kGroupRanks];
+  {
+    const int64_t g = first + t_lo + it / split;
+#pragma unroll
+    for (int k = 0; k < kGroupRanks; ++k) {
+      p0[k] = -1;
+      p1[k] = -1;
+      if (k < nq0) {
+        const int32_t* r = s_inv[k] + g * E;
+        p0[k] = lane < E ? __ldg(r + lane) : -1;
+        p1[k] = lane + 32 < E ? __ldg(r + lane + 32) : -1;
+      }
+    }
+  }
+  for (; it < items; it += nwarps) {
+    const int64_t t = t_lo + it / split;
+    const int64_t g = first + t;
+    const int64_t u0 = (it % split) * upi;
+    const int64_t u1 = min(units, u0 + upi);
+    float acc[kMaxUPL][V];
+#pragma unroll
+    for (int j = 0; j < kMaxUPL; ++j)
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[j][i] = 0.0f;
+    for (int q0 = 0; q0 < world; q0 += kGroupRanks) {
+      const int nq = world - q0 < kGroupRanks ? world - q0 : kGroupRanks;
+      if (q0 > 0) {                                      // later groups: loaded here
+#pragma unroll
+        for (int k = 0; k < kGroupRanks; ++k) {
+          p0[k] = -1;
+          p1[k] = -1;
+          if (k < nq) {
+            const int32_t* r = s_inv[q0 + k] + g * E;
+            p0[k] = lane < E ? __ldg(r + lane) : -1;
+            p1[k] = lane + 32 < E ? __ldg(r + lane + 32) : -1;
+          }
+        }
+      }
+      __syncwarp();                                      // the previous lists are consumed
+      int F = 0;
+#pragma unroll
+      for (int k = 0; k < kGroupRanks; ++k) {
+        if (k < nq) {
+          F += compact_pair(p0[k], p1[k], max_rows, rows + F, err, lane);
+          if (lane == 0) ends[k] = F;
+        }
+      }
+      __syncwarp();
+      if (q0 + kGroupRanks >= world) {                   // next item's first group, in flight
+        const int64_t itn = it + nwarps;
+        if (itn < items) {
+          const int64_t gn = first + t_lo + itn / split;
+#pragma unroll
+          for (int k = 0; k < kGroupRanks; ++k) {
+            p0[k] = -1;
+            p1[k] = -1;
+            if (k < nq0) {
+              const int32_t* r = s_inv[k] + gn * E;
+              p0[k] = lane < E ? __ldg(r + lane) : -1;
+              p1[k] = lane + 32 < E ? __ldg(r + lane + 32) : -1;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxUPL; ++j) {
+        const int64_t u = u0 + lane + 32 * j;
+        if (u < u1)
+          fold_group<DI, DP, VEC>(s_eo, q0, nq, rows, ends, hidden, u, aligned, acc[j]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxUPL; ++j) {
+      const int64_t u = u0 + lane + 32 * j;
+      if (u < u1) {
+        if constexpr (VEC) store8<DO>(out + t * hidden + u * kVec, acc[j]);
+        else store1<DO>(out + t * hidden + u, acc[j][0]);
+      }
+    }
+  }
+}
+
+template <class DI, class DP, class DO>
+int launch(const void* const* eos, const void* const* invs, int world, int rank,
+           const int32_t* offs, const int32_t* ep_tokens, int64_t capacity, int64_t max_rows,
+           int E, void* out, int64_t local, int64_t hidden, int32_t* err, cudaStream_t stream) {
+  using TO = typename DO::T;
+  const bool vec = hidden % kVec == 0 && aligned16(out);
+  const int64_t units = vec ? hidden / kVec : hidden;
+  const int64_t split64 = (units + 32 * kMaxUPL - 1) / (32 * kMaxUPL);
+  const int split = (int)(split64 < 1 ? 1 : split64);
+  auto k = vec ? ep_combine_warp<DI, DP, DO, true> : ep_combine_warp<DI, DP, DO, false>;
+  const int64_t warps = local * split;
+  int grid;
+  if (int rc = persistent_grid((const void*)k, 0, (warps + kThreads / 32 - 1) / (kThreads / 32),
+                               &grid))
+    return rc;
+  launch_kernel(k, grid, 0, stream, eos, invs, world, rank, offs, ep_tokens, capacity, max_rows,
+                E, static_cast<TO*>(out), local, hidden, split, err);
+  return check_launch();
+}
+
+// partial_dt and out_dt are each either the expert outputs' dtype or fp32
+template <class DI>
+int dispatch(moe_dtype partial_dt, moe_dtype out_dt, const void* const* eos,
+             const void* const* invs, int world, int rank, const int32_t* offs,
+             const int32_t* ep_tokens, int64_t capacity, int64_t max_rows, int E, void* out,
+             int64_t local, int64_t hidden, int32_t* err, cudaStream_t stream) {
+  const bool p32 = partial_dt == MOE_FP32, o32 = out_dt == MOE_FP32;
+#define MOE_EPC_ARGS eos, invs, world, rank, offs, ep_tokens, capacity, max_rows, E, out, local, \
+                     hidden, err, stream
+  if (p32 && o32) return launch<DI, F32, F32>(MOE_EPC_ARGS);
+  if (p32) return launch<DI, F32, DI>(MOE_EPC_ARGS);
+  if (o32) return launch<DI, DI, F32>(MOE_EPC_ARGS);
+  return launch<DI, DI, DI>(MOE_EPC_ARGS);
+#undef MOE_EPC_ARGS
+}
+
+}  // namespace
+
+int max_ep_combine_world() { return kMaxWorld; }
+int max_ep_combine_experts() { return kMaxE; }
+
+int launch_unpermute_reduce_scatter(const void* const* expert_outputs, moe_dtype eo_dt,
+                                    int64_t max_rows, const void* const* inverse_maps,
+                                    int num_local_experts, int64_t capacity_rows,
+                                    const int32_t* ep_tokens, int world, int rank,
+                                    const int32_t* rank_token_offset, moe_dtype partial_dt,
+                                    void* out, moe_dtype out_dt, int64_t local_tokens,
+                                    int64_t hidden, int32_t* err, cudaStream_t stream) {
+#define MOE_EPC_ARGS partial_dt, out_dt, expert_outputs, inverse_maps, world, rank, \
+                     rank_token_offset, ep_tokens, capacity_rows, max_rows, num_local_experts, \
+                     out, local_tokens, hidden, err, stream
+  switch (eo_dt) {
+    case MOE_BF16: return dispatch<BF16>(MOE_EPC_ARGS);
+    case MOE_FP16: return dispatch<F16>(MOE_EPC_ARGS);
+    default: return dispatch<F32>(MOE_EPC_ARGS);
+  }
+#undef MOE_EPC_ARGS
+}
+
+}  // namespace moe

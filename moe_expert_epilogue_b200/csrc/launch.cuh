@@ -62,6 +62,15 @@ int launch_swiglu_clamped_bwd(const void* x, const float* probs, const void* gra
                               void* grad_x, float* grad_probs, int64_t rows, int64_t inter,
                               int64_t ld_x, int64_t ld_gy, int64_t ld_gx, float limit,
                               moe_dtype dt, cudaStream_t stream);
+int max_ep_combine_world();
+int max_ep_combine_experts();
+int launch_unpermute_reduce_scatter(const void* const* expert_outputs, moe_dtype eo_dt,
+                                    int64_t max_rows, const void* const* inverse_maps,
+                                    int num_local_experts, int64_t capacity_rows,
+                                    const int32_t* ep_tokens, int world, int rank,
+                                    const int32_t* rank_token_offset, moe_dtype partial_dt,
+                                    void* out, moe_dtype out_dt, int64_t local_tokens,
+                                    int64_t hidden, int32_t* err, cudaStream_t stream);
 int max_reduce_scatter_world();
 int launch_ordered_reduce_scatter_v(const void* const* bufs, int64_t byte_off, int world, int rank,
                                     const int32_t* offs, const int32_t* ep_tokens,

@@ -290,3 +290,41 @@ def ordered_reduce_scatter_v(buffers, rank, rank_token_offset, ep_tokens, capaci
                                       out.shape[0], hidden, moe_dtype(in_dtype),
                                       moe_dtype(out.dtype), dev_err, stream)
     return out
+
+
+def unpermute_reduce_scatter(expert_outputs, eo_dtype, max_rows, inverse_maps, num_local_experts,
+                             capacity_rows, ep_tokens, rank, rank_token_offset, hidden,
+                             local_tokens=None, out=None, out_dtype=None, partial_dtype=None,
+                             dev_err=None, stream=None):
+    """This rank's rows of the EP combine: every rank's fixed-order unpermute
+    and the rank-order reduce-scatter of the results, in one kernel.
+
+    expert_outputs, inverse_maps: int64 device tensors [world] of pointers
+    (rank order) to each rank's [max_rows, hidden] expert rows of `eo_dtype`
+    and int32 [capacity_rows, num_local_experts] inverse map; ep_tokens int32
+    [1] and rank_token_offset int32 [world] on the device.  partial_dtype
+    (default eo_dtype) is the dtype the two-step form would store its partial
+    sums in.  Returns out [local_tokens, hidden] (out_dtype, default eo_dtype)."""
+    for t, name in ((expert_outputs, "expert_outputs"), (inverse_maps, "inverse_maps")):
+        if t.dim() != 1:
+            raise ValueError(f"{name} must be a vector of device pointers")
+        _check(t, name, dtype=torch.int64)
+    world = expert_outputs.numel()
+    _check(inverse_maps, "inverse_maps", numel=world)
+    _check(rank_token_offset, "rank_token_offset", dtype=torch.int32, numel=world)
+    _check(ep_tokens, "ep_tokens", dtype=torch.int32, numel=1)
+    _check(dev_err, "dev_err", dtype=torch.int32, numel=1)
+    if out is None:
+        if local_tokens is None:
+            raise ValueError("give local_tokens or out")
+        out = torch.empty(local_tokens, hidden, dtype=out_dtype or eo_dtype,
+                          device=expert_outputs.device)
+    _two_d(out, "out")
+    _check(out, "out", dtype=_FLOATS, shape=(out.shape[0], hidden))
+    _cuda(expert_outputs, inverse_maps, rank_token_offset, ep_tokens, out, dev_err)
+    _abi.moe_unpermute_reduce_scatter(expert_outputs, moe_dtype(eo_dtype), int(max_rows),
+                                      inverse_maps, int(num_local_experts), int(capacity_rows),
+                                      ep_tokens, world, int(rank), rank_token_offset,
+                                      moe_dtype(partial_dtype or eo_dtype), out,
+                                      moe_dtype(out.dtype), out.shape[0], hidden, dev_err, stream)
+    return out

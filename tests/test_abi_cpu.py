@@ -117,6 +117,27 @@ def test_reduce_scatter_validation(lib):
     f(*dict(ok, local_tokens=0, buffers=None).values())          # nothing to do: a no-op
 
 
+def test_ep_combine_validation(lib):
+    f = _abi.moe_unpermute_reduce_scatter
+    ok = dict(expert_outputs=FAKE, eo_dt=_abi.MOE_BF16, max_rows=100, inverse_maps=FAKE,
+              num_local_experts=8, capacity_rows=50, ep_tokens=FAKE, world=4, rank=1,
+              rank_token_offset=FAKE, partial_dt=_abi.MOE_BF16, out=FAKE, out_dt=_abi.MOE_BF16,
+              local_tokens=10, hidden=64)
+
+    def st(**kw):
+        return _status(f, *dict(ok, **kw).values())
+    # partial and output dtypes: the expert outputs' dtype or fp32
+    assert st(partial_dt=_abi.MOE_FP16) == _abi.MOE_ERR_DTYPE
+    assert st(out_dt=_abi.MOE_FP16) == _abi.MOE_ERR_DTYPE
+    assert st(num_local_experts=65) == _abi.MOE_ERR_SHAPE
+    assert st(num_local_experts=0) == _abi.MOE_ERR_SHAPE
+    assert st(world=65) == _abi.MOE_ERR_SHAPE and st(rank=4) == _abi.MOE_ERR_SHAPE
+    assert st(max_rows=2 ** 31) == _abi.MOE_ERR_SHAPE
+    assert st(inverse_maps=None) == _abi.MOE_ERR_NULL
+    assert st(expert_outputs=FAKE + 4) == _abi.MOE_ERR_ALIGN
+    f(*dict(ok, local_tokens=0, expert_outputs=None).values())   # nothing to do: a no-op
+
+
 def test_ipc_argument_checks(lib):
     import ctypes
     assert lib.moe_symm_alloc(16, None) == _abi.MOE_ERR_NULL

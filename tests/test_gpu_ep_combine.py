@@ -1,0 +1,158 @@
+"""Parity of the EP-combine kernel (every rank's unpermute and the rank-order
+reduce-scatter in one kernel) with the CPU oracle and with the two library
+kernels it fuses (gpu).
+
+Every rank's expert rows and inverse map live on this one GPU; the kernel
+reads them through the pointer tables exactly as it reads peers' memory, and
+runs once per rank (the launches never wait on one another).  Bit-exact: the
+sum orders (experts ascending within a rank, ranks ascending) and the
+rounding of each rank's partial are fixed by the definition."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_expert_epilogue_b200 import _abi, inputs, ops
+from tests._util import assert_bits_equal, bits
+
+pytestmark = pytest.mark.gpu
+
+ODT = {torch.bfloat16: oracle.BF16, torch.float16: oracle.F16, torch.float32: oracle.F32}
+KIND = {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "bf16"}
+
+
+def _tables(dev, case, shift=None):
+    """Device copies of every rank's expert rows and inverse map, and their
+    pointer tables; shift = (rank, bytes) moves one rank's expert rows off
+    16-byte alignment."""
+    keep, eo_ptrs, inv_ptrs = [], [], []
+    for q, (eo, inv) in enumerate(zip(case.expert_outputs, case.inverse_maps)):
+        extra = shift[1] if shift and shift[0] == q else 0
+        raw = torch.zeros(extra + eo.numel() * eo.element_size(), dtype=torch.uint8, device=dev)
+        blk = raw[extra:].view(eo.dtype).view(eo.shape)
+        blk.copy_(eo.to(dev))
+        inv_d = inv.to(dev)
+        keep += [raw, inv_d]
+        eo_ptrs.append(raw.data_ptr() + extra)
+        inv_ptrs.append(inv_d.data_ptr())
+    return (torch.tensor(eo_ptrs, dtype=torch.int64, device=dev),
+            torch.tensor(inv_ptrs, dtype=torch.int64, device=dev), keep)
+
+
+def _run(dev, case, eo_t, inv_t, rank, out_dtype, partial_dtype, init, ep_tokens=None,
+         offsets=None, err=None):
+    E = case.inverse_maps[0].shape[1]
+    hidden = case.expert_outputs[0].shape[1]
+    offs = case.rank_token_offset if offsets is None else torch.tensor(offsets, dtype=torch.int32)
+    ep = torch.tensor([case.tokens if ep_tokens is None else ep_tokens], dtype=torch.int32,
+                      device=dev)
+    out = init.to(dev)
+    ops.unpermute_reduce_scatter(eo_t, case.expert_outputs[0].dtype, case.max_rows, inv_t, E,
+                                 case.tokens, ep, rank, offs.to(dev), hidden, out=out,
+                                 partial_dtype=partial_dtype, dev_err=err)
+    torch.cuda.synchronize()
+    return out.cpu()
+
+
+def _oracle(case, rank, out_dtype, partial_dtype, init, ep_tokens=None, offsets=None):
+    eo_dt = case.expert_outputs[0].dtype
+    offs = case.rank_token_offset.numpy() if offsets is None else np.asarray(offsets, np.int32)
+    return oracle.unpermute_reduce_scatter(
+        [bits(e) for e in case.expert_outputs], ODT[eo_dt], [bits(i) for i in case.inverse_maps],
+        case.tokens if ep_tokens is None else ep_tokens, rank, offs, ODT[partial_dtype],
+        bits(init), ODT[out_dtype])
+
+
+CASES = [  # world, tokens, top_k, experts per rank, align, hidden
+    (1, 40, 4, 8, 4, 64), (2, 61, 2, 4, 4, 24), (4, 200, 8, 16, 16, 1032),
+    (8, 300, 8, 8, 128, 512), (3, 50, 3, 5, 2, 13), (9, 77, 4, 2, 8, 96), (17, 64, 4, 1, 4, 40),
+    (2, 40, 8, 64, 4, 64)]
+DTYPES = [  # expert outputs, partial blocks, output
+    (torch.bfloat16, torch.bfloat16, torch.bfloat16), (torch.bfloat16, torch.float32, torch.bfloat16),
+    (torch.bfloat16, torch.float32, torch.float32), (torch.float16, torch.float16, torch.float32),
+    (torch.float32, torch.float32, torch.float32)]
+
+
+@pytest.mark.parametrize("world,tokens,top_k,epr,align,hidden", CASES)
+@pytest.mark.parametrize("eo_dtype,partial_dtype,out_dtype", DTYPES)
+def test_ep_combine_bitwise_every_rank(cuda_device, world, tokens, top_k, epr, align, hidden,
+                                       eo_dtype, partial_dtype, out_dtype):
+    case = inputs.ep_combine_inputs(world, tokens, top_k, epr, align, hidden, dtype=eo_dtype,
+                                    seed=world * 1000 + hidden)
+    eo_t, inv_t, keep = _tables(cuda_device, case)
+    for rank in range(world):
+        init = torch.full((case.counts[rank], hidden), -2.5, dtype=out_dtype)
+        got = _run(cuda_device, case, eo_t, inv_t, rank, out_dtype, partial_dtype, init)
+        want, err = _oracle(case, rank, out_dtype, partial_dtype, init)
+        assert err == 0
+        assert_bits_equal(bits(got), want, f"rank {rank}", kind=KIND[out_dtype])
+
+
+def _two_step(dev, case, rank, partial_dtype, out_dtype):
+    """The pages' form with the library's own kernels: each rank's unpermute
+    into a partial block, then the reduce-scatter of the blocks."""
+    hidden = case.expert_outputs[0].shape[1]
+    blocks = []
+    vt = torch.tensor([case.tokens], dtype=torch.int32, device=dev)
+    for eo, inv in zip(case.expert_outputs, case.inverse_maps):
+        blk = torch.zeros(case.tokens, hidden, dtype=partial_dtype, device=dev)
+        ops.unpermute_ordered(eo.to(dev), inv.to(dev), vt, blk)
+        blocks.append(blk)
+    out = torch.zeros(case.counts[rank], hidden, dtype=out_dtype, device=dev)
+    ops.ordered_reduce_scatter_v(ops.pointer_table(blocks), rank, case.rank_token_offset.to(dev),
+                                 vt, case.tokens, hidden, partial_dtype, out=out)
+    torch.cuda.synchronize()
+    return out.cpu()
+
+
+@pytest.mark.parametrize("partial_dtype,out_dtype", [(torch.bfloat16, torch.bfloat16),
+                                                     (torch.float32, torch.bfloat16)])
+def test_ep_combine_equals_unpermute_then_reduce_scatter(cuda_device, partial_dtype, out_dtype):
+    """8 EP ranks, 8192 tokens, top-8 of 64 experts (8 per rank), hidden 4096:
+    the fused kernel gives the bits of the two library kernels it replaces,
+    for every rank's rows."""
+    case = inputs.ep_combine_inputs(8, 8192, 8, 8, 128, 4096, seed=3, device="cpu")
+    eo_t, inv_t, keep = _tables(cuda_device, case)
+    for rank in range(8):
+        init = torch.zeros(case.counts[rank], 4096, dtype=out_dtype)
+        got = _run(cuda_device, case, eo_t, inv_t, rank, out_dtype, partial_dtype, init)
+        assert_bits_equal(bits(got), bits(_two_step(cuda_device, case, rank, partial_dtype,
+                                                    out_dtype)), f"rank {rank}")
+
+
+@pytest.mark.parametrize("shift", [(0, 2), (2, 8)])
+def test_ep_combine_unaligned_rows(cuda_device, shift):
+    case = inputs.ep_combine_inputs(4, 120, 4, 4, 8, 264, seed=5)
+    eo_t, inv_t, keep = _tables(cuda_device, case, shift)
+    for rank in range(4):
+        init = torch.zeros(case.counts[rank], 264, dtype=torch.bfloat16)
+        got = _run(cuda_device, case, eo_t, inv_t, rank, torch.bfloat16, torch.bfloat16, init)
+        want, _ = _oracle(case, rank, torch.bfloat16, torch.bfloat16, init)
+        assert_bits_equal(bits(got), want, f"rank {rank}")
+
+
+def test_ep_combine_bad_rows_and_entries(cuda_device):
+    case = inputs.ep_combine_inputs(3, 60, 3, 4, 4, 32, seed=6)
+    init = torch.full((10, 32), 7.0)
+    eo_t, inv_t, keep = _tables(cuda_device, case)
+    for offsets, ep in [([0, 55, 0], 60), ([0, -3, 0], 60), ([0, 50, 0], 80)]:
+        err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+        got = _run(cuda_device, case, eo_t, inv_t, 1, torch.float32, torch.float32, init,
+                   ep_tokens=ep, offsets=offsets, err=err)
+        want, oerr = _oracle(case, 1, torch.float32, torch.float32, init, ep_tokens=ep,
+                             offsets=offsets)
+        assert int(err) == _abi.MOE_DEVERR_COUNT and oerr & _abi.MOE_DEVERR_COUNT
+        assert np.array_equal(bits(got).view(np.uint32), want.view(np.uint32)), (offsets, ep)
+    # an inverse-map entry past the expert rows, in rank 1's own tokens: skipped, reported
+    bad = case.inverse_maps[2].clone()
+    t = int(case.rank_token_offset[1])
+    e = int(torch.nonzero(bad[t] >= 0)[0, 0]) if (bad[t] >= 0).any() else 0
+    bad[t, e] = case.max_rows + 5
+    case.inverse_maps[2] = bad
+    eo_t, inv_t, keep = _tables(cuda_device, case)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    init = torch.zeros(case.counts[1], 32)
+    got = _run(cuda_device, case, eo_t, inv_t, 1, torch.float32, torch.float32, init, err=err)
+    want, oerr = _oracle(case, 1, torch.float32, torch.float32, init)
+    assert int(err) == _abi.MOE_DEVERR_INVERSE and oerr == _abi.MOE_DEVERR_INVERSE
+    assert np.array_equal(bits(got).view(np.uint32), want.view(np.uint32))

@@ -125,3 +125,17 @@ def test_mixed_devices_are_rejected():
             self.device = dev
     with pytest.raises(ValueError, match="different devices"):
         ops._cuda(FakeCuda("cuda:0"), FakeCuda("cuda:1"))
+
+
+def test_ep_combine():
+    tab, offs, ep = z(3, dtype=i64), z(3, dtype=i32), z(1, dtype=i32)
+    with pytest.raises(ValueError, match="elements"):
+        ops.unpermute_reduce_scatter(tab, bf, 10, z(2, dtype=i64), 4, 20, ep, 0, offs, 8,
+                                     local_tokens=2)
+    with pytest.raises(TypeError, match="inverse_maps"):
+        ops.unpermute_reduce_scatter(tab, bf, 10, z(3, dtype=i32), 4, 20, ep, 0, offs, 8,
+                                     local_tokens=2)
+    with pytest.raises(ValueError, match="shape"):
+        ops.unpermute_reduce_scatter(tab, bf, 10, tab, 4, 20, ep, 0, offs, 8, out=z(2, 9))
+    _device_error(lambda: ops.unpermute_reduce_scatter(tab, bf, 10, tab, 4, 20, ep, 0, offs, 8,
+                                                       local_tokens=2))
