@@ -21,14 +21,14 @@
 //
 // One warp per item = (token, 1/split of the row).  For a group of up to 8
 // ranks the warp loads the token's inverse-map rows of all of them at once
-// (the first group of the next item is prefetched), compacts them into one
-// rank-ordered list of rows in shared memory, and then, per 16-byte unit of
-// the row, keeps up to 8 expert rows' loads in flight, closing each rank's
-// partial in rank order (ranks without rows contribute +0, as their partial
-// block row would).
+// (the first group of the next item is prefetched) and compacts them into one
+// rank-ordered list of row pointers in shared memory, each entry tagged with
+// the number of rank partials to close before it; then, per 16-byte unit of
+// the row, it keeps up to 8 expert rows' loads in flight and closes each
+// rank's partial in rank order (ranks without rows contribute +0, as their
+// partial block row would).
 #include "common.cuh"
 #include "launch.cuh"
-#include "rowlist.cuh"
 
 namespace moe {
 namespace {
@@ -36,28 +36,39 @@ namespace {
 constexpr int kMaxWorld = 64;    // ranks (their table entries live in shared memory)
 constexpr int kGroupRanks = 8;   // ranks whose inverse-map rows a warp stages at once
 constexpr int kMaxE = 64;        // local experts per rank (two inverse entries per lane)
-constexpr int kMaxUPL = 4;       // units per lane per item: split keeps items <= 128 units
-constexpr int kRowsInFlight = 8;
+#ifndef MOE_EPC_UPL
+#define MOE_EPC_UPL 1
+#endif
+constexpr int kMaxUPL = MOE_EPC_UPL;  // units per lane per item: split keeps items <= 32 * kMaxUPL units
+#ifndef MOE_EPC_ROWS
+#define MOE_EPC_ROWS 8
+#endif
+constexpr int kRowsInFlight = MOE_EPC_ROWS;
 
 // A unit of a row: 8 elements (16-byte loads) or 1 element.
 template <class D, bool VEC> struct Unit;
 template <class D> struct Unit<D, true> {
   static constexpr int V = kVec;
   using Raw = Raw8<D>;
-  __device__ __forceinline__ static Raw load(const typename D::T* p, bool aligned) {
-    if (aligned) return load8<D>(p);
-    Raw r;                                             // element loads, same bits
-    typename D::T* dst = reinterpret_cast<typename D::T*>(&r);
+  template <bool ALIGNED>
+  __device__ __forceinline__ static Raw load(const typename D::T* p) {
+    if constexpr (ALIGNED) {
+      return load8<D>(p);
+    } else {
+      Raw r;                                           // element loads, same bits
+      typename D::T* dst = reinterpret_cast<typename D::T*>(&r);
 #pragma unroll
-    for (int i = 0; i < kVec; ++i) dst[i] = p[i];
-    return r;
+      for (int i = 0; i < kVec; ++i) dst[i] = p[i];
+      return r;
+    }
   }
   __device__ __forceinline__ static void widen(const Raw& r, float (&v)[kVec]) { widen8<D>(r, v); }
 };
 template <class D> struct Unit<D, false> {
   static constexpr int V = 1;
   struct Raw { float v; };
-  __device__ __forceinline__ static Raw load(const typename D::T* p, bool) { return {load1<D>(p)}; }
+  template <bool ALIGNED>
+  __device__ __forceinline__ static Raw load(const typename D::T* p) { return {load1<D>(p)}; }
   __device__ __forceinline__ static void widen(const Raw& r, float (&v)[1]) { v[0] = r.v; }
 };
 
@@ -71,45 +82,66 @@ __device__ __forceinline__ void round_partial(float (&p)[V]) {
   }
 }
 
-// Folds the partials of ranks q0 .. q0+nq-1 for one unit into acc, rank order.
-// rows[0 .. ends[nq-1]) are the ranks' compacted expert rows, rank by rank.
-template <class DI, class DP, bool VEC>
-__device__ __forceinline__ void fold_group(const typename DI::T* const* eo, int q0, int nq,
-                                           const int32_t* rows, const int32_t* ends,
-                                           int64_t hidden, int64_t u, bool aligned,
-                                           float (&acc)[Unit<DI, VEC>::V]) {
+// Appends rank k's live inverse entries (one per lane; two with TWO) to the
+// warp's list as row pointers, in expert order.  The first appended entry
+// carries `gap`: how many open partials must be closed before it is added
+// (the ranks from the open one up to k).  Returns the number appended.
+template <class T, bool TWO>
+__device__ __forceinline__ int append_rank(int32_t r0, int32_t r1, int64_t max_rows,
+                                           const T* base, int64_t hidden, int gap,
+                                           const T** ptrs, uint8_t* gaps, int32_t* err,
+                                           int lane) {
+  if (r0 >= max_rows) { flag_error(err, MOE_DEVERR_INVERSE); r0 = -1; }
+  if (TWO && r1 >= max_rows) { flag_error(err, MOE_DEVERR_INVERSE); r1 = -1; }
+  const unsigned below = (1u << lane) - 1u;
+  const unsigned m0 = __ballot_sync(0xffffffffu, r0 >= 0);
+  const unsigned m1 = TWO ? __ballot_sync(0xffffffffu, r1 >= 0) : 0u;
+  if (r0 >= 0) {
+    const int pos = __popc(m0 & below);
+    ptrs[pos] = base + (int64_t)r0 * hidden;
+    gaps[pos] = pos == 0 ? (uint8_t)gap : (uint8_t)0;
+  }
+  if (TWO && r1 >= 0) {
+    const int pos = __popc(m0) + __popc(m1 & below);
+    ptrs[pos] = base + (int64_t)r1 * hidden;
+    gaps[pos] = pos == 0 ? (uint8_t)gap : (uint8_t)0;
+  }
+  return __popc(m0) + __popc(m1);
+}
+
+// Rounds the open partial to DP and folds it into acc in rank order (rank 0's
+// partial is the sum's first term); the next rank's partial starts at +0.
+template <class DP, int V>
+__device__ __forceinline__ void close_partial(float (&part)[V], float (&acc)[V], bool first) {
+  round_partial<DP, V>(part);
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    acc[i] = first ? part[i] : acc[i] + part[i];
+    part[i] = 0.0f;
+  }
+}
+
+// One unit of the row: the list's rows (kRowsInFlight loads in flight), each
+// rank's partial closed in rank order, `trailing` closes after the last row.
+template <class DI, class DP, bool VEC, bool ALIGNED>
+__device__ __forceinline__ void fold_unit(const typename DI::T* const* ptrs, const uint8_t* gaps,
+                                          int F, int trailing, int q0, int64_t u,
+                                          float (&acc)[Unit<DI, VEC>::V]) {
   using U = Unit<DI, VEC>;
   constexpr int V = U::V;
   float part[V];
 #pragma unroll
   for (int i = 0; i < V; ++i) part[i] = 0.0f;
-  const int F = ends[nq - 1];
-  int q = 0;        // rank (within the group) whose partial is open
-  int kq = 0;       // rank of the next row to load
+  int q = q0;                                           // global rank of the open partial
   for (int f0 = 0; f0 < F; f0 += kRowsInFlight) {
     typename U::Raw raw[kRowsInFlight];
-    int rk[kRowsInFlight];
 #pragma unroll
-    for (int j = 0; j < kRowsInFlight; ++j) {
-      const int f = f0 + j;
-      rk[j] = nq;
-      if (f < F) {                                       // warp-uniform
-        while (f >= ends[kq]) ++kq;
-        rk[j] = kq;
-        raw[j] = U::load(eo[q0 + kq] + (int64_t)rows[f] * hidden + u * V, aligned);
-      }
-    }
+    for (int j = 0; j < kRowsInFlight; ++j)
+      if (f0 + j < F) raw[j] = U::template load<ALIGNED>(ptrs[f0 + j] + u * V);
 #pragma unroll
     for (int j = 0; j < kRowsInFlight; ++j) {
       if (f0 + j < F) {
-        for (; q < rk[j]; ++q) {                         // close the ranks before this row's
-          round_partial<DP, V>(part);
-#pragma unroll
-          for (int i = 0; i < V; ++i) {
-            acc[i] = (q0 + q == 0) ? part[i] : acc[i] + part[i];
-            part[i] = 0.0f;
-          }
-        }
+        for (int c = gaps[f0 + j]; c > 0; --c, ++q) close_partial<DP, V>(part, acc, q == 0);
         float v[V];
         U::widen(raw[j], v);
 #pragma unroll
@@ -117,30 +149,111 @@ __device__ __forceinline__ void fold_group(const typename DI::T* const* eo, int 
       }
     }
   }
-  for (; q < nq; ++q) {                                  // the rest, empty ones included
-    round_partial<DP, V>(part);
+  for (int c = trailing; c > 0; --c, ++q) close_partial<DP, V>(part, acc, q == 0);
+}
+
+// The token-local inverse-map rows of ranks q0 .. q0+nq-1 for global row g:
+// one entry per lane (TWO: two, for more than 32 local experts).
+template <bool TWO>
+__device__ __forceinline__ void load_group(const int32_t* const* inv, int q0, int nq, int64_t g,
+                                           int E, int lane, int32_t (&p0)[kGroupRanks],
+                                           int32_t (&p1)[kGroupRanks]) {
 #pragma unroll
-    for (int i = 0; i < V; ++i) {
-      acc[i] = (q0 + q == 0) ? part[i] : acc[i] + part[i];
-      part[i] = 0.0f;
+  for (int k = 0; k < kGroupRanks; ++k) {
+    p0[k] = -1;
+    if (TWO) p1[k] = -1;
+    if (k < nq) {
+      const int32_t* r = inv[q0 + k] + g * E;
+      p0[k] = lane < E ? __ldg(r + lane) : -1;
+      if (TWO) p1[k] = lane + 32 < E ? __ldg(r + lane + 32) : -1;
     }
   }
 }
 
-template <class DI, class DP, class DO, bool VEC>
-__global__ void __launch_bounds__(kThreads)
+// The warp's items: (token, slice of the row) pairs, strided over the grid
+// with a division-free cursor.
+template <class DI, class DP, class DO, bool VEC, bool TWO, bool ALIGNED>
+__device__ __forceinline__ void combine_items(
+    const typename DI::T* const* eo, const int32_t* const* inv, const typename DI::T** ptrs,
+    uint8_t* gaps,
+    int world, int64_t first, int64_t t_lo, int64_t t_hi, int split, int64_t units,
+    int64_t hidden, int64_t max_rows, int E, typename DO::T* __restrict__ out, int32_t* err,
+    int lane, int64_t it0, int64_t nwarps) {
+  constexpr int V = Unit<DI, VEC>::V;
+  const int64_t n_tok = t_hi - t_lo;
+  const int64_t upi = (units + split - 1) / split;       // units per item, <= 32 * kMaxUPL
+  const int nq0 = world < kGroupRanks ? world : kGroupRanks;
+  RowCursor cur(it0, nwarps, split);                      // (token, slice) of item it0
+  if (cur.r >= n_tok) return;                             // warp-uniform
+  int32_t p0[kGroupRanks], p1[kGroupRanks];
+  load_group<TWO>(inv, 0, nq0, first + t_lo + cur.r, E, lane, p0, p1);
+  while (cur.r < n_tok) {
+    const int64_t t = t_lo + cur.r;
+    const int64_t g = first + t;
+    const int64_t u0 = cur.c * upi;
+    const int64_t u1 = min(units, u0 + upi);
+    RowCursor nxt = cur;
+    nxt.advance();
+    float acc[kMaxUPL][V];
+#pragma unroll
+    for (int j = 0; j < kMaxUPL; ++j)
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[j][i] = 0.0f;
+    for (int q0 = 0; q0 < world; q0 += kGroupRanks) {
+      const int nq = world - q0 < kGroupRanks ? world - q0 : kGroupRanks;
+      if (q0 > 0) load_group<TWO>(inv, q0, nq, g, E, lane, p0, p1);   // later groups
+      __syncwarp();                                      // the previous list is consumed
+      int F = 0, open = 0;                               // open: the rank whose partial is open
+#pragma unroll
+      for (int k = 0; k < kGroupRanks; ++k) {
+        if (k < nq) {
+          const int c = append_rank<typename DI::T, TWO>(p0[k], p1[k], max_rows, eo[q0 + k],
+                                                         hidden, k - open, ptrs + F, gaps + F,
+                                                         err, lane);
+          if (c > 0) open = k;
+          F += c;
+        }
+      }
+      const int trailing = nq - open;
+      __syncwarp();
+      if (q0 + kGroupRanks >= world && nxt.r < n_tok)   // next item's first group, in flight
+        load_group<TWO>(inv, 0, nq0, first + t_lo + nxt.r, E, lane, p0, p1);
+#pragma unroll
+      for (int j = 0; j < kMaxUPL; ++j) {
+        const int64_t u = u0 + lane + 32 * j;
+        if (u < u1)
+          fold_unit<DI, DP, VEC, ALIGNED>(ptrs, gaps, F, trailing, q0, u, acc[j]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxUPL; ++j) {
+      const int64_t u = u0 + lane + 32 * j;
+      if (u < u1) {
+        if constexpr (VEC) store8<DO>(out + t * hidden + u * kVec, acc[j]);
+        else store1<DO>(out + t * hidden + u, acc[j][0]);
+      }
+    }
+    cur = nxt;
+  }
+}
+
+#ifndef MOE_EPC_MIN_BLOCKS
+#define MOE_EPC_MIN_BLOCKS 0
+#endif
+
+template <class DI, class DP, class DO, bool VEC, bool TWO>
+__global__ void __launch_bounds__(kThreads, MOE_EPC_MIN_BLOCKS)
 ep_combine_warp(const void* const* __restrict__ eo_tab, const void* const* __restrict__ inv_tab,
                 int world, int rank, const int32_t* __restrict__ offs,
                 const int32_t* __restrict__ ep_tokens, int64_t capacity, int64_t max_rows,
                 int E, typename DO::T* __restrict__ out, int64_t local, int64_t hidden,
                 int split, int32_t* err) {
   using TI = typename DI::T;
-  using U = Unit<DI, VEC>;
-  constexpr int V = U::V;
+  constexpr int V = Unit<DI, VEC>::V;
   __shared__ const TI* s_eo[kMaxWorld];
   __shared__ const int32_t* s_inv[kMaxWorld];
-  __shared__ int32_t s_rows[kThreads / 32][kGroupRanks * kMaxE];
-  __shared__ int32_t s_ends[kThreads / 32][kGroupRanks];
+  __shared__ const TI* s_ptrs[kThreads / 32][kGroupRanks * kMaxE];
+  __shared__ uint8_t s_gaps[kThreads / 32][kGroupRanks * kMaxE];
   pdl_prologue();
   // this rank's rows whose token lies inside the data (as the reduce-scatter)
   const int64_t first = __ldg(offs + rank);
@@ -161,95 +274,19 @@ ep_combine_warp(const void* const* __restrict__ eo_tab, const void* const* __res
   }
   const bool aligned = __syncthreads_or(misaligned) == 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int32_t* rows = s_rows[warp];
-  int32_t* ends = s_ends[warp];
-  const int64_t units = hidden / V;
-  const int64_t upi = (units + split - 1) / split;       // units per item, <= 32 * kMaxUPL
-  const int64_t items = (t_hi - t_lo) * split;
+  const int64_t it0 = (int64_t)blockIdx.x * (kThreads / 32) + warp;
   const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
-  const int nq0 = world < kGroupRanks ? world : kGroupRanks;
-  int64_t it = (int64_t)blockIdx.x * (kThreads / 32) + warp;
-  if (it >= items) return;                               // warp-uniform; no barrier follows
-  int32_t p0[kGroupRanks], p1[kGroupRanks];
-  {
-    const int64_t g = first + t_lo + it / split;
-#pragma unroll
-    for (int k = 0; k < kGroupRanks; ++k) {
-      p0[k] = -1;
-      p1[k] = -1;
-      if (k < nq0) {
-        const int32_t* r = s_inv[k] + g * E;
-        p0[k] = lane < E ? __ldg(r + lane) : -1;
-        p1[k] = lane + 32 < E ? __ldg(r + lane + 32) : -1;
-      }
-    }
+#define MOE_EPC_ITEMS(AL)                                                                    \
+  combine_items<DI, DP, DO, VEC, TWO, AL>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world,   \
+                                          first, t_lo, t_hi, split, hidden / V, hidden,     \
+                                          max_rows, E, out, err, lane, it0, nwarps)
+  if constexpr (VEC) {
+    if (aligned) MOE_EPC_ITEMS(true);
+    else MOE_EPC_ITEMS(false);                           // a buffer off 16-byte alignment
+  } else {
+    MOE_EPC_ITEMS(true);
   }
-  for (; it < items; it += nwarps) {
-    const int64_t t = t_lo + it / split;
-    const int64_t g = first + t;
-    const int64_t u0 = (it % split) * upi;
-    const int64_t u1 = min(units, u0 + upi);
-    float acc[kMaxUPL][V];
-#pragma unroll
-    for (int j = 0; j < kMaxUPL; ++j)
-#pragma unroll
-      for (int i = 0; i < V; ++i) acc[j][i] = 0.0f;
-    for (int q0 = 0; q0 < world; q0 += kGroupRanks) {
-      const int nq = world - q0 < kGroupRanks ? world - q0 : kGroupRanks;
-      if (q0 > 0) {                                      // later groups: loaded here
-#pragma unroll
-        for (int k = 0; k < kGroupRanks; ++k) {
-          p0[k] = -1;
-          p1[k] = -1;
-          if (k < nq) {
-            const int32_t* r = s_inv[q0 + k] + g * E;
-            p0[k] = lane < E ? __ldg(r + lane) : -1;
-            p1[k] = lane + 32 < E ? __ldg(r + lane + 32) : -1;
-          }
-        }
-      }
-      __syncwarp();                                      // the previous lists are consumed
-      int F = 0;
-#pragma unroll
-      for (int k = 0; k < kGroupRanks; ++k) {
-        if (k < nq) {
-          F += compact_pair(p0[k], p1[k], max_rows, rows + F, err, lane);
-          if (lane == 0) ends[k] = F;
-        }
-      }
-      __syncwarp();
-      if (q0 + kGroupRanks >= world) {                   // next item's first group, in flight
-        const int64_t itn = it + nwarps;
-        if (itn < items) {
-          const int64_t gn = first + t_lo + itn / split;
-#pragma unroll
-          for (int k = 0; k < kGroupRanks; ++k) {
-            p0[k] = -1;
-            p1[k] = -1;
-            if (k < nq0) {
-              const int32_t* r = s_inv[k] + gn * E;
-              p0[k] = lane < E ? __ldg(r + lane) : -1;
-              p1[k] = lane + 32 < E ? __ldg(r + lane + 32) : -1;
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < kMaxUPL; ++j) {
-        const int64_t u = u0 + lane + 32 * j;
-        if (u < u1)
-          fold_group<DI, DP, VEC>(s_eo, q0, nq, rows, ends, hidden, u, aligned, acc[j]);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kMaxUPL; ++j) {
-      const int64_t u = u0 + lane + 32 * j;
-      if (u < u1) {
-        if constexpr (VEC) store8<DO>(out + t * hidden + u * kVec, acc[j]);
-        else store1<DO>(out + t * hidden + u, acc[j][0]);
-      }
-    }
-  }
+#undef MOE_EPC_ITEMS
 }
 
 template <class DI, class DP, class DO>
@@ -261,7 +298,10 @@ int launch(const void* const* eos, const void* const* invs, int world, int rank,
   const int64_t units = vec ? hidden / kVec : hidden;
   const int64_t split64 = (units + 32 * kMaxUPL - 1) / (32 * kMaxUPL);
   const int split = (int)(split64 < 1 ? 1 : split64);
-  auto k = vec ? ep_combine_warp<DI, DP, DO, true> : ep_combine_warp<DI, DP, DO, false>;
+  const bool two = E > 32;
+  auto k = vec ? (two ? ep_combine_warp<DI, DP, DO, true, true> : ep_combine_warp<DI, DP, DO, true, false>)
+               : (two ? ep_combine_warp<DI, DP, DO, false, true>
+                      : ep_combine_warp<DI, DP, DO, false, false>);
   const int64_t warps = local * split;
   int grid;
   if (int rc = persistent_grid((const void*)k, 0, (warps + kThreads / 32 - 1) / (kThreads / 32),
