@@ -36,14 +36,10 @@ namespace {
 constexpr int kMaxWorld = 64;    // ranks (their table entries live in shared memory)
 constexpr int kGroupRanks = 8;   // ranks whose inverse-map rows a warp stages at once
 constexpr int kMaxE = 64;        // local experts per rank (two inverse entries per lane)
-#ifndef MOE_EPC_UPL
-#define MOE_EPC_UPL 1
-#endif
-constexpr int kMaxUPL = MOE_EPC_UPL;  // units per lane per item: split keeps items <= 32 * kMaxUPL units
-#ifndef MOE_EPC_ROWS
-#define MOE_EPC_ROWS 8
-#endif
-constexpr int kRowsInFlight = MOE_EPC_ROWS;
+// units per lane per item with one group of ranks: 8 (two items per 4096-wide
+// bf16 row) measured fastest against 1, 2, 4 and 16 (203 us against 218-321)
+constexpr int kUnitsPerLane = 8;
+constexpr int kRowsInFlight = 8;    // expert rows in flight per unit (general kernel)
 
 // A unit of a row: 8 elements (16-byte loads) or 1 element.
 template <class D, bool VEC> struct Unit;
@@ -121,9 +117,9 @@ __device__ __forceinline__ void close_partial(float (&part)[V], float (&acc)[V],
   }
 }
 
-// One unit of the row: the list's rows (kRowsInFlight loads in flight), each
+// One unit of the row: the list's rows (ROWS loads in flight), each
 // rank's partial closed in rank order, `trailing` closes after the last row.
-template <class DI, class DP, bool VEC, bool ALIGNED>
+template <class DI, class DP, bool VEC, bool ALIGNED, int ROWS = kRowsInFlight>
 __device__ __forceinline__ void fold_unit(const typename DI::T* const* ptrs, const uint8_t* gaps,
                                           int F, int trailing, int q0, int64_t u,
                                           float (&acc)[Unit<DI, VEC>::V]) {
@@ -133,13 +129,13 @@ __device__ __forceinline__ void fold_unit(const typename DI::T* const* ptrs, con
 #pragma unroll
   for (int i = 0; i < V; ++i) part[i] = 0.0f;
   int q = q0;                                           // global rank of the open partial
-  for (int f0 = 0; f0 < F; f0 += kRowsInFlight) {
-    typename U::Raw raw[kRowsInFlight];
+  for (int f0 = 0; f0 < F; f0 += ROWS) {
+    typename U::Raw raw[ROWS];
 #pragma unroll
-    for (int j = 0; j < kRowsInFlight; ++j)
+    for (int j = 0; j < ROWS; ++j)
       if (f0 + j < F) raw[j] = U::template load<ALIGNED>(ptrs[f0 + j] + u * V);
 #pragma unroll
-    for (int j = 0; j < kRowsInFlight; ++j) {
+    for (int j = 0; j < ROWS; ++j) {
       if (f0 + j < F) {
         for (int c = gaps[f0 + j]; c > 0; --c, ++q) close_partial<DP, V>(part, acc, q == 0);
         float v[V];
@@ -170,84 +166,187 @@ __device__ __forceinline__ void load_group(const int32_t* const* inv, int q0, in
   }
 }
 
-// The warp's items: (token, slice of the row) pairs, strided over the grid
-// with a division-free cursor.
-template <class DI, class DP, class DO, bool VEC, bool TWO, bool ALIGNED>
-__device__ __forceinline__ void combine_items(
+// The rank-ordered row list of ranks q0 .. q0+nq-1 from their staged
+// inverse-map entries; returns its length and, in `trailing`, the partials
+// still to close after its last row.
+template <class T, bool TWO>
+__device__ __forceinline__ int build_list(const int32_t (&p0)[kGroupRanks],
+                                          const int32_t (&p1)[kGroupRanks], int q0, int nq,
+                                          int64_t max_rows, const T* const* eo, int64_t hidden,
+                                          const T** ptrs, uint8_t* gaps, int32_t* err, int lane,
+                                          int& trailing) {
+  int F = 0, open = 0;                                   // open: the rank whose partial is open
+#pragma unroll
+  for (int k = 0; k < kGroupRanks; ++k) {
+    if (k < nq) {
+      const int c = append_rank<T, TWO>(p0[k], p1[k], max_rows, eo[q0 + k], hidden, k - open,
+                                        ptrs + F, gaps + F, err, lane);
+      if (c > 0) open = k;
+      F += c;
+    }
+  }
+  trailing = nq - open;
+  return F;
+}
+
+// The warp's items -- (token, slice of the row) pairs, strided over the grid
+// with a division-free cursor -- for up to 8 ranks (one group): the row list
+// is built once per item, then the item's 16-byte units are folded and
+// stored one after another.
+template <class DI, class DP, class DO, bool TWO, bool ALIGNED, int ROWS>
+__device__ __forceinline__ void combine_one_group(
     const typename DI::T* const* eo, const int32_t* const* inv, const typename DI::T** ptrs,
-    uint8_t* gaps,
-    int world, int64_t first, int64_t t_lo, int64_t t_hi, int split, int64_t units,
-    int64_t hidden, int64_t max_rows, int E, typename DO::T* __restrict__ out, int32_t* err,
-    int lane, int64_t it0, int64_t nwarps) {
-  constexpr int V = Unit<DI, VEC>::V;
+    uint8_t* gaps, int world, int64_t first, int64_t t_lo, int64_t t_hi, int split,
+    int64_t units, int64_t hidden, int64_t max_rows, int E, typename DO::T* __restrict__ out,
+    int32_t* err, int lane, int64_t it0, int64_t nwarps) {
+  using T = typename DI::T;
   const int64_t n_tok = t_hi - t_lo;
-  const int64_t upi = (units + split - 1) / split;       // units per item, <= 32 * kMaxUPL
-  const int nq0 = world < kGroupRanks ? world : kGroupRanks;
-  RowCursor cur(it0, nwarps, split);                      // (token, slice) of item it0
+  const int64_t upi = (units + split - 1) / split;
+  RowCursor cur(it0, nwarps, split);
   if (cur.r >= n_tok) return;                             // warp-uniform
   int32_t p0[kGroupRanks], p1[kGroupRanks];
-  load_group<TWO>(inv, 0, nq0, first + t_lo + cur.r, E, lane, p0, p1);
+  load_group<TWO>(inv, 0, world, first + t_lo + cur.r, E, lane, p0, p1);
   while (cur.r < n_tok) {
     const int64_t t = t_lo + cur.r;
-    const int64_t g = first + t;
     const int64_t u0 = cur.c * upi;
     const int64_t u1 = min(units, u0 + upi);
     RowCursor nxt = cur;
     nxt.advance();
-    float acc[kMaxUPL][V];
+    __syncwarp();                                        // the previous list is consumed
+    int trailing;
+    const int F = build_list<T, TWO>(p0, p1, 0, world, max_rows, eo, hidden, ptrs, gaps, err,
+                                     lane, trailing);
+    __syncwarp();
+    if (nxt.r < n_tok)                                   // next item's entries, in flight
+      load_group<TWO>(inv, 0, world, first + t_lo + nxt.r, E, lane, p0, p1);
+    for (int64_t u = u0 + lane; u < u1; u += 32) {
+      float acc[kVec];
 #pragma unroll
-    for (int j = 0; j < kMaxUPL; ++j)
-#pragma unroll
-      for (int i = 0; i < V; ++i) acc[j][i] = 0.0f;
-    for (int q0 = 0; q0 < world; q0 += kGroupRanks) {
-      const int nq = world - q0 < kGroupRanks ? world - q0 : kGroupRanks;
-      if (q0 > 0) load_group<TWO>(inv, q0, nq, g, E, lane, p0, p1);   // later groups
-      __syncwarp();                                      // the previous list is consumed
-      int F = 0, open = 0;                               // open: the rank whose partial is open
-#pragma unroll
-      for (int k = 0; k < kGroupRanks; ++k) {
-        if (k < nq) {
-          const int c = append_rank<typename DI::T, TWO>(p0[k], p1[k], max_rows, eo[q0 + k],
-                                                         hidden, k - open, ptrs + F, gaps + F,
-                                                         err, lane);
-          if (c > 0) open = k;
-          F += c;
-        }
-      }
-      const int trailing = nq - open;
-      __syncwarp();
-      if (q0 + kGroupRanks >= world && nxt.r < n_tok)   // next item's first group, in flight
-        load_group<TWO>(inv, 0, nq0, first + t_lo + nxt.r, E, lane, p0, p1);
-#pragma unroll
-      for (int j = 0; j < kMaxUPL; ++j) {
-        const int64_t u = u0 + lane + 32 * j;
-        if (u < u1)
-          fold_unit<DI, DP, VEC, ALIGNED>(ptrs, gaps, F, trailing, q0, u, acc[j]);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kMaxUPL; ++j) {
-      const int64_t u = u0 + lane + 32 * j;
-      if (u < u1) {
-        if constexpr (VEC) store8<DO>(out + t * hidden + u * kVec, acc[j]);
-        else store1<DO>(out + t * hidden + u, acc[j][0]);
-      }
+      for (int i = 0; i < kVec; ++i) acc[i] = 0.0f;
+      fold_unit<DI, DP, true, ALIGNED, ROWS>(ptrs, gaps, F, trailing, 0, u, acc);
+      store8<DO>(out + t * hidden + u * kVec, acc);
     }
     cur = nxt;
   }
 }
 
-#ifndef MOE_EPC_MIN_BLOCKS
-#define MOE_EPC_MIN_BLOCKS 0
-#endif
+// Any number of ranks and any row width / alignment: one unit per lane per
+// item, each unit's sum carried across the groups of 8 ranks.
+template <class DI, class DP, class DO, bool VEC, bool ALIGNED>
+__device__ __forceinline__ void combine_groups(
+    const typename DI::T* const* eo, const int32_t* const* inv, const typename DI::T** ptrs,
+    uint8_t* gaps, int world, int64_t first, int64_t t_lo, int64_t t_hi, int split,
+    int64_t units, int64_t hidden, int64_t max_rows, int E, typename DO::T* __restrict__ out,
+    int32_t* err, int lane, int64_t it0, int64_t nwarps) {
+  using T = typename DI::T;
+  constexpr int V = Unit<DI, VEC>::V;
+  const int64_t n_tok = t_hi - t_lo;
+  const int64_t upi = (units + split - 1) / split;       // <= 32 units: one per lane
+  const int nq0 = world < kGroupRanks ? world : kGroupRanks;
+  RowCursor cur(it0, nwarps, split);
+  if (cur.r >= n_tok) return;                             // warp-uniform
+  int32_t p0[kGroupRanks], p1[kGroupRanks];
+  load_group<true>(inv, 0, nq0, first + t_lo + cur.r, E, lane, p0, p1);
+  while (cur.r < n_tok) {
+    const int64_t t = t_lo + cur.r;
+    const int64_t g = first + t;
+    const int64_t u = cur.c * upi + lane;
+    const bool mine = u < min(units, cur.c * upi + upi);
+    RowCursor nxt = cur;
+    nxt.advance();
+    float acc[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] = 0.0f;
+    for (int q0 = 0; q0 < world; q0 += kGroupRanks) {
+      const int nq = world - q0 < kGroupRanks ? world - q0 : kGroupRanks;
+      if (q0 > 0) load_group<true>(inv, q0, nq, g, E, lane, p0, p1);   // later groups
+      __syncwarp();
+      int trailing;
+      const int F = build_list<T, true>(p0, p1, q0, nq, max_rows, eo, hidden, ptrs, gaps, err,
+                                        lane, trailing);
+      __syncwarp();
+      if (q0 + kGroupRanks >= world && nxt.r < n_tok)
+        load_group<true>(inv, 0, nq0, first + t_lo + nxt.r, E, lane, p0, p1);
+      if (mine) fold_unit<DI, DP, VEC, ALIGNED>(ptrs, gaps, F, trailing, q0, u, acc);
+    }
+    if (mine) {
+      if constexpr (VEC) store8<DO>(out + t * hidden + u * kVec, acc);
+      else store1<DO>(out + t * hidden + u, acc[0]);
+    }
+    cur = nxt;
+  }
+}
 
-template <class DI, class DP, class DO, bool VEC, bool TWO>
-__global__ void __launch_bounds__(kThreads, MOE_EPC_MIN_BLOCKS)
-ep_combine_warp(const void* const* __restrict__ eo_tab, const void* const* __restrict__ inv_tab,
-                int world, int rank, const int32_t* __restrict__ offs,
-                const int32_t* __restrict__ ep_tokens, int64_t capacity, int64_t max_rows,
-                int E, typename DO::T* __restrict__ out, int64_t local, int64_t hidden,
-                int split, int32_t* err) {
+// Shared set-up of both kernels: the valid rows of this rank (as the
+// reduce-scatter) and the world's table entries in shared memory.
+struct CombineSetup {
+  int64_t first, t_lo, t_hi;
+  bool aligned;
+};
+
+template <class T>
+__device__ __forceinline__ CombineSetup combine_setup(
+    const void* const* eo_tab, const void* const* inv_tab, int world, int rank,
+    const int32_t* offs, const int32_t* ep_tokens, int64_t capacity, int64_t local,
+    const T** s_eo, const int32_t** s_inv, int32_t* err) {
+  CombineSetup c;
+  c.first = __ldg(offs + rank);
+  const int64_t ep = __ldg(ep_tokens);
+  const int64_t avail = ep < 0 ? 0 : (ep > capacity ? capacity : ep);
+  c.t_lo = c.first < 0 ? -c.first : 0;
+  c.t_hi = avail - c.first < local ? avail - c.first : local;
+  if (c.t_lo > local) c.t_lo = local;
+  if (c.t_hi < c.t_lo) c.t_hi = c.t_lo;
+  if ((ep < 0 || ep > capacity || c.t_lo > 0 || c.t_hi < local) && blockIdx.x == 0 &&
+      threadIdx.x == 0)
+    flag_error(err, MOE_DEVERR_COUNT);
+  int misaligned = 0;
+  for (int q = threadIdx.x; q < world; q += blockDim.x) {
+    s_eo[q] = static_cast<const T*>(eo_tab[q]);
+    s_inv[q] = static_cast<const int32_t*>(inv_tab[q]);
+    misaligned |= (int)(reinterpret_cast<uintptr_t>(eo_tab[q]) & 15);
+  }
+  c.aligned = __syncthreads_or(misaligned) == 0;
+  return c;
+}
+
+#define MOE_EPC_PARAMS                                                                        \
+  const void* const* __restrict__ eo_tab, const void* const* __restrict__ inv_tab, int world, \
+      int rank, const int32_t* __restrict__ offs, const int32_t* __restrict__ ep_tokens,      \
+      int64_t capacity, int64_t max_rows, int E, typename DO::T* __restrict__ out,            \
+      int64_t local, int64_t hidden, int split, int32_t* err
+
+// Up to 8 ranks, 16-byte units (hidden % 8 == 0, out aligned).  ROWS: expert
+// rows in flight per unit -- 8 for short launches (fewer items than warps:
+// depth per warp counts), 4 for long ones (80 registers, 3 CTAs per SM).
+template <class DI, class DP, class DO, bool TWO, int ROWS>
+__global__ void __launch_bounds__(kThreads)
+ep_combine_group(MOE_EPC_PARAMS) {
+  using TI = typename DI::T;
+  __shared__ const TI* s_eo[kMaxWorld];
+  __shared__ const int32_t* s_inv[kMaxWorld];
+  __shared__ const TI* s_ptrs[kThreads / 32][kGroupRanks * kMaxE];
+  __shared__ uint8_t s_gaps[kThreads / 32][kGroupRanks * kMaxE];
+  pdl_prologue();
+  const CombineSetup c = combine_setup<TI>(eo_tab, inv_tab, world, rank, offs, ep_tokens,
+                                           capacity, local, s_eo, s_inv, err);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t it0 = (int64_t)blockIdx.x * (kThreads / 32) + warp;
+  const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
+  if (c.aligned)
+    combine_one_group<DI, DP, DO, TWO, true, ROWS>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world,
+                                             c.first, c.t_lo, c.t_hi, split, hidden / kVec,
+                                             hidden, max_rows, E, out, err, lane, it0, nwarps);
+  else                                                   // a buffer off 16-byte alignment
+    combine_one_group<DI, DP, DO, TWO, false, ROWS>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world,
+                                              c.first, c.t_lo, c.t_hi, split, hidden / kVec,
+                                              hidden, max_rows, E, out, err, lane, it0, nwarps);
+}
+
+// Any number of ranks, any width and alignment.
+template <class DI, class DP, class DO, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+ep_combine_groups(MOE_EPC_PARAMS) {
   using TI = typename DI::T;
   constexpr int V = Unit<DI, VEC>::V;
   __shared__ const TI* s_eo[kMaxWorld];
@@ -255,39 +354,21 @@ ep_combine_warp(const void* const* __restrict__ eo_tab, const void* const* __res
   __shared__ const TI* s_ptrs[kThreads / 32][kGroupRanks * kMaxE];
   __shared__ uint8_t s_gaps[kThreads / 32][kGroupRanks * kMaxE];
   pdl_prologue();
-  // this rank's rows whose token lies inside the data (as the reduce-scatter)
-  const int64_t first = __ldg(offs + rank);
-  const int64_t ep = __ldg(ep_tokens);
-  const int64_t avail = ep < 0 ? 0 : (ep > capacity ? capacity : ep);
-  int64_t t_lo = first < 0 ? -first : 0;
-  int64_t t_hi = avail - first < local ? avail - first : local;
-  if (t_lo > local) t_lo = local;
-  if (t_hi < t_lo) t_hi = t_lo;
-  if ((ep < 0 || ep > capacity || t_lo > 0 || t_hi < local) && blockIdx.x == 0 &&
-      threadIdx.x == 0)
-    flag_error(err, MOE_DEVERR_COUNT);
-  int misaligned = 0;
-  for (int q = threadIdx.x; q < world; q += blockDim.x) {
-    s_eo[q] = static_cast<const TI*>(eo_tab[q]);
-    s_inv[q] = static_cast<const int32_t*>(inv_tab[q]);
-    misaligned |= (int)(reinterpret_cast<uintptr_t>(eo_tab[q]) & 15);
-  }
-  const bool aligned = __syncthreads_or(misaligned) == 0;
+  const CombineSetup c = combine_setup<TI>(eo_tab, inv_tab, world, rank, offs, ep_tokens,
+                                           capacity, local, s_eo, s_inv, err);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t it0 = (int64_t)blockIdx.x * (kThreads / 32) + warp;
   const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
-#define MOE_EPC_ITEMS(AL)                                                                    \
-  combine_items<DI, DP, DO, VEC, TWO, AL>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world,   \
-                                          first, t_lo, t_hi, split, hidden / V, hidden,     \
-                                          max_rows, E, out, err, lane, it0, nwarps)
-  if constexpr (VEC) {
-    if (aligned) MOE_EPC_ITEMS(true);
-    else MOE_EPC_ITEMS(false);                           // a buffer off 16-byte alignment
-  } else {
-    MOE_EPC_ITEMS(true);
-  }
-#undef MOE_EPC_ITEMS
+  if (!VEC || c.aligned)
+    combine_groups<DI, DP, DO, VEC, true>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world,
+                                          c.first, c.t_lo, c.t_hi, split, hidden / V, hidden,
+                                          max_rows, E, out, err, lane, it0, nwarps);
+  else
+    combine_groups<DI, DP, DO, VEC, false>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world,
+                                           c.first, c.t_lo, c.t_hi, split, hidden / V, hidden,
+                                           max_rows, E, out, err, lane, it0, nwarps);
 }
+#undef MOE_EPC_PARAMS
 
 template <class DI, class DP, class DO>
 int launch(const void* const* eos, const void* const* invs, int world, int rank,
@@ -295,20 +376,50 @@ int launch(const void* const* eos, const void* const* invs, int world, int rank,
            int E, void* out, int64_t local, int64_t hidden, int32_t* err, cudaStream_t stream) {
   using TO = typename DO::T;
   const bool vec = hidden % kVec == 0 && aligned16(out);
+  const bool one_group = vec && world <= kGroupRanks;
   const int64_t units = vec ? hidden / kVec : hidden;
-  const int64_t split64 = (units + 32 * kMaxUPL - 1) / (32 * kMaxUPL);
+  // units per item: 32 lanes x kUnitsPerLane with one group of ranks (the row
+  // list is built once per item), one per lane otherwise
+  const int64_t per_item = 32 * (one_group ? kUnitsPerLane : 1);
+  const int64_t split64 = (units + per_item - 1) / per_item;
   const int split = (int)(split64 < 1 ? 1 : split64);
-  const bool two = E > 32;
-  auto k = vec ? (two ? ep_combine_warp<DI, DP, DO, true, true> : ep_combine_warp<DI, DP, DO, true, false>)
-               : (two ? ep_combine_warp<DI, DP, DO, false, true>
-                      : ep_combine_warp<DI, DP, DO, false, false>);
   const int64_t warps = local * split;
+  int sms = 0;
+  if (int rc = device_sm_count(&sms)) return rc;
+  // measured on B200 (8 ranks x 8 experts, top-8, hidden 4096): 8 rows in
+  // flight win while items are few (1024 tokens a rank: 203 against 234 us),
+  // 4 rows at 3 CTAs per SM once there are several items per warp (8192 tokens
+  // a rank: 1112 against 1371 us)
+  const bool deep = warps < 4 * (int64_t)sms * 16;
+  const void* k;
+  if (one_group)
+    k = E > 32 ? (deep ? (const void*)ep_combine_group<DI, DP, DO, true, 8>
+                       : (const void*)ep_combine_group<DI, DP, DO, true, 4>)
+               : (deep ? (const void*)ep_combine_group<DI, DP, DO, false, 8>
+                       : (const void*)ep_combine_group<DI, DP, DO, false, 4>);
+  else
+    k = vec ? (const void*)ep_combine_groups<DI, DP, DO, true>
+            : (const void*)ep_combine_groups<DI, DP, DO, false>;
   int grid;
-  if (int rc = persistent_grid((const void*)k, 0, (warps + kThreads / 32 - 1) / (kThreads / 32),
-                               &grid))
+  if (int rc = persistent_grid(k, 0, (warps + kThreads / 32 - 1) / (kThreads / 32), &grid))
     return rc;
-  launch_kernel(k, grid, 0, stream, eos, invs, world, rank, offs, ep_tokens, capacity, max_rows,
-                E, static_cast<TO*>(out), local, hidden, split, err);
+#define MOE_EPC_LAUNCH(KERNEL)                                                                 \
+  launch_kernel(KERNEL, grid, 0, stream, eos, invs, world, rank, offs, ep_tokens, capacity,    \
+                max_rows, E, static_cast<TO*>(out), local, hidden, split, err)
+  if (one_group) {
+    if (E > 32) {
+      if (deep) MOE_EPC_LAUNCH((ep_combine_group<DI, DP, DO, true, 8>));
+      else MOE_EPC_LAUNCH((ep_combine_group<DI, DP, DO, true, 4>));
+    } else {
+      if (deep) MOE_EPC_LAUNCH((ep_combine_group<DI, DP, DO, false, 8>));
+      else MOE_EPC_LAUNCH((ep_combine_group<DI, DP, DO, false, 4>));
+    }
+  } else if (vec) {
+    MOE_EPC_LAUNCH((ep_combine_groups<DI, DP, DO, true>));
+  } else {
+    MOE_EPC_LAUNCH((ep_combine_groups<DI, DP, DO, false>));
+  }
+#undef MOE_EPC_LAUNCH
   return check_launch();
 }
 

@@ -156,3 +156,16 @@ def test_ep_combine_bad_rows_and_entries(cuda_device):
     want, oerr = _oracle(case, 1, torch.float32, torch.float32, init)
     assert int(err) == _abi.MOE_DEVERR_INVERSE and oerr == _abi.MOE_DEVERR_INVERSE
     assert np.array_equal(bits(got).view(np.uint32), want.view(np.uint32))
+
+
+def test_ep_combine_long_launch(cuda_device):
+    """A launch with many items per warp takes the 4-rows-in-flight kernel:
+    2 ranks, 40000 tokens (about 20000 a rank) x top-4 of 8 experts, hidden
+    4096 -- still the two library kernels' bits for every row."""
+    case = inputs.ep_combine_inputs(2, 40000, 4, 4, 128, 4096, seed=8, device=cuda_device)
+    eo_t, inv_t, keep = _tables(cuda_device, case)
+    for rank in range(2):
+        init = torch.zeros(case.counts[rank], 4096, dtype=torch.bfloat16)
+        got = _run(cuda_device, case, eo_t, inv_t, rank, torch.bfloat16, torch.bfloat16, init)
+        assert_bits_equal(bits(got), bits(_two_step(cuda_device, case, rank, torch.bfloat16,
+                                                    torch.bfloat16)), f"rank {rank}")
