@@ -6,7 +6,7 @@ sweep reaches combinations the hand-picked tests do not -- odd widths, tiny and
 ragged sizes, unaligned views that take the element-wise paths, short live
 prefixes -- and every failure replays from its case index.  Pass criteria are
 the ops' own: bit-exact for the router-weight multiply, the unpermute, the
-residual add, the fused chain and the reduce-scatter; within 1 ulp of the
+residual add, the fused chain, the reduce-scatter and the EP combine; within 1 ulp of the
 16-bit dtype for the SwiGLU forms and the soft-clamped squared ReLU; the
 reduction tolerance for the probability gradients.
 """
@@ -240,3 +240,38 @@ def test_fuzz_reduce_scatter(cuda_device, case):
                           f"case {case}: world {world} rank {rank} tokens {tokens} hidden "
                           f"{hidden} {in_dt}->{out_dt} byte offset {byte_off}",
                           kind=KIND.get(out_dt, "bf16"))
+
+
+@pytest.mark.parametrize("case", range(N_CASES))
+def test_fuzz_ep_combine(cuda_device, case):
+    r = _rng(case, 7)
+    world = int(r.integers(1, 12))
+    top_k = int(r.integers(1, 9))
+    epr = int(r.integers(max(1, -(-top_k // world)), 40))
+    tokens, hidden = int(r.integers(1, 200)), int(r.integers(1, 700))
+    eo_dt = DT[int(r.integers(0, 3))]
+    p_dt = [eo_dt, torch.float32][int(r.integers(0, 2))]
+    o_dt = [eo_dt, torch.float32][int(r.integers(0, 2))]
+    ec = inputs.ep_combine_inputs(world, tokens, top_k, epr, int(r.choice([1, 4, 16])), hidden,
+                                  dtype=eo_dt, seed=case)
+    keep = [e.to(cuda_device) for e in ec.expert_outputs] + \
+        [i.to(cuda_device) for i in ec.inverse_maps]
+    eo_t, inv_t = ops.pointer_table(keep[:world]), ops.pointer_table(keep[world:])
+    ep = torch.tensor([tokens], dtype=torch.int32, device=cuda_device)
+    offs = ec.rank_token_offset.to(cuda_device)
+    eos = [bits(e) for e in ec.expert_outputs]
+    invs = [bits(i) for i in ec.inverse_maps]
+    for rank in range(world):
+        init = torch.full((ec.counts[rank], hidden), 1.25, dtype=o_dt)
+        out = init.to(cuda_device)
+        ops.unpermute_reduce_scatter(eo_t, eo_dt, ec.max_rows, inv_t, epr, tokens, ep, rank, offs,
+                                     hidden, out=out, partial_dtype=p_dt)
+        torch.cuda.synchronize()
+        want, err = oracle.unpermute_reduce_scatter(eos, ODT[eo_dt], invs, tokens, rank,
+                                                    ec.rank_token_offset.numpy(), ODT[p_dt],
+                                                    bits(init), ODT[o_dt])
+        assert err == 0
+        assert_bits_equal(bits(out), want,
+                          f"case {case}: world {world} rank {rank} top-{top_k} of {world}x{epr} "
+                          f"tokens {tokens} hidden {hidden} {eo_dt}/{p_dt}/{o_dt}",
+                          kind=KIND.get(o_dt, "bf16"))
