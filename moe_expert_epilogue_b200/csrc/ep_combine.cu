@@ -36,9 +36,7 @@ namespace {
 constexpr int kMaxWorld = 64;    // ranks (their table entries live in shared memory)
 constexpr int kGroupRanks = 8;   // ranks whose inverse-map rows a warp stages at once
 constexpr int kMaxE = 64;        // local experts per rank (two inverse entries per lane)
-// units per lane per item with one group of ranks: 8 (two items per 4096-wide
-// bf16 row) measured fastest against 1, 2, 4 and 16 (203 us against 218-321)
-constexpr int kUnitsPerLane = 8;
+constexpr int kRowsGroup = 4;       // expert rows in flight per unit (one-group kernel)
 constexpr int kRowsInFlight = 8;    // expert rows in flight per unit (general kernel)
 
 // A unit of a row: 8 elements (16-byte loads) or 1 element.
@@ -316,10 +314,10 @@ __device__ __forceinline__ CombineSetup combine_setup(
       int64_t capacity, int64_t max_rows, int E, typename DO::T* __restrict__ out,            \
       int64_t local, int64_t hidden, int split, int32_t* err
 
-// Up to 8 ranks, 16-byte units (hidden % 8 == 0, out aligned).  ROWS: expert
-// rows in flight per unit -- 8 for short launches (fewer items than warps:
-// depth per warp counts), 4 for long ones (80 registers, 3 CTAs per SM).
-template <class DI, class DP, class DO, bool TWO, int ROWS>
+// Up to 8 ranks, 16-byte units (hidden % 8 == 0, out aligned); 4 expert rows
+// in flight per unit keep it at 80 registers, 3 CTAs per SM (8 rows: 104
+// registers, 2 CTAs, slower except on the shortest launches).
+template <class DI, class DP, class DO, bool TWO>
 __global__ void __launch_bounds__(kThreads)
 ep_combine_group(MOE_EPC_PARAMS) {
   using TI = typename DI::T;
@@ -334,11 +332,11 @@ ep_combine_group(MOE_EPC_PARAMS) {
   const int64_t it0 = (int64_t)blockIdx.x * (kThreads / 32) + warp;
   const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
   if (c.aligned)
-    combine_one_group<DI, DP, DO, TWO, true, ROWS>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world,
+    combine_one_group<DI, DP, DO, TWO, true, kRowsGroup>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world,
                                              c.first, c.t_lo, c.t_hi, split, hidden / kVec,
                                              hidden, max_rows, E, out, err, lane, it0, nwarps);
   else                                                   // a buffer off 16-byte alignment
-    combine_one_group<DI, DP, DO, TWO, false, ROWS>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world,
+    combine_one_group<DI, DP, DO, TWO, false, kRowsGroup>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world,
                                               c.first, c.t_lo, c.t_hi, split, hidden / kVec,
                                               hidden, max_rows, E, out, err, lane, it0, nwarps);
 }
@@ -378,25 +376,28 @@ int launch(const void* const* eos, const void* const* invs, int world, int rank,
   const bool vec = hidden % kVec == 0 && aligned16(out);
   const bool one_group = vec && world <= kGroupRanks;
   const int64_t units = vec ? hidden / kVec : hidden;
-  // units per item: 32 lanes x kUnitsPerLane with one group of ranks (the row
-  // list is built once per item), one per lane otherwise
-  const int64_t per_item = 32 * (one_group ? kUnitsPerLane : 1);
+  int sms = 0;
+  if (int rc = device_sm_count(&sms)) return rc;
+  // Units per item: one per lane across groups of ranks.  With one group, 4
+  // per lane once there are at least two items per resident warp (3 CTAs of
+  // 8 warps per SM), else 2, so that short launches still spread over the
+  // GPU.  Measured on B200, 8 ranks x 8 experts, top-8, hidden 4096, 4 rows in
+  // flight: 1024 tokens a rank 203.5 us (2 per lane) against 225.6 (4);
+  // 4096 tokens a rank 598.8 (4) against 614.6 (2) and 763.3 for the earlier
+  // 8 rows in flight x 8 per lane.
+  int per_lane = 1;
+  if (one_group) {
+    const int64_t items4 = local * ((units + 32 * 4 - 1) / (32 * 4));
+    per_lane = items4 >= 2 * (int64_t)sms * 24 ? 4 : 2;
+  }
+  const int64_t per_item = 32 * (int64_t)per_lane;
   const int64_t split64 = (units + per_item - 1) / per_item;
   const int split = (int)(split64 < 1 ? 1 : split64);
   const int64_t warps = local * split;
-  int sms = 0;
-  if (int rc = device_sm_count(&sms)) return rc;
-  // measured on B200 (8 ranks x 8 experts, top-8, hidden 4096): 8 rows in
-  // flight win while items are few (1024 tokens a rank: 203 against 234 us),
-  // 4 rows at 3 CTAs per SM once there are several items per warp (8192 tokens
-  // a rank: 1112 against 1371 us)
-  const bool deep = warps < 4 * (int64_t)sms * 16;
   const void* k;
   if (one_group)
-    k = E > 32 ? (deep ? (const void*)ep_combine_group<DI, DP, DO, true, 8>
-                       : (const void*)ep_combine_group<DI, DP, DO, true, 4>)
-               : (deep ? (const void*)ep_combine_group<DI, DP, DO, false, 8>
-                       : (const void*)ep_combine_group<DI, DP, DO, false, 4>);
+    k = E > 32 ? (const void*)ep_combine_group<DI, DP, DO, true>
+               : (const void*)ep_combine_group<DI, DP, DO, false>;
   else
     k = vec ? (const void*)ep_combine_groups<DI, DP, DO, true>
             : (const void*)ep_combine_groups<DI, DP, DO, false>;
@@ -407,13 +408,8 @@ int launch(const void* const* eos, const void* const* invs, int world, int rank,
   launch_kernel(KERNEL, grid, 0, stream, eos, invs, world, rank, offs, ep_tokens, capacity,    \
                 max_rows, E, static_cast<TO*>(out), local, hidden, split, err)
   if (one_group) {
-    if (E > 32) {
-      if (deep) MOE_EPC_LAUNCH((ep_combine_group<DI, DP, DO, true, 8>));
-      else MOE_EPC_LAUNCH((ep_combine_group<DI, DP, DO, true, 4>));
-    } else {
-      if (deep) MOE_EPC_LAUNCH((ep_combine_group<DI, DP, DO, false, 8>));
-      else MOE_EPC_LAUNCH((ep_combine_group<DI, DP, DO, false, 4>));
-    }
+    if (E > 32) MOE_EPC_LAUNCH((ep_combine_group<DI, DP, DO, true>));
+    else MOE_EPC_LAUNCH((ep_combine_group<DI, DP, DO, false>));
   } else if (vec) {
     MOE_EPC_LAUNCH((ep_combine_groups<DI, DP, DO, true>));
   } else {
