@@ -24,9 +24,9 @@
 // (the first group of the next item is prefetched) and compacts them into one
 // rank-ordered list of row pointers in shared memory, each entry tagged with
 // the number of rank partials to close before it; then, per 16-byte unit of
-// the row, it keeps up to 8 expert rows' loads in flight and closes each
-// rank's partial in rank order (ranks without rows contribute +0, as their
-// partial block row would).
+// the row, it keeps 4 expert rows' loads in flight (8 in the kernel for more
+// than 8 ranks or odd widths) and closes each rank's partial in rank order
+// (ranks without rows contribute +0, as their partial block row would).
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -36,8 +36,8 @@ namespace {
 constexpr int kMaxWorld = 64;    // ranks (their table entries live in shared memory)
 constexpr int kGroupRanks = 8;   // ranks whose inverse-map rows a warp stages at once
 constexpr int kMaxE = 64;        // local experts per rank (two inverse entries per lane)
-constexpr int kRowsGroup = 4;       // expert rows in flight per unit (one-group kernel)
-constexpr int kRowsInFlight = 8;    // expert rows in flight per unit (general kernel)
+constexpr int kRowsGroup = 4;    // expert rows in flight per unit (one-group kernel)
+constexpr int kRowsInFlight = 8; // expert rows in flight per unit (general kernel)
 
 // A unit of a row: 8 elements (16-byte loads) or 1 element.
 template <class D, bool VEC> struct Unit;
@@ -332,11 +332,13 @@ ep_combine_group(MOE_EPC_PARAMS) {
   const int64_t it0 = (int64_t)blockIdx.x * (kThreads / 32) + warp;
   const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
   if (c.aligned)
-    combine_one_group<DI, DP, DO, TWO, true, kRowsGroup>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world,
+    combine_one_group<DI, DP, DO, TWO, true, kRowsGroup>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp],
+                                                         world,
                                              c.first, c.t_lo, c.t_hi, split, hidden / kVec,
                                              hidden, max_rows, E, out, err, lane, it0, nwarps);
   else                                                   // a buffer off 16-byte alignment
-    combine_one_group<DI, DP, DO, TWO, false, kRowsGroup>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world,
+    combine_one_group<DI, DP, DO, TWO, false, kRowsGroup>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp],
+                                                          world,
                                               c.first, c.t_lo, c.t_hi, split, hidden / kVec,
                                               hidden, max_rows, E, out, err, lane, it0, nwarps);
 }
