@@ -332,15 +332,13 @@ ep_combine_group(MOE_EPC_PARAMS) {
   const int64_t it0 = (int64_t)blockIdx.x * (kThreads / 32) + warp;
   const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
   if (c.aligned)
-    combine_one_group<DI, DP, DO, TWO, true, kRowsGroup>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp],
-                                                         world,
-                                             c.first, c.t_lo, c.t_hi, split, hidden / kVec,
-                                             hidden, max_rows, E, out, err, lane, it0, nwarps);
+    combine_one_group<DI, DP, DO, TWO, true, kRowsGroup>(
+        s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world, c.first, c.t_lo, c.t_hi, split,
+        hidden / kVec, hidden, max_rows, E, out, err, lane, it0, nwarps);
   else                                                   // a buffer off 16-byte alignment
-    combine_one_group<DI, DP, DO, TWO, false, kRowsGroup>(s_eo, s_inv, s_ptrs[warp], s_gaps[warp],
-                                                          world,
-                                              c.first, c.t_lo, c.t_hi, split, hidden / kVec,
-                                              hidden, max_rows, E, out, err, lane, it0, nwarps);
+    combine_one_group<DI, DP, DO, TWO, false, kRowsGroup>(
+        s_eo, s_inv, s_ptrs[warp], s_gaps[warp], world, c.first, c.t_lo, c.t_hi, split,
+        hidden / kVec, hidden, max_rows, E, out, err, lane, it0, nwarps);
 }
 
 // Any number of ranks, any width and alignment.
