@@ -1,10 +1,12 @@
-"""Rank-order reduce-scatter between the processes of one node.
+"""Rank-order reduce-scatter and EP combine between the processes of one node.
 
 (core.inference.moe.batch_invariant: ordered_reduce_scatter_v.)  Every EP rank
 writes its partial results for the tokens of all ranks into a buffer that every
 other rank can read (`SymmetricBuffer`); `ordered_reduce_scatter_v` then sums,
 on each rank, the rows that rank owns over all ranks in rank order (fp32, one
-rounding), reading the peers' buffers directly over NVLink with plain loads.
+rounding), reading the peers' buffers directly over NVLink with plain loads;
+`unpermute_reduce_scatter` does the same straight from every rank's expert
+rows (the unpermute fused in).
 
 Ordering is stream-ordered and host-free: a one-element all-reduce on the
 process group before the launch (every rank's inputs are complete) and after
@@ -92,6 +94,12 @@ class SymmetricBuffer:
         raw = self.backend.view(self.local, self.nbytes, self.device)
         return raw[byte_offset:byte_offset + numel * esize].view(dtype).view(*shape)
 
+    def table_at(self, byte_offset: int = 0) -> torch.Tensor:
+        """The ranks' buffers from `byte_offset`, as a device pointer table."""
+        if byte_offset < 0 or byte_offset >= max(1, self.nbytes):
+            raise ValueError("offset outside the buffer")
+        return self.backend.table([p + byte_offset for p in self.ptrs], self.device)
+
     def _release(self):
         for q, p in enumerate(self.ptrs):
             if q != self.rank:
@@ -142,4 +150,34 @@ def ordered_reduce_scatter_v(output: torch.Tensor, symm: SymmetricBuffer,
                                  capacity_rows, hidden, in_dtype, out=output,
                                  input_byte_offset=input_byte_offset, dev_err=dev_err)
     stream_barrier(symm.group, symm.device)
+    return output
+
+
+def unpermute_reduce_scatter(output: torch.Tensor, experts: SymmetricBuffer,
+                             inverse_maps: SymmetricBuffer, eo_dtype: torch.dtype, max_rows: int,
+                             hidden: int, num_local_experts: int, capacity_rows: int,
+                             rank_token_offset: torch.Tensor, ep_tokens: torch.Tensor,
+                             eo_byte_offset: int = 0, inv_byte_offset: int = 0,
+                             partial_dtype=None, dev_err=None) -> torch.Tensor:
+    """Collective over experts.group: the EP combine.  Every rank holds its
+    experts' output rows ([max_rows, hidden] of eo_dtype at eo_byte_offset of
+    `experts`) and its inverse map over the token rows of all ranks (int32
+    [capacity_rows, num_local_experts] at inv_byte_offset of `inverse_maps`);
+    this rank's `output` [local_tokens, hidden] gets, per token, every rank's
+    expert-order partial sum folded in rank order -- the unpermute and the
+    rank-order reduce-scatter in one kernel, launched on the current stream
+    between two stream barriers."""
+    esize = torch.empty((), dtype=eo_dtype).element_size()
+    if eo_byte_offset + max_rows * hidden * esize > experts.nbytes or \
+            inv_byte_offset + capacity_rows * num_local_experts * 4 > inverse_maps.nbytes:
+        raise ValueError("a block does not fit in its symmetric buffer")
+    if experts.world != inverse_maps.world or experts.rank != inverse_maps.rank:
+        raise ValueError("both buffers must span the same group")
+    stream_barrier(experts.group, experts.device)
+    ops.unpermute_reduce_scatter(experts.table_at(eo_byte_offset), eo_dtype, max_rows,
+                                 inverse_maps.table_at(inv_byte_offset), num_local_experts,
+                                 capacity_rows, ep_tokens, experts.rank, rank_token_offset,
+                                 hidden, out=output, partial_dtype=partial_dtype,
+                                 dev_err=dev_err)
+    stream_barrier(experts.group, experts.device)
     return output

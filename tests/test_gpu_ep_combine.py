@@ -169,3 +169,68 @@ def test_ep_combine_long_launch(cuda_device):
         got = _run(cuda_device, case, eo_t, inv_t, rank, torch.bfloat16, torch.bfloat16, init)
         assert_bits_equal(bits(got), bits(_two_step(cuda_device, case, rank, torch.bfloat16,
                                                     torch.bfloat16)), f"rank {rank}")
+
+
+# ------------------------------------------------------- two processes, IPC
+
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _ipc_worker(rank, world, port, q):
+    import os
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import torch.distributed as dist
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        from moe_expert_epilogue_b200 import symmetric
+        dev = torch.device("cuda", 0)
+        ec = inputs.ep_combine_inputs(world, 300, 4, 4, 16, 512, seed=19)
+        experts = symmetric.SymmetricBuffer(256 + ec.max_rows * 512 * 2, device=dev)
+        maps = symmetric.SymmetricBuffer(300 * 4 * 4, device=dev)
+        experts.view(torch.bfloat16, (ec.max_rows, 512), 256).copy_(ec.expert_outputs[rank].to(dev))
+        maps.view(torch.int32, (300, 4)).copy_(ec.inverse_maps[rank].to(dev))
+        out = torch.empty(ec.counts[rank], 512, dtype=torch.bfloat16, device=dev)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        symmetric.unpermute_reduce_scatter(out, experts, maps, torch.bfloat16, ec.max_rows, 512, 4,
+                                           300, ec.rank_token_offset.to(dev),
+                                           torch.tensor([300], dtype=torch.int32, device=dev),
+                                           eo_byte_offset=256, dev_err=err)
+        res = (rank, bits(out.cpu()), int(err))
+        experts.close()
+        maps.close()
+        q.put(res)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ep_combine_two_processes_cuda_ipc(cuda_device):
+    """Two processes on this GPU, each publishing its expert rows and inverse
+    map in CUDA-IPC-mapped buffers; the collective wrapper combines over both
+    (host barriers under gloo; the kernels never wait on one another)."""
+    import torch.multiprocessing as mp
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ipc_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=240) for _ in range(world)), key=lambda r: r[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    ec = inputs.ep_combine_inputs(world, 300, 4, 4, 16, 512, seed=19)
+    for rank, got, err in res:
+        assert err == 0
+        want, _ = oracle.unpermute_reduce_scatter(
+            [bits(e) for e in ec.expert_outputs], oracle.BF16, [bits(i) for i in ec.inverse_maps],
+            300, rank, ec.rank_token_offset.numpy(), oracle.BF16,
+            np.zeros((ec.counts[rank], 512), np.uint16), oracle.BF16)
+        assert_bits_equal(got, want, f"rank {rank} over IPC")
