@@ -29,7 +29,7 @@
 namespace moe {
 namespace {
 
-template <class D> constexpr int kRowsAhead = D::kBytes == 4 ? 4 : 8;
+template <class D> constexpr int kRowsAhead = 4;
 
 template <class D, bool VEC, bool SMALL_E>
 __global__ void __launch_bounds__(kThreads)
@@ -140,15 +140,15 @@ epilogue_fused_kernel(const typename D::T* __restrict__ eo, const float* __restr
 // already loaded during the previous item) into its own shared-memory list,
 // so warps never wait for each other; items = tokens * SPLIT keep the load
 // balanced across the persistent grid.
-// Three resident CTAs per SM (at most 85 registers a thread): more warps to
-// hide the gather latency; measured 126 us against 138 us with the compiler's
-// own choice (102 registers, two CTAs) at 8192 tokens x top-8, hidden 4096.
-#ifndef MOE_FUSED_MIN_BLOCKS
-#define MOE_FUSED_MIN_BLOCKS 3
-#endif
+// More resident warps hide the gather latency better than more rows in flight
+// per warp: 4 rows at 4 CTAs per SM (64 registers) for the 16-bit types,
+// measured 122.5 us against 127.6 (8 rows, 3 CTAs) and 138 (8 rows, the
+// compiler's 102 registers, 2 CTAs) at 8192 tokens x top-8, hidden 4096; fp32
+// keeps 3 CTAs (4 would spill).
+template <class D> constexpr int kFusedMinBlocks = D::kBytes == 4 ? 3 : 4;
 
 template <class D, int SPLIT>
-__global__ void __launch_bounds__(kThreads, MOE_FUSED_MIN_BLOCKS)
+__global__ void __launch_bounds__(kThreads, kFusedMinBlocks<D>)
 epilogue_fused_warp(const typename D::T* __restrict__ eo, const float* __restrict__ row_probs,
                     int64_t max_rows, const int32_t* __restrict__ inv,
                     const int32_t* __restrict__ valid_tokens,
