@@ -768,3 +768,41 @@ def test_ep_combine_rounds_each_rank_partial():
     out_f, _ = oracle.unpermute_reduce_scatter(eos, oracle.F32, invs, 1, 0, [0, 1], oracle.F32,
                                                np.zeros((1, 1), np.float32), oracle.F32)
     assert out_b[0, 0] == 1.0 + 2.0 ** -8 and out_f[0, 0] == 1.0 + 2.0 ** -7
+
+
+# ------------------------------------------------------------ identities
+
+@pytest.mark.parametrize("x_dtype,out_dtype", [(torch.bfloat16, torch.bfloat16),
+                                               (torch.float32, torch.bfloat16),
+                                               (torch.bfloat16, torch.float16)])
+def test_router_weight_unit_probs_is_a_cast(x_dtype, out_dtype):
+    """probs = 1 is the identity weighting: x * 1 is exact, so the forward is a
+    plain dtype conversion of x (torch's), and grad_x one of grad_out."""
+    odt = {torch.bfloat16: oracle.BF16, torch.float16: oracle.F16, torch.float32: oracle.F32}
+    g = torch.Generator().manual_seed(31)
+    x = (torch.randn(33, 70, generator=g) * 5).to(x_dtype)
+    ones = np.ones(33, np.float32)
+    out = oracle.router_weight_fwd(bits(x), odt[x_dtype], ones, odt[out_dtype])
+    assert_bits_equal(out, bits(x.to(out_dtype)), "fwd with unit probs",
+                      kind="f16" if out_dtype == torch.float16 else "bf16")
+    gx, _, _ = oracle.router_weight_bwd(bits(x), odt[x_dtype], None, odt[out_dtype], ones)
+    assert_bits_equal(gx, bits(x.to(out_dtype)), "grad_x with unit probs",
+                      kind="f16" if out_dtype == torch.float16 else "bf16")
+
+
+def test_unpermute_single_expert_is_a_copy():
+    """A token routed to one local expert gets that expert row exactly (+0 + x
+    is x for every x but -0), converted by torch to the output dtype."""
+    g = torch.Generator().manual_seed(32)
+    eo = (torch.randn(10, 24, generator=g) * 3).to(torch.bfloat16)
+    inv = np.full((6, 4), -1, np.int32)
+    rows = [7, 2, 9, 0, 5, 3]
+    for t, r in enumerate(rows):
+        inv[t, t % 4] = r
+    for odt, tdt in ((oracle.BF16, torch.bfloat16), (oracle.F32, torch.float32)):
+        out, err = oracle.unpermute_ordered(bits(eo), oracle.BF16, inv, 6,
+                                            np.zeros((6, 24), oracle._storage_np(odt)), odt)
+        assert err == 0
+        want = eo[torch.tensor(rows)].to(tdt)
+        want = torch.where(want == 0, torch.zeros((), dtype=tdt), want)   # -0 becomes +0
+        assert_bits_equal(out, bits(want), f"copy to {tdt}")
