@@ -9,7 +9,9 @@
  * It also checks that a bad argument returns MOE_ERR_LIMIT without a launch, and
  * runs the rank-order reduce-scatter over three buffers from moe_symm_alloc
  * (exact integers: block q holds (q + 1) * (row * 16 + col + 1), so rank 1's
- * rows 4..7 sum to 6 * (row * 16 + col + 1)), after exporting an IPC handle.
+ * rows 4..7 sum to 6 * (row * 16 + col + 1)), after exporting an IPC handle,
+ * and the EP combine over two ranks' fp32 expert rows (token t of rank q's
+ * expert e: inverse map entry, rows holding small integers, exact sums).
  * Exit status 0 on success.
  */
 #include <stdio.h>
@@ -108,6 +110,64 @@ int main(void) {
       }
     for (int q = 0; q < W; ++q) CHECK(moe_symm_free(blocks[q]));
     CHECK(cudaFree(table));
+    CHECK(cudaFree(offs));
+    CHECK(cudaFree(ep));
+    CHECK(cudaFree(out));
+  }
+  /* EP combine: 2 ranks x 2 experts, 4 tokens, hidden 8, fp32.  Rank q's
+     expert rows: row r holds 100 * q + 10 * r + col.  Token t uses rank 0's
+     row t (expert 0) and rank 1's row 3 - t (expert 1); rank 1 owns tokens
+     2..3, so out[i] = (10 * t + col) + (100 + 10 * (3 - t) + col). */
+  {
+    enum { W = 2, E = 2, T = 4, H = 8, ROWS = 4 };
+    float hrows[ROWS * H];
+    int32_t hinv[T * E];
+    float* eo[W];
+    int32_t* inv[W];
+    for (int q = 0; q < W; ++q) {
+      for (int r = 0; r < ROWS; ++r)
+        for (int c = 0; c < H; ++c) hrows[r * H + c] = (float)(100 * q + 10 * r + c);
+      for (int t = 0; t < T; ++t) {
+        hinv[t * E + 0] = q == 0 ? t : -1;
+        hinv[t * E + 1] = q == 1 ? 3 - t : -1;
+      }
+      CHECK(cudaMalloc((void**)&eo[q], sizeof(hrows)));
+      CHECK(cudaMemcpy(eo[q], hrows, sizeof(hrows), cudaMemcpyHostToDevice));
+      CHECK(cudaMalloc((void**)&inv[q], sizeof(hinv)));
+      CHECK(cudaMemcpy(inv[q], hinv, sizeof(hinv), cudaMemcpyHostToDevice));
+    }
+    void **eo_t, **inv_t;
+    int32_t *offs, *ep;
+    float* out;
+    const int32_t h_offs[W] = {0, 2}, h_ep = T;
+    CHECK(cudaMalloc((void**)&eo_t, sizeof(eo)));
+    CHECK(cudaMemcpy(eo_t, eo, sizeof(eo), cudaMemcpyHostToDevice));
+    CHECK(cudaMalloc((void**)&inv_t, sizeof(inv)));
+    CHECK(cudaMemcpy(inv_t, inv, sizeof(inv), cudaMemcpyHostToDevice));
+    CHECK(cudaMalloc((void**)&offs, sizeof(h_offs)));
+    CHECK(cudaMemcpy(offs, h_offs, sizeof(h_offs), cudaMemcpyHostToDevice));
+    CHECK(cudaMalloc((void**)&ep, sizeof(h_ep)));
+    CHECK(cudaMemcpy(ep, &h_ep, sizeof(h_ep), cudaMemcpyHostToDevice));
+    CHECK(cudaMalloc((void**)&out, 2 * H * sizeof(float)));
+    CHECK(moe_unpermute_reduce_scatter((const void* const*)eo_t, MOE_FP32, ROWS,
+                                       (const int32_t* const*)inv_t, E, T, ep, W, 1, offs,
+                                       MOE_FP32, out, MOE_FP32, 2, H, NULL, 0));
+    float ho[2 * H];
+    CHECK(cudaMemcpy(ho, out, sizeof(ho), cudaMemcpyDeviceToHost));
+    for (int i = 0; i < 2 * H; ++i) {
+      const int t = 2 + i / H, c = i % H;
+      const float want = (float)((10 * t + c) + (100 + 10 * (3 - t) + c));
+      if (ho[i] != want) {
+        fprintf(stderr, "EP combine: element %d is %g, want %g\n", i, ho[i], want);
+        return 1;
+      }
+    }
+    for (int q = 0; q < W; ++q) {
+      CHECK(cudaFree(eo[q]));
+      CHECK(cudaFree(inv[q]));
+    }
+    CHECK(cudaFree(eo_t));
+    CHECK(cudaFree(inv_t));
     CHECK(cudaFree(offs));
     CHECK(cudaFree(ep));
     CHECK(cudaFree(out));
