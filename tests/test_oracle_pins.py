@@ -806,3 +806,28 @@ def test_unpermute_single_expert_is_a_copy():
         want = eo[torch.tensor(rows)].to(tdt)
         want = torch.where(want == 0, torch.zeros((), dtype=tdt), want)   # -0 becomes +0
         assert_bits_equal(out, bits(want), f"copy to {tdt}")
+
+
+# --------------------------------------------------- seeded random sweeps
+
+@pytest.mark.parametrize("case", range(8))
+def test_random_shapes_residual_and_router_weight_vs_torch(case):
+    """Random shapes and dtypes: the residual add equals torch's two adds and
+    the router-weight forward torch's fp32 multiply and cast, bit for bit."""
+    rng = np.random.default_rng(100 + case)
+    dts = [torch.bfloat16, torch.float16, torch.float32]
+    odt = {torch.bfloat16: oracle.BF16, torch.float16: oracle.F16, torch.float32: oracle.F32}
+    g = torch.Generator().manual_seed(case)
+    dt = dts[case % 3]
+    shape = (int(rng.integers(1, 50)), int(rng.integers(1, 90)))
+    e, s_, r = ((torch.randn(*shape, generator=g) * 4).to(dt) for _ in range(3))
+    assert_bits_equal(oracle.residual_add(bits(e), bits(s_), bits(r), odt[dt]),
+                      bits(r + (e + s_)) if dt == torch.float32 else
+                      bits((r.float() + (e.float() + s_.float()).to(dt).float()).to(dt)),
+                      "residual", kind="f16" if dt == torch.float16 else "bf16")
+    x_dt, o_dt = dts[int(rng.integers(0, 3))], dts[int(rng.integers(0, 3))]
+    x = (torch.randn(*shape, generator=g) * 3).to(x_dt)
+    p = torch.rand(shape[0], 1, generator=g) + 0.01
+    assert_bits_equal(oracle.router_weight_fwd(bits(x), odt[x_dt], bits(p), odt[o_dt]),
+                      bits((x.float() * p).to(o_dt)), "router weight",
+                      kind="f16" if o_dt == torch.float16 else "bf16")
