@@ -1,5 +1,5 @@
 #!/usr/bin/env python
-"""Throughput of the MoE expert-epilogue pass on B200: achieved HBM GB/s.
+"""Clamped-SwiGLU fwd+bwd throughput on B200 inside the MoE expert-epilogue pass.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -15,21 +15,31 @@ inputs that are resident in HBM before timing starts:
     residual add                    [32768, 7168] bf16; its expert_output's first
                                     16384 rows are the router-weight forward's output
 
-value = algorithmic bytes of all steps on all ranks / max-over-ranks device
-time (CUDA events on the launching stream, barrier + synchronize on both
-sides).  Per-kernel durations come from CUDA events around each launch on
-every 10th timed step (event records between kernels would stop the
-programmatic launch overlap on every step).  Every kernel's working set
-exceeds the 126 MB L2, so no flush is needed between steps.  Multi-GPU runs
-(torchrun) are weak scaling: each rank runs the full step on its own inputs;
-the only collectives are the barrier and the max of the timings.
+The headline (`value`, `ms_per_step`) is the metric the line names: the
+clamped-SwiGLU forward + backward (the two launches run back to back at the
+start of every step) in achieved HBM GB/s = their algorithmic bytes over the
+time between a CUDA event recorded before the forward and one recorded after
+the backward, summed over all K timed steps (one more event between the two
+launches splits the time per kernel); max over ranks.  The whole step is
+reported under `step` (its bytes over the time of the K steps).  The other
+kernels get CUDA events around each launch on every 10th timed step (event
+records between kernels stop programmatic launch overlap).  Every kernel's
+working set exceeds the 126 MB L2, so no flush is needed between steps.
+Multi-GPU runs (torchrun) are weak scaling: each rank runs the full step on its
+own inputs; the data path has no collective, the barrier and the max of the
+timings are the only ones.  With N > 1 the line also carries `collectives`:
+the rank-order reduce-scatter and the EP combine across the N ranks over
+their peer-mapped buffers, timed after the step.
 
 The line also carries `e2e` (the same step through the public API with every
 input copied from pinned host memory and every output copied back inside the
-timed region, pipelined), `next_rows` (the bounded SwiGLU, the fused chain and
-the rank-order reduce-scatter, timed after the step), `clocks`, `roofline` and
-`cpu_baseline` (the CPU oracle, one core and all cores).  `--impl reference`
-times the CPU oracle alone on every host core.
+timed region, pipelined), `configs` (the workload's other configurations:
+the small SwiGLU, the router-weight output-dtype / save_x variants, the
+residual add in three dtypes alone and chained after the router-weight
+forward, the fp32-output unpermute), `next_rows` (the bounded SwiGLU, the
+fused chain, the reduce-scatter and the EP combine, timed after the step),
+`clocks`, `roofline` and `cpu_baseline` (the CPU oracle, one core and all
+cores).  `--impl reference` times the CPU oracle alone on every host core.
 """
 from __future__ import annotations
 
@@ -73,6 +83,8 @@ WORKLOAD_NAME = ("moe_expert_epilogue_pass: clamped SwiGLU fwd+bwd rows=65536 in
                  "router-weight fwd+bwd [16384,7168]; permuted SQRELU/SQRELU_CLAMP/SWIGLU + "
                  "ordered unpermute (8192 tok, top-8 of 64, align 128, width 1536, hidden 4096); "
                  "residual add [32768,7168]; all bf16 with fp32 probs")
+HEADLINE_NAME = ("clamped SwiGLU fwd+bwd: rows=65536 (8192 tokens x top-8), inter=2048, L=10, "
+                 "x bf16 [65536, 4096] ~N(0, 3^2), fp32 top-8 softmax probs, grad_y bf16 ~N(0,1)")
 
 
 def algorithmic_bytes(n_used: int, scale: float = 1.0) -> dict:
@@ -121,8 +133,11 @@ GROUPS = {  # kernel -> the input group it needs
     "act_sqrelu": "act", "act_sqrelu_clamp": "act", "act_swiglu": "act",
     "unpermute": "unpermute", "residual_add": "residual",
 }
-ORDER = ["swiglu_fwd", "router_weight_fwd", "act_sqrelu", "act_sqrelu_clamp", "act_swiglu",
-         "unpermute", "residual_add", "router_weight_bwd", "swiglu_bwd"]
+# The clamped SwiGLU's forward and backward open every step back to back: the
+# headline brackets the two with one event pair.
+ORDER = ["swiglu_fwd", "swiglu_bwd", "router_weight_fwd", "act_sqrelu", "act_sqrelu_clamp",
+         "act_swiglu", "unpermute", "residual_add", "router_weight_bwd"]
+HEAD = ("swiglu_fwd", "swiglu_bwd")
 
 
 class Batch:
@@ -264,7 +279,8 @@ def measure_next_rows(device, seed, reps, peak, scale=1.0, only=None):
     if only in (None, "ordered_reduce_scatter_v"):
         out.update(_measure_reduce_scatter(device, seed, reps, peak, T, H))
     if only in (None, "unpermute_reduce_scatter"):
-        out.update(_measure_ep_combine(device, seed, reps, peak, T, K, E, A, H))
+        out.update(_measure_ep_combine(device, seed, reps, peak, T, K, E, A, H,
+                                       long_tokens=8192 if scale == 1.0 else None))
     return out
 
 
@@ -281,7 +297,8 @@ def _graph_time(fn, reps, device):
     return ms
 
 
-def _measure_ep_combine(device, seed, reps, peak, T, K, E, A, H, world=RS_WORLD):
+def _measure_ep_combine(device, seed, reps, peak, T, K, E, A, H, world=RS_WORLD,
+                        long_tokens=8192):
     """EP combine with every rank's expert rows on this GPU: the fused kernel
     (one launch per rank) against the pages' two steps with the library's own
     kernels (each rank's unpermute into a partial block, then one
@@ -312,13 +329,37 @@ def _measure_ep_combine(device, seed, reps, peak, T, K, E, A, H, world=RS_WORLD)
     nb_f = live * H * 2 + world * T * (E // world) * 4 + T * H * 2
     nb_2 = (live * H * 2 + world * T * (E // world) * 4 + world * T * H * 2) \
         + (world * T * H * 2 + T * H * 2)
-    return {"unpermute_reduce_scatter": {
+    res = {
         "shape": f"{world} ranks x {E // world} experts, {T} tokens top-{K}, hidden {H}, bf16, "
                  f"all ranks' expert rows on one GPU, one launch per rank",
         "us": round(ms_f * 1e3, 2), "bytes": nb_f, "gbs": round(nb_f / ms_f / 1e6, 1),
         "frac": round(nb_f / ms_f / 1e6 / peak, 4),
         "two_step_us": round(ms_2 * 1e3, 2), "two_step_bytes": nb_2,
-        "speedup_vs_two_step": round(ms_2 / ms_f, 3)}}
+        "speedup_vs_two_step": round(ms_2 / ms_f, 3)}
+    del case, eo_t, inv_t, outs, blocks, blk_t
+    torch.cuda.empty_cache()
+    if long_tokens:                       # longer launches: long_tokens tokens a rank
+        TL = long_tokens * world
+        case = inputs.ep_combine_inputs(world, TL, K, E // world, A, H, seed=seed + 10,
+                                        device=device)
+        eo_t = ops.pointer_table(case.expert_outputs)
+        inv_t = ops.pointer_table(case.inverse_maps)
+        ep = torch.tensor([TL], dtype=torch.int32, device=device)
+        outs = [torch.empty(c, H, dtype=torch.bfloat16, device=device) for c in case.counts]
+
+        def fused_long():
+            for r in range(world):
+                ops.unpermute_reduce_scatter(eo_t, torch.bfloat16, case.max_rows, inv_t,
+                                             E // world, TL, ep, r, case.rank_token_offset, H,
+                                             out=outs[r])
+        ms = _graph_time(fused_long, max(3, reps // 4), device)
+        nb = TL * K * H * 2 + world * TL * (E // world) * 4 + TL * H * 2
+        res["long"] = {"shape": f"{TL} tokens ({long_tokens} a rank), otherwise as above",
+                       "us": round(ms * 1e3, 2), "bytes": nb, "gbs": round(nb / ms / 1e6, 1),
+                       "frac": round(nb / ms / 1e6 / peak, 4)}
+        del case, eo_t, inv_t, outs
+        torch.cuda.empty_cache()
+    return {"unpermute_reduce_scatter": res}
 
 
 def _measure_reduce_scatter(device, seed, reps, peak, T, H, world=RS_WORLD):
@@ -394,6 +435,289 @@ def _measure_fused(device, seed, reps, peak, T, K, E, A, H):
         "chained_three_launches_us": round(ms_c * 1e3, 2), "chained_bytes": nb_c,
         "speedup_vs_chained": round(ms_c / ms_f, 3)}
     return out
+
+
+# ---------------------------------------------------------------- configurations
+
+CONFIG_ROWS = ("swiglu_small", "router_weight", "residual_add", "unpermute_fp32_out")
+L2_FLUSH_BYTES = 256 << 20   # twice the 126 MB L2
+
+
+def _entry(ms, nbytes, peak, **extra):
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return dict(us=round(ms * 1e3, 2), bytes=nbytes, gbs=round(gbs, 1),
+                frac=round(gbs / peak, 4), **extra)
+
+
+def measure_configs(device, seed, reps, peak, only=None):
+    """The workload's configurations the step does not run, each timed alone
+    after the step (outside its timed region): the small SwiGLU (latency-bound,
+    L2 flushed before every pair), the router-weight multiply with fp32 output
+    and with and without saved x, the residual add in bf16 / fp16 / fp32 alone
+    and chained after the router-weight forward of the same output dtype, and
+    the unpermute into fp32.  Inputs larger than L2 except the small SwiGLU."""
+    out = {}
+    if only in (None, "swiglu_small"):
+        out["swiglu_small"] = _measure_swiglu_small(device, seed, max(reps, 50), peak)
+    if only in (None, "router_weight"):
+        out["router_weight"] = _measure_router_variants(device, seed, reps, peak)
+    if only in (None, "residual_add"):
+        out["residual_add"] = _measure_residual_variants(device, seed, reps, peak)
+    if only in (None, "unpermute_fp32_out"):
+        out["unpermute_fp32_out"] = _measure_unpermute_fp32(device, seed, reps, peak)
+    torch.cuda.empty_cache()
+    return out
+
+
+def _measure_swiglu_small(device, seed, reps, peak):
+    """rows 256, inter 512 (x ~N(0, 2^2), probs ~U(0,1)), L = 7 and inf: per
+    launch with the L2 flushed before every fwd/bwd pair (cold), and replayed
+    as a CUDA graph with the 1 MB working set in L2 (hot)."""
+    from moe_expert_epilogue_b200 import inputs, ops
+    R, I = 256, 512
+    d = inputs.swiglu_inputs(R, I, sigma=2.0, seed=seed, device=device)
+    x, p, gy = d["x"], d["probs"], d["grad_y"]
+    y, gx = torch.empty(R, I, dtype=torch.bfloat16, device=device), torch.empty_like(x)
+    gp = torch.empty(R, 1, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    nb_f, nb_b = R * (6 * I + 4), R * (10 * I + 8)
+    res = {"shape": f"rows {R}, inter {I}, bf16; latency-bound (the working set fits in L2)"}
+    for L in (7.0, float("inf")):
+        fwd = lambda: ops.swiglu_clamped_fwd(x, p, L, out=y)  # noqa: E731
+        bwd = lambda: ops.swiglu_clamped_bwd(x, p, gy, L, grad_x=gx, grad_probs=gp)  # noqa: E731
+        for _ in range(3):
+            fwd()
+            bwd()
+        evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(reps)]
+        for e in evs:
+            flush.zero_()
+            e[0].record()
+            fwd()
+            e[1].record()
+            bwd()
+            e[2].record()
+        torch.cuda.synchronize(device)
+        tf = sorted(e[0].elapsed_time(e[1]) for e in evs)[reps // 2]
+        tb = sorted(e[1].elapsed_time(e[2]) for e in evs)[reps // 2]
+        hot_f = _graph_time(fwd, reps, device)      # one launch is shorter than its host call
+        hot_b = _graph_time(bwd, reps, device)
+        key = "L7" if L == 7.0 else "Linf"
+        res[key] = {"fwd_cold": _entry(tf, nb_f, peak, rows_per_s=R / (tf * 1e-3)),
+                    "bwd_cold": _entry(tb, nb_b, peak, rows_per_s=R / (tb * 1e-3)),
+                    "fwd_hot_us": round(hot_f * 1e3, 2), "bwd_hot_us": round(hot_b * 1e3, 2),
+                    "timing": f"median of {reps} flushed launches; hot = mean of {reps} "
+                              "graph replays of one launch (working set in L2)"}
+    return res
+
+
+def _measure_router_variants(device, seed, reps, peak):
+    """[16384, 7168] bf16 x, U(0.01, 1) probs: the forward into bf16 and fp32,
+    the backward from a bf16 and an fp32 gradient, with x saved (grad_probs
+    computed) and without (x not read)."""
+    from moe_expert_epilogue_b200 import inputs, ops
+    Rr, H = ROUTER["rows"], ROUTER["hidden"]
+    d = inputs.router_weight_inputs(Rr, H, seed=seed + 1, device=device)
+    x, p, g16 = d["x"], d["probs"], d["grad_out"]
+    g32 = g16.float()
+    n = Rr * H
+    o16 = torch.empty(Rr, H, dtype=torch.bfloat16, device=device)
+    o32 = torch.empty(Rr, H, dtype=torch.float32, device=device)
+    gx = torch.empty(Rr, H, dtype=torch.bfloat16, device=device)
+    gp = torch.empty(Rr, 1, device=device)
+    res = {"shape": f"[{Rr}, {H}] bf16 x, fp32 probs"}
+    runs = {
+        "fwd_out_bf16": (lambda: ops.router_weight_mul_fwd(x, p, out=o16), n * 4 + Rr * 4),
+        "fwd_out_fp32": (lambda: ops.router_weight_mul_fwd(x, p, out=o32), n * 6 + Rr * 4),
+        "bwd_g_bf16_save_x": (lambda: ops.router_weight_mul_bwd(g16, x, p, grad_x=gx,
+                                                                grad_probs=gp), n * 6 + Rr * 8),
+        "bwd_g_bf16_no_x": (lambda: ops.router_weight_mul_bwd(g16, None, p, torch.bfloat16,
+                                                              grad_x=gx), n * 4 + Rr * 4),
+        "bwd_g_fp32_save_x": (lambda: ops.router_weight_mul_bwd(g32, x, p, grad_x=gx,
+                                                                grad_probs=gp), n * 8 + Rr * 8),
+        "bwd_g_fp32_no_x": (lambda: ops.router_weight_mul_bwd(g32, None, p, torch.bfloat16,
+                                                              grad_x=gx), n * 6 + Rr * 4),
+    }
+    for name, (fn, nb) in runs.items():
+        ms = time_launches(fn, reps, device)
+        res[name] = _entry(ms, nb, peak, rows_per_s=Rr / (ms * 1e-3))
+    return res
+
+
+def _measure_residual_variants(device, seed, reps, peak):
+    """[32768, 7168] N(0,1) in bf16, fp16 and fp32: the residual add alone, and
+    chained after the router-weight forward that produces its expert output
+    (bf16 x of the same shape, U(0.01, 1) probs, output in the add's dtype) on
+    one stream as one epilogue pass."""
+    from moe_expert_epilogue_b200 import inputs, ops
+    R, H = RESIDUAL["rows"], RESIDUAL["hidden"]
+    n = R * H
+    rw = inputs.router_weight_inputs(R, H, seed=seed + 6, device=device)
+    x, p = rw["x"], rw["probs"]
+    del rw
+    res = {"shape": f"[{R}, {H}]"}
+    for dt, name in ((torch.bfloat16, "bf16"), (torch.float16, "fp16"), (torch.float32, "fp32")):
+        t = inputs.residual_inputs((R, H), dt, seed=seed + 6, device=device)
+        e, s, r = t["expert_output"], t["shared_expert_output"], t["residual"]
+        o = torch.empty_like(r)
+        es = o.element_size()
+        ms = time_launches(lambda: ops.residual_add(e, s, r, out=o), reps, device)
+        res[name] = _entry(ms, 4 * n * es, peak, rows_per_s=R / (ms * 1e-3))
+
+        def chain():
+            ops.router_weight_mul_fwd(x, p, out=e)
+            ops.residual_add(e, s, r, out=o)
+        ms = time_launches(chain, reps, device)
+        nb = (n * 2 + n * es + R * 4) + 4 * n * es
+        res[name + "_chained"] = _entry(ms, nb, peak, rows_per_s=R / (ms * 1e-3))
+        del t, e, s, r, o
+        torch.cuda.empty_cache()
+    return res
+
+
+def _measure_unpermute_fp32(device, seed, reps, peak):
+    """The fixed-order unpermute of the step's routing (8192 tokens, top-8 of
+    64, hidden 4096, bf16 expert rows) into an fp32 output."""
+    from moe_expert_epilogue_b200 import inputs, ops
+    P = PERMUTED
+    rt = inputs.routing(P["tokens"], P["top_k"], P["experts"], P["align"], seed=seed + 2,
+                        device=device)
+    eo = inputs.expert_output_input(rt, P["hidden"], seed=seed + 5, device=device)
+    valid = torch.tensor([rt.tokens], dtype=torch.int32, device=device)
+    o = torch.empty(rt.tokens, P["hidden"], dtype=torch.float32, device=device)
+    ms = time_launches(lambda: ops.unpermute_ordered(eo, rt.inverse_map, valid, o), reps, device)
+    live = rt.tokens * rt.top_k
+    nb = live * P["hidden"] * 2 + rt.tokens * P["experts"] * 4 + rt.tokens * P["hidden"] * 4
+    return _entry(ms, nb, peak, rows_per_s=rt.tokens / (ms * 1e-3),
+                  shape=f"{rt.tokens} tokens x top-{rt.top_k} of {P['experts']}, hidden "
+                        f"{P['hidden']}, bf16 -> fp32")
+
+
+# ---------------------------------------------------------------- collectives (N > 1)
+
+PEER_GBS = 770.0   # measured peer copy on this node type, per direction per GPU
+
+
+class _Clock:
+    """CUDA events on the current stream (host clock on a CPU process group)."""
+
+    def __init__(self, device):
+        self.cuda = device.type == "cuda"
+        self.device = device
+
+    def mark(self):
+        if self.cuda:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            return e
+        return time.perf_counter()
+
+    def ms(self, a, b):
+        if self.cuda:
+            torch.cuda.synchronize(self.device)
+            return a.elapsed_time(b)
+        return (b - a) * 1e3
+
+
+def measure_collectives(device, seed, reps, tokens=8192, hidden=4096, top_k=8,
+                        experts_per_rank=8, backend=None, return_outputs=False):
+    """The exchange steps across the ranks of the process group (one per GPU),
+    timed after the step: the rank-order reduce-scatter (every rank's block of
+    bf16 partials for all `tokens` token rows in a symmetric buffer) and the EP
+    combine (every rank's expert rows and inverse map in two symmetric
+    buffers), both through `symmetric` -- peer buffers read over NVLink with
+    plain loads.  Per collective: the kernel alone (CUDA events around the
+    launch, between the two stream barriers; max over ranks) and the whole
+    call (barriers included); NVLink bytes are the rows this rank reads from
+    its peers.  `backend` replaces the CUDA IPC mapping (CPU tests)."""
+    import torch.distributed as dist
+    from moe_expert_epilogue_b200 import inputs, symmetric
+    rank, world = dist.get_rank(), dist.get_world_size()
+    clock = _Clock(device)
+    out, outputs = {"world": world}, {}
+    peak_hbm, _ = hbm_peak()
+    dt, H = torch.bfloat16, hidden
+
+    def run(call):
+        """call(hooks) runs one collective; hooks = (before, after) run around
+        its launch.  Returns the mean kernel and whole-call ms, max over ranks."""
+        for _ in range(2):
+            call(None)
+        kern, whole = [], []
+        for _ in range(reps):
+            marks = []
+            hook = lambda: marks.append(clock.mark())  # noqa: E731
+            a = clock.mark()
+            call((hook, hook))
+            b = clock.mark()
+            kern.append(clock.ms(marks[0], marks[1]))
+            whole.append(clock.ms(a, b))
+        return (max_over_ranks(sum(kern) / reps, device),
+                max_over_ranks(sum(whole) / reps, device))
+
+    def entry(k_ms, w_ms, local_bytes, remote_bytes, **extra):
+        t_link = remote_bytes / (PEER_GBS * 1e9) * 1e3
+        t_hbm = local_bytes / (peak_hbm * 1e9) * 1e3
+        return dict(kernel_us=round(k_ms * 1e3, 2), call_us=round(w_ms * 1e3, 2),
+                    bytes_read_written=local_bytes, nvlink_bytes=remote_bytes,
+                    nvlink_gbs=round(remote_bytes / (k_ms * 1e-3) / 1e9, 1),
+                    frac=round(max(t_link, t_hbm) / k_ms, 4),
+                    roofline=f"max(NVLink bytes / {PEER_GBS:g} GB/s measured peer copy, "
+                             f"bytes / {peak_hbm:g} GB/s HBM) / kernel time", **extra)
+
+    # rank-order reduce-scatter
+    case = inputs.reduce_scatter_inputs(world, tokens, H, seed=seed + 8, device=device)
+    cap, mine = tokens, case.counts[rank]
+    symm = symmetric.SymmetricBuffer(cap * H * 2, device=device, backend=backend)
+    symm.view(dt, (cap, H)).copy_(case.buffers[rank])
+    offs, ep = case.rank_token_offset, torch.tensor([case.ep_tokens], dtype=torch.int32,
+                                                    device=device)
+    rs_out = torch.empty(mine, H, dtype=dt, device=device)
+    del case
+
+    k, w = run(lambda hooks: symmetric.ordered_reduce_scatter_v(
+        rs_out, symm, offs, ep, cap, H, dt, launch_hooks=hooks))
+    out["ordered_reduce_scatter_v"] = entry(
+        k, w, mine * H * 2 * (world + 1), mine * H * 2 * (world - 1),
+        shape=f"{world} ranks, {tokens} token rows x hidden {H} bf16 partials per rank, "
+              f"{mine} rows on this rank")
+    if return_outputs:
+        outputs["ordered_reduce_scatter_v"] = rs_out.clone()
+    symm.close()
+    del rs_out
+
+    # EP combine
+    ec = inputs.ep_combine_inputs(world, tokens, top_k, experts_per_rank, 128, H,
+                                  seed=seed + 9, device=device)
+    mine, first = ec.counts[rank], int(ec.rank_token_offset[rank])
+    experts = symmetric.SymmetricBuffer(ec.max_rows * H * 2, device=device, backend=backend)
+    maps = symmetric.SymmetricBuffer(tokens * experts_per_rank * 4, device=device,
+                                     backend=backend)
+    experts.view(dt, (ec.max_rows, H)).copy_(ec.expert_outputs[rank])
+    maps.view(torch.int32, (tokens, experts_per_rank)).copy_(ec.inverse_maps[rank])
+    rows_from = [int((m[first:first + mine] >= 0).sum()) for m in ec.inverse_maps]
+    remote_rows = sum(r for q, r in enumerate(rows_from) if q != rank)
+    ep_t = torch.tensor([tokens], dtype=torch.int32, device=device)
+    offs = ec.rank_token_offset
+    ec_out = torch.empty(mine, H, dtype=dt, device=device)
+    max_rows = ec.max_rows
+    del ec
+
+    k, w = run(lambda hooks: symmetric.unpermute_reduce_scatter(
+        ec_out, experts, maps, dt, max_rows, H, experts_per_rank, tokens, offs, ep_t,
+        launch_hooks=hooks))
+    meta = mine * experts_per_rank * 4
+    out["unpermute_reduce_scatter"] = entry(
+        k, w, sum(rows_from) * H * 2 + world * meta + mine * H * 2,
+        remote_rows * H * 2 + (world - 1) * meta,
+        shape=f"{world} ranks x {experts_per_rank} experts, {tokens} tokens top-{top_k}, "
+              f"hidden {H} bf16, {mine} tokens on this rank")
+    if return_outputs:
+        outputs["unpermute_reduce_scatter"] = ec_out.clone()
+    experts.close()
+    maps.close()
+    if device.type != "cuda":
+        out["note"] = "CPU process group: protocol check only, times are not GPU times"
+    return (out, outputs) if return_outputs else out
 
 
 # ---------------------------------------------------------------- distributed
@@ -528,6 +852,19 @@ def ncu_traffic(kernel: str):
 
 # ---------------------------------------------------------------- our arm
 
+def _kernel_stats(times_ms, nbytes, rows, peak):
+    """Mean / median of one kernel's event durations and its GB/s."""
+    times = sorted(times_ms)
+    avg_ms = sum(times) / len(times)
+    gbs = nbytes / (avg_ms * 1e-3) / 1e9
+    st = {"us": round(avg_ms * 1e3, 2), "median_us": round(times[len(times) // 2] * 1e3, 2),
+          "bytes": nbytes, "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+          "launches_timed": len(times), "share": None}
+    if rows:
+        st["rows_per_s"] = rows / (avg_ms * 1e-3)
+    return st
+
+
 def run_ours(args):
     from moe_expert_epilogue_b200 import build as mbuild
     rank, local_rank, world = dist_env()
@@ -545,17 +882,21 @@ def run_ours(args):
         barrier(device)
 
     only = set(args.kernel.split(",")) if args.kernel else None
-    if only and len(only) == 1 and next(iter(only)) in NEXT_ROWS:
-        # a next-row op alone (profiling captures): warm-ups, then --steps launches
+    if only and len(only) == 1 and next(iter(only)) in NEXT_ROWS + CONFIG_ROWS:
+        # a next-row op or a configuration alone (profiling captures)
         peak, _ = hbm_peak()
-        res = measure_next_rows(device, 1000 * rank, args.steps, peak, args.scale,
-                                only=next(iter(only)))
+        name = next(iter(only))
+        if name in NEXT_ROWS:
+            res = measure_next_rows(device, 1000 * rank, args.steps, peak, args.scale, only=name)
+        else:
+            res = measure_configs(device, 1000 * rank, args.steps, peak, only=name)
         if rank == 0:
             print(json.dumps({"kernel": args.kernel, "scale": args.scale, "result": res}),
                   flush=True)
         return
     if only and not only <= set(ORDER):
-        raise SystemExit(f"unknown --kernel {args.kernel}; choose from {ORDER + list(NEXT_ROWS)}")
+        raise SystemExit(f"unknown --kernel {args.kernel}; choose from "
+                         f"{ORDER + list(NEXT_ROWS) + list(CONFIG_ROWS)}")
     batch = Batch(device, seed=1000 * rank, scale=args.scale, kernels=only)
     kernels = batch.kernels()
     nbytes = algorithmic_bytes(batch.rt.n_used, args.scale)
@@ -563,6 +904,7 @@ def run_ours(args):
     rows = rows_per_launch(args.scale)
     bytes_per_step = sum(nbytes.values())
     stream = torch.cuda.current_stream(device)
+    head = all(h in nbytes for h in HEAD)
 
     for _ in range(args.warmup):
         for _, fn in kernels:
@@ -572,99 +914,142 @@ def run_ours(args):
     K = args.steps
     every = max(1, args.event_every)
     probed = [k for k in range(K) if k % every == every - 1] or [K - 1]
-    ev = {name: {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for k in probed} for name, _ in kernels}
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    # the SwiGLU pair: events before the forward, between the two, after the backward
+    hev = [(mk(), mk(), mk()) for _ in range(K)] if head else None
+    ev = {name: {k: (mk(), mk()) for k in probed} for name, _ in kernels if name not in HEAD
+          or not head}
+    t_start, t_end = mk(), mk()
     sampler = ClockSampler(device.index) if not args.no_clocks else contextlib.nullcontext()
     with sampler:
         barrier(device)
         torch.cuda.synchronize(device)
         t_start.record(stream)
         for k in range(K):
-            if k in probed:                # per-kernel events on every `every`-th step
-                for name, fn in kernels:
+            probe = k in probed
+            for name, fn in kernels:
+                if head and name == HEAD[0]:
+                    hev[k][0].record(stream)
+                    fn()
+                    hev[k][1].record(stream)
+                elif head and name == HEAD[1]:
+                    fn()
+                    hev[k][2].record(stream)
+                elif probe:
                     ev[name][k][0].record(stream)
                     fn()
                     ev[name][k][1].record(stream)
-            else:
-                for _, fn in kernels:
+                else:
                     fn()
         t_end.record(stream)
         torch.cuda.synchronize(device)
         barrier(device)
-    elapsed_ms = t_start.elapsed_time(t_end)
-    max_ms = max_over_ranks(elapsed_ms, device)
+    step_ms = t_start.elapsed_time(t_end)
+    max_step_ms = max_over_ranks(step_ms, device)
     clocks = sampler.summary() if not args.no_clocks else None
 
     per_kernel = {}
     peak, peak_kind = hbm_peak()
     for name, _ in kernels:
-        times = sorted(a.elapsed_time(b) for a, b in ev[name].values())
-        avg_ms = sum(times) / len(times)
-        gbs = nbytes[name] / (avg_ms * 1e-3) / 1e9
-        per_kernel[name] = {"us": round(avg_ms * 1e3, 2), "median_us": round(times[len(times) // 2] * 1e3, 2),
-                            "bytes": nbytes[name], "gbs": round(gbs, 1),
-                            "frac": round(gbs / peak, 4),
-                            "share": None}
-        if rows[name]:
-            per_kernel[name]["rows_per_s"] = rows[name] / (avg_ms * 1e-3)
+        if head and name in HEAD:
+            i = HEAD.index(name)
+            times = [e[i].elapsed_time(e[i + 1]) for e in hev]
+        else:
+            times = [a.elapsed_time(b) for a, b in ev[name].values()]
+        per_kernel[name] = _kernel_stats(times, nbytes[name], rows[name], peak)
     total_kernel_ms = sum(v["us"] for v in per_kernel.values())
     for v in per_kernel.values():
         v["share"] = round(v["us"] / total_kernel_ms, 4)
-    dominant = max(per_kernel, key=lambda n: per_kernel[n]["us"])
-    d = per_kernel[dominant]
 
-    e2e = None
+    # the headline: the SwiGLU pair over all K steps (else, for a --kernel
+    # subset without it, the selected kernels' whole steps)
+    if head:
+        head_bytes = nbytes[HEAD[0]] + nbytes[HEAD[1]]
+        head_ms = sum(e[0].elapsed_time(e[2]) for e in hev)
+    else:
+        head_bytes, head_ms = bytes_per_step, step_ms
+    max_head_ms = max_over_ranks(head_ms, device)
+    value = aggregate_value(head_bytes, K, world, max_head_ms * 1e-3)
+    dom_set = HEAD if head else list(per_kernel)
+    dominant = max(dom_set, key=lambda n: per_kernel[n]["us"])
+    d = per_kernel[dominant]
+    step_dom = max(per_kernel, key=lambda n: per_kernel[n]["us"])
+    sd = per_kernel[step_dom]
+    sw = None
+    if head:
+        us = max_head_ms * 1e3 / K
+        sw = {"us_per_step": round(us, 2), "bytes": head_bytes,
+              "gbs": round(head_bytes / (us * 1e-6) / 1e9, 1),
+              "frac": round(head_bytes / (us * 1e-6) / 1e9 / peak, 4),
+              "rows_per_s": rows[HEAD[0]] / (us * 1e-6),
+              "fwd_frac": per_kernel[HEAD[0]]["frac"], "bwd_frac": per_kernel[HEAD[1]]["frac"],
+              "steps_timed": K}
+
+    e2e = e2e_step = None
     if not args.no_e2e and not args.kernel:
-        e2e = run_e2e(batch, nbytes, args, device, 1000 * rank)
+        e2e_step = run_e2e(args, device, 1000 * rank, first=batch)
+        if head:
+            e2e = run_e2e(args, device, 1000 * rank + 11, names=HEAD)
     n_used, n_kernels = batch.rt.n_used, len(kernels)
-    next_rows = None
-    if not args.kernel and not args.no_next_rows:
+    next_rows = configs = collectives = None
+    if not args.kernel:
         del batch, kernels
         torch.cuda.empty_cache()
-        next_rows = measure_next_rows(device, 1000 * rank, 20, peak)
+        if not args.no_configs:
+            configs = measure_configs(device, 1000 * rank, 20, peak)
+        if not args.no_next_rows:
+            next_rows = measure_next_rows(device, 1000 * rank, 20, peak)
+        if world > 1 and not args.no_collectives:
+            collectives = measure_collectives(device, 1000, 20)
 
-    sw = None
-    if "swiglu_fwd" in per_kernel and "swiglu_bwd" in per_kernel:
-        sw_bytes = nbytes["swiglu_fwd"] + nbytes["swiglu_bwd"]
-        sw_us = per_kernel["swiglu_fwd"]["us"] + per_kernel["swiglu_bwd"]["us"]
-        sw_gbs = sw_bytes / (sw_us * 1e-6) / 1e9
-        sw = {"gbs": round(sw_gbs, 1), "frac": round(sw_gbs / peak, 4),
-              "rows_per_s": rows["swiglu_fwd"] / (sw_us * 1e-6),
-              "fwd_frac": per_kernel["swiglu_fwd"]["frac"],
-              "bwd_frac": per_kernel["swiglu_bwd"]["frac"]}
-    workload = WORKLOAD_NAME if not args.kernel and args.scale == 1.0 else \
-        f"{args.kernel or 'all'} at scale {args.scale:g} of: {WORKLOAD_NAME}"
+    if args.kernel or args.scale != 1.0:
+        workload = f"{args.kernel or 'all'} at scale {args.scale:g} of: {WORKLOAD_NAME}"
+    else:
+        workload = HEADLINE_NAME
     line = {
         "metric": METRIC,
-        "value": round(aggregate_value(bytes_per_step, K, world, max_ms * 1e-3), 1),
+        "value": round(value, 1),
         "unit": "GB/s",
         "n_gpus": world,
         "steps": K,
         "warmup": args.warmup,
-        "ms_per_step": round(max_ms / K, 4),
+        "ms_per_step": round(max_head_ms / K, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": workload, "bytes_per_step": bytes_per_step,
+        "config": {"workload": workload, "bytes_per_step": head_bytes,
+                   "timed_in": "every step of the pass: " + WORKLOAD_NAME,
                    "l2": "no flush: every kernel streams > 126 MB (inputs larger than L2)",
                    "parallelism": f"weak: {world} independent replica(s), one per GPU",
-                   "per_kernel_events": f"on {len(probed)} of the {K} timed steps (every "
-                                        f"{every}th); the other steps run without event records",
+                   "per_kernel_events": f"SwiGLU fwd / bwd on all {K} timed steps; the other "
+                                        f"kernels on {len(probed)} of them (every {every}th)",
                    "n_used": n_used},
         "swiglu_fwd_bwd": sw,
         "roofline": {"kernel": dominant, "bound": "hbm", "achieved": d["gbs"], "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": d["frac"],
                      "algorithmic_bytes": d["bytes"],
-                     "traffic": ncu_traffic(dominant) if args.scale == 1.0 else None},
+                     "traffic": ncu_traffic(dominant) if args.scale == 1.0 else None,
+                     "region": ({"kernels": list(HEAD), "achieved": sw["gbs"],
+                                 "frac": sw["frac"], "algorithmic_bytes": head_bytes}
+                                if sw else None)},
+        "step": {"ms": round(max_step_ms / K, 4), "bytes": bytes_per_step,
+                 "gbs": round(aggregate_value(bytes_per_step, K, world, max_step_ms * 1e-3), 1),
+                 "frac": round(aggregate_value(bytes_per_step, K, 1, max_step_ms * 1e-3) / peak, 4),
+                 "kernels": n_kernels, "e2e": e2e_step,
+                 "roofline": {"kernel": step_dom, "achieved": sd["gbs"], "frac": sd["frac"],
+                              "algorithmic_bytes": sd["bytes"],
+                              "traffic": ncu_traffic(step_dom) if args.scale == 1.0 else None}},
         "kernels": per_kernel,
         "gpu_launches": K * n_kernels,
         "clocks": clocks,
         "e2e": e2e,
+        "configs": configs,
         "next_rows": next_rows,
     }
+    if collectives is not None:
+        line["collectives"] = collectives
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.kernel:
         line["cpu_baseline"] = cpu_baseline(args.cpu_sample or 0.25, steps=1)
     if rank == 0:
@@ -674,16 +1059,21 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_e2e(batch, nbytes, args, device, seed):
-    """The same step through the public API with inputs in pinned host memory:
-    every step copies all of its inputs host -> device, runs the kernels and
-    copies all of its outputs device -> host, all inside the timed region.
-    Steps are pipelined as a user would drive them: two device buffer sets,
-    a copy-in stream, the compute stream and a copy-out stream, so step k's
-    kernels overlap step k+1's inputs and step k-1's outputs on the host link.
-    Events order every reuse of a buffer set."""
-    sets = [batch, Batch(device, seed=seed + 7, scale=args.scale)]
+def run_e2e(args, device, seed, names=None, first=None):
+    """The step's kernels `names` (default: all) through the public API with
+    inputs in pinned host memory: every step copies all of their inputs host
+    -> device, runs the kernels and copies all of their outputs device -> host,
+    all inside the timed region.  Steps are pipelined as a user would drive
+    them: two device buffer sets (`first`, if given, is one of them), a copy-in
+    stream, the compute stream and a copy-out stream, so step k's kernels
+    overlap step k+1's inputs and step k-1's outputs on the host link.  Events
+    order every reuse of a buffer set."""
+    sets = [first or Batch(device, seed=seed, scale=args.scale, kernels=names),
+            Batch(device, seed=seed + 7, scale=args.scale, kernels=names)]
+    batch = sets[0]
     kernel_sets = [b.kernels() for b in sets]
+    nb = algorithmic_bytes(batch.rt.n_used, args.scale)
+    step_bytes = sum(nb[n] for n, _ in kernel_sets[0])
     host_in = {k: torch.empty_like(getattr(batch, k), device="cpu").pin_memory()
                for k in batch.inputs}
     for k, h in host_in.items():
@@ -733,86 +1123,108 @@ def run_e2e(batch, nbytes, args, device, seed):
     barrier(device)
     ms = max_over_ranks(a.elapsed_time(z), device)
     _, _, world = dist_env()
-    return {"value": round(aggregate_value(sum(nbytes.values()), n, world, ms * 1e-3), 2),
+    return {"value": round(aggregate_value(step_bytes, n, world, ms * 1e-3), 2),
             "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": n, "ms_per_step": round(ms / n, 3),
+            "kernels": [name for name, _ in kernel_sets[0]],
             "pipeline": "2 device buffer sets; copy-in, compute and copy-out streams"}
 
 
 # ---------------------------------------------------------------- CPU oracle
 
-def cpu_sample_workload(frac: float, seed: int = 0):
-    """A bounded sample of the same workload on the host: the first `frac` of
-    the rows (tokens) of every op, same distributions."""
-    import numpy as np  # noqa: F401
+def cpu_sample_workload(frac: float, seed: int = 0, whole_pass: bool = False):
+    """A bounded sample of the same workload on the host, same distributions:
+    the first `frac` of the SwiGLU rows (the headline), or with `whole_pass`
+    the first `frac` of the rows (tokens) of every op of the step."""
     from moe_expert_epilogue_b200 import inputs
     R = max(8, int(SWIGLU["rows"] * frac) // 8 * 8)
+    sw = inputs.swiglu_inputs(R, SWIGLU["inter"], sigma=SWIGLU["sigma"], probs="topk_softmax",
+                              seed=seed)
+    w = dict(R=R, sw=sw, whole_pass=whole_pass)
+    if not whole_pass:
+        return w
     Rr = max(1, int(ROUTER["rows"] * frac))
     T = max(8, int(PERMUTED["tokens"] * frac))
     Rs = max(1, int(RESIDUAL["rows"] * frac))
-    sw = inputs.swiglu_inputs(R, SWIGLU["inter"], sigma=SWIGLU["sigma"], probs="topk_softmax",
-                              seed=seed)
     rw = inputs.router_weight_inputs(Rr, ROUTER["hidden"], seed=seed + 1)
     rt = inputs.routing(T, PERMUTED["top_k"], PERMUTED["experts"], PERMUTED["align"], seed=seed + 2)
     ax = inputs.permuted_activation_input(rt, PERMUTED["width"], swiglu=False, seed=seed + 3)
     ax2 = inputs.permuted_activation_input(rt, PERMUTED["width"], swiglu=True, seed=seed + 4)
     eo = inputs.expert_output_input(rt, PERMUTED["hidden"], seed=seed + 5)
     res = inputs.residual_inputs((Rs, RESIDUAL["hidden"]), torch.bfloat16, seed=seed + 6)
-    return dict(R=R, Rr=Rr, T=T, Rs=Rs, sw=sw, rw=rw, rt=rt, ax=ax, ax2=ax2, eo=eo, res=res)
+    w.update(Rr=Rr, T=T, Rs=Rs, rw=rw, rt=rt, ax=ax, ax2=ax2, eo=eo, res=res)
+    return w
 
 
 def oracle_step(w):
-    """One pass of the oracle over the sampled workload; returns its algorithmic bytes."""
+    """One pass of the oracle over the sampled workload (the SwiGLU fwd + bwd,
+    or every op of the step); returns its algorithmic bytes."""
     import numpy as np
     import oracle
     from moe_expert_epilogue_b200.inputs import bits
     L, I, W, Hu = SWIGLU["limit"], SWIGLU["inter"], PERMUTED["width"], PERMUTED["hidden"]
-    sw, rw, rt, res = w["sw"], w["rw"], w["rt"], w["res"]
+    sw, R = w["sw"], w["R"]
     xb, pb, gb = bits(sw["x"]), bits(sw["probs"]), bits(sw["grad_y"])
     oracle.swiglu_clamped_fwd(xb, pb, L)
-    rxb, rpb, rgb = bits(rw["x"]), bits(rw["probs"]), bits(rw["grad_out"])
-    e = oracle.router_weight_fwd(rxb, oracle.BF16, rpb, oracle.BF16)
-    pm, pr = bits(rt.permutation_map), bits(rt.probs)
-    init = np.zeros((rt.max_rows, W), np.uint16)
-    for act, x in ((oracle.SQRELU, w["ax"]), (oracle.SQRELU_CLAMP, w["ax"]), (oracle.SWIGLU, w["ax2"])):
-        oracle.act_with_probs_permuted(act, bits(x), init, pm, rt.n_used, pr, W, PERMUTED["scale"],
-                                       True)
-    oracle.unpermute_ordered(bits(w["eo"]), oracle.BF16, bits(rt.inverse_map), rt.tokens,
-                             np.zeros((rt.tokens, Hu), np.uint16), oracle.BF16)
-    ee = bits(res["expert_output"]).copy()
-    ee[: min(ee.shape[0], e.shape[0])] = e[: ee.shape[0]]
-    oracle.residual_add(ee, bits(res["shared_expert_output"]), bits(res["residual"]), oracle.BF16)
-    oracle.router_weight_bwd(rgb, oracle.BF16, rxb, oracle.BF16, rpb)
+    nbytes = R * (2 * I * 2 + 4 + I * 2) + R * (2 * I * 2 + I * 2 + 4 + 2 * I * 2 + 4)
+    if w["whole_pass"]:
+        rw, rt, res = w["rw"], w["rt"], w["res"]
+        rxb, rpb, rgb = bits(rw["x"]), bits(rw["probs"]), bits(rw["grad_out"])
+        e = oracle.router_weight_fwd(rxb, oracle.BF16, rpb, oracle.BF16)
+        pm, pr = bits(rt.permutation_map), bits(rt.probs)
+        init = np.zeros((rt.max_rows, W), np.uint16)
+        for act, x in ((oracle.SQRELU, w["ax"]), (oracle.SQRELU_CLAMP, w["ax"]),
+                       (oracle.SWIGLU, w["ax2"])):
+            oracle.act_with_probs_permuted(act, bits(x), init, pm, rt.n_used, pr, W,
+                                           PERMUTED["scale"], True)
+        oracle.unpermute_ordered(bits(w["eo"]), oracle.BF16, bits(rt.inverse_map), rt.tokens,
+                                 np.zeros((rt.tokens, Hu), np.uint16), oracle.BF16)
+        ee = bits(res["expert_output"]).copy()
+        ee[: min(ee.shape[0], e.shape[0])] = e[: ee.shape[0]]
+        oracle.residual_add(ee, bits(res["shared_expert_output"]), bits(res["residual"]),
+                            oracle.BF16)
+        oracle.router_weight_bwd(rgb, oracle.BF16, rxb, oracle.BF16, rpb)
+        live = rt.tokens * rt.top_k
+        Rr, Rs, T = w["Rr"], w["Rs"], w["T"]
+        meta = 4 * rt.n_used + 4 * live
+        nbytes += (Rr * ROUTER["hidden"] * 4 + Rr * 4 + Rr * ROUTER["hidden"] * 6 + Rr * 8
+                   + 2 * (live * W * 2 + rt.n_used * W * 2 + meta)
+                   + (live * 2 * W * 2 + rt.n_used * W * 2 + meta)
+                   + live * Hu * 2 + T * rt.experts * 4 + T * Hu * 2
+                   + 4 * Rs * RESIDUAL["hidden"] * 2)
     oracle.swiglu_clamped_bwd(xb, pb, gb, L)
-    live = rt.tokens * rt.top_k
-    R, Rr, Rs, T = w["R"], w["Rr"], w["Rs"], w["T"]
-    meta = 4 * rt.n_used + 4 * live
-    return (R * (2 * I * 2 + 4 + I * 2) + R * (2 * I * 2 + I * 2 + 4 + 2 * I * 2 + 4)
-            + Rr * ROUTER["hidden"] * 4 + Rr * 4 + Rr * ROUTER["hidden"] * 6 + Rr * 8
-            + 2 * (live * W * 2 + rt.n_used * W * 2 + meta)
-            + (live * 2 * W * 2 + rt.n_used * W * 2 + meta)
-            + live * Hu * 2 + T * rt.experts * 4 + T * Hu * 2
-            + 4 * Rs * RESIDUAL["hidden"] * 2)
+    return nbytes
 
 
-def cpu_baseline(frac, steps=1, all_cores=True):
-    """The oracle on the host: single-threaded on the first `frac` of every
-    op's rows, and (all_cores) the same fraction split over one process per
-    host core."""
-    w = cpu_sample_workload(frac)
+def _time_oracle(frac, steps, whole_pass=False):
+    w = cpu_sample_workload(frac, whole_pass=whole_pass)
     t0 = time.perf_counter()
     b = 0
     for _ in range(steps):
         b += oracle_step(w)
-    dt = time.perf_counter() - t0
+    return b, time.perf_counter() - t0, w
+
+
+def cpu_baseline(frac, steps=1, all_cores=True):
+    """The oracle on the host, on the headline's workload: single-threaded on
+    the first `frac` of the SwiGLU rows, and (all_cores) the same fraction
+    split over one process per host core; `step` is the whole pass on one
+    core (the first `frac` of every op's rows)."""
+    b, dt, w = _time_oracle(frac, steps)
     out = {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
            "seconds": round(dt, 2), "host_cpu": _cpu_model(), "host_nproc": os.cpu_count(),
-           "sample": f"first {frac:g} of the rows/tokens of every op of the step "
-                     f"(swiglu rows {w['R']}, router rows {w['Rr']}, tokens {w['T']}, "
-                     f"residual rows {w['Rs']}); single-threaded C oracle, -O2"}
+           "sample": f"clamped SwiGLU fwd+bwd on the first {w['R']} of the {SWIGLU['rows']} "
+                     f"rows (inter {SWIGLU['inter']}, L {SWIGLU['limit']:g}); single-threaded "
+                     "C oracle, -O2"}
     del w
     if all_cores and (os.cpu_count() or 1) > 1:
         out["all_cores"] = oracle_pool(frac, os.cpu_count(), warmup=1, steps=4 * max(1, steps))
+    b, dt, w = _time_oracle(frac, 1, whole_pass=True)
+    out["step"] = {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": 1,
+                   "seconds": round(dt, 2),
+                   "sample": f"first {frac:g} of the rows/tokens of every op of the step "
+                             f"(swiglu rows {w['R']}, router rows {w['Rr']}, tokens {w['T']}, "
+                             f"residual rows {w['Rs']}); single-threaded C oracle"}
     return out
 
 
@@ -835,7 +1247,7 @@ def _oracle_worker(frac, seed, warmup, steps, barrier_, q):
 
 def oracle_pool(frac_total, n, warmup=1, steps=1):
     """The oracle as it stands on `n` host processes (spawned), each on its own
-    seeded sample of frac_total / n of every op's rows: aggregate GB/s = all
+    seeded sample of frac_total / n of the SwiGLU rows: aggregate GB/s = all
     processes' algorithmic bytes / the slowest process's time."""
     import multiprocessing as mp
     import oracle
@@ -864,8 +1276,8 @@ def oracle_pool(frac_total, n, warmup=1, steps=1):
     return {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": n, "kind": "oracle",
             "seconds": round(dt, 2),
             "sample": f"{n} processes, each its own seeded sample of {frac_total / n:.4g} of the "
-                      f"rows/tokens of every op ({frac_total:g} in total), {steps} timed "
-                      "pass(es) after a warm-up; single-threaded C oracle in each"}
+                      f"SwiGLU rows ({frac_total:g} in total), {steps} timed pass(es) of fwd+bwd "
+                      "after a warm-up; single-threaded C oracle in each"}
 
 
 def _cpu_model():
@@ -879,13 +1291,13 @@ def _cpu_model():
 
 
 def reference_fraction(args, cores=1) -> float:
-    """Row fraction of every op the oracle runs per step in the reference arm
-    (split over `cores` processes): --cpu-sample if given, else sized so that
-    the warm-up and timed steps take about two minutes on a host that needs
-    ~17 s of one core per full step, capped at half the workload (host memory)."""
+    """Fraction of the SwiGLU rows the oracle runs per step in the reference
+    arm (split over `cores` processes): --cpu-sample if given, else sized so
+    that the warm-up and timed steps take about two minutes on a host that
+    needs ~4 s of one core per full fwd + bwd, capped at half the rows."""
     if args.cpu_sample is not None:
         return args.cpu_sample
-    return max(0.005, min(0.5, 120.0 * cores / (17.0 * max(1, args.steps + args.warmup))))
+    return max(0.005, min(0.5, 120.0 * cores / (4.0 * max(1, args.steps + args.warmup))))
 
 
 def run_reference(args):
@@ -903,7 +1315,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(pool["seconds"] / args.steps * 1e3, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD_NAME, "sample_fraction": args.cpu_sample},
+        "config": {"workload": HEADLINE_NAME, "sample_fraction": args.cpu_sample},
         "cpu_baseline": pool,
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -931,6 +1343,10 @@ def main(argv=None):
                          "between kernels stop programmatic launch overlap)")
     ap.add_argument("--no-next-rows", action="store_true",
                     help="skip the separately timed ops beyond the step")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the separately timed configurations beyond the step")
+    ap.add_argument("--no-collectives", action="store_true",
+                    help="with N > 1: skip the cross-rank reduce-scatter and EP combine")
     ap.add_argument("--kernel", default=None,
                     help="comma-separated kernels to run alone (profiling); default: the whole step")
     ap.add_argument("--scale", type=float, default=1.0,

@@ -137,18 +137,25 @@ def stream_barrier(group=None, device=None):
 def ordered_reduce_scatter_v(output: torch.Tensor, symm: SymmetricBuffer,
                              rank_token_offset: torch.Tensor, ep_tokens: torch.Tensor,
                              capacity_rows: int, hidden: int, in_dtype: torch.dtype,
-                             input_byte_offset: int = 0, dev_err=None) -> torch.Tensor:
+                             input_byte_offset: int = 0, dev_err=None,
+                             launch_hooks=None) -> torch.Tensor:
     """Collective over symm.group: this rank's `output` [local_tokens, hidden]
     = the rank-order fp32 sum of its token rows over every rank's block
     ([capacity_rows, hidden] of in_dtype at input_byte_offset in the symmetric
-    buffer), launched on the current stream between two stream barriers."""
+    buffer), launched on the current stream between two stream barriers.
+    `launch_hooks`, a (before, after) pair of callables, runs just around the
+    launch, inside the barriers (e.g. to record timing events)."""
     esize = torch.empty((), dtype=in_dtype).element_size()
     if input_byte_offset + capacity_rows * hidden * esize > symm.nbytes:
         raise ValueError("the input block does not fit in the symmetric buffer")
     stream_barrier(symm.group, symm.device)
+    if launch_hooks:
+        launch_hooks[0]()
     ops.ordered_reduce_scatter_v(symm.table, symm.rank, rank_token_offset, ep_tokens,
                                  capacity_rows, hidden, in_dtype, out=output,
                                  input_byte_offset=input_byte_offset, dev_err=dev_err)
+    if launch_hooks:
+        launch_hooks[1]()
     stream_barrier(symm.group, symm.device)
     return output
 
@@ -158,7 +165,7 @@ def unpermute_reduce_scatter(output: torch.Tensor, experts: SymmetricBuffer,
                              hidden: int, num_local_experts: int, capacity_rows: int,
                              rank_token_offset: torch.Tensor, ep_tokens: torch.Tensor,
                              eo_byte_offset: int = 0, inv_byte_offset: int = 0,
-                             partial_dtype=None, dev_err=None) -> torch.Tensor:
+                             partial_dtype=None, dev_err=None, launch_hooks=None) -> torch.Tensor:
     """Collective over experts.group: the EP combine.  Every rank holds its
     experts' output rows ([max_rows, hidden] of eo_dtype at eo_byte_offset of
     `experts`) and its inverse map over the token rows of all ranks (int32
@@ -166,7 +173,7 @@ def unpermute_reduce_scatter(output: torch.Tensor, experts: SymmetricBuffer,
     this rank's `output` [local_tokens, hidden] gets, per token, every rank's
     expert-order partial sum folded in rank order -- the unpermute and the
     rank-order reduce-scatter in one kernel, launched on the current stream
-    between two stream barriers."""
+    between two stream barriers (`launch_hooks` as for ordered_reduce_scatter_v)."""
     esize = torch.empty((), dtype=eo_dtype).element_size()
     if eo_byte_offset + max_rows * hidden * esize > experts.nbytes or \
             inv_byte_offset + capacity_rows * num_local_experts * 4 > inverse_maps.nbytes:
@@ -174,10 +181,14 @@ def unpermute_reduce_scatter(output: torch.Tensor, experts: SymmetricBuffer,
     if experts.world != inverse_maps.world or experts.rank != inverse_maps.rank:
         raise ValueError("both buffers must span the same group")
     stream_barrier(experts.group, experts.device)
+    if launch_hooks:
+        launch_hooks[0]()
     ops.unpermute_reduce_scatter(experts.table_at(eo_byte_offset), eo_dtype, max_rows,
                                  inverse_maps.table_at(inv_byte_offset), num_local_experts,
                                  capacity_rows, ep_tokens, experts.rank, rank_token_offset,
                                  hidden, out=output, partial_dtype=partial_dtype,
                                  dev_err=dev_err)
+    if launch_hooks:
+        launch_hooks[1]()
     stream_barrier(experts.group, experts.device)
     return output
