@@ -51,20 +51,17 @@ def test_residual_add_in_place_and_unaligned(cuda_device, dtype):
 
 
 @pytest.mark.parametrize("dtype", DTYPES)
-def test_residual_add_full_workload_sampled(cuda_device, dtype):
-    """[32768, 7168], all inputs N(0,1): the full launch, checked on a sample
-    of elements (the op is elementwise)."""
+def test_residual_add_full_workload_whole_tensor(cuda_device, dtype):
+    """[32768, 7168], all inputs N(0,1): the full launch, every element
+    against the oracle."""
     shape = (32768, 7168)
     d = inputs.residual_inputs(shape, dtype, seed=0)
     e, s, r = (d[k].to(cuda_device) for k in ("expert_output", "shared_expert_output", "residual"))
     out = ops.residual_add(e, s, r)
     torch.cuda.synchronize()
-    rng = np.random.default_rng(4)
-    idx = np.unique(np.concatenate([[0, e.numel() - 1], rng.integers(0, e.numel(), 200000)]))
-    ti = torch.from_numpy(idx)
-    ref = oracle.residual_add(*(bits(d[k].reshape(-1)[ti]) for k in
+    ref = oracle.residual_add(*(bits(d[k]) for k in
                                 ("expert_output", "shared_expert_output", "residual")), ODT[dtype])
-    assert_bits_equal(bits(out.reshape(-1).cpu()[ti]), ref, "residual add", kind=_kind(dtype))
+    assert_bits_equal(bits(out), ref, "residual add", kind=_kind(dtype))
     assert_bits_equal(bits(out), bits(r + (e + s)), "whole tensor vs torch", kind=_kind(dtype))
 
 
