@@ -10,6 +10,8 @@
 // 8-element chunks.  The backward with the probability gradient walks rows
 // like the SwiGLU backward: W threads per row, fixed column assignment, fixed
 // reduction tree, no fp32 intermediate ever leaves the registers.
+#include <type_traits>
+
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -65,6 +67,54 @@ scale_rows_vec(const typename DI::T* __restrict__ in, const void* __restrict__ p
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = v[i] * p[k];
         store8<DO>(out + off[k], v);
+      }
+    }
+  }
+}
+
+// A 16-bit input scaled into fp32: units of 4 elements, so that a warp's
+// 8-byte loads cover 256 contiguous bytes and its 16-byte stores 512 (with
+// 8-element units each fp32 store instruction would cover every other 16
+// bytes of a 1 KB span).  U units' loads in flight per thread.
+template <class DI, int U>
+__global__ void __launch_bounds__(kThreads)
+scale_rows_to_f32(const uint16_t* __restrict__ in, const void* __restrict__ probs, int p_dt,
+                  float* __restrict__ out, int64_t rows, int64_t hidden) {
+  pdl_prologue();
+  const int64_t upr = hidden / 4;
+  const int64_t total = rows * upr;
+  const int64_t S = (int64_t)gridDim.x * kThreads;
+  int64_t q = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (q >= total) return;
+  RowCursor cur(q, S, upr);
+  for (; q < total; q += U * S) {
+    uint2 raw[U];
+    float p[U];
+    int64_t off[U];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      if (q + k * S < total) {
+        off[k] = cur.r * hidden + cur.c * 4;
+        asm("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+            : "=r"(raw[k].x), "=r"(raw[k].y)
+            : "l"(in + off[k]));
+        p[k] = load_prob(probs, p_dt, cur.r);
+      }
+      cur.advance();
+    }
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      if (q + k * S < total) {
+        float v[4];
+        if constexpr (std::is_same<DI, BF16>::value) {
+          v[0] = bf16_lo(raw[k].x); v[1] = bf16_hi(raw[k].x);
+          v[2] = bf16_lo(raw[k].y); v[3] = bf16_hi(raw[k].y);
+        } else {
+          v[0] = f16_to_f32((uint16_t)(raw[k].x & 0xffffu)); v[1] = f16_to_f32((uint16_t)(raw[k].x >> 16));
+          v[2] = f16_to_f32((uint16_t)(raw[k].y & 0xffffu)); v[3] = f16_to_f32((uint16_t)(raw[k].y >> 16));
+        }
+        st_stream(out + off[k], make_uint4(__float_as_uint(v[0] * p[k]), __float_as_uint(v[1] * p[k]),
+                                           __float_as_uint(v[2] * p[k]), __float_as_uint(v[3] * p[k])));
       }
     }
   }
@@ -174,6 +224,19 @@ int launch_scale(const void* in, const void* probs, int p_dt, void* out, int64_t
   const auto* i = static_cast<const typename DI::T*>(in);
   auto* o = static_cast<typename DO::T*>(out);
   int grid;
+  if constexpr (DI::kBytes == 2 && DO::kBytes == 4) {
+    if (hidden % 4 == 0 && aligned16(out) && (reinterpret_cast<uintptr_t>(in) & 7u) == 0) {
+      constexpr int U = 4;
+      auto k = scale_rows_to_f32<DI, U>;
+      const int64_t units = rows * (hidden / 4);
+      if (int rc = persistent_grid((const void*)k, 0, (units + kThreads * U - 1) / (kThreads * U),
+                                   &grid))
+        return rc;
+      launch_kernel(k, grid, 0, stream, static_cast<const uint16_t*>(in), probs, p_dt,
+                    static_cast<float*>(out), rows, hidden);
+      return check_launch();
+    }
+  }
   if (hidden % kVec == 0 && aligned16(in) && aligned16(out)) {
     auto k = scale_rows_vec<DI, DO>;
     const int64_t units = rows * (hidden / kVec);

@@ -29,6 +29,30 @@ def test_router_weight_fwd_bitwise(cuda_device, rows, hidden, x_dtype, out_dtype
     assert_bits_equal(bits(out), ref, "fwd", kind="f16" if out_dtype == torch.float16 else "bf16")
 
 
+@pytest.mark.parametrize("x_dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("hidden", [4096, 1004, 12, 7])
+@pytest.mark.parametrize("x_shift,out_shift", [(0, 0), (4, 0), (2, 0), (0, 2)])
+def test_router_weight_fwd_16bit_to_fp32_layouts(cuda_device, x_dtype, hidden, x_shift,
+                                                 out_shift):
+    """A 16-bit input scaled into fp32, with rows of 4-element units (hidden %
+    4 == 0) and without, inputs 8-byte but not 16-byte aligned (x_shift 4),
+    4-byte aligned (2), and an fp32 output off 16-byte alignment: every path
+    gives the oracle's bits."""
+    rows = 37
+    d = inputs.router_weight_inputs(rows, hidden, seed=hidden + x_shift)
+    x = d["x"].to(x_dtype)
+    xbuf = torch.zeros(rows * hidden + x_shift, dtype=x_dtype, device=cuda_device)
+    xd = xbuf[x_shift:].view(rows, hidden)
+    xd.copy_(x.to(cuda_device))
+    obuf = torch.full((rows * hidden + out_shift,), 7.0, device=cuda_device)
+    od = obuf[out_shift:].view(rows, hidden)
+    ops.router_weight_mul_fwd(xd, d["probs"].to(cuda_device), torch.float32, out=od)
+    torch.cuda.synchronize()
+    ref = oracle.router_weight_fwd(bits(x), ODT[x_dtype], bits(d["probs"]), oracle.F32)
+    assert_bits_equal(bits(od), ref, "fwd")
+    assert (obuf[:out_shift] == 7.0).all()
+
+
 @pytest.mark.parametrize("rows,hidden", [(129, 7176), (300, 1001), (1, 8), (3000, 40)])
 @pytest.mark.parametrize("g_dtype", [torch.bfloat16, torch.float32, torch.float16])
 @pytest.mark.parametrize("x_dtype", [torch.bfloat16, torch.float32])
