@@ -95,8 +95,15 @@ enum {
   MOE_DEVERR_COUNT = 1,  /* *n_used / *valid_tokens outside [0, max]: clamped    */
   MOE_DEVERR_MAP = 2,    /* permutation_map entry >= num_probs: row skipped       */
   MOE_DEVERR_INVERSE = 4, /* inverse_map entry >= max_rows: contribution skipped  */
-  MOE_DEVERR_TIMEOUT = 8  /* a kernel's barrier wait gave up after ~1 s (a copy that
-                             never completed); the affected rows were not written  */
+  MOE_DEVERR_TIMEOUT = 8  /* a kernel's barrier wait gave up (~1 s: a shared-memory
+                             copy or a consumer that never completed).  The rows the
+                             waiting warps had not reached were not written.  Before
+                             exiting, a CTA waits (bounded again) for every copy it
+                             issued; if that wait gives up as well, a copy may land in
+                             shared memory after the CTA has exited, where another
+                             kernel's CTA may live.  Treat the bit as fatal for the
+                             results of everything enqueued after the call on the
+                             device: discard them and rebuild the CUDA context.     */
 };
 
 /* Human-readable name of a status code (static storage). */
@@ -108,10 +115,13 @@ MOE_API int moe_last_cuda_error(void);
 /* Library ABI version, currently 1. */
 MOE_API int moe_abi_version(void);
 
-/* Error bits recorded on the current device by kernels that have no dev_err
- * argument (today: the TMA-staged clamped-SwiGLU forward, MOE_DEVERR_TIMEOUT).
- * Synchronous: waits for the device, copies the word into *bits and, if
- * `clear`, resets it.  Returns MOE_OK, MOE_ERR_NULL or MOE_ERR_CUDA. */
+/* Error bits recorded on the current device by calls that were given no
+ * error word of their own (today: the TMA-staged clamped-SwiGLU forward
+ * through moe_swiglu_clamped_fwd, or _ex with dev_err NULL:
+ * MOE_DEVERR_TIMEOUT).  One word per device, shared by every stream and
+ * thread; pass dev_err to moe_swiglu_clamped_fwd_ex to keep a call's bits
+ * apart.  Synchronous: waits for the device, copies the word into *bits and,
+ * if `clear`, resets it.  Returns MOE_OK, MOE_ERR_NULL or MOE_ERR_CUDA. */
 MOE_API int moe_device_errors(int32_t* bits, int clear);
 
 /* ------------------------------------------------------------------------
@@ -130,6 +140,16 @@ MOE_API int moe_device_errors(int32_t* bits, int clear);
 MOE_API int moe_swiglu_clamped_fwd(const void* x, const float* probs, void* y, int64_t rows,
                            int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
                            moe_dtype dt, cudaStream_t stream);
+
+/* moe_swiglu_clamped_fwd with an error word of the caller's: dev_err
+ * (optional int32, device memory, 4-byte aligned) receives MOE_DEVERR_TIMEOUT
+ * if the TMA-staged kernel (bf16 / fp16, contiguous 16-byte aligned rows of
+ * at least 512 columns) gave up a barrier wait; with dev_err NULL the bit
+ * goes to the per-device word of moe_device_errors().  Same computation,
+ * arguments and status codes as moe_swiglu_clamped_fwd. */
+MOE_API int moe_swiglu_clamped_fwd_ex(const void* x, const float* probs, void* y, int64_t rows,
+                                      int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
+                                      moe_dtype dt, int32_t* dev_err, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * Clamped SwiGLU, one-pass backward.
@@ -405,6 +425,30 @@ MOE_API int moe_unpermute_reduce_scatter(const void* const* expert_outputs, moe_
                                          const int32_t* rank_token_offset, moe_dtype partial_dt,
                                          void* out, moe_dtype out_dt, int64_t local_tokens,
                                          int64_t hidden, int32_t* dev_err, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Test hook of the failure path of the bounded waits (no counterpart on the
+ * pages; for tests of the error handling, not for production use).
+ * The TMA-staged clamped-SwiGLU forward on contiguous x [rows, 2*inter] and
+ * y [rows, inter] with `grid` CTAs, except that the copy of row `stall_row`
+ * is never issued and its barrier never arrived on: the consumer of that row
+ * gives up after `wait_cycles` SM cycles, and so does every warp of its CTA
+ * that later waits on it (the producer for a free stage, the other consumers
+ * for rows that were never filled).  The CTA then drains its issued copies
+ * and exits: no copy is left in flight and no wait is unbounded.  *dev_err
+ * receives MOE_DEVERR_TIMEOUT; the other CTAs' rows (r % grid != stall_row %
+ * grid) are written as by moe_swiglu_clamped_fwd, row stall_row is not
+ * written, and the CUDA context stays usable.
+ * dt        MOE_BF16 or MOE_FP16; rows >= 1; inter a multiple of 8, >= 512 and
+ *           small enough for the shared-memory ring (MOE_ERR_SHAPE otherwise)
+ * grid      1 .. min(rows, SM count);  stall_row in [0, rows)
+ * wait_cycles  1000 .. 2^31
+ * x, y      16-byte aligned (MOE_ERR_ALIGN);  dev_err required (MOE_ERR_NULL)
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_test_swiglu_fwd_stalled(const void* x, const float* probs, void* y,
+                                        int64_t rows, int64_t inter, float limit, moe_dtype dt,
+                                        int32_t grid, int64_t stall_row, int64_t wait_cycles,
+                                        int32_t* dev_err, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * Buffers shared between the processes of one node (CUDA IPC): the plumbing

@@ -28,6 +28,8 @@ _P, _I64, _I32, _F, _I = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctype
 # name -> argtypes (every entry point returns int)
 SIGNATURES = {
     "moe_swiglu_clamped_fwd": [_P, _P, _P, _I64, _I64, _I64, _I64, _F, _I, _P],
+    "moe_swiglu_clamped_fwd_ex": [_P, _P, _P, _I64, _I64, _I64, _I64, _F, _I, _P, _P],
+    "moe_test_swiglu_fwd_stalled": [_P, _P, _P, _I64, _I64, _F, _I, _I32, _I64, _I64, _P, _P],
     "moe_swiglu_clamped_bwd": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _F, _I, _P],
     "moe_router_weight_mul_fwd": [_P, _I, _P, _P, _I, _I64, _I64, _P],
     "moe_router_weight_mul_bwd": [_P, _I, _P, _I, _P, _P, _P, _I64, _I64, _P],
@@ -119,6 +121,18 @@ def moe_swiglu_clamped_fwd(x, probs, y, rows, inter, ld_x, ld_y, limit, dt=MOE_B
                            stream=None):
     _call("moe_swiglu_clamped_fwd", ptr(x), ptr(probs), ptr(y), rows, inter, ld_x, ld_y,
           float(limit), dt, stream_handle(stream))
+
+
+def moe_swiglu_clamped_fwd_ex(x, probs, y, rows, inter, ld_x, ld_y, limit, dt=MOE_BF16,
+                              dev_err=None, stream=None):
+    _call("moe_swiglu_clamped_fwd_ex", ptr(x), ptr(probs), ptr(y), rows, inter, ld_x, ld_y,
+          float(limit), dt, ptr(dev_err), stream_handle(stream))
+
+
+def moe_test_swiglu_fwd_stalled(x, probs, y, rows, inter, limit, dt, grid, stall_row,
+                                wait_cycles, dev_err, stream=None):
+    _call("moe_test_swiglu_fwd_stalled", ptr(x), ptr(probs), ptr(y), rows, inter, float(limit),
+          dt, grid, stall_row, wait_cycles, ptr(dev_err), stream_handle(stream))
 
 
 def moe_swiglu_clamped_bwd(x, probs, grad_y, grad_x, grad_probs, rows, inter, ld_x, ld_gy,

@@ -16,6 +16,7 @@
 
 #include "common.cuh"
 #include "launch.cuh"
+#include "tma.cuh"
 
 namespace moe {
 
@@ -26,9 +27,27 @@ thread_local int g_last_cuda_error = 0;
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sms[kMaxDevices];
 
+// Resident CTAs per SM by (kernel, dynamic shared memory, device): the same
+// kernel launched with more shared memory may fit fewer CTAs on an SM.
+struct OccKey {
+  const void* kernel;
+  size_t smem;
+  int device;
+  bool operator==(const OccKey& o) const {
+    return kernel == o.kernel && smem == o.smem && device == o.device;
+  }
+};
+struct OccKeyHash {
+  size_t operator()(const OccKey& k) const {
+    size_t h = std::hash<const void*>()(k.kernel);
+    h ^= std::hash<size_t>()(k.smem) + 0x9e3779b97f4a7c15ull + (h << 6) + (h >> 2);
+    h ^= std::hash<int>()(k.device) + 0x9e3779b97f4a7c15ull + (h << 6) + (h >> 2);
+    return h;
+  }
+};
 std::mutex g_occ_mutex;
-std::unordered_map<const void*, int>& occ_cache() {
-  static std::unordered_map<const void*, int> m;
+std::unordered_map<OccKey, int, OccKeyHash>& occ_cache() {
+  static std::unordered_map<OccKey, int, OccKeyHash> m;
   return m;
 }
 
@@ -87,18 +106,22 @@ int check_launch() {
 int persistent_grid(const void* kernel, size_t smem, int64_t useful_blocks, int* grid) {
   int sms = 0;
   if (int rc = device_sms(&sms)) return rc;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const OccKey key{kernel, smem, dev};
   int per_sm = 0;
   {
     std::lock_guard<std::mutex> lock(g_occ_mutex);
     auto& m = occ_cache();
-    auto it = m.find(kernel);
+    auto it = m.find(key);
     if (it != m.end()) {
       per_sm = it->second;
     } else {
-      cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem);
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem);
       if (e != cudaSuccess) return cuda_fail(e);
       if (per_sm < 1) per_sm = 1;
-      m.emplace(kernel, per_sm);
+      m.emplace(key, per_sm);
     }
   }
   int64_t g = (int64_t)sms * per_sm;
@@ -143,9 +166,9 @@ int moe_last_cuda_error(void) { return g_last_cuda_error; }
 
 int moe_abi_version(void) { return 1; }
 
-int moe_swiglu_clamped_fwd(const void* x, const float* probs, void* y, int64_t rows,
-                           int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
-                           moe_dtype dt, cudaStream_t stream) {
+int moe_swiglu_clamped_fwd_ex(const void* x, const float* probs, void* y, int64_t rows,
+                              int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
+                              moe_dtype dt, int32_t* dev_err, cudaStream_t stream) {
   if (!dtype_ok(dt)) return MOE_ERR_DTYPE;
   if (rows < 0 || inter < 0 || ld_x < 2 * inter || ld_y < inter) return MOE_ERR_SHAPE;
   if (!product_ok(rows, ld_x) || !product_ok(rows, ld_y)) return MOE_ERR_SHAPE;
@@ -153,8 +176,38 @@ int moe_swiglu_clamped_fwd(const void* x, const float* probs, void* y, int64_t r
   if (rows == 0 || inter == 0) return MOE_OK;
   if (!x || !probs || !y) return MOE_ERR_NULL;
   const int64_t es = dtype_size(dt);
-  if (!aligned_to(x, es) || !aligned_to(y, es) || !aligned_to(probs, 4)) return MOE_ERR_ALIGN;
-  return launch_swiglu_clamped_fwd(x, probs, y, rows, inter, ld_x, ld_y, limit, dt, stream);
+  if (!aligned_to(x, es) || !aligned_to(y, es) || !aligned_to(probs, 4) ||
+      !aligned_to(dev_err, 4))
+    return MOE_ERR_ALIGN;
+  return launch_swiglu_clamped_fwd(x, probs, y, rows, inter, ld_x, ld_y, limit, dt, dev_err,
+                                   stream);
+}
+
+int moe_swiglu_clamped_fwd(const void* x, const float* probs, void* y, int64_t rows,
+                           int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
+                           moe_dtype dt, cudaStream_t stream) {
+  return moe_swiglu_clamped_fwd_ex(x, probs, y, rows, inter, ld_x, ld_y, limit, dt, nullptr,
+                                   stream);
+}
+
+int moe_test_swiglu_fwd_stalled(const void* x, const float* probs, void* y, int64_t rows,
+                                int64_t inter, float limit, moe_dtype dt, int32_t grid,
+                                int64_t stall_row, int64_t wait_cycles, int32_t* dev_err,
+                                cudaStream_t stream) {
+  if (dt != MOE_BF16 && dt != MOE_FP16) return MOE_ERR_DTYPE;
+  int sms = 0;
+  if (int rc = device_sm_count(&sms)) return rc;
+  if (rows < 1 || !product_ok(rows, 2 * inter) || !tma_forward_applies(inter, dt) ||
+      grid < 1 || grid > sms || (int64_t)grid > rows || stall_row < 0 || stall_row >= rows ||
+      wait_cycles < 1000 || wait_cycles > tma::kWaitCycles)
+    return MOE_ERR_SHAPE;
+  if (!limit_ok(limit)) return MOE_ERR_LIMIT;
+  if (!x || !probs || !y || !dev_err) return MOE_ERR_NULL;
+  if (!aligned_to(x, 16) || !aligned_to(y, 16) || !aligned_to(probs, 4) ||
+      !aligned_to(dev_err, 4))
+    return MOE_ERR_ALIGN;
+  return launch_swiglu_fwd_stalled(x, probs, y, rows, inter, limit, dt, grid, stall_row,
+                                   (long long)wait_cycles, dev_err, stream);
 }
 
 int moe_swiglu_clamped_bwd(const void* x, const float* probs, const void* grad_y,

@@ -27,8 +27,11 @@
 // the row, it keeps 4 expert rows' loads in flight (8 in the kernel for more
 // than 8 ranks or odd widths) and closes each rank's partial in rank order
 // (ranks without rows contribute +0, as their partial block row would).
+#include <type_traits>
+
 #include "common.cuh"
 #include "launch.cuh"
+#include "tma.cuh"
 
 namespace moe {
 namespace {
@@ -229,8 +232,9 @@ __device__ __forceinline__ void combine_one_group(
 }
 
 // Any number of ranks and any row width / alignment: one unit per lane per
-// item, each unit's sum carried across the groups of 8 ranks.
-template <class DI, class DP, class DO, bool VEC, bool ALIGNED>
+// item, each unit's sum carried across the groups of 8 ranks, ROWS expert
+// rows' loads in flight per unit.
+template <class DI, class DP, class DO, bool VEC, bool ALIGNED, int ROWS = kRowsInFlight>
 __device__ __forceinline__ void combine_groups(
     const typename DI::T* const* eo, const int32_t* const* inv, const typename DI::T** ptrs,
     uint8_t* gaps, int world, int64_t first, int64_t t_lo, int64_t t_hi, int split,
@@ -265,7 +269,7 @@ __device__ __forceinline__ void combine_groups(
       __syncwarp();
       if (q0 + kGroupRanks >= world && nxt.r < n_tok)
         load_group<true>(inv, 0, nq0, first + t_lo + nxt.r, E, lane, p0, p1);
-      if (mine) fold_unit<DI, DP, VEC, ALIGNED>(ptrs, gaps, F, trailing, q0, u, acc);
+      if (mine) fold_unit<DI, DP, VEC, ALIGNED, ROWS>(ptrs, gaps, F, trailing, q0, u, acc);
     }
     if (mine) {
       if constexpr (VEC) store8<DO>(out + t * hidden + u * kVec, acc);
@@ -368,12 +372,435 @@ ep_combine_groups(MOE_EPC_PARAMS) {
 }
 #undef MOE_EPC_PARAMS
 
+// ------------------------------------------------------------------------
+// TMA-staged EP combine (up to 32 * kTmaBatches (rank, local expert) pairs,
+// hidden % 8 == 0): one CTA per SM, one producer warp and kTmaWarps consumer
+// warps around a ring of shared-memory stages of up to R expert-row chunks.
+//
+// Work items are (token, chunk of up to kChunkUnits 8-element units of the
+// row, at most kRowBytes); each CTA takes a contiguous range of them, so the
+// chunks of one token follow each other and share its row list.  The producer
+// loads the token's inverse-map entries of all ranks (the next token's are in
+// flight while it works) and compacts them into the rank-ordered list of
+// (rank, row) pairs with the partial-close counts; the item's rows go to
+// ceil(F / R) consecutive stages, and producer lane j fills the item's j-th
+// stage: waits for it to be free, writes its header (item, rows, closes before
+// each row, first / last stage of the item) and issues one 1-D bulk copy
+// (cp.async.bulk, no multicast) per row chunk.  Consumer thread u folds unit
+// u of every row of a stage as it lands, in list order, closes each rank's
+// partial in rank order (rounded to DP), and stores the item's unit after its
+// last stage.  The expert rows are read once, by the copy engine, with up to
+// a ring of row chunks (~190 KB) in flight per SM.
+//
+// Barriers: full[s] completes when the producer's arrival and the stage's
+// bytes are in; empty[s] when the kTmaWarps consumer warps have read it.  Every
+// wait is bounded: a timeout sets MOE_DEVERR_TIMEOUT and ends the warp; the
+// producer drains every copy it issued before its CTA exits.  The producer
+// ends the stream with a header marked `done`.
+//
+// If an expert-output base is not 16-byte aligned (no bulk copy can read it),
+// every warp of the CTA runs the general register-staged combine instead,
+// with 2 rows' loads in flight (it shares the kernel's register budget).
+
+// Timeouts of the TMA-staged kernel for calls given no error word (per
+// device; moe_device_errors() reads it with the forward SwiGLU's word).
+__device__ int32_t g_epc_errors;
+
+#ifndef MOE_EPC_UNITS
+#define MOE_EPC_UNITS 1
+#endif
+// Units (8 elements) of a row chunk per consumer thread: 1 -> 16 consumer
+// warps, one CTA per SM; 2 -> 8 consumer warps and two CTAs per SM, each with
+// half the ring.
+constexpr int kUnitsPerThread = MOE_EPC_UNITS;
+constexpr int kTmaWarps = 16 / kUnitsPerThread;     // consumer warps
+constexpr int kTmaEpcThreads = 32 * (kTmaWarps + 1);
+constexpr int kTmaCtasPerSm = kUnitsPerThread;
+constexpr int kChunkUnits = 512;                    // units per row chunk at most
+constexpr int kRowBytes = 8192;                     // at most this much of a row per copy
+constexpr int kMaxStages = 32;
+constexpr int kTmaBatches = 2;                      // inverse entries per producer lane
+constexpr size_t kEpcSmemMax = 200 * 1024 / kTmaCtasPerSm;
+
+enum : uint8_t { kFirst = 1, kLast = 2, kDone = 4 };
+
+struct __align__(16) StageHeader {
+  int64_t t;                    // token row of the output
+  int64_t col;                  // first column of the chunk
+  uint64_t gaps;                // byte j: partials to close before row j
+  uint8_t rows;                 // rows in this stage
+  uint8_t flags;                // kFirst / kLast (of the item) / kDone
+  uint8_t trailing;             // partials to close after the item's last row (kLast)
+  uint8_t pad[5];
+};
+static_assert(sizeof(StageHeader) == 32, "stage header layout");
+
+// Dynamic shared memory of the kernel: the ring, the headers, the barriers
+// and the producer's row list, in that order.
+struct EpcSmem {
+  size_t headers, bars, list_rows, list_q, list_gaps, total;
+  __host__ __device__ EpcSmem(int stages, size_t stage_bytes) {
+    headers = (size_t)stages * stage_bytes;
+    bars = headers + (size_t)stages * sizeof(StageHeader);
+    list_rows = bars + (size_t)2 * stages * sizeof(uint64_t);
+    list_q = list_rows + (size_t)32 * kTmaBatches * sizeof(int32_t);
+    list_gaps = list_q + (size_t)32 * kTmaBatches;
+    total = list_gaps + (size_t)32 * kTmaBatches + 8;    // 8: the last 64-bit gap read
+  }
+};
+
+// Compacts the token's entries (lane entry b is the flattened pair
+// f = 32 b + lane, rank q[b]) into the list -- rank order, then expert order --
+// with each row's partial-close count; returns the list length, and in
+// `trailing` the partials left to close after its last row.
+__device__ __forceinline__ int build_tma_list(const int32_t (&ent)[kTmaBatches],
+                                              const int (&q)[kTmaBatches], int world,
+                                              int64_t max_rows, int32_t* rows, uint8_t* qs,
+                                              uint8_t* gaps, int32_t* err, int lane,
+                                              int& trailing) {
+  const unsigned below = (1u << lane) - 1u;
+  int F = 0, carry_q = 0;                      // carry_q: rank of the last listed row
+#pragma unroll
+  for (int b = 0; b < kTmaBatches; ++b) {
+    int32_t r = ent[b];
+    if (r >= max_rows) { flag_error(err, MOE_DEVERR_INVERSE); r = -1; }
+    const unsigned m = __ballot_sync(0xffffffffu, r >= 0);
+    const unsigned pm = m & below;
+    const int q_prev = __shfl_sync(0xffffffffu, q[b], pm ? 31 - __clz(pm) : 0);
+    if (r >= 0) {
+      const int pos = F + __popc(pm);
+      rows[pos] = r;
+      qs[pos] = (uint8_t)q[b];
+      gaps[pos] = (uint8_t)(q[b] - (pm ? q_prev : carry_q));
+    }
+    if (m) carry_q = __shfl_sync(0xffffffffu, q[b], 31 - __clz(m));
+    F += __popc(m);
+  }
+  trailing = world - carry_q;
+  __syncwarp();
+  return F;
+}
+
+// Row folds: fold_first, p = v + 0 (a partial's first row: +0 + v, which
+// turns a -0 row into +0 as the definition's +0 start does); fold_add,
+// p = p + v.
+template <class D, bool FIRST>
+__device__ __forceinline__ void fold_row(float (&p)[kVec], const Raw8<D>& r) {
+  float v[kVec];
+  widen8<D>(r, v);
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) p[i] = FIRST ? v[i] + 0.0f : p[i] + v[i];
+}
+
+// Closes the open rank partial (n rows since it opened) into the rank-order
+// sum: acc += round_DP(part).  acc starts at -0, the identity of fp32
+// addition (-0 + x == x for every x, +0 and -0 included), so the first rank's
+// close leaves exactly its partial, as the definition's first term.  A partial
+// of fewer than two rows is +0 or +0 + v with v a value of the input dtype,
+// which DP (the input dtype or fp32) represents exactly: it is not rounded.
+// `empties` ranks without rows follow it: each adds +0, and since
+// (acc + 0) + 0 == acc + 0 they collapse into one add.  The branches are
+// uniform across the warp (every thread walks the same rows).
+template <class DP>
+__device__ __forceinline__ void close_rank(float (&part)[kVec], float (&acc)[kVec], int n,
+                                           bool empties) {
+  if (DP::kBytes == 2 && n >= 2) round_partial<DP, kVec>(part);
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) acc[i] = acc[i] + part[i];
+  if (empties) {
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) acc[i] = acc[i] + 0.0f;
+  }
+}
+
+template <class DI, class DP, class DO, int R>
+__global__ void __launch_bounds__(kTmaEpcThreads, kTmaCtasPerSm)
+ep_combine_tma(const void* const* __restrict__ eo_tab, const void* const* __restrict__ inv_tab,
+               int world, int rank, const int32_t* __restrict__ offs,
+               const int32_t* __restrict__ ep_tokens, int64_t capacity, int64_t max_rows, int E,
+               typename DO::T* __restrict__ out, int64_t local, int64_t hidden, int64_t chunk,
+               int stages, int32_t* err) {
+  static_assert(R >= 1 && R <= 8, "a stage header holds up to 8 closes");
+  using TI = typename DI::T;
+  __shared__ const TI* s_eo[kMaxWorld];
+  __shared__ const int32_t* s_inv[kMaxWorld];
+  extern __shared__ __align__(128) uint8_t smem[];
+  pdl_prologue();
+  const CombineSetup c = combine_setup<TI>(eo_tab, inv_tab, world, rank, offs, ep_tokens,
+                                           capacity, local, s_eo, s_inv, err);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int32_t* const errw = err ? err : &g_epc_errors;
+  if (!c.aligned) {                                     // no bulk copy can read a base
+    const TI** ptrs = reinterpret_cast<const TI**>(smem) + (size_t)warp * kGroupRanks * kMaxE;
+    uint8_t* gaps = smem + (size_t)(kTmaWarps + 1) * kGroupRanks * kMaxE * sizeof(void*) +
+                    (size_t)warp * kGroupRanks * kMaxE;
+    const int64_t units = hidden / kVec;
+    const int64_t split = (units + 31) / 32;
+    combine_groups<DI, DP, DO, true, false, 2>(
+        s_eo, s_inv, ptrs, gaps, world, c.first, c.t_lo, c.t_hi, (int)split, units, hidden,
+        max_rows, E, out, err, lane, (int64_t)blockIdx.x * (kTmaWarps + 1) + warp,
+        (int64_t)gridDim.x * (kTmaWarps + 1));
+    return;
+  }
+  const size_t row_bytes = (size_t)chunk * sizeof(TI);
+  const size_t stage_bytes = (size_t)R * row_bytes;
+  const EpcSmem lay(stages, stage_bytes);
+  StageHeader* hdr = reinterpret_cast<StageHeader*>(smem + lay.headers);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars);
+  uint64_t* empty = full + stages;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      tma::mbar_init(&full[s], 1);
+      tma::mbar_init(&empty[s], kTmaWarps);
+    }
+    tma::mbar_init_fence();
+  }
+  __syncthreads();
+  const int64_t split = (hidden + chunk - 1) / chunk;
+  const int64_t n_items = (c.t_hi - c.t_lo) * split;
+  const int64_t lo = n_items * blockIdx.x / gridDim.x;
+  const int64_t hi = n_items * (blockIdx.x + 1) / gridDim.x;
+
+  if (warp == 0) {                                      // producer
+    int32_t* l_rows = reinterpret_cast<int32_t*>(smem + lay.list_rows);
+    uint8_t* l_q = smem + lay.list_q;
+    uint8_t* l_gaps = smem + lay.list_gaps;
+    // this lane's (rank, local expert) pairs, fixed for the whole launch
+    int qb[kTmaBatches];
+    const int32_t* pb[kTmaBatches];
+#pragma unroll
+    for (int b = 0; b < kTmaBatches; ++b) {
+      const int f = 32 * b + lane;
+      qb[b] = f < world * E ? f / E : world;
+      pb[b] = f < world * E ? s_inv[qb[b]] + f % E : nullptr;
+    }
+    int32_t ent[kTmaBatches];
+#pragma unroll
+    for (int b = 0; b < kTmaBatches; ++b) {
+      const int64_t g = c.first + c.t_lo + lo / split;
+      ent[b] = pb[b] && lo < hi ? __ldg(pb[b] + g * E) : -1;
+    }
+    const int64_t last_t = c.t_lo + (hi - 1) / split;
+    const int per_round = stages < 32 ? stages : 32;   // lanes filling distinct stages at once
+    uint32_t k = 0;                                     // stages filled so far
+    bool failed = false;
+    int F = 0, trailing = 0;
+    int64_t t = c.t_lo + lo / split, ci = lo % split;
+    for (int64_t item = lo; item < hi && !failed; ++item) {
+      if (item == lo || ci == 0) {                     // a new token: its row list
+        F = build_tma_list(ent, qb, world, max_rows, l_rows, l_q, l_gaps, err, lane, trailing);
+        if (t < last_t) {                              // the next token's entries, in flight
+#pragma unroll
+          for (int b = 0; b < kTmaBatches; ++b)
+            ent[b] = pb[b] ? __ldg(pb[b] + (c.first + t + 1) * E) : -1;
+        }
+      }
+      const int64_t col = ci * chunk;
+      const uint32_t bytes = (uint32_t)((hidden - col < chunk ? hidden - col : chunk) *
+                                        (int64_t)sizeof(TI));
+      const int nst = F > 0 ? (F + R - 1) / R : 1;     // stages of this item
+      for (int j0 = 0; j0 < nst && !failed; j0 += per_round) {
+        const int cnt = nst - j0 < per_round ? nst - j0 : per_round;
+        const int j = j0 + lane;                        // this lane's stage of the item
+        const uint32_t kk = k + lane;
+        const int s = (int)(kk % stages);
+        bool ok = true;
+        if (lane < cnt && kk >= (uint32_t)stages)       // wait until the stage is free
+          ok = tma::mbar_wait(&empty[s], (kk / stages - 1) & 1);
+        if (!__all_sync(0xffffffffu, ok)) {
+          if (lane == 0) atomicOr(errw, MOE_DEVERR_TIMEOUT);
+          failed = true;
+          break;
+        }
+        if (lane < cnt) {
+          const int r0 = j * R;
+          const int nr = F - r0 < R ? F - r0 : R;       // <= 0 only for a row-less item
+          StageHeader& h = hdr[s];
+          uint64_t g8 = 0;
+          for (int i = 0; i < nr; ++i) g8 |= (uint64_t)l_gaps[r0 + i] << (8 * i);
+          h.t = t;
+          h.col = col;
+          h.gaps = g8;
+          h.rows = (uint8_t)(nr > 0 ? nr : 0);
+          h.flags = (uint8_t)((j == 0 ? kFirst : 0) | (j == nst - 1 ? kLast : 0));
+          h.trailing = (uint8_t)trailing;
+          if (nr > 0) {
+            tma::mbar_arrive_expect_tx(&full[s], (uint32_t)nr * bytes);
+            for (int i = 0; i < nr; ++i) {
+              const TI* src = s_eo[l_q[r0 + i]] + (int64_t)l_rows[r0 + i] * hidden + col;
+              tma::bulk_load(smem + (size_t)s * stage_bytes + (size_t)i * row_bytes, src, bytes,
+                             &full[s]);
+            }
+          } else {
+            tma::mbar_arrive(&full[s]);
+          }
+        }
+        k += (uint32_t)cnt;
+      }
+      __syncwarp();                                    // the list is read before it changes
+      if (++ci == split) { ci = 0; ++t; }
+    }
+    if (!failed) {                                     // end of stream
+      const int s = (int)(k % stages);
+      bool ok = true;
+      if (lane == 0 && k >= (uint32_t)stages) ok = tma::mbar_wait(&empty[s], (k / stages - 1) & 1);
+      if (lane == 0) {
+        if (ok) {
+          hdr[s].flags = kDone;
+          tma::mbar_arrive(&full[s]);
+          ++k;
+        } else {
+          atomicOr(errw, MOE_DEVERR_TIMEOUT);
+        }
+      }
+      k = __shfl_sync(0xffffffffu, k, 0);
+    }
+    if (lane == 0) {                                   // drain: every issued fill has landed
+      for (int s = 0; s < stages && (uint32_t)s < k; ++s) {
+        const uint32_t last = s + ((k - 1 - s) / stages) * stages;
+        if (!tma::mbar_wait(&full[s], (last / stages) & 1)) atomicOr(errw, MOE_DEVERR_TIMEOUT);
+      }
+    }
+    return;
+  }
+
+  // consumers: thread u folds units u, u + 32 * kTmaWarps, ... of every row of
+  // a stage as it lands
+  constexpr int U = kUnitsPerThread;
+  constexpr int kStride = 32 * kTmaWarps;
+  const int u0 = threadIdx.x - 32;
+  const int64_t width0 = hidden < chunk ? hidden : chunk;
+  const bool act_any = (int64_t)u0 * kVec < width0;
+  float acc[U][kVec] = {}, part[U][kVec] = {};
+  int n = 0;                                           // rows in the open partial
+  int s = 0;
+  uint32_t phase = 0;
+  for (;;) {
+    const bool ok = tma::mbar_wait(&full[s], phase);
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (lane == 0) atomicOr(errw, MOE_DEVERR_TIMEOUT);
+      return;
+    }
+    const StageHeader& h = hdr[s];
+    const uint8_t flags = h.flags;
+    if (flags & kDone) return;
+    if (act_any) {
+      const int64_t col = h.col;
+      const int64_t width = hidden - col < chunk ? hidden - col : chunk;
+      if (flags & kFirst) {                            // a new item: -0 sum, +0 partial
+#pragma unroll
+        for (int x = 0; x < U; ++x)
+#pragma unroll
+          for (int i = 0; i < kVec; ++i) {
+            acc[x][i] = -0.0f;
+            part[x][i] = 0.0f;
+          }
+        n = 0;
+      }
+      const int nr = h.rows;
+      uint64_t gaps = h.gaps;
+      const TI* st = reinterpret_cast<const TI*>(smem + (size_t)s * stage_bytes) +
+                     (size_t)u0 * kVec;
+      bool mine[U];
+      Raw8<DI> raw[R][U];
+#pragma unroll
+      for (int x = 0; x < U; ++x) mine[x] = (int64_t)(u0 + x * kStride) * kVec < width;
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int x = 0; x < U; ++x)
+          if (i < nr && mine[x])
+            raw[i][x] = tma::lds8<DI>(st + (size_t)i * chunk + (size_t)x * kStride * kVec);
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        if (i < nr) {
+          const int g = (int)(gaps & 0xffu);
+          gaps >>= 8;
+          if (g > 0) {                                 // the row opens a rank
+#pragma unroll
+            for (int x = 0; x < U; ++x) {
+              close_rank<DP>(part[x], acc[x], n, g > 1);
+              fold_row<DI, true>(part[x], raw[i][x]);
+            }
+            n = 1;
+          } else {
+#pragma unroll
+            for (int x = 0; x < U; ++x) fold_row<DI, false>(part[x], raw[i][x]);
+            ++n;
+          }
+        }
+      }
+      if (flags & kLast) {
+        const int g = h.trailing;                      // >= 1: the open rank, then empties
+#pragma unroll
+        for (int x = 0; x < U; ++x) {
+          close_rank<DP>(part[x], acc[x], n, g > 1);
+          if (mine[x])
+            store8<DO>(out + h.t * hidden + col + (int64_t)(u0 + x * kStride) * kVec, acc[x]);
+        }
+      }
+    }
+    __syncwarp();                                      // the warp has read the stage
+    if (lane == 0) tma::mbar_arrive(&empty[s]);
+    if (++s == stages) {
+      s = 0;
+      phase ^= 1u;
+    }
+  }
+}
+
+#ifndef MOE_EPC_TMA
+#define MOE_EPC_TMA 1
+#endif
+
+#ifndef MOE_EPC_STAGE_ROWS
+#define MOE_EPC_STAGE_ROWS 4
+#endif
+
+template <class DI, class DP, class DO>
+int launch_tma(const void* const* eos, const void* const* invs, int world, int rank,
+               const int32_t* offs, const int32_t* ep_tokens, int64_t capacity, int64_t max_rows,
+               int E, void* out, int64_t local, int64_t hidden, int32_t* err,
+               cudaStream_t stream) {
+  using TI = typename DI::T;
+  constexpr int R = MOE_EPC_STAGE_ROWS;
+  // row chunks of at most kRowBytes (and one unit per consumer thread)
+  int64_t units = hidden / kVec;
+  if (units > kChunkUnits) units = kChunkUnits;
+  if (units * kVec * (int64_t)sizeof(TI) > kRowBytes) units = kRowBytes / (kVec * sizeof(TI));
+  const int64_t chunk = units * kVec;
+  const size_t stage_bytes = (size_t)R * chunk * sizeof(TI);
+  int stages = kMaxStages;
+  while (stages >= 3 && EpcSmem(stages, stage_bytes).total > kEpcSmemMax) --stages;
+  if (stages < 3) return -1;
+  // the misaligned-base path carves per-warp row lists out of the same memory
+  const size_t lists = (size_t)(kTmaWarps + 1) * kGroupRanks * kMaxE * (sizeof(void*) + 1);
+  size_t smem = EpcSmem(stages, stage_bytes).total;
+  if (smem < lists) smem = lists;
+  auto k = ep_combine_tma<DI, DP, DO, R>;
+  if (int rc = ensure_smem_limit((const void*)k, kEpcSmemMax)) return rc;
+  int sms = 0;
+  if (int rc = device_sm_count(&sms)) return rc;
+  const int64_t items = local * ((hidden + chunk - 1) / chunk);
+  const int64_t ctas = (int64_t)sms * kTmaCtasPerSm;
+  const int grid = (int)(items < ctas ? items : ctas);
+  launch_kernel_block(k, grid, kTmaEpcThreads, smem, stream, eos, invs, world, rank, offs,
+                      ep_tokens, capacity, max_rows, E, static_cast<typename DO::T*>(out), local,
+                      hidden, chunk, stages, err);
+  return check_launch();
+}
+
 template <class DI, class DP, class DO>
 int launch(const void* const* eos, const void* const* invs, int world, int rank,
            const int32_t* offs, const int32_t* ep_tokens, int64_t capacity, int64_t max_rows,
            int E, void* out, int64_t local, int64_t hidden, int32_t* err, cudaStream_t stream) {
   using TO = typename DO::T;
   const bool vec = hidden % kVec == 0 && aligned16(out);
+  if (MOE_EPC_TMA && vec && world * E <= 32 * kTmaBatches) {
+    const int rc = launch_tma<DI, DP, DO>(eos, invs, world, rank, offs, ep_tokens, capacity,
+                                          max_rows, E, out, local, hidden, err, stream);
+    if (rc >= 0) return rc;
+  }
   const bool one_group = vec && world <= kGroupRanks;
   const int64_t units = vec ? hidden / kVec : hidden;
   int sms = 0;
@@ -438,6 +865,17 @@ int dispatch(moe_dtype partial_dt, moe_dtype out_dt, const void* const* eos,
 }  // namespace
 
 int max_ep_combine_world() { return kMaxWorld; }
+
+int ep_combine_device_errors(int32_t* bits, int clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(bits, g_epc_errors, sizeof(int32_t));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (clear) {
+    const int32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_epc_errors, &zero, sizeof(int32_t));
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return MOE_OK;
+}
 int max_ep_combine_experts() { return kMaxE; }
 
 int launch_unpermute_reduce_scatter(const void* const* expert_outputs, moe_dtype eo_dt,

@@ -14,8 +14,8 @@ int cuda_fail(cudaError_t e);
 
 // Persistent grid for `kernel` launched with kThreads threads and `smem`
 // bytes of dynamic shared memory: resident CTAs per SM (occupancy, cached per
-// kernel) times the SM count of the current device (cached per device), but
-// no more than `useful_blocks`, and at least 1.
+// kernel, shared-memory size and device) times the SM count of the current
+// device (cached per device), but no more than `useful_blocks`, and at least 1.
 int persistent_grid(const void* kernel, size_t smem, int64_t useful_blocks, int* grid);
 
 // MOE_ERR_CUDA if the launch just issued failed.
@@ -57,12 +57,23 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Launchers (one per op family); arguments already validated.
 int launch_swiglu_clamped_fwd(const void* x, const float* probs, void* y, int64_t rows,
                               int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
-                              moe_dtype dt, cudaStream_t stream);
+                              moe_dtype dt, int32_t* dev_err, cudaStream_t stream);
+// 1 if the forward of rows of `inter` columns of dt takes the TMA-staged kernel
+// (given contiguous, 16-byte aligned tensors).
+int tma_forward_applies(int64_t inter, moe_dtype dt);
+// The TMA-staged forward with one row's fill withheld (tests of the bounded
+// waits; contiguous x and y, arguments validated by the caller).
+int launch_swiglu_fwd_stalled(const void* x, const float* probs, void* y, int64_t rows,
+                              int64_t inter, float limit, moe_dtype dt, int grid,
+                              int64_t stall_row, long long wait_cycles, int32_t* dev_err,
+                              cudaStream_t stream);
 int launch_swiglu_clamped_bwd(const void* x, const float* probs, const void* grad_y,
                               void* grad_x, float* grad_probs, int64_t rows, int64_t inter,
                               int64_t ld_x, int64_t ld_gy, int64_t ld_gx, float limit,
                               moe_dtype dt, cudaStream_t stream);
 int max_ep_combine_world();
+// Copies (and optionally clears) the EP combine's per-device timeout word.
+int ep_combine_device_errors(int32_t* bits, int clear);
 int max_ep_combine_experts();
 int launch_unpermute_reduce_scatter(const void* const* expert_outputs, moe_dtype eo_dt,
                                     int64_t max_rows, const void* const* inverse_maps,

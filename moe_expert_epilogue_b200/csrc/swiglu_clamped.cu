@@ -112,7 +112,8 @@ swiglu_fwd_rows(const typename D::T* __restrict__ x, const float* __restrict__ p
 }
 
 // Errors recorded by the kernels of this file that wait on barriers (bits
-// MOE_DEVERR_*), per device; read and cleared by moe_device_errors().
+// MOE_DEVERR_*), per device, when the caller gives no error word of its own;
+// read and cleared by moe_device_errors().
 __device__ int32_t g_device_errors;
 
 constexpr int kTmaConsumers = 8;
@@ -124,18 +125,27 @@ constexpr size_t kTmaSmemMax = 200 * 1024;
 // filled and emptied by one consumer in order, so a stage has at most one fill
 // outstanding and the barrier parities are unambiguous.  full[s] completes a
 // phase when the producer's arrival and the row's bytes are in; empty[s] when
-// the consumer has read the row.  Every wait is bounded: on a timeout the
-// waiting warp records MOE_DEVERR_TIMEOUT and stops; the producer then waits
-// (bounded again) for every copy it issued before its CTA exits.
-template <class D, int S>
+// the consumer has read the row.  Every wait is bounded: a consumer's wait for
+// its row and the producer's wait for a free stage give up after `wait_cycles`
+// SM cycles; the waiting warp then ORs MOE_DEVERR_TIMEOUT into `err` (the
+// caller's word, else g_device_errors) and stops, and the producer waits
+// (bounded again, kWaitCycles) for every copy it issued before its CTA exits,
+// so no copy is left in flight on the normal timeout path.
+//
+// STALL (tests of that failure path only): the producer neither arrives on
+// nor copies into the stage of row `stall_row`, so that row's consumer waits
+// for a phase that never completes and times out; nothing is left in flight
+// (the drain skips the fill that was never issued).
+template <class D, int S, bool STALL>
 __global__ void __launch_bounds__(kTmaThreads, 1)
 swiglu_fwd_tma(const typename D::T* __restrict__ x, const float* __restrict__ probs,
                typename D::T* __restrict__ y, int64_t rows, int64_t inter, int64_t ld_x,
-               int64_t ld_y, float L) {
+               int64_t ld_y, float L, int32_t* err, long long wait_cycles, int64_t stall_row) {
   static_assert(S % kTmaConsumers == 0, "each stage must belong to one consumer warp");
   pdl_prologue();
   using T = typename D::T;
   extern __shared__ __align__(128) uint8_t smem[];
+  int32_t* const errw = err ? err : &g_device_errors;
   const uint32_t stage_bytes = (uint32_t)(2 * inter * sizeof(T));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * stage_bytes);
   uint64_t* empty = full + S;
@@ -149,24 +159,30 @@ swiglu_fwd_tma(const typename D::T* __restrict__ x, const float* __restrict__ pr
   }
   __syncthreads();
   const int64_t my_rows = rows > blockIdx.x ? (rows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  // the CTA-local index of the row that is never filled (STALL only)
+  const int64_t k_stall = (STALL && stall_row >= 0 && stall_row % gridDim.x == blockIdx.x)
+                              ? stall_row / gridDim.x : -1;
   if (warp == 0) {                                        // producer
     if (lane != 0) return;
     int64_t k = 0;
     for (; k < my_rows; ++k) {
       const int s = (int)(k % S);
       const uint32_t n = (uint32_t)(k / S);
-      if (n > 0 && !tma::mbar_wait(&empty[s], (n - 1) & 1)) {
-        atomicOr(&g_device_errors, MOE_DEVERR_TIMEOUT);
+      if (n > 0 && !tma::mbar_wait(&empty[s], (n - 1) & 1, wait_cycles)) {
+        atomicOr(errw, MOE_DEVERR_TIMEOUT);
         break;
       }
+      if (STALL && k == k_stall) continue;
       const int64_t r = blockIdx.x + k * gridDim.x;
       tma::mbar_arrive_expect_tx(&full[s], stage_bytes);
       tma::bulk_load(smem + (size_t)s * stage_bytes, x + r * ld_x, stage_bytes, &full[s]);
     }
     for (int s = 0; s < S && s < k; ++s) {                // drain every issued copy
-      const int64_t last = s + ((k - 1 - s) / S) * S;
+      int64_t last = s + ((k - 1 - s) / S) * S;
+      if (STALL && last == k_stall) last -= S;            // that fill was never issued
+      if (last < 0) continue;
       if (!tma::mbar_wait(&full[s], (uint32_t)(last / S) & 1))
-        atomicOr(&g_device_errors, MOE_DEVERR_TIMEOUT);
+        atomicOr(errw, MOE_DEVERR_TIMEOUT);
     }
     return;
   }
@@ -175,8 +191,11 @@ swiglu_fwd_tma(const typename D::T* __restrict__ x, const float* __restrict__ pr
   const FwdMath f{L};
   for (int64_t k = cw; k < my_rows; k += kTmaConsumers) {
     const int s = (int)(k % S);
-    if (!tma::mbar_wait(&full[s], (uint32_t)(k / S) & 1)) {
-      if (lane == 0) atomicOr(&g_device_errors, MOE_DEVERR_TIMEOUT);
+    // every lane polls; the warp gives up as one if any lane did (a phase that
+    // completes just as the limit passes cannot split the warp)
+    const bool ok = tma::mbar_wait(&full[s], (uint32_t)(k / S) & 1, wait_cycles);
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (lane == 0) atomicOr(errw, MOE_DEVERR_TIMEOUT);
       return;
     }
     const int64_t r = blockIdx.x + k * gridDim.x;
@@ -194,6 +213,30 @@ swiglu_fwd_tma(const typename D::T* __restrict__ x, const float* __restrict__ pr
     __syncwarp();                                          // every lane has read the stage
     if (lane == 0) tma::mbar_arrive(&empty[s]);
   }
+}
+
+// Stages of the TMA ring for rows of `inter` columns of T: 16, or 8 for
+// longer rows, or 0 when even 8 do not fit.
+template <class T>
+int tma_stages(int64_t inter) {
+  const size_t stage = (size_t)2 * inter * sizeof(T);
+  return 16 * stage + 256 <= kTmaSmemMax ? 16 : 8 * stage + 128 <= kTmaSmemMax ? 8 : 0;
+}
+
+// Launches the TMA-staged forward with `grid` CTAs (one per SM at most).
+template <class D, bool STALL>
+int launch_fwd_tma(const typename D::T* x, const float* probs, typename D::T* y, int64_t rows,
+                   int64_t inter, int64_t ld_x, int64_t ld_y, float limit, int grid,
+                   int32_t* err, long long wait_cycles, int64_t stall_row,
+                   cudaStream_t stream) {
+  using T = typename D::T;
+  const int S = tma_stages<T>(inter);
+  auto k = S == 16 ? swiglu_fwd_tma<D, 16, STALL> : swiglu_fwd_tma<D, 8, STALL>;
+  const size_t smem = (size_t)S * 2 * inter * sizeof(T) + 2 * (size_t)S * sizeof(uint64_t);
+  if (int rc = ensure_smem_limit((const void*)k, kTmaSmemMax)) return rc;
+  launch_kernel_block(k, grid, kTmaThreads, smem, stream, x, probs, y, rows, inter, ld_x, ld_y,
+                      limit, err, wait_cycles, stall_row);
+  return check_launch();
 }
 
 // Flat grid-stride forward over (row, chunk) pairs, for short rows.
@@ -417,7 +460,7 @@ constexpr int kBwdRowThreads = MOE_SWIGLU_BWD_ROW_THREADS;
 
 template <class D>
 int fwd(const void* xv, const float* probs, void* yv, int64_t rows, int64_t inter, int64_t ld_x,
-        int64_t ld_y, float limit, cudaStream_t stream) {
+        int64_t ld_y, float limit, int32_t* err, cudaStream_t stream) {
   using T = typename D::T;
   const T* x = static_cast<const T*>(xv);
   T* y = static_cast<T*>(yv);
@@ -425,19 +468,12 @@ int fwd(const void* xv, const float* probs, void* yv, int64_t rows, int64_t inte
                    aligned16(y);
   int grid;
   if constexpr (D::kBytes == 2) {
-    // TMA ring: 16 stages of one row, or 8 for longer rows, if it fits
-    const size_t stage = (size_t)2 * inter * sizeof(T);
-    const int S = 16 * stage + 256 <= kTmaSmemMax ? 16 : 8 * stage + 128 <= kTmaSmemMax ? 8 : 0;
-    if (MOE_SWIGLU_FWD_TMA && vec && inter / kVec >= 64 && S > 0) {
-      auto k = S == 16 ? swiglu_fwd_tma<D, 16> : swiglu_fwd_tma<D, 8>;
-      const size_t smem = (size_t)S * stage + 2 * (size_t)S * sizeof(uint64_t);
-      if (int rc = ensure_smem_limit((const void*)k, kTmaSmemMax)) return rc;
+    if (MOE_SWIGLU_FWD_TMA && vec && inter / kVec >= 64 && tma_stages<T>(inter) > 0) {
       int sms = 0;
       if (int rc = device_sm_count(&sms)) return rc;
       grid = (int)(rows < sms ? rows : sms);
-      launch_kernel_block(k, grid, kTmaThreads, smem, stream, x, probs, y, rows, inter, ld_x,
-                          ld_y, limit);
-      return check_launch();
+      return launch_fwd_tma<D, false>(x, probs, y, rows, inter, ld_x, ld_y, limit, grid, err,
+                                      tma::kWaitCycles, -1, stream);
     }
   }
   if (vec && inter / kVec >= 64) {
@@ -510,12 +546,30 @@ int bwd(const void* xv, const float* probs, const void* gyv, void* gxv, float* g
 
 int launch_swiglu_clamped_fwd(const void* x, const float* probs, void* y, int64_t rows,
                               int64_t inter, int64_t ld_x, int64_t ld_y, float limit,
-                              moe_dtype dt, cudaStream_t stream) {
+                              moe_dtype dt, int32_t* dev_err, cudaStream_t stream) {
   switch (dt) {
-    case MOE_BF16: return fwd<BF16>(x, probs, y, rows, inter, ld_x, ld_y, limit, stream);
-    case MOE_FP16: return fwd<F16>(x, probs, y, rows, inter, ld_x, ld_y, limit, stream);
-    default: return fwd<F32>(x, probs, y, rows, inter, ld_x, ld_y, limit, stream);
+    case MOE_BF16: return fwd<BF16>(x, probs, y, rows, inter, ld_x, ld_y, limit, dev_err, stream);
+    case MOE_FP16: return fwd<F16>(x, probs, y, rows, inter, ld_x, ld_y, limit, dev_err, stream);
+    default: return fwd<F32>(x, probs, y, rows, inter, ld_x, ld_y, limit, dev_err, stream);
   }
+}
+
+int tma_forward_applies(int64_t inter, moe_dtype dt) {
+  if (dt == MOE_FP32 || inter % kVec != 0 || inter / kVec < 64) return 0;
+  return tma_stages<uint16_t>(inter) > 0;
+}
+
+int launch_swiglu_fwd_stalled(const void* x, const float* probs, void* y, int64_t rows,
+                              int64_t inter, float limit, moe_dtype dt, int grid,
+                              int64_t stall_row, long long wait_cycles, int32_t* dev_err,
+                              cudaStream_t stream) {
+  if (dt == MOE_BF16)
+    return launch_fwd_tma<BF16, true>(static_cast<const uint16_t*>(x), probs,
+                                      static_cast<uint16_t*>(y), rows, inter, 2 * inter, inter,
+                                      limit, grid, dev_err, wait_cycles, stall_row, stream);
+  return launch_fwd_tma<F16, true>(static_cast<const uint16_t*>(x), probs,
+                                   static_cast<uint16_t*>(y), rows, inter, 2 * inter, inter,
+                                   limit, grid, dev_err, wait_cycles, stall_row, stream);
 }
 
 int launch_swiglu_clamped_bwd(const void* x, const float* probs, const void* grad_y,
@@ -546,5 +600,8 @@ extern "C" int moe_device_errors(int32_t* bits, int clear) {
     e = cudaMemcpyToSymbol(moe::g_device_errors, &zero, sizeof(int32_t));
     if (e != cudaSuccess) return moe::cuda_fail(e);
   }
+  int32_t epc = 0;
+  if (int rc = moe::ep_combine_device_errors(&epc, clear)) return rc;
+  *bits |= epc;
   return MOE_OK;
 }

@@ -39,8 +39,9 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 }
 
 // Waits for the completion of the barrier phase with the given parity;
-// false once kWaitCycles have passed without it.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// false once `limit` SM cycles have passed without it.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          long long limit = kWaitCycles) {
   const long long t0 = clock64();
   while (true) {
     uint32_t done;
@@ -51,7 +52,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
         : "r"(smem_addr(bar)), "r"(parity)
         : "memory");
     if (done) return true;
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
 }
 

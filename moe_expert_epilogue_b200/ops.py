@@ -73,8 +73,10 @@ def _two_d(t, name):
     return t.shape
 
 
-def swiglu_clamped_fwd(x, probs, limit, out=None, stream=None):
-    """y = silu(clamp(gate, max=L)) * clamp(up, -L, L) * probs, in x's dtype."""
+def swiglu_clamped_fwd(x, probs, limit, out=None, dev_err=None, stream=None):
+    """y = silu(clamp(gate, max=L)) * clamp(up, -L, L) * probs, in x's dtype.
+    dev_err (int32 [1], optional) receives MOE_DEVERR_TIMEOUT if a barrier
+    wait of the TMA-staged kernel gave up."""
     rows, two_i = _two_d(x, "x")
     if two_i % 2:
         raise ValueError("x must hold [gate | up]: an even number of columns")
@@ -85,9 +87,10 @@ def swiglu_clamped_fwd(x, probs, limit, out=None, stream=None):
     _check(out, "out", dtype=x.dtype, shape=(rows, inter), contiguous=False)
     ld_x, ld_y = _rows_stride(x, "x"), _rows_stride(out, "out")
     _flat_probs(probs, rows)
-    _cuda(x, probs, out)
-    _abi.moe_swiglu_clamped_fwd(x, probs, out, rows, inter, ld_x, ld_y, limit,
-                                moe_dtype(x.dtype), stream)
+    _check(dev_err, "dev_err", dtype=torch.int32, numel=1)
+    _cuda(x, probs, out, dev_err)
+    _abi.moe_swiglu_clamped_fwd_ex(x, probs, out, rows, inter, ld_x, ld_y, limit,
+                                   moe_dtype(x.dtype), dev_err, stream)
     return out
 
 

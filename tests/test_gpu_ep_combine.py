@@ -88,6 +88,76 @@ def test_ep_combine_bitwise_every_rank(cuda_device, world, tokens, top_k, epr, a
         assert_bits_equal(bits(got), want, f"rank {rank}", kind=KIND[out_dtype])
 
 
+# Shapes aimed at the TMA-staged kernel (up to 64 (rank, local expert) pairs,
+# hidden % 8 == 0): lists longer than one stage of 8 rows, rows cut into chunks
+# of 2048 columns with a ragged last chunk, a one-unit row; and one shape past
+# 64 pairs, which takes the register-staged kernel.
+CASES_TMA = [  # world, tokens, top_k, experts per rank, align, hidden
+    (2, 50, 20, 16, 4, 264), (4, 100, 12, 16, 8, 4104), (8, 64, 8, 8, 16, 7168),
+    (1, 33, 1, 1, 1, 8), (9, 60, 4, 8, 8, 96)]
+
+
+@pytest.mark.parametrize("world,tokens,top_k,epr,align,hidden", CASES_TMA)
+@pytest.mark.parametrize("eo_dtype,partial_dtype,out_dtype", DTYPES)
+def test_ep_combine_stages_and_chunks(cuda_device, world, tokens, top_k, epr, align, hidden,
+                                      eo_dtype, partial_dtype, out_dtype):
+    case = inputs.ep_combine_inputs(world, tokens, top_k, epr, align, hidden, dtype=eo_dtype,
+                                    seed=world * 77 + hidden)
+    eo_t, inv_t, keep = _tables(cuda_device, case)
+    _abi.moe_device_errors(clear=True)
+    for rank in range(world):
+        init = torch.full((case.counts[rank], hidden), -2.5, dtype=out_dtype)
+        got = _run(cuda_device, case, eo_t, inv_t, rank, out_dtype, partial_dtype, init)
+        want, err = _oracle(case, rank, out_dtype, partial_dtype, init)
+        assert err == 0
+        assert_bits_equal(bits(got), want, f"rank {rank}", kind=KIND[out_dtype])
+    assert _abi.moe_device_errors(clear=True) == 0
+
+
+def test_ep_combine_tokens_without_rows(cuda_device):
+    """Tokens none of whose experts any rank holds (all inverse entries < 0)
+    get the empty rank-order sum, +0, like their all-zero partial block rows;
+    the tokens around them are unaffected."""
+    case = inputs.ep_combine_inputs(4, 90, 4, 4, 8, 2056, seed=12)
+    for q in range(4):
+        inv = case.inverse_maps[q].clone()
+        inv[::7] = -1
+        inv[40:44] = -1
+        case.inverse_maps[q] = inv
+    eo_t, inv_t, keep = _tables(cuda_device, case)
+    for rank in range(4):
+        init = torch.full((case.counts[rank], 2056), 9.0, dtype=torch.bfloat16)
+        got = _run(cuda_device, case, eo_t, inv_t, rank, torch.bfloat16, torch.bfloat16, init)
+        want, err = _oracle(case, rank, torch.bfloat16, torch.bfloat16, init)
+        assert err == 0
+        assert_bits_equal(bits(got), want, f"rank {rank}")
+
+
+@pytest.mark.parametrize("partial_dtype", [torch.bfloat16, torch.float32])
+def test_ep_combine_subnormal_and_signed_zero_rows(cuda_device, partial_dtype):
+    """Expert rows of bf16 subnormals, signed zeros and their negations: the
+    packed adds keep subnormal operands and sums (no flush to zero), and a
+    one-row partial of -0 still becomes +0 + -0 = +0 as in the two steps."""
+    case = inputs.ep_combine_inputs(2, 64, 4, 4, 8, 4096, seed=21)
+    g = torch.Generator().manual_seed(22)
+    for q in range(2):
+        eo = case.expert_outputs[q]
+        raw = torch.randint(1, 0x80, eo.shape, generator=g, dtype=torch.int32)  # subnormal bits
+        sign = torch.randint(0, 2, eo.shape, generator=g, dtype=torch.int32) << 15
+        bits16 = (raw | sign).to(torch.int16)
+        bits16[:, ::97] = 0
+        bits16[:, 1::97] = -32768                                              # -0.0
+        case.expert_outputs[q] = bits16.view(torch.bfloat16)
+    eo_t, inv_t, keep = _tables(cuda_device, case)
+    for rank in range(2):
+        init = torch.zeros(case.counts[rank], 4096, dtype=torch.float32)
+        got = _run(cuda_device, case, eo_t, inv_t, rank, torch.float32, partial_dtype, init)
+        want, err = _oracle(case, rank, torch.float32, partial_dtype, init)
+        assert err == 0
+        assert np.array_equal(bits(got).view(np.uint32), want.view(np.uint32)), rank
+        assert (bits(got) != 0).any() and np.isfinite(bits(got)).all()
+
+
 def _two_step(dev, case, rank, partial_dtype, out_dtype):
     """The pages' form with the library's own kernels: each rank's unpermute
     into a partial block, then the reduce-scatter of the blocks."""

@@ -152,25 +152,46 @@ def test_swiglu_cuda_graph_replay(cuda_device):
     _check(d, L, bits(y), bits(gx), bits(gp))
 
 
+def strict_grad_probs_report(got, ref64, abs64, rtol=1e-5, floor=1e-3):
+    """How many rows meet the pure relative bound |got - ref| <= rtol * |ref|,
+    over all rows and over the rows whose sum does not cancel below
+    floor * sum_j |t_j| (the rows where a relative bound is meaningful)."""
+    got = np.asarray(got, np.float64).ravel()
+    err = np.abs(got - ref64)
+    strict = err <= rtol * np.abs(ref64)
+    big = np.abs(ref64) >= floor * abs64
+    return {"rows": int(got.size), "strict_fail": int((~strict).sum()),
+            "rows_not_cancelling": int(big.sum()),
+            "strict_fail_not_cancelling": int((~strict & big).sum()),
+            "max_err_over_ref_not_cancelling": float((err[big] / np.abs(ref64[big])).max())
+            if big.any() else 0.0}
+
+
 @pytest.mark.parametrize("sigma", [3.0, 5.1])
-def test_swiglu_large_workload_sampled_rows(cuda_device, sigma):
+def test_swiglu_large_workload_whole_tensor(cuda_device, sigma):
     """rows = 65536 (8192 tokens x top-8), inter = 2048, L = 10, top-8 softmax
-    probs: the full launch the benchmark times, checked on sampled rows."""
+    probs: the full launches the benchmark times, every element of y and
+    grad_x and every grad_probs row against the oracle."""
     rows, inter, L = 65536, 2048, 10.0
     d = inputs.swiglu_inputs(rows, inter, sigma=sigma, probs="topk_softmax", seed=0)
     x, p, gy = (d[k].to(cuda_device) for k in ("x", "probs", "grad_y"))
     y = ops.swiglu_clamped_fwd(x, p, L)
     gx, gp = ops.swiglu_clamped_bwd(x, p, gy, L)
     torch.cuda.synchronize()
-    rng = np.random.default_rng(int(sigma * 10))
-    idx = np.unique(np.concatenate([[0, 1, rows - 1], rng.integers(0, rows, 509)]))
-    ti = torch.from_numpy(idx)
-    _check(d, L, bits(y.cpu()[ti]), bits(gx.cpu()[ti]), bits(gp.cpu()[ti]), rows_idx=idx)
+    xb, pb, gyb = bits(d["x"]), bits(d["probs"]), bits(d["grad_y"])
+    assert_within_ulp16(bits(y), oracle.swiglu_clamped_fwd(xb, pb, L), 1, what="y")
+    gx_ref, gp_ref, gabs = oracle.swiglu_clamped_bwd(xb, pb, gyb, L)
+    assert_within_ulp16(bits(gx), gx_ref, 1, what="grad_x")
+    got = bits(gp).ravel()
+    assert_sum_close(got, gp_ref, gabs, 1e-5, "grad_probs")
+    rep = strict_grad_probs_report(got, gp_ref, gabs)
+    print(f"\ngrad_probs strict relative 1e-5, sigma {sigma}: {rep}")
+    # where the row sum does not cancel, the pure relative bound holds almost everywhere
+    assert rep["strict_fail_not_cancelling"] <= rep["rows_not_cancelling"] // 100
     # whole-tensor properties: masks exactly where the inputs leave the range
     gate, up = x[:, :inter], x[:, inter:]
     assert bool((gx[:, :inter][gate > L] == 0).all())
     assert bool((gx[:, inter:][(up > L) | (up < -L)] == 0).all())
-    assert bool(torch.isfinite(y.float()).all()) and bool(torch.isfinite(gp).all())
 
 
 # ------------------------------------------------------- fp16 / fp32 storage
@@ -239,3 +260,74 @@ def test_tma_forward_paths_and_no_device_errors(cuda_device):
             assert_within_ulp16(bits(y), ref, 1, kind="bf16" if dt == torch.bfloat16 else "f16",
                                 what=f"tma fwd {rows}x{inter} {dt}")
     assert _abi.moe_device_errors(clear=True) == 0
+
+
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+def test_tma_forward_bounded_wait_runs_out(cuda_device, dt):
+    """The failure path of the TMA forward's bounded waits: the test hook
+    withholds one row's copy and barrier arrival (nothing ever completes that
+    phase), with a wait limit of 2e5 SM cycles.  The row's consumer gives up,
+    the producer then gives up waiting for that stage, the CTA's other
+    consumers give up on the rows that are never filled, every issued copy is
+    drained, and the kernel returns: the caller's error word holds
+    MOE_DEVERR_TIMEOUT, every row of the other CTAs and every row the stalled
+    CTA reached before the stall is correct, the rows it never reached keep
+    their canary, and the context still runs the normal forward."""
+    from moe_expert_epilogue_b200 import _abi
+    rows, inter, L, grid = 300, 2048, 10.0, 4
+    S, C = 16, 8                                       # stages and consumer warps of the ring
+    k_stall, cta = 20, 1
+    stall_row = cta + k_stall * grid
+    d = inputs.swiglu_inputs(rows, inter, sigma=3.0, seed=41)
+    kind = "bf16" if dt == torch.bfloat16 else "f16"
+    odt = oracle.BF16 if dt == torch.bfloat16 else oracle.F16
+    x, p = d["x"].to(dt), d["probs"]
+    ref = oracle.swiglu_clamped_fwd(bits(x), bits(p), L, odt)
+    canary = 0x7FAB if dt == torch.bfloat16 else 0x7DAB      # a NaN no output takes here
+    xd, pd = x.to(cuda_device), p.to(cuda_device)
+    y = torch.full((rows, inter), canary, dtype=torch.int16, device=cuda_device).view(dt)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    _abi.moe_device_errors(clear=True)
+    _abi.moe_test_swiglu_fwd_stalled(xd, pd, y, rows, inter, L, ops.moe_dtype(dt), grid,
+                                     stall_row, 200_000, err)
+    torch.cuda.synchronize()
+    assert int(err) == _abi.MOE_DEVERR_TIMEOUT
+    got = bits(y)
+    r = np.arange(rows)
+    k = r // grid
+    mine = r % grid == cta
+    written = ~mine | (k < k_stall) | ((k > k_stall) & (k < k_stall + S) & ((k - k_stall) % C != 0))
+    never = mine & ((k == k_stall) | (k >= k_stall + S) | ((k > k_stall) & ((k - k_stall) % C == 0)))
+    assert_within_ulp16(got[written], ref[written], 1, kind=kind, what="rows written")
+    assert (got[never] == canary).all(), "rows the stalled CTA never reached"
+    # rows the surviving consumers may or may not have reached: canary or correct
+    rest = ~written & ~never
+    for i in np.flatnonzero(rest):
+        if not (got[i] == canary).all():
+            assert_within_ulp16(got[i], ref[i], 1, kind=kind, what=f"row {i}")
+    # the per-device word was not touched, and the context still works
+    assert _abi.moe_device_errors(clear=True) == 0
+    err.zero_()
+    y2 = ops.swiglu_clamped_fwd(xd, pd, L, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err) == 0
+    assert_within_ulp16(bits(y2), ref, 1, kind=kind, what="normal forward after the timeout")
+
+
+def test_forward_error_word_variants(cuda_device):
+    """moe_swiglu_clamped_fwd_ex with and without an error word computes the
+    same bits as moe_swiglu_clamped_fwd; no bit is set when nothing times out."""
+    from moe_expert_epilogue_b200 import _abi
+    rows, inter, L = 200, 1024, 7.0
+    d = inputs.swiglu_inputs(rows, inter, sigma=3.0, seed=43)
+    x, p = d["x"].to(cuda_device), d["probs"].to(cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    a = torch.empty(rows, inter, dtype=torch.bfloat16, device=cuda_device)
+    b, c = torch.empty_like(a), torch.empty_like(a)
+    _abi.moe_swiglu_clamped_fwd(x, p, a, rows, inter, 2 * inter, inter, L)
+    _abi.moe_swiglu_clamped_fwd_ex(x, p, b, rows, inter, 2 * inter, inter, L, dev_err=err)
+    _abi.moe_swiglu_clamped_fwd_ex(x, p, c, rows, inter, 2 * inter, inter, L, dev_err=None)
+    torch.cuda.synchronize()
+    assert int(err) == 0 and _abi.moe_device_errors(clear=True) == 0
+    assert_bits_equal(bits(a), bits(b), "fwd vs fwd_ex")
+    assert_bits_equal(bits(a), bits(c), "fwd vs fwd_ex without an error word")
