@@ -439,7 +439,8 @@ def _measure_fused(device, seed, reps, peak, T, K, E, A, H):
 
 # ---------------------------------------------------------------- configurations
 
-CONFIG_ROWS = ("swiglu_small", "router_weight", "residual_add", "unpermute_fp32_out")
+CONFIG_ROWS = ("swiglu_small", "router_weight_variants", "residual_add_variants",
+               "unpermute_fp32_out")
 L2_FLUSH_BYTES = 256 << 20   # twice the 126 MB L2
 
 
@@ -459,10 +460,10 @@ def measure_configs(device, seed, reps, peak, only=None):
     out = {}
     if only in (None, "swiglu_small"):
         out["swiglu_small"] = _measure_swiglu_small(device, seed, max(reps, 50), peak)
-    if only in (None, "router_weight"):
-        out["router_weight"] = _measure_router_variants(device, seed, reps, peak)
-    if only in (None, "residual_add"):
-        out["residual_add"] = _measure_residual_variants(device, seed, reps, peak)
+    if only in (None, "router_weight_variants"):
+        out["router_weight_variants"] = _measure_router_variants(device, seed, reps, peak)
+    if only in (None, "residual_add_variants"):
+        out["residual_add_variants"] = _measure_residual_variants(device, seed, reps, peak)
     if only in (None, "unpermute_fp32_out"):
         out["unpermute_fp32_out"] = _measure_unpermute_fp32(device, seed, reps, peak)
     torch.cuda.empty_cache()
@@ -1051,7 +1052,8 @@ def run_ours(args):
     if collectives is not None:
         line["collectives"] = collectives
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.kernel:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_sample or 0.25, steps=1)
+        # about 12 s of one core: every SwiGLU row, 3 passes (~4 s a pass)
+        line["cpu_baseline"] = cpu_baseline(args.cpu_sample or 1.0, steps=3)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -1207,22 +1209,23 @@ def _time_oracle(frac, steps, whole_pass=False):
 
 def cpu_baseline(frac, steps=1, all_cores=True):
     """The oracle on the host, on the headline's workload: single-threaded on
-    the first `frac` of the SwiGLU rows, and (all_cores) the same fraction
-    split over one process per host core; `step` is the whole pass on one
-    core (the first `frac` of every op's rows)."""
+    the first `frac` of the SwiGLU rows, `steps` passes, and (all_cores) the
+    same fraction split over one process per host core; `step` is the whole
+    pass on one core (the first quarter, at most, of every op's rows)."""
     b, dt, w = _time_oracle(frac, steps)
     out = {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
            "seconds": round(dt, 2), "host_cpu": _cpu_model(), "host_nproc": os.cpu_count(),
            "sample": f"clamped SwiGLU fwd+bwd on the first {w['R']} of the {SWIGLU['rows']} "
-                     f"rows (inter {SWIGLU['inter']}, L {SWIGLU['limit']:g}); single-threaded "
-                     "C oracle, -O2"}
+                     f"rows (inter {SWIGLU['inter']}, L {SWIGLU['limit']:g}), {steps} pass(es); "
+                     "single-threaded C oracle, -O2"}
     del w
     if all_cores and (os.cpu_count() or 1) > 1:
-        out["all_cores"] = oracle_pool(frac, os.cpu_count(), warmup=1, steps=4 * max(1, steps))
-    b, dt, w = _time_oracle(frac, 1, whole_pass=True)
+        out["all_cores"] = oracle_pool(frac, os.cpu_count(), warmup=1, steps=max(1, steps))
+    fs = min(frac, 0.25)
+    b, dt, w = _time_oracle(fs, 1, whole_pass=True)
     out["step"] = {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": 1,
                    "seconds": round(dt, 2),
-                   "sample": f"first {frac:g} of the rows/tokens of every op of the step "
+                   "sample": f"first {fs:g} of the rows/tokens of every op of the step "
                              f"(swiglu rows {w['R']}, router rows {w['Rr']}, tokens {w['T']}, "
                              f"residual rows {w['Rs']}); single-threaded C oracle"}
     return out
@@ -1332,9 +1335,9 @@ def main(argv=None):
                     help="pipelined end-to-end steps (fill and drain of the copy pipeline "
                          "are amortised over them)")
     ap.add_argument("--cpu-sample", type=float, default=None,
-                    help="fraction of the rows of every op the CPU oracle runs (default: "
-                         "0.25 for the cpu_baseline; sized to the step count for the "
-                         "reference arm)")
+                    help="fraction of the SwiGLU rows the CPU oracle runs (default: all of "
+                         "them, 3 passes, for the cpu_baseline; sized to the step count for "
+                         "the reference arm)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")

@@ -15,9 +15,14 @@
 //   out[t, :] = out_dt(acc)
 // -- the bits of the two-step form, with no partial blocks written or read:
 // each partial lives in registers, and the peers' expert rows and
-// inverse-map rows are read once, directly (plain loads; no bulk copies, no
-// multicast).  The kernel never waits on another rank: the caller orders the
-// launch after every rank's expert outputs are complete.
+// inverse-map rows are read once, directly (1-D bulk copies into shared
+// memory in the TMA-staged kernel, plain loads in the register-staged ones;
+// never with multicast).  The kernel never waits on another rank: the caller
+// orders the launch after every rank's expert outputs are complete.
+//
+// Up to 64 (rank, local expert) pairs and rows of a multiple of 8 elements
+// take the TMA-staged kernel (ep_combine_tma, below); otherwise the
+// register-staged ones:
 //
 // One warp per item = (token, 1/split of the row).  For a group of up to 8
 // ranks the warp loads the token's inverse-map rows of all of them at once
@@ -420,7 +425,10 @@ constexpr int kChunkUnits = 512;                    // units per row chunk at mo
 constexpr int kRowBytes = 8192;                     // at most this much of a row per copy
 constexpr int kMaxStages = 32;
 constexpr int kTmaBatches = 2;                      // inverse entries per producer lane
-constexpr size_t kEpcSmemMax = 200 * 1024 / kTmaCtasPerSm;
+#ifndef MOE_EPC_SMEM_KB
+#define MOE_EPC_SMEM_KB 200
+#endif
+constexpr size_t kEpcSmemMax = (size_t)MOE_EPC_SMEM_KB * 1024 / kTmaCtasPerSm;
 
 enum : uint8_t { kFirst = 1, kLast = 2, kDone = 4 };
 
