@@ -217,9 +217,17 @@ swiglu_fwd_tma(const typename D::T* __restrict__ x, const float* __restrict__ pr
 
 // Stages of the TMA ring for rows of `inter` columns of T: 16, or 8 for
 // longer rows, or 0 when even 8 do not fit.
+#ifndef MOE_SWIGLU_FWD_STAGES
+#define MOE_SWIGLU_FWD_STAGES 16
+#endif
+constexpr int kTmaStagesMax = MOE_SWIGLU_FWD_STAGES;   // 16 or 24
+static_assert(kTmaStagesMax == 16 || kTmaStagesMax == 24, "16 or 24 ring stages");
+
 template <class T>
 int tma_stages(int64_t inter) {
   const size_t stage = (size_t)2 * inter * sizeof(T);
+  if (kTmaStagesMax > 16 && kTmaStagesMax * stage + 16 * kTmaStagesMax <= kTmaSmemMax)
+    return kTmaStagesMax;
   return 16 * stage + 256 <= kTmaSmemMax ? 16 : 8 * stage + 128 <= kTmaSmemMax ? 8 : 0;
 }
 
@@ -231,7 +239,9 @@ int launch_fwd_tma(const typename D::T* x, const float* probs, typename D::T* y,
                    cudaStream_t stream) {
   using T = typename D::T;
   const int S = tma_stages<T>(inter);
-  auto k = S == 16 ? swiglu_fwd_tma<D, 16, STALL> : swiglu_fwd_tma<D, 8, STALL>;
+  auto k = S == kTmaStagesMax ? swiglu_fwd_tma<D, kTmaStagesMax, STALL>
+          : S == 16          ? swiglu_fwd_tma<D, 16, STALL>
+                             : swiglu_fwd_tma<D, 8, STALL>;
   const size_t smem = (size_t)S * 2 * inter * sizeof(T) + 2 * (size_t)S * sizeof(uint64_t);
   if (int rc = ensure_smem_limit((const void*)k, kTmaSmemMax)) return rc;
   launch_kernel_block(k, grid, kTmaThreads, smem, stream, x, probs, y, rows, inter, ld_x, ld_y,
