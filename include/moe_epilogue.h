@@ -399,7 +399,10 @@ MOE_API int moe_ordered_reduce_scatter_v(const void* const* buffers, int64_t inp
  * expert_outputs     DEVICE array of `world` pointers (rank order) to each
  *                    rank's expert-grouped rows, eo_dt [max_rows, hidden]
  *                    contiguous, addressable from this GPU (own memory, or a
- *                    peer's mapped with moe_ipc_open); read with plain loads
+ *                    peer's mapped with moe_ipc_open); read with 1-D bulk copies
+ *                    into shared memory (16-byte aligned bases, hidden % 8 == 0,
+ *                    up to 64 (rank, local expert) pairs) or plain loads, never
+ *                    with multicast
  * inverse_maps       DEVICE array of `world` pointers to each rank's int32
  *                    [capacity_rows, num_local_experts] inverse map over the
  *                    token rows of all ranks (row in that rank's expert
