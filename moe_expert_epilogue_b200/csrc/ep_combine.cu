@@ -411,24 +411,16 @@ ep_combine_groups(MOE_EPC_PARAMS) {
 // device; moe_device_errors() reads it with the forward SwiGLU's word).
 __device__ int32_t g_epc_errors;
 
-#ifndef MOE_EPC_UNITS
-#define MOE_EPC_UNITS 1
-#endif
-// Units (8 elements) of a row chunk per consumer thread: 1 -> 16 consumer
-// warps, one CTA per SM; 2 -> 8 consumer warps and two CTAs per SM, each with
-// half the ring.
-constexpr int kUnitsPerThread = MOE_EPC_UNITS;
-constexpr int kTmaWarps = 16 / kUnitsPerThread;     // consumer warps
+constexpr int kTmaWarps = 16;                       // consumer warps
 constexpr int kTmaEpcThreads = 32 * (kTmaWarps + 1);
-constexpr int kTmaCtasPerSm = kUnitsPerThread;
-constexpr int kChunkUnits = 512;                    // units per row chunk at most
+constexpr int kChunkUnits = 32 * kTmaWarps;         // at most one unit per consumer thread
 constexpr int kRowBytes = 8192;                     // at most this much of a row per copy
 constexpr int kMaxStages = 32;
 constexpr int kTmaBatches = 2;                      // inverse entries per producer lane
 #ifndef MOE_EPC_SMEM_KB
 #define MOE_EPC_SMEM_KB 200
 #endif
-constexpr size_t kEpcSmemMax = (size_t)MOE_EPC_SMEM_KB * 1024 / kTmaCtasPerSm;
+constexpr size_t kEpcSmemMax = (size_t)MOE_EPC_SMEM_KB * 1024;
 
 enum : uint8_t { kFirst = 1, kLast = 2, kDone = 4 };
 
@@ -522,7 +514,7 @@ __device__ __forceinline__ void close_rank(float (&part)[kVec], float (&acc)[kVe
 }
 
 template <class DI, class DP, class DO, int R>
-__global__ void __launch_bounds__(kTmaEpcThreads, kTmaCtasPerSm)
+__global__ void __launch_bounds__(kTmaEpcThreads, 1)
 ep_combine_tma(const void* const* __restrict__ eo_tab, const void* const* __restrict__ inv_tab,
                int world, int rank, const int32_t* __restrict__ offs,
                const int32_t* __restrict__ ep_tokens, int64_t capacity, int64_t max_rows, int E,
@@ -672,14 +664,11 @@ ep_combine_tma(const void* const* __restrict__ eo_tab, const void* const* __rest
     return;
   }
 
-  // consumers: thread u folds units u, u + 32 * kTmaWarps, ... of every row of
-  // a stage as it lands
-  constexpr int U = kUnitsPerThread;
-  constexpr int kStride = 32 * kTmaWarps;
-  const int u0 = threadIdx.x - 32;
+  // consumers: thread u folds unit u of every row of a stage as it lands
+  const int u = threadIdx.x - 32;
   const int64_t width0 = hidden < chunk ? hidden : chunk;
-  const bool act_any = (int64_t)u0 * kVec < width0;
-  float acc[U][kVec] = {}, part[U][kVec] = {};
+  const bool act_any = (int64_t)u * kVec < width0;
+  float acc[kVec] = {}, part[kVec] = {};
   int n = 0;                                           // rows in the open partial
   int s = 0;
   uint32_t phase = 0;
@@ -694,58 +683,41 @@ ep_combine_tma(const void* const* __restrict__ eo_tab, const void* const* __rest
     if (flags & kDone) return;
     if (act_any) {
       const int64_t col = h.col;
-      const int64_t width = hidden - col < chunk ? hidden - col : chunk;
       if (flags & kFirst) {                            // a new item: -0 sum, +0 partial
 #pragma unroll
-        for (int x = 0; x < U; ++x)
-#pragma unroll
-          for (int i = 0; i < kVec; ++i) {
-            acc[x][i] = -0.0f;
-            part[x][i] = 0.0f;
-          }
+        for (int i = 0; i < kVec; ++i) {
+          acc[i] = -0.0f;
+          part[i] = 0.0f;
+        }
         n = 0;
       }
+      const bool mine = (int64_t)u * kVec < (hidden - col < chunk ? hidden - col : chunk);
       const int nr = h.rows;
       uint64_t gaps = h.gaps;
       const TI* st = reinterpret_cast<const TI*>(smem + (size_t)s * stage_bytes) +
-                     (size_t)u0 * kVec;
-      bool mine[U];
-      Raw8<DI> raw[R][U];
-#pragma unroll
-      for (int x = 0; x < U; ++x) mine[x] = (int64_t)(u0 + x * kStride) * kVec < width;
+                     (size_t)u * kVec;
+      Raw8<DI> raw[R];
 #pragma unroll
       for (int i = 0; i < R; ++i)
-#pragma unroll
-        for (int x = 0; x < U; ++x)
-          if (i < nr && mine[x])
-            raw[i][x] = tma::lds8<DI>(st + (size_t)i * chunk + (size_t)x * kStride * kVec);
+        if (i < nr && mine) raw[i] = tma::lds8<DI>(st + (size_t)i * chunk);
 #pragma unroll
       for (int i = 0; i < R; ++i) {
         if (i < nr) {
           const int g = (int)(gaps & 0xffu);
           gaps >>= 8;
           if (g > 0) {                                 // the row opens a rank
-#pragma unroll
-            for (int x = 0; x < U; ++x) {
-              close_rank<DP>(part[x], acc[x], n, g > 1);
-              fold_row<DI, true>(part[x], raw[i][x]);
-            }
+            close_rank<DP>(part, acc, n, g > 1);
+            fold_row<DI, true>(part, raw[i]);
             n = 1;
           } else {
-#pragma unroll
-            for (int x = 0; x < U; ++x) fold_row<DI, false>(part[x], raw[i][x]);
+            fold_row<DI, false>(part, raw[i]);
             ++n;
           }
         }
       }
       if (flags & kLast) {
-        const int g = h.trailing;                      // >= 1: the open rank, then empties
-#pragma unroll
-        for (int x = 0; x < U; ++x) {
-          close_rank<DP>(part[x], acc[x], n, g > 1);
-          if (mine[x])
-            store8<DO>(out + h.t * hidden + col + (int64_t)(u0 + x * kStride) * kVec, acc[x]);
-        }
+        close_rank<DP>(part, acc, n, h.trailing > 1);  // the open rank, then empties
+        if (mine) store8<DO>(out + h.t * hidden + col + (int64_t)u * kVec, acc);
       }
     }
     __syncwarp();                                      // the warp has read the stage
@@ -790,8 +762,7 @@ int launch_tma(const void* const* eos, const void* const* invs, int world, int r
   int sms = 0;
   if (int rc = device_sm_count(&sms)) return rc;
   const int64_t items = local * ((hidden + chunk - 1) / chunk);
-  const int64_t ctas = (int64_t)sms * kTmaCtasPerSm;
-  const int grid = (int)(items < ctas ? items : ctas);
+  const int grid = (int)(items < sms ? items : sms);
   launch_kernel_block(k, grid, kTmaEpcThreads, smem, stream, eos, invs, world, rank, offs,
                       ep_tokens, capacity, max_rows, E, static_cast<typename DO::T*>(out), local,
                       hidden, chunk, stages, err);
