@@ -9,11 +9,21 @@
 //
 // p = probs[permutation_map[r]].  Rows r < *n_used with a negative map entry
 // are alignment padding: zero-filled when zero_padding is set, otherwise not
-// touched.  Rows r >= *n_used are neither read nor written.  The kernel is a
-// fixed persistent grid whose warps stride over rows up to the
+// touched.  Rows r >= *n_used are neither read nor written.  Both kernels are
+// fixed grids (sized from max_rows) that stride over the rows up to the
 // device-resident bound, so a captured graph stays valid as n_used changes,
 // and every output element is computed by the same instruction sequence
 // whatever the grid (batch invariance).
+//
+// Rows of a multiple of 16 columns with 32-byte aligned bases take the flat
+// kernel: one 32-byte chunk per thread per step, grid-strided in row-major
+// order over all live rows, 4 CTAs per SM.  Measured on B200 at 8192 tokens x
+// top-8, width 1536, against one warp per row at full occupancy: 70.6 against
+// 75.0 us (SQRELU), 72.3 against 75.1 (SQRELU_CLAMP), 101.6 against 106.1
+// (SWIGLU), bit-identical outputs.  A streaming copy behaves the same way: each
+// load instruction of the grid covering one contiguous window, with few CTAs,
+// beats many warps each on its own row.  Other layouts take the warp-per-row
+// kernel.
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -50,10 +60,89 @@ __device__ __forceinline__ int64_t live_rows(const int32_t* n_used, int64_t max_
   return n;
 }
 
-// One warp owns one row at a time (warps stride over rows up to the
-// device-resident bound); lanes take 8-column chunks lane, lane + 32, ...
-// The next row's map entry is fetched while the current row streams, so the
-// row's data loads never wait on the map lookup.
+// Eight elements of one 16-byte chunk: a (and, for SWIGLU, the matching up
+// chunk b) in, eight bf16 results packed out.
+template <int ACT>
+__device__ __forceinline__ uint4 act8(const uint4& a, const uint4& b, float p, float scale,
+                                     float inv_scale) {
+  float av[8], o[8];
+  unpack_bf16x8(a, av);
+  if constexpr (ACT == MOE_ACT_SQRELU) {
+    // the squares are rounded to bf16 two at a time (packed conversion), then
+    // widened back for the fp32 probability multiply
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const float r0 = av[i] < 0.0f ? 0.0f : av[i];
+      const float r1 = av[i + 1] < 0.0f ? 0.0f : av[i + 1];
+      const uint32_t sq = pack_bf16x2(r0 * r0, r1 * r1);
+      o[i] = bf16_lo(sq) * p;
+      o[i + 1] = bf16_hi(sq) * p;
+    }
+  } else {
+    float bv[8];
+    if constexpr (ACT == MOE_ACT_SWIGLU) unpack_bf16x8(b, bv);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      o[i] = act_one<ACT>(av[i], ACT == MOE_ACT_SWIGLU ? bv[i] : 0.0f, p, scale, inv_scale);
+  }
+  return make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                    pack_bf16x2(o[6], o[7]));
+}
+
+// Flat kernel: threads stride over the (row, 16-column chunk) pairs of the
+// live rows in row-major order, so each load instruction of the whole grid
+// covers one contiguous window of the input.  The (row, chunk) cursor
+// advances by the grid stride without a division, and the map entry of the
+// next step's row is fetched a step ahead, so the data load never waits on it.
+template <int ACT>
+__global__ void __launch_bounds__(kThreads)
+act_flat_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ out,
+                const int32_t* __restrict__ pmap, const int32_t* __restrict__ n_used,
+                const float* __restrict__ probs, int64_t num_probs, int64_t max_rows,
+                int64_t width, float scale, int zero_padding, int32_t* err) {
+  constexpr int64_t CH = 16;                             // elements per chunk (32 bytes)
+  pdl_prologue();
+  const int64_t rows = live_rows(n_used, max_rows, err);
+  const float inv_scale = 1.0f / scale;
+  const int64_t upr = width / CH;                        // chunks per row
+  const int64_t in_w = ACT == MOE_ACT_SWIGLU ? 2 * width : width;
+  const int64_t total = rows * upr;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (i >= total) return;
+  RowCursor cur(i, stride, upr);
+  int32_t m_next = __ldg(pmap + cur.r);
+  for (; i < total; i += stride) {
+    const int64_t r = cur.r, c = cur.c;
+    const int32_t m = m_next;
+    cur.advance();
+    if (i + stride < total) m_next = __ldg(pmap + cur.r);
+    uint16_t* op = out + r * width + c * CH;
+    if (m < 0) {                                         // alignment padding row
+      if (zero_padding) {
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        st_stream32(op, z, z);
+      }
+      continue;
+    }
+    if (m >= num_probs) {
+      if (c == 0) flag_error(err, MOE_DEVERR_MAP);
+      continue;
+    }
+    const uint16_t* xp = x + r * in_w + c * CH;
+    const u4x2 a = ld_stream32(xp);
+    u4x2 b;
+    if constexpr (ACT == MOE_ACT_SWIGLU) b = ld_stream32(xp + width);
+    const float p = __ldg(probs + m);
+    st_stream32(op, act8<ACT>(a.lo, b.lo, p, scale, inv_scale),
+                act8<ACT>(a.hi, b.hi, p, scale, inv_scale));
+  }
+}
+
+// Warp-per-row kernel (other layouts): one warp owns one row at a time (warps
+// stride over rows up to the device-resident bound); lanes take 8-column
+// chunks lane, lane + 32, ...  The next row's map entry is fetched while the
+// current row streams, so the row's data loads never wait on the map lookup.
 #ifndef MOE_ACT_MIN_BLOCKS
 #define MOE_ACT_MIN_BLOCKS 0
 #endif
@@ -119,27 +208,7 @@ act_permuted_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ out,
         const int64_t c = c0 + 32 * k;
         if (c < upr) {
           if constexpr (VEC) {
-            float av[8], bv[8], o[8];
-            unpack_bf16x8(a[k], av);
-            if constexpr (ACT == MOE_ACT_SWIGLU) unpack_bf16x8(b[k], bv);
-            if constexpr (ACT == MOE_ACT_SQRELU) {
-              // the squares are rounded to bf16 two at a time (packed conversion),
-              // then widened back for the fp32 probability multiply
-#pragma unroll
-              for (int i = 0; i < 8; i += 2) {
-                const float r0 = av[i] < 0.0f ? 0.0f : av[i];
-                const float r1 = av[i + 1] < 0.0f ? 0.0f : av[i + 1];
-                const uint32_t sq = pack_bf16x2(r0 * r0, r1 * r1);
-                o[i] = bf16_lo(sq) * p;
-                o[i + 1] = bf16_hi(sq) * p;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                o[i] = act_one<ACT>(av[i], ACT == MOE_ACT_SWIGLU ? bv[i] : 0.0f, p, scale,
-                                   inv_scale);
-            }
-            store8<BF16>(orow + c * kVec, o);
+            st_stream(orow + c * kVec, act8<ACT>(a[k], b[k], p, scale, inv_scale));
           } else {
             const float av = __uint_as_float(a[k].x << 16);
             const float bv = ACT == MOE_ACT_SWIGLU ? __uint_as_float(b[k].x << 16) : 0.0f;
@@ -151,8 +220,31 @@ act_permuted_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ out,
   }
 }
 
-// Chunks per lane loaded ahead: 6 single-stream loads, or 3 chunks of the
-// two-stream SwiGLU input.
+// CTAs per SM of the flat kernel (measured at 1 / 2 / 3 / 4 / 6: 4 best; 2
+// chunks per thread at 2 / 3 / 4 CTAs per SM were not faster).
+#ifndef MOE_ACT_FLAT_CTAS
+#define MOE_ACT_FLAT_CTAS 4
+#endif
+
+template <int ACT>
+int launch_act_flat(const uint16_t* x, uint16_t* out, const int32_t* pmap, const int32_t* n_used,
+                    const float* probs, int64_t num_probs, int64_t max_rows, int64_t width,
+                    float scale, int zero_padding, int32_t* err, cudaStream_t stream) {
+  auto k = act_flat_kernel<ACT>;
+  int sms = 0, resident = 0;
+  if (int rc = device_sm_count(&sms)) return rc;
+  if (int rc = persistent_grid((const void*)k, 0, INT64_MAX, &resident)) return rc;
+  const int64_t useful = (max_rows * (width / 16) + kThreads - 1) / kThreads;
+  int64_t g = (int64_t)sms * MOE_ACT_FLAT_CTAS;
+  if (resident < g) g = resident;
+  if (useful < g) g = useful;
+  launch_kernel(k, (int)(g < 1 ? 1 : g), 0, stream, x, out, pmap, n_used, probs, num_probs,
+                max_rows, width, scale, zero_padding, err);
+  return check_launch();
+}
+
+// Chunks per lane loaded ahead in the warp-per-row kernel: 6 single-stream
+// loads, or 3 chunks of the two-stream SwiGLU input.
 #ifndef MOE_ACT_LOADS_AHEAD
 #define MOE_ACT_LOADS_AHEAD 6
 #endif
@@ -181,20 +273,22 @@ int launch_act_with_probs_permuted(moe_act act, const uint16_t* x, uint16_t* out
                                    const float* probs, int64_t num_probs, int64_t max_rows,
                                    int64_t width, float clamp_scale, int zero_padding,
                                    int32_t* dev_err, cudaStream_t stream) {
+  const bool flat = width % 16 == 0 && aligned32(x) && aligned32(out);
   const bool vec = width % kVec == 0 && aligned16(x) && aligned16(out);
 #define MOE_ACT_ARGS x, out, permutation_map, n_used, probs, num_probs, max_rows, width, \
                      clamp_scale, zero_padding, dev_err, stream
+#define MOE_ACT_PICK(A)                                                       \
+  (flat ? launch_act_flat<A>(MOE_ACT_ARGS)                                    \
+   : vec ? launch_act<A, true>(MOE_ACT_ARGS) : launch_act<A, false>(MOE_ACT_ARGS))
   switch (act) {
     case MOE_ACT_SQRELU:
-      return vec ? launch_act<MOE_ACT_SQRELU, true>(MOE_ACT_ARGS)
-                 : launch_act<MOE_ACT_SQRELU, false>(MOE_ACT_ARGS);
+      return MOE_ACT_PICK(MOE_ACT_SQRELU);
     case MOE_ACT_SQRELU_CLAMP:
-      return vec ? launch_act<MOE_ACT_SQRELU_CLAMP, true>(MOE_ACT_ARGS)
-                 : launch_act<MOE_ACT_SQRELU_CLAMP, false>(MOE_ACT_ARGS);
+      return MOE_ACT_PICK(MOE_ACT_SQRELU_CLAMP);
     default:
-      return vec ? launch_act<MOE_ACT_SWIGLU, true>(MOE_ACT_ARGS)
-                 : launch_act<MOE_ACT_SWIGLU, false>(MOE_ACT_ARGS);
+      return MOE_ACT_PICK(MOE_ACT_SWIGLU);
   }
+#undef MOE_ACT_PICK
 #undef MOE_ACT_ARGS
 }
 

@@ -45,6 +45,18 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return v;
 }
 
+// 32-byte form of ld_stream (sm_100 256-bit global access): one instruction
+// per lane moves two 16-byte chunks.  The address must be 32-byte aligned.
+struct u4x2 { uint4 lo, hi; };
+__device__ __forceinline__ u4x2 ld_stream32(const void* p) {
+  u4x2 v;
+  asm("ld.global.nc.L1::no_allocate.L2::256B.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(v.lo.x), "=r"(v.lo.y), "=r"(v.lo.z), "=r"(v.lo.w),
+        "=r"(v.hi.x), "=r"(v.hi.y), "=r"(v.hi.z), "=r"(v.hi.w)
+      : "l"(p));
+  return v;
+}
+
 // 16-byte coherent load, no L1 allocation: for data that the same kernel
 // also writes (the in-place residual add).
 __device__ __forceinline__ uint4 ld_coherent(const void* p) {
@@ -70,6 +82,14 @@ __device__ __forceinline__ void st_stream(void* p, uint4 v) {
   asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};"
 #endif
                ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// 32-byte store, no L1 allocation; the address must be 32-byte aligned.
+__device__ __forceinline__ void st_stream32(void* p, const uint4& lo, const uint4& hi) {
+  asm volatile("st.global.L1::no_allocate.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+               ::"l"(p), "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w),
+                 "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
                : "memory");
 }
 
@@ -198,6 +218,17 @@ template <> __device__ __forceinline__ void widen8<F32>(const Raw8<F32>& r, floa
   v[2] = __uint_as_float(r.w[0].z); v[3] = __uint_as_float(r.w[0].w);
   v[4] = __uint_as_float(r.w[1].x); v[5] = __uint_as_float(r.w[1].y);
   v[6] = __uint_as_float(r.w[1].z); v[7] = __uint_as_float(r.w[1].w);
+}
+
+// Round 8 fp32 values to a 16-bit storage dtype (RNE), packed into 16 bytes.
+template <class D> __device__ __forceinline__ uint4 pack8(const float (&v)[8]);
+template <> __device__ __forceinline__ uint4 pack8<BF16>(const float (&v)[8]) {
+  return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                    pack_bf16x2(v[6], v[7]));
+}
+template <> __device__ __forceinline__ uint4 pack8<F16>(const float (&v)[8]) {
+  return make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]),
+                    pack_f16x2(v[6], v[7]));
 }
 
 // Round 8 fp32 values to the storage dtype (RNE) and store them.

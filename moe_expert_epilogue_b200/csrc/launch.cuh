@@ -53,6 +53,7 @@ int device_sm_count(int* sms);
 int ensure_smem_limit(const void* kernel, size_t smem);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // Launchers (one per op family); arguments already validated.
 int launch_swiglu_clamped_fwd(const void* x, const float* probs, void* y, int64_t rows,

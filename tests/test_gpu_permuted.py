@@ -76,6 +76,76 @@ def test_act_permuted_full_workload_whole_tensor(cuda_device, act, oact, tol):
     assert (got[:rt.n_used][pm[:rt.n_used] < 0] == 0).all()
 
 
+def _placed(t, dev, offset_elems):
+    """t copied to the device at an element offset inside a larger buffer."""
+    flat = torch.empty(t.numel() + offset_elems, dtype=t.dtype, device=dev)
+    v = flat[offset_elems:].view(t.shape)
+    v.copy_(t.to(dev))
+    return v
+
+
+# (width, x offset, out offset) in elements: the flat 32-byte kernel (width a
+# multiple of 16, both bases 32-byte aligned), the warp-per-row 16-byte kernel
+# (width 8 mod 16, or a base only 16-byte aligned) and the per-element kernel
+# (a base off 16-byte alignment).
+LAYOUTS = [(1536, 0, 0), (48, 0, 0), (16, 0, 0), (1544, 0, 0), (1536, 8, 0), (1536, 0, 8),
+           (1536, 1, 0)]
+
+
+@pytest.mark.parametrize("act,oact,tol", ACTS)
+@pytest.mark.parametrize("zero_padding", [False, True])
+@pytest.mark.parametrize("width,x_off,out_off", LAYOUTS)
+def test_act_permuted_layouts(cuda_device, act, oact, tol, zero_padding, width, x_off, out_off):
+    """Every kernel the layout selects, on a ragged routing (300 tokens, top-3 of
+    7 experts, rows padded to 16) with the live-row bound cut short, against
+    the oracle; untouched rows keep their canary."""
+    rt = inputs.routing(300, 3, 7, 16, seed=width + x_off)
+    n_used = rt.n_used - 5
+    x = inputs.permuted_activation_input(rt, width, swiglu=(oact == oracle.SWIGLU), seed=width)
+    canary = torch.full((rt.max_rows, width), CANARY, dtype=torch.int16).view(torch.bfloat16)
+    out = _placed(canary, cuda_device, out_off)
+    ops.act_with_probs_permuted(act, _placed(x, cuda_device, x_off),
+                                rt.permutation_map.to(cuda_device),
+                                torch.tensor([n_used], dtype=torch.int32, device=cuda_device),
+                                rt.probs.to(cuda_device), 7.0, zero_padding, out=out)
+    torch.cuda.synchronize()
+    ref, err = oracle.act_with_probs_permuted(oact, bits(x), bits(canary),
+                                              bits(rt.permutation_map), n_used, bits(rt.probs),
+                                              width, 7.0, zero_padding)
+    assert err == 0
+    got = bits(out)
+    if tol == 0:
+        assert_bits_equal(got, ref, "act")
+    else:
+        assert_within_ulp16(got, ref, tol, what="act")
+    assert (got[n_used:] == CANARY).all()
+
+
+@pytest.mark.parametrize("act", [a for a, _, _ in ACTS])
+def test_act_permuted_flat_kernel_batch_invariant(cuda_device, act):
+    """The flat kernel's grid and stride follow max_rows: the same live rows in
+    a buffer of 3x the rows (123 against 369 CTAs, so every chunk falls at
+    another stride phase) give the same bits."""
+    rt = inputs.routing(100, 2, 8, 16, seed=11)
+    width = 1536
+    x = inputs.permuted_activation_input(rt, width, swiglu=act == _abi.MOE_ACT_SWIGLU, seed=12)
+    small = _run_act(cuda_device, act, rt, x, width, 7.0, True)
+    R = rt.max_rows
+    big_x = torch.zeros((3 * R,) + tuple(x.shape[1:]), dtype=x.dtype)
+    big_x[:R] = x
+    big_pm = torch.full((3 * R,), -1, dtype=torch.int32)
+    big_pm[:R] = rt.permutation_map
+    out = torch.full((3 * R, width), CANARY, dtype=torch.int16, device=cuda_device) \
+        .view(torch.bfloat16)
+    ops.act_with_probs_permuted(act, big_x.to(cuda_device), big_pm.to(cuda_device),
+                                torch.tensor([rt.n_used], dtype=torch.int32, device=cuda_device),
+                                rt.probs.to(cuda_device), 7.0, True, out=out)
+    torch.cuda.synchronize()
+    got = bits(out)
+    assert_bits_equal(got[:R], small, "same rows, larger buffer")
+    assert (got[R:] == CANARY).all()
+
+
 def test_act_permuted_bad_metadata_sets_error_bits(cuda_device):
     rt = inputs.routing(40, 2, 4, 8, seed=3)
     width = 16
