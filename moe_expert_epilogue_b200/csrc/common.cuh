@@ -57,6 +57,17 @@ __device__ __forceinline__ u4x2 ld_stream32(const void* p) {
   return v;
 }
 
+// 32-byte form of ld_coherent; the address must be 32-byte aligned.
+__device__ __forceinline__ u4x2 ld_coherent32(const void* p) {
+  u4x2 v;
+  asm volatile("ld.global.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v.lo.x), "=r"(v.lo.y), "=r"(v.lo.z), "=r"(v.lo.w),
+                 "=r"(v.hi.x), "=r"(v.hi.y), "=r"(v.hi.z), "=r"(v.hi.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
 // 16-byte coherent load, no L1 allocation: for data that the same kernel
 // also writes (the in-place residual add).
 __device__ __forceinline__ uint4 ld_coherent(const void* p) {

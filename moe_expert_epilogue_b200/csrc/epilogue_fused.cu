@@ -18,10 +18,11 @@
 // rounded multiply (__fmul_rn), so it is never fused into the step-2 add, for
 // fp32 as for the 16-bit types.
 //
-// Structure: the unpermute's -- one CTA per token at a time, row lists
-// compacted one token ahead by warp 0, one barrier per token; each thread
-// gathers up to 8 rows of an 8-column chunk (and the rows' probabilities,
-// which stay in L1) with the shared and residual chunks in flight beside them.
+// Structure: the unpermute's -- a warp per (token, column range) with its own
+// row list for E <= 64 (below), else one CTA per token at a time with row
+// lists compacted one token ahead by warp 0 and one barrier per token; each
+// thread gathers the rows of its chunk (and the rows' probabilities, which
+// stay in L1) with the shared and residual chunks in flight beside them.
 #include "common.cuh"
 #include "launch.cuh"
 #include "rowlist.cuh"
@@ -140,15 +141,30 @@ epilogue_fused_kernel(const typename D::T* __restrict__ eo, const float* __restr
 // already loaded during the previous item) into its own shared-memory list,
 // so warps never wait for each other; items = tokens * SPLIT keep the load
 // balanced across the persistent grid.
-// More resident warps hide the gather latency better than more rows in flight
-// per warp: 4 rows at 4 CTAs per SM (64 registers) for the 16-bit types,
-// measured 122.5 us against 127.6 (8 rows, 3 CTAs) and 138 (8 rows, the
-// compiler's 102 registers, 2 CTAs) at 8192 tokens x top-8, hidden 4096; fp32
-// keeps 3 CTAs (4 would spill).
+// CH is the columns per lane per load.  With 16-byte loads (CH = 8) more
+// resident warps hide the gather latency better than more rows in flight per
+// warp: 4 rows at 4 CTAs per SM (64 registers) for the 16-bit types, measured
+// 122.5 us against 127.6 (8 rows, 3 CTAs) and 138 (8 rows, the compiler's 102
+// registers, 2 CTAs) at 8192 tokens x top-8, hidden 4096; fp32 keeps 3 CTAs (4
+// would spill).  16-bit types with hidden % 16 == 0 and 32-byte aligned bases
+// take 32-byte loads (CH = 16): 4 rows in flight at 2 CTAs per SM, 119.5 us
+// against 122.6 on the same shape, bit-identical (2 rows at 3 CTAs: 124.1).
 template <class D> constexpr int kFusedMinBlocks = D::kBytes == 4 ? 3 : 4;
+#ifndef MOE_FUSED_WIDE
+#define MOE_FUSED_WIDE 1
+#endif
+#ifndef MOE_FUSED_WIDE_ROWS
+#define MOE_FUSED_WIDE_ROWS 4
+#endif
+#ifndef MOE_FUSED_WIDE_MIN_BLOCKS
+#define MOE_FUSED_WIDE_MIN_BLOCKS 2
+#endif
+#ifndef MOE_FUSED_WIDE_ROUNDS
+#define MOE_FUSED_WIDE_ROUNDS 4
+#endif
 
-template <class D, int SPLIT>
-__global__ void __launch_bounds__(kThreads, kFusedMinBlocks<D>)
+template <class D, int SPLIT, int CH>
+__global__ void __launch_bounds__(kThreads, CH == 16 ? MOE_FUSED_WIDE_MIN_BLOCKS : kFusedMinBlocks<D>)
 epilogue_fused_warp(const typename D::T* __restrict__ eo, const float* __restrict__ row_probs,
                     int64_t max_rows, const int32_t* __restrict__ inv,
                     const int32_t* __restrict__ valid_tokens,
@@ -164,7 +180,7 @@ epilogue_fused_warp(const typename D::T* __restrict__ eo, const float* __restric
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
   const int64_t items = n * SPLIT;
-  const int64_t cpr = hidden / kVec;
+  const int64_t cpr = hidden / CH;
   const int64_t cpi = (cpr + SPLIT - 1) / SPLIT;          // chunks per item
   int32_t* list = s_list[warp];
   int64_t it = (int64_t)blockIdx.x * (kThreads / 32) + warp;
@@ -176,6 +192,7 @@ epilogue_fused_warp(const typename D::T* __restrict__ eo, const float* __restric
     p1 = lane + 32 < E ? __ldg(row + lane + 32) : -1;
   }
   constexpr int B = kRowsAhead<D>;
+  constexpr int WB = MOE_FUSED_WIDE_ROWS;
   for (; it < items; it += nwarps) {
     const int64_t t = it / SPLIT;
     __syncwarp();                                          // the previous list is consumed
@@ -190,49 +207,109 @@ epilogue_fused_warp(const typename D::T* __restrict__ eo, const float* __restric
     const int64_t base = t * hidden;
     const int64_t c_end = min(cpr, (it % SPLIT + 1) * cpi);
     for (int64_t c = (it % SPLIT) * cpi + lane; c < c_end; c += 32) {
-      const Raw8<D> rs = load8<D>(shared + base + c * kVec);
-      const Raw8<D> rr = load8<D, false>(residual + base + c * kVec);  // may alias out
-      float acc[8];
+      if constexpr (CH == 8) {
+        const Raw8<D> rs = load8<D>(shared + base + c * kVec);
+        const Raw8<D> rr = load8<D, false>(residual + base + c * kVec);  // may alias out
+        float acc[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-      for (int j0 = 0; j0 < count; j0 += B) {
-        Raw8<D> raw[B];
-        float p[B];
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        for (int j0 = 0; j0 < count; j0 += B) {
+          Raw8<D> raw[B];
+          float p[B];
 #pragma unroll
-        for (int j = 0; j < B; ++j) {
-          if (j0 + j < count) {
-            const int64_t row = list[j0 + j];
-            raw[j] = load8<D>(eo + row * hidden + c * kVec);
-            p[j] = __ldg(row_probs + row);
+          for (int j = 0; j < B; ++j) {
+            if (j0 + j < count) {
+              const int64_t row = list[j0 + j];
+              raw[j] = load8<D>(eo + row * hidden + c * kVec);
+              p[j] = __ldg(row_probs + row);
+            }
           }
-        }
 #pragma unroll
-        for (int j = 0; j < B; ++j) {
-          if (j0 + j < count) {
-            float v[8];
-            widen8<D>(raw[j], v);
+          for (int j = 0; j < B; ++j) {
+            if (j0 + j < count) {
+              float v[8];
+              widen8<D>(raw[j], v);
 #pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-              float w0 = __fmul_rn(v[i], p[j]), w1 = __fmul_rn(v[i + 1], p[j]);
-              round2<D>(w0, w1);
-              acc[i] = acc[i] + w0;
-              acc[i + 1] = acc[i + 1] + w1;
+              for (int i = 0; i < 8; i += 2) {
+                float w0 = __fmul_rn(v[i], p[j]), w1 = __fmul_rn(v[i + 1], p[j]);
+                round2<D>(w0, w1);
+                acc[i] = acc[i] + w0;
+                acc[i + 1] = acc[i + 1] + w1;
+              }
             }
           }
         }
-      }
-      float vs[8], vr[8];
-      widen8<D>(rs, vs);
-      widen8<D>(rr, vr);
+        float vs[8], vr[8];
+        widen8<D>(rs, vs);
+        widen8<D>(rr, vr);
 #pragma unroll
-      for (int i = 0; i < 8; i += 2) {
-        round2<D>(acc[i], acc[i + 1]);
-        float t0 = acc[i] + vs[i], t1 = acc[i + 1] + vs[i + 1];
-        round2<D>(t0, t1);
-        acc[i] = vr[i] + t0;
-        acc[i + 1] = vr[i + 1] + t1;
+        for (int i = 0; i < 8; i += 2) {
+          round2<D>(acc[i], acc[i + 1]);
+          float t0 = acc[i] + vs[i], t1 = acc[i + 1] + vs[i + 1];
+          round2<D>(t0, t1);
+          acc[i] = vr[i] + t0;
+          acc[i + 1] = vr[i + 1] + t1;
+        }
+        store8<D>(out + base + c * kVec, acc);
+      } else {
+        // 16 columns per lane: 32-byte loads and store (16-bit types)
+        const u4x2 rs = ld_stream32(shared + base + c * 16);
+        const u4x2 rr = ld_coherent32(residual + base + c * 16);   // may alias out
+        float acc[2][8];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[h][i] = 0.0f;
+        for (int j0 = 0; j0 < count; j0 += WB) {
+          u4x2 raw[WB];
+          float p[WB];
+#pragma unroll
+          for (int j = 0; j < WB; ++j) {
+            if (j0 + j < count) {
+              const int64_t row = list[j0 + j];
+              raw[j] = ld_stream32(eo + row * hidden + c * 16);
+              p[j] = __ldg(row_probs + row);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < WB; ++j) {
+            if (j0 + j < count) {
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                Raw8<D> r8;
+                r8.w[0] = h ? raw[j].hi : raw[j].lo;
+                float v[8];
+                widen8<D>(r8, v);
+#pragma unroll
+                for (int i = 0; i < 8; i += 2) {
+                  float w0 = __fmul_rn(v[i], p[j]), w1 = __fmul_rn(v[i + 1], p[j]);
+                  round2<D>(w0, w1);
+                  acc[h][i] = acc[h][i] + w0;
+                  acc[h][i + 1] = acc[h][i + 1] + w1;
+                }
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          Raw8<D> s8, r8;
+          s8.w[0] = h ? rs.hi : rs.lo;
+          r8.w[0] = h ? rr.hi : rr.lo;
+          float vs[8], vr[8];
+          widen8<D>(s8, vs);
+          widen8<D>(r8, vr);
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            round2<D>(acc[h][i], acc[h][i + 1]);
+            float t0 = acc[h][i] + vs[i], t1 = acc[h][i + 1] + vs[i + 1];
+            round2<D>(t0, t1);
+            acc[h][i] = vr[i] + t0;
+            acc[h][i + 1] = vr[i + 1] + t1;
+          }
+        }
+        st_stream32(out + base + c * 16, pack8<D>(acc[0]), pack8<D>(acc[1]));
       }
-      store8<D>(out + base + c * kVec, acc);
     }
   }
 }
@@ -241,6 +318,12 @@ epilogue_fused_warp(const typename D::T* __restrict__ eo, const float* __restric
 #define MOE_FUSED_WARP_ITEMS 1
 #endif
 
+template <class D, int CH>
+auto fused_warp_for(int split) {
+  return split == 8 ? epilogue_fused_warp<D, 8, CH> : split == 4 ? epilogue_fused_warp<D, 4, CH>
+       : split == 2 ? epilogue_fused_warp<D, 2, CH> : epilogue_fused_warp<D, 1, CH>;
+}
+
 template <class D>
 int launch(const void* eo, const float* row_probs, int64_t max_rows, const int32_t* inv,
            const int32_t* valid_tokens, const void* shared, const void* residual, void* out,
@@ -248,12 +331,17 @@ int launch(const void* eo, const float* row_probs, int64_t max_rows, const int32
   using T = typename D::T;
   const bool vec = hidden % kVec == 0 && aligned16(eo) && aligned16(shared) &&
                    aligned16(residual) && aligned16(out);
+  bool wide = false;
+  if constexpr (D::kBytes == 2)
+    wide = MOE_FUSED_WIDE && hidden % 16 == 0 && aligned32(eo) && aligned32(shared) &&
+           aligned32(residual) && aligned32(out);
   if (MOE_FUSED_WARP_ITEMS && vec && E <= 64) {
-    // SPLIT: items per token, the largest power of two <= chunks per row / 128
-    const int64_t cpr = hidden / kVec;
-    const int split = cpr >= 1024 ? 8 : cpr >= 512 ? 4 : cpr >= 256 ? 2 : 1;
-    auto k = split == 8 ? epilogue_fused_warp<D, 8> : split == 4 ? epilogue_fused_warp<D, 4>
-           : split == 2 ? epilogue_fused_warp<D, 2> : epilogue_fused_warp<D, 1>;
+    // SPLIT: items per token, the largest power of two <= chunks per row / (32 x rounds)
+    const int64_t per = wide ? hidden / 16 / (32 * MOE_FUSED_WIDE_ROUNDS) : hidden / kVec / 128;
+    const int split = per >= 8 ? 8 : per >= 4 ? 4 : per >= 2 ? 2 : 1;
+    auto k = fused_warp_for<D, 8>(split);
+    if constexpr (D::kBytes == 2)
+      if (wide) k = fused_warp_for<D, 16>(split);
     int grid;
     const int64_t warps = tokens * split;
     if (int rc = persistent_grid((const void*)k, 0, (warps + kThreads / 32 - 1) / (kThreads / 32),

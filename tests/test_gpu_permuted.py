@@ -186,7 +186,8 @@ def _run_unpermute(dev, rt, eo, out_dtype, valid, inv=None, err=None):
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32, torch.float16])
 @pytest.mark.parametrize("tokens,top_k,experts,align,hidden,valid", [
     (50, 2, 4, 4, 72, 50), (300, 8, 64, 16, 1001, 290), (129, 6, 10, 128, 4096, 100),
-    (200, 4, 100, 8, 264, 200), (70, 2, 65, 4, 16, 69), (3000, 8, 64, 16, 512, 2999)])
+    (200, 4, 100, 8, 264, 200), (70, 2, 65, 4, 16, 69), (3000, 8, 64, 16, 512, 2999),
+    (90, 5, 12, 4, 48, 90)])
 def test_unpermute_bitwise(cuda_device, in_dtype, out_dtype, tokens, top_k, experts, align, hidden,
                            valid):
     rt = inputs.routing(tokens, top_k, experts, align, seed=hidden)
@@ -211,12 +212,15 @@ def test_unpermute_full_workload_bitwise(cuda_device, out_dtype):
     assert_bits_equal(got, ref, "unpermute")
 
 
-def test_unpermute_order_witness_and_bad_entries(cuda_device):
+@pytest.mark.parametrize("hidden", [8, 16])
+def test_unpermute_order_witness_and_bad_entries(cuda_device, hidden):
     # contributions 1, 2^24, -2^24 in expert order 0, 1, 2: fp32 gives 0, not 1
+    # (hidden 8: 16-byte loads; 16: 32-byte loads)
     rt = inputs.Routing(2, 3, 3, 1, 3, 3, torch.tensor([0, 1, 2], dtype=torch.int32),
                         torch.tensor([[0, 1, 2], [2, 1, 0]], dtype=torch.int32),
                         torch.ones(6), torch.tensor([2, 2, 2]))
-    eo = torch.tensor([[1.0] * 8, [2.0 ** 24] * 8, [-(2.0 ** 24)] * 8], dtype=torch.bfloat16)
+    eo = torch.tensor([[1.0] * hidden, [2.0 ** 24] * hidden, [-(2.0 ** 24)] * hidden],
+                      dtype=torch.bfloat16)
     got = _run_unpermute(cuda_device, rt, eo, torch.float32, 2)
     assert (got[0] == 0.0).all() and (got[1] == 1.0).all()
     err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
@@ -225,6 +229,31 @@ def test_unpermute_order_witness_and_bad_entries(cuda_device):
     got = _run_unpermute(cuda_device, rt, eo, torch.float32, 5, inv=inv, err=err)
     assert int(err) == _abi.MOE_DEVERR_COUNT | _abi.MOE_DEVERR_INVERSE
     assert (got[0] == 1.0 - 2.0 ** 24).all()
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("eo_off_bytes,out_off_bytes", [(0, 0), (16, 0), (0, 16), (2, 0)])
+def test_unpermute_layouts(cuda_device, out_dtype, eo_off_bytes, out_off_bytes):
+    """32-byte aligned bases (32-byte loads), 16-byte aligned ones (16-byte
+    loads) and an unaligned input (the per-element kernel), hidden 4096."""
+    rt = inputs.routing(257, 8, 64, 16, seed=21)
+    hidden = 4096
+    eo = inputs.expert_output_input(rt, hidden, seed=22)
+    e_off = eo_off_bytes // 2
+    o_off = out_off_bytes // (2 if out_dtype == torch.bfloat16 else 4)
+    flat_e = torch.empty(eo.numel() + e_off, dtype=eo.dtype, device=cuda_device)
+    eo_d = flat_e[e_off:].view(eo.shape)
+    eo_d.copy_(eo.to(cuda_device))
+    flat_o = torch.full((rt.tokens * hidden + o_off,), 3.0, dtype=out_dtype, device=cuda_device)
+    out = flat_o[o_off:].view(rt.tokens, hidden)
+    vt = torch.tensor([rt.tokens - 3], dtype=torch.int32, device=cuda_device)
+    ops.unpermute_ordered(eo_d, rt.inverse_map.to(cuda_device), vt, out)
+    torch.cuda.synchronize()
+    init = bits(torch.full((rt.tokens, hidden), 3.0, dtype=out_dtype))
+    ref, err = oracle.unpermute_ordered(bits(eo), oracle.BF16, bits(rt.inverse_map),
+                                        rt.tokens - 3, init, ODT[out_dtype])
+    assert err == 0
+    assert_bits_equal(bits(out), ref, "unpermute")
 
 
 def test_unpermute_batch_invariant(cuda_device):
