@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle
-from moe_expert_epilogue_b200 import inputs, ops
+from moe_expert_epilogue_b200 import _abi, inputs, ops
 from tests._util import assert_bits_equal, assert_sum_close, bits
 
 pytestmark = pytest.mark.gpu
@@ -53,7 +53,8 @@ def test_router_weight_fwd_16bit_to_fp32_layouts(cuda_device, x_dtype, hidden, x
     assert (obuf[:out_shift] == 7.0).all()
 
 
-@pytest.mark.parametrize("rows,hidden", [(129, 7176), (300, 1001), (1, 8), (3000, 40)])
+@pytest.mark.parametrize("rows,hidden", [(129, 7176), (300, 1001), (1, 8), (3000, 40),
+                                         (257, 7168), (64, 48), (5, 16), (33, 4096)])
 @pytest.mark.parametrize("g_dtype", [torch.bfloat16, torch.float32, torch.float16])
 @pytest.mark.parametrize("x_dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("save_x", [True, False])
@@ -72,6 +73,31 @@ def test_router_weight_bwd(cuda_device, rows, hidden, g_dtype, x_dtype, save_x):
         assert_sum_close(bits(gp).ravel(), gp_ref, gabs, 1e-5, "grad_probs")
     else:
         assert gp is None
+
+
+@pytest.mark.parametrize("g_off,x_off,gx_off", [(0, 0, 0), (8, 0, 0), (0, 8, 0), (0, 0, 8)])
+def test_router_weight_bwd_layouts(cuda_device, g_off, x_off, gx_off):
+    """Bases 32-byte aligned (32-byte loads) or only 16-byte aligned (an
+    offset of 8 bf16 elements: 16-byte loads), 7168-wide rows."""
+    rows, hidden = 200, 7168
+    d = inputs.router_weight_inputs(rows, hidden, seed=17)
+
+    def placed(t, off):
+        buf = torch.empty(t.numel() + off, dtype=t.dtype, device=cuda_device)
+        v = buf[off:].view(t.shape)
+        v.copy_(t.to(cuda_device))
+        return v
+
+    g, x = placed(d["grad_out"], g_off), placed(d["x"], x_off)
+    gx = placed(torch.full((rows, hidden), 5.0, dtype=torch.bfloat16), gx_off)
+    gp = torch.empty(rows, dtype=torch.float32, device=cuda_device)
+    _abi.moe_router_weight_mul_bwd(g, _abi.MOE_BF16, x, _abi.MOE_BF16,
+                                   d["probs"].to(cuda_device), gx, gp, rows, hidden, None)
+    torch.cuda.synchronize()
+    gx_ref, gp_ref, gabs = oracle.router_weight_bwd(bits(d["grad_out"]), oracle.BF16,
+                                                    bits(d["x"]), oracle.BF16, bits(d["probs"]))
+    assert_bits_equal(bits(gx), gx_ref, "grad_x")
+    assert_sum_close(bits(gp).ravel(), gp_ref, gabs, 1e-5, "grad_probs")
 
 
 def test_router_weight_unaligned(cuda_device):
