@@ -348,15 +348,20 @@ struct RowCursor {
 // launched with programmatic stream serialisation allowed and begins with
 // this prologue: griddepcontrol.wait blocks until the grids this one depends
 // on (the previous work in the stream) have completed and their memory is
-// visible -- so nothing is read early -- and launch_dependents lets the next
-// kernel's CTAs be scheduled onto SMs as this kernel's CTAs retire, hiding
-// the launch latency and the tail of each kernel boundary.  Without a
-// programmatic dependency both instructions are no-ops.
+// visible -- so nothing is read early.  The dependents' trigger is left
+// implicit (at CTA exit), so the next kernel's grid is launched as this one
+// completes, hiding the launch latency, and its CTAs never share an SM with
+// this kernel's running ones.  An explicit launch_dependents at the top
+// (MOE_PDL_TRIGGER=1) lets the next grid's CTAs become resident early, where
+// a kernel runs fewer CTAs per SM than fit, and wait there: measured on B200
+// over the nine-kernel epilogue step, 1154 us per step against 1113 with the
+// implicit trigger and 1126 without PDL.  Without a programmatic dependency
+// the wait is a no-op.
 #ifndef MOE_PDL
 #define MOE_PDL 1
 #endif
 #ifndef MOE_PDL_TRIGGER
-#define MOE_PDL_TRIGGER 1
+#define MOE_PDL_TRIGGER 0
 #endif
 __device__ __forceinline__ void pdl_prologue() {
 #if MOE_PDL
