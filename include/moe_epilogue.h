@@ -25,8 +25,11 @@
  *   - Alignment: every pointer must be aligned to its element size
  *     (MOE_ERR_ALIGN otherwise).  16-byte aligned pointers and leading
  *     dimensions / widths that are multiples of 8 elements take the
- *     vectorised path; anything else takes an element-wise path inside the
- *     same kernel family with identical results.
+ *     vectorised path (for 16-bit data, 32-byte aligned pointers and widths
+ *     that are multiples of 16 take 32-byte accesses where that is faster);
+ *     anything else takes an element-wise path inside the same kernel family
+ *     with identical results (grad_probs, a reduction: within its stated
+ *     tolerance, its order fixed for a given layout).
  *   - Aliasing: outputs must not overlap inputs, except that
  *     moe_residual_add and moe_epilogue_fused may run in place
  *     (out == residual).

@@ -8,12 +8,14 @@
 // increasing local expert id.  fp32 sequential adds, no atomics: the bits of
 // a token depend only on that token's rows, never on the grid or the batch.
 //
-// One CTA owns one token at a time (persistent loop up to the
-// device-resident valid_tokens).  Warp 0 compacts a token's inverse-map row
-// into an ordered list of live rows in shared memory (ballot + popc keeps
-// the increasing-expert order), one token ahead; every thread takes 8-column
-// chunks of the hidden dimension and issues the loads of up to 8 contributing
-// rows before it adds them in list order.
+// For E <= 64 a warp owns one (token, column range) item at a time and
+// compacts the token's inverse-map row itself (unpermute_warp); otherwise one
+// CTA owns one token at a time (persistent loop up to the device-resident
+// valid_tokens) and warp 0 compacts a token's inverse-map row into an ordered
+// list of live rows in shared memory, one token ahead.  Either way the
+// compaction (ballot + popc) keeps the increasing-expert order, and every
+// thread issues the loads of up to 8 contributing rows of its chunk (8 or 16
+// columns) before it adds them in list order.
 #include "common.cuh"
 #include "launch.cuh"
 #include "rowlist.cuh"
