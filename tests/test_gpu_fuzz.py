@@ -275,3 +275,108 @@ def test_fuzz_ep_combine(cuda_device, case):
                           f"case {case}: world {world} rank {rank} top-{top_k} of {world}x{epr} "
                           f"tokens {tokens} hidden {hidden} {eo_dt}/{p_dt}/{o_dt}",
                           kind=KIND.get(o_dt, "bf16"))
+
+
+H16 = [torch.bfloat16, torch.float16]
+
+
+@pytest.mark.parametrize("case", range(N_CASES))
+def test_fuzz_32_byte_paths(cuda_device, case):
+    """Widths that are multiples of 16 with bases offset by 0, 8 or 16 elements
+    (32-byte aligned, only 16-byte aligned, 32-byte aligned again): the flat
+    activation, the unpermute and fused chain, the residual add, the
+    router-weight backward and the bounded SwiGLU, each against the oracle."""
+    r = _rng(case, 8)
+    off = int(r.choice([0, 8, 16]))
+    what = f"case {case} off {off}"
+    # permuted activation
+    rt = _routing(r, case)
+    act, oact, tol = [(ops.MOE_ACT_SQRELU, oracle.SQRELU, 0),
+                      (ops.MOE_ACT_SQRELU_CLAMP, oracle.SQRELU_CLAMP, 1),
+                      (ops.MOE_ACT_SWIGLU, oracle.SWIGLU, 1)][case % 3]
+    width = 16 * int(r.integers(1, 100))
+    zero_padding = bool(r.integers(0, 2))
+    n_used = int(r.integers(0, rt.n_used + 1)) if case % 2 else rt.n_used
+    x = inputs.permuted_activation_input(rt, width, swiglu=act == ops.MOE_ACT_SWIGLU, seed=case)
+    canary = torch.full((rt.max_rows, width), 0x1234, dtype=torch.int16).view(torch.bfloat16)
+    out = _place(canary, cuda_device, off)
+    ops.act_with_probs_permuted(act, _place(x, cuda_device, off),
+                                rt.permutation_map.to(cuda_device),
+                                torch.tensor([n_used], dtype=torch.int32, device=cuda_device),
+                                rt.probs.to(cuda_device), 7.0, zero_padding, out=out)
+    torch.cuda.synchronize()
+    ref, err = oracle.act_with_probs_permuted(oact, bits(x), bits(canary), bits(rt.permutation_map),
+                                              n_used, bits(rt.probs), width, 7.0, zero_padding)
+    assert err == 0
+    w_what = f"act {act} width {width} n_used {n_used}/{rt.n_used} " + what
+    if tol == 0:
+        assert_bits_equal(bits(out), ref, w_what)
+    else:
+        assert_within_ulp16(bits(out), ref, tol, what=w_what)
+    # unpermute and fused chain
+    hidden = 16 * int(r.integers(1, 80))
+    in_dt, out_dt = H16[int(r.integers(0, 2))], DT[int(r.integers(0, 3))]
+    valid = int(r.integers(0, rt.tokens + 1))
+    eo = inputs.expert_output_input(rt, hidden, dtype=in_dt, seed=case + 1)
+    eod = _place(eo, cuda_device, off)
+    vt = torch.tensor([valid], dtype=torch.int32, device=cuda_device)
+    init = torch.full((rt.tokens, hidden), 2.5, dtype=out_dt)
+    uo = _place(init, cuda_device, off)
+    ops.unpermute_ordered(eod, rt.inverse_map.to(cuda_device), vt, uo)
+    pm = rt.permutation_map
+    rp = torch.where(pm >= 0, rt.probs[pm.clamp(min=0).long()], torch.zeros(())).float()
+    res = inputs.residual_inputs((rt.tokens, hidden), in_dt, seed=case + 2)
+    finit = torch.full((rt.tokens, hidden), -1.5, dtype=in_dt)
+    fo = _place(finit, cuda_device, off)
+    ops.epilogue_fused(eod, rp.to(cuda_device), rt.inverse_map.to(cuda_device), vt,
+                       _place(res["shared_expert_output"], cuda_device, off),
+                       _place(res["residual"], cuda_device, off), out=fo)
+    torch.cuda.synchronize()
+    u_what = f"hidden {hidden} {in_dt}->{out_dt} valid {valid}/{rt.tokens} " + what
+    uref, err = oracle.unpermute_ordered(bits(eo), ODT[in_dt], bits(rt.inverse_map), valid,
+                                         bits(init), ODT[out_dt])
+    assert err == 0
+    assert_bits_equal(bits(uo), uref, "unpermute " + u_what, kind=KIND.get(out_dt, "bf16"))
+    fref, err = oracle.epilogue_chain(bits(eo), bits(rp), bits(rt.inverse_map), valid,
+                                      bits(res["shared_expert_output"]), bits(res["residual"]),
+                                      bits(finit), ODT[in_dt])
+    assert err == 0
+    assert_bits_equal(bits(fo), fref, "fused " + u_what, kind=KIND.get(in_dt, "bf16"))
+    # residual add, possibly in place
+    dt = H16[case % 2]
+    n = int(r.integers(1, 200000))
+    e, s, rr = (_randn((n,), 1.0, case * 3 + k, dt) for k in range(3))
+    ed, sd, rd = (_place(t, cuda_device, off) for t in (e, s, rr))
+    in_place = bool(r.integers(0, 2))
+    ro = ops.residual_add(ed, sd, rd, out=rd if in_place else None)
+    torch.cuda.synchronize()
+    assert_bits_equal(bits(ro), oracle.residual_add(bits(e), bits(s), bits(rr), ODT[dt]),
+                      f"residual n {n} in place {in_place} " + what, kind=KIND[dt])
+    # router-weight backward with x saved
+    rows, rh = int(r.integers(1, 300)), 16 * int(r.integers(1, 500))
+    g_dt, x_dt = H16[int(r.integers(0, 2))], H16[int(r.integers(0, 2))]
+    xw = _randn((rows, rh), 1.0, case + 3, x_dt)
+    gw = _randn((rows, rh), 1.0, case + 4, g_dt)
+    pw = torch.rand(rows, 1, generator=torch.Generator().manual_seed(case)) + 0.01
+    gx, gp = ops.router_weight_mul_bwd(_place(gw, cuda_device, off), _place(xw, cuda_device, off),
+                                       pw.to(cuda_device))
+    torch.cuda.synchronize()
+    gx_ref, gp_ref, gabs = oracle.router_weight_bwd(bits(gw), ODT[g_dt], bits(xw), ODT[x_dt],
+                                                    bits(pw))
+    rw_what = f"router bwd {rows}x{rh} g {g_dt} x {x_dt} " + what
+    assert_bits_equal(bits(gx), gx_ref, "grad_x " + rw_what, kind=KIND[x_dt])
+    assert_sum_close(bits(gp).ravel(), gp_ref, gabs, 1e-5, "grad_probs " + rw_what)
+    # bounded weighted SwiGLU
+    brows, half_n = int(r.integers(1, 300)), 16 * int(r.integers(1, 60))
+    y = _randn((brows, 2 * half_n), 3.0, case + 5, torch.bfloat16)
+    wb = torch.rand(brows, generator=torch.Generator().manual_seed(case + 6))
+    bound = int(r.integers(0, brows * half_n + 1))
+    bcan = torch.full((brows, half_n), 0x1234, dtype=torch.int16).view(torch.bfloat16)
+    bo = _place(bcan, cuda_device, off)
+    ops.weighted_silu_mul_bounded(_place(y, cuda_device, off), wb.to(cuda_device),
+                                  torch.tensor([bound], dtype=torch.int64, device=cuda_device),
+                                  out=bo)
+    torch.cuda.synchronize()
+    bref, err = oracle.weighted_silu_mul_bounded(bits(y), bits(wb), bits(bcan), bound)
+    assert err == 0
+    assert_within_ulp16(bits(bo), bref, 1, what=f"bounded {brows}x{half_n} bound {bound} " + what)
