@@ -6,6 +6,13 @@ Each ``csrc/*.cu`` is compiled to an object for ``sm_100a`` only (no PTX for
 other targets), then linked with the static CUDA runtime into one shared
 library next to this file, so the library loads on any machine with an NVIDIA
 driver and no CUDA toolkit.  The build needs no GPU.
+
+Tuning builds: ``MOE_BUILD_DEFINES="NAME=VALUE ..."`` in the environment adds
+``-DNAME=VALUE`` for the kernels' compile-time knobs (the ``MOE_*`` macros of
+``csrc``).  The defines of the library on disk are kept in a stamp file beside
+it, and the library counts as up to date only when they equal the
+environment's, so ``MOE_BUILD_DEFINES=... python bench.py`` rebuilds with the
+knobs and a later plain run rebuilds the defaults.
 """
 from __future__ import annotations
 
@@ -22,6 +29,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libmoe_epilogue.so")
+STAMP = LIB + ".defines"
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
@@ -44,11 +52,31 @@ def _deps():
         glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
+def defines() -> list:
+    """The tuning defines requested by MOE_BUILD_DEFINES (sorted), each
+    NAME or NAME=VALUE with NAME a MOE_* macro and VALUE an integer."""
+    out = []
+    for d in os.environ.get("MOE_BUILD_DEFINES", "").split():
+        name, _, value = d.partition("=")
+        if not name.startswith("MOE_") or not name.replace("_", "").isalnum() or \
+                (value and not value.lstrip("-").isdigit()):
+            raise ValueError(f"MOE_BUILD_DEFINES: bad define {d!r} (want MOE_NAME=integer)")
+        out.append(d)
+    return sorted(out)
+
+
+def built_defines() -> list:
+    if not os.path.exists(STAMP):
+        return []
+    with open(STAMP) as f:
+        return sorted(f.read().split())
+
+
 def up_to_date() -> bool:
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(p) <= t for p in _deps())
+    return all(os.path.getmtime(p) <= t for p in _deps()) and built_defines() == defines()
 
 
 def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
@@ -56,7 +84,9 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         return LIB
     os.makedirs(BUILD, exist_ok=True)
     cc = nvcc()
+    defs = defines()
     extra = ["-Xptxas", "-v"] if ptxas_info else []
+    extra += [f"-D{d}" for d in defs]
 
     def compile_one(src):
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
@@ -80,6 +110,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(" ".join(defs))
     return LIB
 
 
