@@ -258,15 +258,16 @@ def time_launches(fn, reps, device):
 
 
 NEXT_ROWS = ("weighted_silu_mul_bounded", "epilogue_fused", "ordered_reduce_scatter_v",
-             "unpermute_reduce_scatter")
+             "unpermute_reduce_scatter", "dtype_variants")
 RS_WORLD = 8  # EP ranks of the rank-order reduce-scatter, all blocks on this GPU
 
 
 def measure_next_rows(device, seed, reps, peak, scale=1.0, only=None):
     """The ops beyond the step: the device-bounded weighted SwiGLU, the fused
     router-weight -> unpermute -> residual chain (against the same chain as
-    three launches) and the rank-order reduce-scatter.  Timed after the step,
-    outside its timed region."""
+    three launches), the rank-order reduce-scatter, the EP combine and the
+    other storage dtypes of the SwiGLU and the router-weight probabilities.
+    Timed after the step, outside its timed region."""
     from moe_expert_epilogue_b200 import inputs, ops
     out = {}
     T = scaled(scale)["permuted"]["tokens"]
@@ -281,6 +282,54 @@ def measure_next_rows(device, seed, reps, peak, scale=1.0, only=None):
     if only in (None, "unpermute_reduce_scatter"):
         out.update(_measure_ep_combine(device, seed, reps, peak, T, K, E, A, H,
                                        long_tokens=8192 if scale == 1.0 else None))
+    if only in (None, "dtype_variants"):
+        out["dtype_variants"] = _measure_dtype_variants(device, seed, reps, peak, scale)
+    return out
+
+
+def _measure_dtype_variants(device, seed, reps, peak, scale=1.0):
+    """The other storage dtypes of the hot path's ops: the clamped SwiGLU fwd and
+    bwd in fp16 and fp32 at the headline shape, and the router-weight fwd and
+    bwd (x saved) with bf16 and fp16 routing probabilities at [16384, 7168]."""
+    from moe_expert_epilogue_b200 import ops
+    out = {}
+    R, I, L = int(SWIGLU["rows"] * scale), SWIGLU["inter"], SWIGLU["limit"]
+    g = torch.Generator(device=device).manual_seed(seed + 41)
+    for dt, name in ((torch.float16, "fp16"), (torch.float32, "fp32")):
+        es = torch.empty((), dtype=dt).element_size()
+        x = (torch.randn(R, 2 * I, generator=g, device=device) * SWIGLU["sigma"]).to(dt)
+        gy = torch.randn(R, I, generator=g, device=device).to(dt)
+        p = torch.rand(R, 1, generator=g, device=device)
+        y = torch.empty(R, I, dtype=dt, device=device)
+        gx = torch.empty(R, 2 * I, dtype=dt, device=device)
+        gp = torch.empty(R, 1, dtype=torch.float32, device=device)
+        ms_f = time_launches(lambda: ops.swiglu_clamped_fwd(x, p, L, out=y), reps, device)
+        ms_b = time_launches(lambda: ops.swiglu_clamped_bwd(x, p, gy, L, grad_x=gx, grad_probs=gp),
+                             reps, device)
+        nb_f = R * (2 * I * es + 4 + I * es)
+        nb_b = R * (2 * I * es + I * es + 4 + 2 * I * es + 4)
+        out[f"swiglu_{name}"] = {"shape": f"rows {R}, inter {I}, L {L}, {name}",
+                                 "fwd": _entry(ms_f, nb_f, peak), "bwd": _entry(ms_b, nb_b, peak),
+                                 "pair": _entry(ms_f + ms_b, nb_f + nb_b, peak)}
+        del x, gy, y, gx
+    Rr, H = int(ROUTER["rows"] * scale), ROUTER["hidden"]
+    x = torch.randn(Rr, H, generator=g, device=device).to(torch.bfloat16)
+    gr = torch.randn(Rr, H, generator=g, device=device).to(torch.bfloat16)
+    o = torch.empty_like(x)
+    gxr = torch.empty_like(x)
+    for pdt, name in ((torch.bfloat16, "bf16"), (torch.float16, "fp16")):
+        p = (torch.rand(Rr, 1, generator=g, device=device) + 0.01).to(pdt)
+        gpr = torch.empty(Rr, 1, dtype=pdt, device=device)
+        ms_f = time_launches(lambda: ops.router_weight_mul_fwd(x, p, torch.bfloat16, out=o), reps,
+                             device)
+        ms_b = time_launches(lambda: ops.router_weight_mul_bwd(gr, x, p, grad_x=gxr,
+                                                               grad_probs=gpr), reps, device)
+        nb_f = Rr * (H * 2 * 2 + 2)
+        nb_b = Rr * (H * 2 * 3 + 2 + 2)
+        out[f"router_weight_probs_{name}"] = {
+            "shape": f"[{Rr}, {H}] bf16 x, {name} probs",
+            "fwd": _entry(ms_f, nb_f, peak), "bwd_save_x": _entry(ms_b, nb_b, peak)}
+    torch.cuda.empty_cache()
     return out
 
 

@@ -146,8 +146,9 @@ MOE_API int moe_swiglu_clamped_fwd(const void* x, const float* probs, void* y, i
 
 /* moe_swiglu_clamped_fwd with an error word of the caller's: dev_err
  * (optional int32, device memory, 4-byte aligned) receives MOE_DEVERR_TIMEOUT
- * if the TMA-staged kernel (bf16 / fp16, contiguous 16-byte aligned rows of
- * at least 512 columns) gave up a barrier wait; with dev_err NULL the bit
+ * if the TMA-staged kernel (contiguous 16-byte aligned rows of at least 512
+ * columns that fit its shared-memory ring: up to 6392 columns in bf16 / fp16,
+ * 3192 in fp32) gave up a barrier wait; with dev_err NULL the bit
  * goes to the per-device word of moe_device_errors().  Same computation,
  * arguments and status codes as moe_swiglu_clamped_fwd. */
 MOE_API int moe_swiglu_clamped_fwd_ex(const void* x, const float* probs, void* y, int64_t rows,

@@ -8,16 +8,17 @@
 //   d_up   = dy * p * silu(gc)        on -L <= u <= L
 //   d_p    = sum_j dy * silu(gc) * uc
 //
-// Forward, 16-bit types: TMA-staged.  One CTA per SM; a producer thread
-// copies whole rows (gate | up, one cp.async.bulk each) into a ring of S
-// shared-memory stages, and 8 consumer warps compute rows out of shared
-// memory, writing y straight to global memory -- S rows (up to ~200 KB) in
-// flight per SM without holding them in registers (measured 4 % faster than
-// the register-staged kernel at rows 65536, inter 2048).  Otherwise (fp32,
-// rows too long for the ring): one warp per row (warps stride over the rows),
-// the row's probability loaded once, U chunks of 8 columns per lane in flight
-// (two loads each: gate, up), one 16-byte store per chunk (two for fp32); a
-// flat grid-stride variant serves rows shorter than 64 chunks.  Backward: W threads
+// Forward: TMA-staged.  One CTA per SM; a producer thread copies whole rows
+// (gate | up, one cp.async.bulk each) into a ring of S shared-memory stages
+// (16, or 8 for rows too long for 16 -- fp32 rows of more than 1592 columns),
+// and 8 consumer warps compute rows out of shared memory, writing y straight
+// to global memory -- S rows (up to ~200 KB) in flight per SM without holding
+// them in registers (measured at rows 65536, inter 2048: 4 % faster than the
+// register-staged kernel in bf16, 14 % in fp32).  Rows too long even for 8
+// stages: one warp per row (warps stride over the rows), the row's
+// probability loaded once, U chunks of 8 columns per lane in flight (two
+// loads each: gate, up), one 16-byte store per chunk (two for fp32); a flat
+// grid-stride variant serves rows shorter than 64 chunks.  Backward: W threads
 // own one row (one warp for the vectorised path), walk its chunks with a fixed
 // column assignment, write d_gate / d_up straight into the two halves of
 // grad_x and reduce the row's probability gradient with a fixed tree
@@ -481,14 +482,12 @@ int fwd(const void* xv, const float* probs, void* yv, int64_t rows, int64_t inte
   const bool vec = inter % kVec == 0 && ld_x % kVec == 0 && ld_y % kVec == 0 && aligned16(x) &&
                    aligned16(y);
   int grid;
-  if constexpr (D::kBytes == 2) {
-    if (MOE_SWIGLU_FWD_TMA && vec && inter / kVec >= 64 && tma_stages<T>(inter) > 0) {
-      int sms = 0;
-      if (int rc = device_sm_count(&sms)) return rc;
-      grid = (int)(rows < sms ? rows : sms);
-      return launch_fwd_tma<D, false>(x, probs, y, rows, inter, ld_x, ld_y, limit, grid, err,
-                                      tma::kWaitCycles, -1, stream);
-    }
+  if (MOE_SWIGLU_FWD_TMA && vec && inter / kVec >= 64 && tma_stages<T>(inter) > 0) {
+    int sms = 0;
+    if (int rc = device_sm_count(&sms)) return rc;
+    grid = (int)(rows < sms ? rows : sms);
+    return launch_fwd_tma<D, false>(x, probs, y, rows, inter, ld_x, ld_y, limit, grid, err,
+                                    tma::kWaitCycles, -1, stream);
   }
   if (vec && inter / kVec >= 64) {
     auto k = swiglu_fwd_rows<D, unroll_for<D>(MOE_SWIGLU_FWD_ROW_UNROLL)>;
@@ -569,8 +568,8 @@ int launch_swiglu_clamped_fwd(const void* x, const float* probs, void* y, int64_
 }
 
 int tma_forward_applies(int64_t inter, moe_dtype dt) {
-  if (dt == MOE_FP32 || inter % kVec != 0 || inter / kVec < 64) return 0;
-  return tma_stages<uint16_t>(inter) > 0;
+  if (inter % kVec != 0 || inter / kVec < 64) return 0;
+  return dt == MOE_FP32 ? tma_stages<float>(inter) > 0 : tma_stages<uint16_t>(inter) > 0;
 }
 
 int launch_swiglu_fwd_stalled(const void* x, const float* probs, void* y, int64_t rows,

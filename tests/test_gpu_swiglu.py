@@ -214,7 +214,8 @@ def _f32_bwd_scale(x, p, dy, limit):
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.float32])
 @pytest.mark.parametrize("rows,inter,limit", [(256, 512, 7.0), (300, 2048, 10.0),
-                                              (97, 1001, 7.0), (64, 40, float("inf"))])
+                                              (97, 1001, 7.0), (64, 40, float("inf")),
+                                              (2048, 3072, 10.0), (300, 3200, 7.0)])
 def test_swiglu_fp16_fp32_parity(cuda_device, dtype, rows, inter, limit):
     d = inputs.swiglu_inputs(rows, inter, sigma=3.0, limit=7.0, plant_ties=True, seed=rows)
     if dtype == torch.float32:
