@@ -348,7 +348,33 @@ __device__ __forceinline__ float row_reduce(float acc, float (*red)[kThreads / 3
 #define MOE_SWIGLU_BWD_MIN_BLOCKS_ATTR __launch_bounds__(kThreads)
 #endif
 
-template <class D, int W, int U>
+// An 8-element chunk of D: one 16-byte access for the 16-bit types; two for
+// fp32, or one 32-byte access when A32 (32-byte aligned fp32 rows).
+template <class D, bool A32>
+__device__ __forceinline__ Raw8<D> load_chunk(const typename D::T* p) {
+  if constexpr (A32) {
+    const u4x2 v = ld_stream32(p);
+    Raw8<D> r;
+    r.w[0] = v.lo;
+    r.w[1] = v.hi;
+    return r;
+  } else {
+    return load8<D>(p);
+  }
+}
+template <class D, bool A32>
+__device__ __forceinline__ void store_chunk(typename D::T* p, const float (&v)[8]) {
+  if constexpr (A32) {
+    st_stream32(p, make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
+                              __float_as_uint(v[3])),
+                make_uint4(__float_as_uint(v[4]), __float_as_uint(v[5]), __float_as_uint(v[6]),
+                           __float_as_uint(v[7])));
+  } else {
+    store8<D>(p, v);
+  }
+}
+
+template <class D, int W, int U, bool A32 = false>
 __global__ void MOE_SWIGLU_BWD_MIN_BLOCKS_ATTR
 swiglu_bwd_vec(const typename D::T* __restrict__ x, const float* __restrict__ probs,
                const typename D::T* __restrict__ gy, typename D::T* __restrict__ gx,
@@ -374,9 +400,9 @@ swiglu_bwd_vec(const typename D::T* __restrict__ x, const float* __restrict__ pr
         for (int k = 0; k < U; ++k) {
           const int64_t c = c0 + (int64_t)k * W;
           if (c < cpr) {
-            gw[k] = load8<D>(xr + c * kVec);
-            uw[k] = load8<D>(xr + inter + c * kVec);
-            dw[k] = load8<D>(gyr + c * kVec);
+            gw[k] = load_chunk<D, A32>(xr + c * kVec);
+            uw[k] = load_chunk<D, A32>(xr + inter + c * kVec);
+            dw[k] = load_chunk<D, A32>(gyr + c * kVec);
           }
         }
 #pragma unroll
@@ -394,8 +420,8 @@ swiglu_bwd_vec(const typename D::T* __restrict__ x, const float* __restrict__ pr
               ou[i] = o.d_up;
               acc += o.t;
             }
-            store8<D>(gxr + c * kVec, og);
-            store8<D>(gxr + inter + c * kVec, ou);
+            store_chunk<D, A32>(gxr + c * kVec, og);
+            store_chunk<D, A32>(gxr + inter + c * kVec, ou);
           }
         }
       }
@@ -465,6 +491,17 @@ inline int threads_per_row(int64_t units) {
 #endif
 #ifndef MOE_SWIGLU_BWD_ROW_THREADS
 #define MOE_SWIGLU_BWD_ROW_THREADS 32
+#endif
+// fp32 rows that are 32-byte aligned take one 32-byte access per 8-element
+// chunk, 4 chunks per lane in flight (141 registers, one CTA per SM).
+// Measured on B200 at 65536 x 2048 fp32: 394.2 us against 457.2 with two
+// 16-byte accesses per chunk (2 chunks per lane), 431.2-431.7 / 423.8-424.1
+// with 2 / 3 chunks of 32 bytes.
+#ifndef MOE_SWIGLU_BWD_F32_WIDE
+#define MOE_SWIGLU_BWD_F32_WIDE 1
+#endif
+#ifndef MOE_SWIGLU_BWD_F32_UNROLL
+#define MOE_SWIGLU_BWD_F32_UNROLL 4
 #endif
 #ifndef MOE_SWIGLU_BWD_UNROLL
 #define MOE_SWIGLU_BWD_UNROLL 4
@@ -538,6 +575,13 @@ int bwd(const void* xv, const float* probs, const void* gyv, void* gxv, float* g
                                         : threads_per_row(vec ? inter / kVec : inter);
   constexpr int U = unroll_for<D>(MOE_SWIGLU_BWD_UNROLL);
 #define MOE_BWD_ARGS stream, x, probs, gy, gx, gp, rows, inter, ld_x, ld_gy, ld_gx, limit
+  if constexpr (D::kBytes == 4) {
+    const bool a32 = MOE_SWIGLU_BWD_F32_WIDE && vec && W == 32 && (inter * 4) % 32 == 0 &&
+                     (ld_x * 4) % 32 == 0 && (ld_gy * 4) % 32 == 0 && (ld_gx * 4) % 32 == 0 &&
+                     aligned32(x) && aligned32(gy) && aligned32(gx);
+    if (a32) return launch_bwd(swiglu_bwd_vec<D, 32, MOE_SWIGLU_BWD_F32_UNROLL, true>, 32,
+                               MOE_BWD_ARGS);
+  }
   if (vec) {
     switch (W) {
       case 32: return launch_bwd(swiglu_bwd_vec<D, 32, U>, 32, MOE_BWD_ARGS);

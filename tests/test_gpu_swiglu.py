@@ -212,6 +212,26 @@ def _f32_bwd_scale(x, p, dy, limit):
     return torch.cat([a * uc.abs() * sg * (1 + gc.abs() * (1 - sg)), a * (gc * sg).abs()], 1)
 
 
+@pytest.mark.parametrize("x_off", [0, 4])
+def test_swiglu_fp32_backward_alignments(cuda_device, x_off):
+    """fp32 backward with 32-byte aligned rows (one 32-byte access per chunk)
+    and with x only 16-byte aligned (two 16-byte accesses), 300 x 1024."""
+    rows, inter, limit = 300, 1024, 7.0
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(rows, 2 * inter, generator=g) * 3.0
+    gy = torch.randn(rows, inter, generator=g)
+    p = torch.rand(rows, 1, generator=g)
+    buf = torch.empty(x.numel() + x_off, dtype=torch.float32, device=cuda_device)
+    xd = buf[x_off:].view(rows, 2 * inter)
+    xd.copy_(x.to(cuda_device))
+    gx, gp = ops.swiglu_clamped_bwd(xd, p.to(cuda_device), gy.to(cuda_device), limit)
+    torch.cuda.synchronize()
+    gx_ref, gp_ref, gabs = oracle.swiglu_clamped_bwd(bits(x), bits(p), bits(gy), limit, oracle.F32)
+    scale = _f32_bwd_scale(x, p, gy, limit).numpy()
+    assert (np.abs(bits(gx) - gx_ref) <= 2 ** -17 * scale + 1e-35).all(), "fp32 grad_x"
+    assert_sum_close(bits(gp).ravel(), gp_ref, gabs, 1e-5, "grad_probs")
+
+
 @pytest.mark.parametrize("dtype", [torch.float16, torch.float32])
 @pytest.mark.parametrize("rows,inter,limit", [(256, 512, 7.0), (300, 2048, 10.0),
                                               (97, 1001, 7.0), (64, 40, float("inf")),
