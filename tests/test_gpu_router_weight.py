@@ -30,14 +30,15 @@ def test_router_weight_fwd_bitwise(cuda_device, rows, hidden, x_dtype, out_dtype
 
 
 @pytest.mark.parametrize("x_dtype", [torch.bfloat16, torch.float16])
-@pytest.mark.parametrize("hidden", [4096, 1004, 12, 7])
-@pytest.mark.parametrize("x_shift,out_shift", [(0, 0), (4, 0), (2, 0), (0, 2)])
+@pytest.mark.parametrize("hidden", [4096, 4104, 1004, 12, 7])
+@pytest.mark.parametrize("x_shift,out_shift", [(0, 0), (4, 0), (2, 0), (0, 2), (0, 4), (8, 0)])
 def test_router_weight_fwd_16bit_to_fp32_layouts(cuda_device, x_dtype, hidden, x_shift,
                                                  out_shift):
-    """A 16-bit input scaled into fp32, with rows of 4-element units (hidden %
-    4 == 0) and without, inputs 8-byte but not 16-byte aligned (x_shift 4),
-    4-byte aligned (2), and an fp32 output off 16-byte alignment: every path
-    gives the oracle's bits."""
+    """A 16-bit input scaled into fp32, with rows of 8- or 4-element units
+    (hidden % 8 == 0, hidden % 4 == 0) and without, inputs 16-byte (x_shift 8),
+    8-byte (4) or 4-byte (2) aligned, and an fp32 output 16- but not 32-byte
+    aligned (out_shift 4) or off 16-byte alignment (2): every path gives the
+    oracle's bits."""
     rows = 37
     d = inputs.router_weight_inputs(rows, hidden, seed=hidden + x_shift)
     x = d["x"].to(x_dtype)
