@@ -231,6 +231,21 @@ template <> __device__ __forceinline__ void widen8<F32>(const Raw8<F32>& r, floa
   v[6] = __uint_as_float(r.w[1].z); v[7] = __uint_as_float(r.w[1].w);
 }
 
+// An 8-element chunk with one 32-byte access where A32 and the type is fp32
+// (a 32-byte aligned address), else as load8 / store8.
+template <class D, bool A32, bool NC = true>
+__device__ __forceinline__ Raw8<D> load8a(const typename D::T* p) {
+  if constexpr (A32 && D::kBytes == 4) {
+    const u4x2 v = NC ? ld_stream32(p) : ld_coherent32(p);
+    Raw8<D> r;
+    r.w[0] = v.lo;
+    r.w[1] = v.hi;
+    return r;
+  } else {
+    return load8<D, NC>(p);
+  }
+}
+
 // Round 8 fp32 values to a 16-bit storage dtype (RNE), packed into 16 bytes.
 template <class D> __device__ __forceinline__ uint4 pack8(const float (&v)[8]);
 template <> __device__ __forceinline__ uint4 pack8<BF16>(const float (&v)[8]) {
@@ -257,6 +272,18 @@ template <> __device__ __forceinline__ void store8<F32>(float* p, const float (&
                           __float_as_uint(v[3])));
   st_stream(p + 4, make_uint4(__float_as_uint(v[4]), __float_as_uint(v[5]),
                               __float_as_uint(v[6]), __float_as_uint(v[7])));
+}
+
+template <class D, bool A32>
+__device__ __forceinline__ void store8a(typename D::T* p, const float (&v)[8]) {
+  if constexpr (A32 && D::kBytes == 4) {
+    st_stream32(p, make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
+                              __float_as_uint(v[3])),
+                make_uint4(__float_as_uint(v[4]), __float_as_uint(v[5]), __float_as_uint(v[6]),
+                           __float_as_uint(v[7])));
+  } else {
+    store8<D>(p, v);
+  }
 }
 
 // ------------------------------------------------------------ math

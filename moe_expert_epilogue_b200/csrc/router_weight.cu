@@ -83,7 +83,7 @@ __device__ __forceinline__ void store_prob(void* p, int dt, int64_t i, float v) 
 }
 
 // out[r, :] = cast(in[r, :] * p[r]) over a [rows, cpr] chunk grid.
-template <class DI, class DO, int PDT>
+template <class DI, class DO, int PDT, bool A32 = false>
 __global__ void __launch_bounds__(kThreads)
 scale_rows_vec(const typename DI::T* __restrict__ in, const void* __restrict__ probs, int p_dt,
                typename DO::T* __restrict__ out, int64_t rows, int64_t hidden) {
@@ -103,12 +103,11 @@ scale_rows_vec(const typename DI::T* __restrict__ in, const void* __restrict__ p
     for (int k = 0; k < U; ++k) {
       if (q + k * S < total) {
         off[k] = cur.r * hidden + cur.c * kVec;
-        raw[k] = load8<DI>(in + off[k]);
+        raw[k] = load8a<DI, A32>(in + off[k]);
         p[k] = load_prob_t<PDT>(probs, p_dt, cur.r);
       }
       cur.advance();
     }
-
 #pragma unroll
     for (int k = 0; k < U; ++k) {
       if (q + k * S < total) {
@@ -116,7 +115,7 @@ scale_rows_vec(const typename DI::T* __restrict__ in, const void* __restrict__ p
         widen8<DI>(raw[k], v);
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = v[i] * p[k];
-        store8<DO>(out + off[k], v);
+        store8a<DO, A32>(out + off[k], v);
       }
     }
   }
@@ -380,6 +379,12 @@ scale_rows_to_f32_wide(const uint16_t* __restrict__ in, const void* __restrict__
 #ifndef MOE_RW_F32OUT_WIDE_U
 #define MOE_RW_F32OUT_WIDE_U 2
 #endif
+// fp32 input or output sides with 32-byte alignment: one 32-byte access per
+// 8-element chunk.  Measured on B200 at [16384, 7168], fp32 grad_out into bf16
+// grad_x (x not saved): 112.8-113.0 us against 117.7.
+#ifndef MOE_RW_F32_WIDE
+#define MOE_RW_F32_WIDE 1
+#endif
 
 template <class DI, class DO, int PDT>
 int launch_scale_t(const void* in, const void* probs, int p_dt, void* out, int64_t rows,
@@ -412,7 +417,10 @@ int launch_scale_t(const void* in, const void* probs, int p_dt, void* out, int64
     }
   }
   if (hidden % kVec == 0 && aligned16(in) && aligned16(out)) {
-    auto k = scale_rows_vec<DI, DO, PDT>;
+    // fp32 sides with 32-byte alignment take one 32-byte access per chunk
+    const bool a32 = MOE_RW_F32_WIDE && (DI::kBytes == 4 || DO::kBytes == 4) &&
+                     (DI::kBytes != 4 || aligned32(in)) && (DO::kBytes != 4 || aligned32(out));
+    auto k = a32 ? scale_rows_vec<DI, DO, PDT, true> : scale_rows_vec<DI, DO, PDT, false>;
     const int64_t units = rows * (hidden / kVec);
     if (int rc = persistent_grid((const void*)k, 0,
                                  (units + kThreads * scale_unroll<DI>() - 1) /

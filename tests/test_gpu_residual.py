@@ -50,23 +50,24 @@ def test_residual_add_in_place_and_unaligned(cuda_device, dtype):
     assert_bits_equal(bits(out), ref, "unaligned", kind=_kind(dtype))
 
 
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("dtype", DTYPES)
 @pytest.mark.parametrize("which", [0, 1, 2, 3])
 def test_residual_add_16_byte_aligned(cuda_device, dtype, which):
     """One of the four tensors 16- but not 32-byte aligned (the 16-byte
     stream instead of the 32-byte one), 10007 elements."""
     n = 10007
+    shift = 16 // torch.empty((), dtype=dtype).element_size()
     d = inputs.residual_inputs((n,), dtype, seed=9)
     names = ("expert_output", "shared_expert_output", "residual")
     ref = oracle.residual_add(*(bits(d[k]) for k in names), ODT[dtype])
     ts = []
     for i, k in enumerate(names):
-        off = 8 if i == which else 0
+        off = shift if i == which else 0
         buf = torch.empty(n + off, dtype=dtype, device=cuda_device)
         ts.append(buf[off:])
         ts[-1].copy_(d[k].to(cuda_device))
-    obuf = torch.empty(n + (8 if which == 3 else 0), dtype=dtype, device=cuda_device)
-    out = obuf[8 if which == 3 else 0:]
+    obuf = torch.empty(n + (shift if which == 3 else 0), dtype=dtype, device=cuda_device)
+    out = obuf[shift if which == 3 else 0:]
     ops.residual_add(*ts, out=out)
     torch.cuda.synchronize()
     assert_bits_equal(bits(out), ref, "16-byte aligned", kind=_kind(dtype))

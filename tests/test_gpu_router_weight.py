@@ -101,6 +101,24 @@ def test_router_weight_bwd_layouts(cuda_device, g_off, x_off, gx_off):
     assert_sum_close(bits(gp).ravel(), gp_ref, gabs, 1e-5, "grad_probs")
 
 
+@pytest.mark.parametrize("off", [0, 4])
+def test_router_weight_bwd_fp32_grad_without_x(cuda_device, off):
+    """fp32 grad_out, x not saved: 32-byte aligned rows (one 32-byte load per
+    chunk) and rows only 16-byte aligned (off 4 floats: two 16-byte loads)."""
+    rows, hidden = 130, 7168
+    d = inputs.router_weight_inputs(rows, hidden, out_dtype=torch.float32, seed=23)
+    buf = torch.empty(rows * hidden + off, dtype=torch.float32, device=cuda_device)
+    g = buf[off:].view(rows, hidden)
+    g.copy_(d["grad_out"].to(cuda_device))
+    gx, gp = ops.router_weight_mul_bwd(g, None, d["probs"].to(cuda_device),
+                                       x_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    gx_ref, _, _ = oracle.router_weight_bwd(bits(d["grad_out"]), oracle.F32, None, oracle.BF16,
+                                            bits(d["probs"]))
+    assert gp is None
+    assert_bits_equal(bits(gx), gx_ref, "grad_x")
+
+
 def test_router_weight_unaligned(cuda_device):
     rows, hidden = 33, 64
     d = inputs.router_weight_inputs(rows, hidden, seed=5)
