@@ -7,8 +7,9 @@
 // Both adds in fp32, each result rounded to the activation dtype, so the
 // output is bit-identical to the two unfused adds.  One flat grid-stride
 // stream: for 16-bit types with 32-byte aligned bases three 32-byte loads and
-// one 32-byte store per 16 elements, otherwise three 16-byte loads and one
-// 16-byte store per 8 elements (two of each for fp32).  In place (out ==
+// one 32-byte store per 16 elements; for fp32 with 32-byte aligned bases the
+// same per 8 elements; otherwise three 16-byte loads and one 16-byte store
+// per 8 elements (two of each for fp32).  In place (out ==
 // residual) is safe: every element is read and written by the same thread,
 // load before store, and the residual is read through the coherent path
 // (never the read-only one).

@@ -7,10 +7,12 @@
 //         grad_p = sum_h g.float() * x.float()               fp32 row reduction
 //
 // The forward and the x-only backward are flat grid-stride streams over
-// 8-element chunks.  The backward with the probability gradient walks rows
-// like the SwiGLU backward: W threads per row, fixed column assignment, fixed
-// reduction tree, no fp32 intermediate ever leaves the registers (16-bit rows
-// with 32-byte alignment: 16-column chunks, otherwise 8).
+// 8-element chunks (an fp32 side 32-byte aligned moves each chunk with one
+// 32-byte access; 16-bit input into fp32 output takes one 16-byte load and one
+// 32-byte store per chunk).  The backward with the probability gradient walks
+// rows like the SwiGLU backward: W threads per row, fixed column assignment,
+// fixed reduction tree, no fp32 intermediate ever leaves the registers (16-bit
+// rows with 32-byte alignment: 16-column chunks, otherwise 8).
 #include <type_traits>
 
 #include "common.cuh"
