@@ -37,7 +37,9 @@ timed region, pipelined), `configs` (the workload's other configurations:
 the small SwiGLU, the router-weight output-dtype / save_x variants, the
 residual add in three dtypes alone and chained after the router-weight
 forward, the fp32-output unpermute), `next_rows` (the bounded SwiGLU, the
-fused chain, the reduce-scatter and the EP combine, timed after the step),
+fused chain, the reduce-scatter, the EP combine, and the other storage dtypes:
+the SwiGLU in fp16 and fp32, the router weight with bf16 and fp16
+probabilities; timed after the step),
 `clocks`, `roofline` and `cpu_baseline` (the CPU oracle, one core and all
 cores).  `--impl reference` times the CPU oracle alone on every host core.
 """
